@@ -1,0 +1,837 @@
+// C ABI of the scorer (include/rm.h, include/rm_ops.h): validation, weight
+// upload, the arena, per-call metadata and the forward launch sequence.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "../../include/rm.h"
+#include "../../include/rm_ops.h"
+#include "common.cuh"
+#include "host.h"
+#include "kernels.h"
+
+namespace rmk {
+
+namespace {
+thread_local char g_msg[512] = "";
+__device__ int32_t g_err_sink[ERR_WORDS];   // error words for handle-less rm_op_* calls
+}  // namespace
+
+int set_error(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define RM_CUDA(call)                                                                  \
+  do {                                                                                 \
+    cudaError_t e_ = (call);                                                           \
+    if (e_ != cudaSuccess)                                                             \
+      return set_error(e_ == cudaErrorMemoryAllocation ? RM_E_NOMEM : RM_E_CUDA,       \
+                       "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+int validate_config(const rm_config* c, bool sched_only, const char** why) {
+  auto bad = [&](const char* m) { *why = m; return RM_E_INVAL; };
+  if (c == nullptr) return bad("config is NULL");
+  if (c->max_len < 1 || c->max_len > 1024) return bad("max_len must be in 1..1024");
+  if (c->sched_max_batch < 1) return bad("sched_max_batch must be >= 1");
+  if (c->sched_c0 < 0 || c->sched_c1 < 0 || c->sched_c0 > (1LL << 40) || c->sched_c1 > (1LL << 40))
+    return bad("sched_c0 and sched_c1 must be in 0..2^40");
+  if (c->sched_table != nullptr) {
+    if (c->sched_table_b < c->sched_max_batch || c->sched_table_l < c->max_len)
+      return bad("sched_table must have >= sched_max_batch rows and >= max_len columns");
+    for (int32_t b = 0; b < c->sched_table_b; ++b)
+      for (int32_t l = 0; l < c->sched_table_l; ++l) {
+        const int64_t v = c->sched_table[static_cast<size_t>(b) * c->sched_table_l + l];
+        if (v < 0 || v > (1LL << 56)) return bad("sched_table entries must be in 0..2^56");
+        if (l > 0 && v < c->sched_table[static_cast<size_t>(b) * c->sched_table_l + l - 1])
+          return bad("sched_table must be non-decreasing along L");
+      }
+  }
+  if (sched_only) return RM_OK;
+  if (c->arch != RM_ENC_POSTLN && c->arch != RM_DEC_PRELN) return bad("arch must be 0 or 1");
+  if (c->n_layers < 1) return bad("n_layers must be >= 1");
+  if (c->hidden < 8 || c->hidden > 4096 || c->hidden % 8 != 0)
+    return bad("hidden must be a multiple of 8 in 8..4096");
+  if (c->n_heads < 1 || c->hidden % c->n_heads != 0) return bad("n_heads must divide hidden");
+  const int d = c->hidden / c->n_heads;
+  if (d % 2 != 0 || d > 128) return bad("head dim hidden/n_heads must be even and <= 128");
+  if (c->ffn < 8 || c->ffn % 8 != 0 || c->ffn > 65536) return bad("ffn must be a multiple of 8");
+  if (c->vocab < 1) return bad("vocab must be >= 1");
+  if (c->max_pos < c->max_len) return bad("max_pos must be >= max_len");
+  if (c->weight_dtype != RM_F32 && c->weight_dtype != RM_BF16) return bad("weight_dtype must be 0 or 1");
+  if (c->gelu != RM_GELU_ERF && c->gelu != RM_GELU_TANH) return bad("gelu must be 0 or 1");
+  if (!(c->ln_eps > 0.0f) || !std::isfinite(c->ln_eps)) return bad("ln_eps must be > 0");
+  if (c->max_batch_seqs < 1) return bad("max_batch_seqs must be >= 1");
+  if (c->max_tokens < 1 || c->max_tokens > (1 << 24)) return bad("max_tokens must be in 1..2^24");
+  return RM_OK;
+}
+
+SchedCost sched_cost_from(const rm_config* c) {
+  SchedCost s;
+  s.bmax = c->sched_max_batch;
+  s.c0 = c->sched_c0;
+  s.c1 = c->sched_c1;
+  if (c->sched_table != nullptr) {
+    s.tb = c->sched_table_b;
+    s.tl = c->sched_table_l;
+    s.table.assign(c->sched_table, c->sched_table + static_cast<size_t>(s.tb) * s.tl);
+  }
+  return s;
+}
+
+namespace {
+
+// ---- weight layout ----
+struct Segment {
+  const char* name;
+  int64_t elems;
+  bool matrix;       // stored bf16 on device (GEMM operand or embedding table)
+};
+
+std::vector<Segment> segments(const rm_config* c) {
+  const int64_t H = c->hidden, F = c->ffn;
+  std::vector<Segment> s;
+  s.push_back({"emb_word", static_cast<int64_t>(c->vocab) * H, true});
+  s.push_back({"emb_pos", static_cast<int64_t>(c->max_pos) * H, true});
+  if (c->arch == RM_ENC_POSTLN) {
+    s.push_back({"ln_emb_g", H, false});
+    s.push_back({"ln_emb_b", H, false});
+  }
+  for (int l = 0; l < c->n_layers; ++l) {
+    s.push_back({"w_qkv", 3 * H * H, true});
+    s.push_back({"b_qkv", 3 * H, false});
+    s.push_back({"w_o", H * H, true});
+    s.push_back({"b_o", H, false});
+    s.push_back({"ln1_g", H, false});
+    s.push_back({"ln1_b", H, false});
+    s.push_back({"w_1", F * H, true});
+    s.push_back({"b_1", F, false});
+    s.push_back({"w_2", H * F, true});
+    s.push_back({"b_2", H, false});
+    s.push_back({"ln2_g", H, false});
+    s.push_back({"ln2_b", H, false});
+  }
+  if (c->arch == RM_DEC_PRELN) {
+    s.push_back({"lnf_g", H, false});
+    s.push_back({"lnf_b", H, false});
+  }
+  s.push_back({"w_r", H, false});
+  s.push_back({"b_r", 1, false});
+  return s;
+}
+
+int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+struct LayerW {
+  bf16 *w_qkv, *w_o, *w_1, *w_2;
+  float *b_qkv, *b_o, *ln1_g, *ln1_b, *b_1, *b_2, *ln2_g, *ln2_b;
+  CUtensorMap tm[4][2];   // [qkv, o, 1, 2][box rows 128, 256]
+};
+
+struct Bucket {
+  ArenaPlan plan;
+  CUtensorMap a_in, a_ctx, a_f;   // A operands: x (encoder) or z (decoder), ctx, f
+};
+
+constexpr int kSlots = 4;
+
+}  // namespace
+}  // namespace rmk
+
+using namespace rmk;
+
+struct rm_handle {
+  rm_config cfg;
+  SchedCost sched;
+  int device = 0, num_sms = 148;
+  void* wbuf = nullptr;
+  bf16 *emb_word = nullptr, *emb_pos = nullptr;
+  float *ln_emb_g = nullptr, *ln_emb_b = nullptr, *lnf_g = nullptr, *lnf_b = nullptr,
+        *w_r = nullptr;
+  float b_r = 0.f;
+  std::vector<LayerW> layers;
+  uint8_t* arena = nullptr;
+  int64_t arena_bytes = 0, fixed_bytes = 0, meta_bytes = 0;
+  int32_t* d_ids = nullptr;
+  float* d_scores = nullptr;
+  uint8_t* d_meta = nullptr;
+  uint8_t* planned = nullptr;
+  int32_t* d_err = nullptr;
+  uint8_t* pinned = nullptr;
+  cudaEvent_t ev[kSlots] = {};
+  int slot = 0;
+  std::map<std::pair<int64_t, int64_t>, Bucket> buckets;
+  int64_t max_peak = 0;
+  cudaStream_t last_stream = nullptr;
+  // measurement
+  int64_t launches = 0, calls = 0;
+  int32_t prof_every = 0;
+  struct ProfRec { int cls; double flops, bytes; cudaEvent_t a, b; };
+  std::vector<ProfRec> prof;
+  std::vector<cudaEvent_t> ev_pool;
+};
+
+namespace {
+
+// Metadata of one call in a staging slot / the device meta region:
+// offsets int32[n+1] | rb_off int32[n+1] | s_off int64[n+1]  (16-byte aligned parts)
+struct MetaLayout {
+  int64_t rb, so, bytes;
+  explicit MetaLayout(int64_t n) {
+    rb = align_up(4 * (n + 1), 16);
+    so = rb + align_up(4 * (n + 1), 16);
+    bytes = so + align_up(8 * (n + 1), 16);
+  }
+};
+
+int host_varlen_meta(const int32_t* off, int32_t n, int32_t nh, int32_t* rb, int64_t* so,
+                     int32_t* max_len) {
+  if (off[0] != 0) return set_error(RM_E_INVAL, "seq_offsets[0] must be 0");
+  rb[0] = 0;
+  so[0] = 0;
+  int32_t ml = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t L = static_cast<int64_t>(off[i + 1]) - off[i];
+    if (L < 1) return set_error(RM_E_INVAL, "sequence %d has length %lld (< 1)", i, (long long)L);
+    ml = std::max<int32_t>(ml, static_cast<int32_t>(L));
+    rb[i + 1] = rb[i] + static_cast<int32_t>((L + 63) / 64);
+    so[i + 1] = so[i] + static_cast<int64_t>(nh) * L * align_up(L, 8);
+  }
+  if (max_len) *max_len = ml;
+  return RM_OK;
+}
+
+int upload_weights(rm_handle* h, const void* weights) {
+  const rm_config* c = &h->cfg;
+  const auto seg = segments(c);
+  const int esz = c->weight_dtype == RM_F32 ? 4 : 2;
+  int64_t nbf = 0, nf = 0, total = 0;
+  for (const auto& s : seg) {
+    if (s.matrix) nbf += align_up(s.elems, 128);
+    else nf += align_up(s.elems, 64);
+    total += s.elems;
+  }
+  const size_t wbytes = static_cast<size_t>(nbf) * 2 + static_cast<size_t>(nf) * 4;
+  RM_CUDA(cudaMalloc(&h->wbuf, wbytes));
+  void* staging = nullptr;
+  RM_CUDA(cudaMalloc(&staging, static_cast<size_t>(total) * esz));
+  cudaError_t e = cudaMemcpy(staging, weights, static_cast<size_t>(total) * esz, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(staging);
+    return set_error(RM_E_CUDA, "weight upload: %s", cudaGetErrorString(e));
+  }
+  bf16* pb = static_cast<bf16*>(h->wbuf);
+  float* pf = reinterpret_cast<float*>(static_cast<uint8_t*>(h->wbuf) + nbf * 2);
+  int64_t src = 0;
+  int layer = -1;
+  for (const auto& s : seg) {
+    const void* from = static_cast<const uint8_t*>(staging) + src * esz;
+    void* dst;
+    if (s.matrix) {
+      dst = pb;
+      e = cvt_to_bf16_launch(from, c->weight_dtype, pb, static_cast<size_t>(s.elems), 0);
+      pb += align_up(s.elems, 128);
+    } else {
+      dst = pf;
+      e = cvt_to_f32_launch(from, c->weight_dtype, pf, static_cast<size_t>(s.elems), 0);
+      pf += align_up(s.elems, 64);
+    }
+    if (e != cudaSuccess) break;
+    const std::string nm = s.name;
+    if (nm == "w_qkv") { h->layers.emplace_back(); ++layer; }
+    LayerW* L = layer >= 0 ? &h->layers[layer] : nullptr;
+    if (nm == "emb_word") h->emb_word = static_cast<bf16*>(dst);
+    else if (nm == "emb_pos") h->emb_pos = static_cast<bf16*>(dst);
+    else if (nm == "ln_emb_g") h->ln_emb_g = static_cast<float*>(dst);
+    else if (nm == "ln_emb_b") h->ln_emb_b = static_cast<float*>(dst);
+    else if (nm == "lnf_g") h->lnf_g = static_cast<float*>(dst);
+    else if (nm == "lnf_b") h->lnf_b = static_cast<float*>(dst);
+    else if (nm == "w_r") h->w_r = static_cast<float*>(dst);
+    else if (nm == "b_r") {
+      // the head bias is also a kernel argument: read it on the host
+      if (c->weight_dtype == RM_F32) {
+        std::memcpy(&h->b_r, static_cast<const uint8_t*>(weights) + src * 4, 4);
+      } else {
+        uint16_t bits;
+        std::memcpy(&bits, static_cast<const uint8_t*>(weights) + src * 2, 2);
+        const uint32_t u = static_cast<uint32_t>(bits) << 16;
+        std::memcpy(&h->b_r, &u, 4);
+      }
+    } else if (L) {
+      if (nm == "w_qkv") L->w_qkv = static_cast<bf16*>(dst);
+      else if (nm == "b_qkv") L->b_qkv = static_cast<float*>(dst);
+      else if (nm == "w_o") L->w_o = static_cast<bf16*>(dst);
+      else if (nm == "b_o") L->b_o = static_cast<float*>(dst);
+      else if (nm == "ln1_g") L->ln1_g = static_cast<float*>(dst);
+      else if (nm == "ln1_b") L->ln1_b = static_cast<float*>(dst);
+      else if (nm == "w_1") L->w_1 = static_cast<bf16*>(dst);
+      else if (nm == "b_1") L->b_1 = static_cast<float*>(dst);
+      else if (nm == "w_2") L->w_2 = static_cast<bf16*>(dst);
+      else if (nm == "b_2") L->b_2 = static_cast<float*>(dst);
+      else if (nm == "ln2_g") L->ln2_g = static_cast<float*>(dst);
+      else if (nm == "ln2_b") L->ln2_b = static_cast<float*>(dst);
+    }
+    src += s.elems;
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  cudaFree(staging);
+  if (e != cudaSuccess) return set_error(RM_E_CUDA, "weight conversion: %s", cudaGetErrorString(e));
+  // TMA maps of every weight matrix, for both column-tile widths
+  const int64_t H = c->hidden, F = c->ffn;
+  for (auto& L : h->layers) {
+    const bf16* mats[4] = {L.w_qkv, L.w_o, L.w_1, L.w_2};
+    const int64_t rows[4] = {3 * H, H, F, H}, cols[4] = {H, H, H, F};
+    for (int m = 0; m < 4; ++m)
+      for (int b = 0; b < 2; ++b) {
+        const char* why = "";
+        if (!make_tmap_bf16(&L.tm[m][b], mats[m], rows[m], cols[m], b ? 256 : 128, &why))
+          return set_error(RM_E_CUDA, "weight tensor map: %s", why);
+      }
+  }
+  return RM_OK;
+}
+
+int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
+  // length buckets: tokens rounded up to 128, score elements to 64 Ki
+  const int64_t Tb = align_up(T, 128), Sb = align_up(std::max<int64_t>(S, 1), 65536);
+  auto key = std::make_pair(Tb, Sb);
+  auto it = h->buckets.find(key);
+  if (it != h->buckets.end()) {
+    *out = &it->second;
+    return RM_OK;
+  }
+  const rm_config* c = &h->cfg;
+  Bucket b;
+  b.plan = plan_arena(c->arch, c->hidden, c->ffn, Tb, Sb);
+  if (h->fixed_bytes + b.plan.peak > h->arena_bytes)
+    return set_error(RM_E_RANGE, "arena plan (%lld bytes) exceeds the reservation",
+                     (long long)b.plan.peak);
+  uint8_t* base = h->planned;
+  const void* a_in = base + (c->arch == RM_DEC_PRELN ? b.plan.off[B_Z] : b.plan.off[B_X]);
+  const char* why = "";
+  if (!make_tmap_bf16(&b.a_in, a_in, Tb, c->hidden, 128, &why) ||
+      !make_tmap_bf16(&b.a_ctx, base + b.plan.off[B_CTX], Tb, c->hidden, 128, &why) ||
+      !make_tmap_bf16(&b.a_f, base + b.plan.off[B_F], Tb, c->ffn, 128, &why))
+    return set_error(RM_E_CUDA, "activation tensor map: %s", why);
+  h->max_peak = std::max(h->max_peak, b.plan.peak);
+  auto res = h->buckets.emplace(key, b);
+  *out = &res.first->second;
+  return RM_OK;
+}
+
+int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[2], int M, int N, int K,
+         const float* bias, void* y, int act, cudaStream_t st) {
+  const int bn = gemm_pick_bn(M, N, h->num_sms);
+  cudaError_t e = gemm_launch(a, b[bn == 256 ? 1 : 0], bn, M, N, K, bias, y, false, act,
+                              h->d_err, st);
+  if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
+  return RM_OK;
+}
+
+#define RM_LAUNCH(call)                                                                   \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return set_error(RM_E_CUDA, "%s: %s", #call, cudaGetErrorString(e_));              \
+  } while (0)
+#define RM_TRY(call)          \
+  do {                        \
+    int r_ = (call);          \
+    if (r_ != RM_OK) return r_; \
+  } while (0)
+
+// Events around one launch when this call is profiled.
+struct ProfScope {
+  rm_handle* h;
+  bool on;
+  cudaEvent_t a = nullptr, b = nullptr;
+  cudaStream_t st;
+  ProfScope(rm_handle* hh, bool enabled, cudaStream_t s) : h(hh), on(enabled), st(s) {
+    if (!on) return;
+    a = take();
+    b = take();
+    if (a == nullptr || b == nullptr || cudaEventRecord(a, st) != cudaSuccess) on = false;
+  }
+  cudaEvent_t take() {
+    if (!h->ev_pool.empty()) {
+      cudaEvent_t e = h->ev_pool.back();
+      h->ev_pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    return cudaEventCreate(&e) == cudaSuccess ? e : nullptr;
+  }
+  void done(int cls, double flops, double bytes) {
+    ++h->launches;
+    if (on && cudaEventRecord(b, st) == cudaSuccess) {
+      h->prof.push_back({cls, flops, bytes, a, b});
+      a = b = nullptr;
+    }
+  }
+  ~ProfScope() {
+    if (a) h->ev_pool.push_back(a);
+    if (b) h->ev_pool.push_back(b);
+  }
+};
+
+#define RM_KERNEL(cls, flops, bytes, call)          \
+  do {                                               \
+    ProfScope ps_(h, prof_on, st);                   \
+    RM_LAUNCH(call);                                 \
+    ps_.done(cls, flops, bytes);                     \
+  } while (0)
+#define RM_GEMM(flops, bytes, call)                  \
+  do {                                               \
+    ProfScope ps_(h, prof_on, st);                   \
+    RM_TRY(call);                                    \
+    ps_.done(RM_K_GEMM, flops, bytes);               \
+  } while (0)
+
+// host_ids != NULL: copy the ids host->device (into the arena) once the call
+// has been validated, and the scores back into host_out at the end.
+int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, const int32_t* offsets,
+               int32_t n, float* d_out, float* host_out, cudaStream_t st) {
+  const rm_config* c = &h->cfg;
+  if (n < 1) return set_error(RM_E_INVAL, "n_seqs must be >= 1");
+  if (n > c->max_batch_seqs)
+    return set_error(RM_E_RANGE, "n_seqs %d exceeds max_batch_seqs %d", n, c->max_batch_seqs);
+  // metadata into the next pinned slot
+  const int slot = h->slot;
+  h->slot = (h->slot + 1) % kSlots;
+  RM_CUDA(cudaEventSynchronize(h->ev[slot]));
+  uint8_t* ps = h->pinned + static_cast<size_t>(slot) * h->meta_bytes;
+  const MetaLayout ml(n);
+  int32_t* p_off = reinterpret_cast<int32_t*>(ps);
+  int32_t* p_rb = reinterpret_cast<int32_t*>(ps + ml.rb);
+  int64_t* p_so = reinterpret_cast<int64_t*>(ps + ml.so);
+  if (offsets[0] != 0) return set_error(RM_E_INVAL, "seq_offsets[0] must be 0");
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t L = static_cast<int64_t>(offsets[i + 1]) - offsets[i];
+    if (L < 1) return set_error(RM_E_INVAL, "sequence %d has length %lld (< 1)", i, (long long)L);
+    if (L > c->max_len)
+      return set_error(RM_E_RANGE, "sequence %d has length %lld > max_len %d", i, (long long)L,
+                       c->max_len);
+  }
+  const int32_t T = offsets[n];
+  if (T > c->max_tokens)
+    return set_error(RM_E_RANGE, "%d tokens exceed max_tokens %d", T, c->max_tokens);
+  std::memcpy(p_off, offsets, 4 * static_cast<size_t>(n + 1));
+  int32_t Lmax = 0;
+  RM_TRY(host_varlen_meta(offsets, n, c->n_heads, p_rb, p_so, &Lmax));
+  const int32_t nrb = p_rb[n];
+  const int64_t S = p_so[n];
+  if (host_ids != nullptr) {
+    RM_CUDA(cudaMemcpyAsync(h->d_ids, host_ids, 4 * static_cast<size_t>(T), cudaMemcpyHostToDevice, st));
+    d_ids = h->d_ids;
+    d_out = h->d_scores;
+  }
+  RM_CUDA(cudaMemcpyAsync(h->d_meta, ps, ml.bytes, cudaMemcpyHostToDevice, st));
+  RM_CUDA(cudaEventRecord(h->ev[slot], st));
+  const int32_t* d_off = reinterpret_cast<const int32_t*>(h->d_meta);
+  const int32_t* d_rb = reinterpret_cast<const int32_t*>(h->d_meta + ml.rb);
+  const int64_t* d_so = reinterpret_cast<const int64_t*>(h->d_meta + ml.so);
+
+  Bucket* bk = nullptr;
+  RM_TRY(get_bucket(h, T, S, &bk));
+  uint8_t* base = h->planned;
+  bf16* x = reinterpret_cast<bf16*>(base + bk->plan.off[B_X]);
+  bf16* z = reinterpret_cast<bf16*>(base + bk->plan.off[B_Z]);
+  bf16* qkv = reinterpret_cast<bf16*>(base + bk->plan.off[B_QKV]);
+  bf16* s = reinterpret_cast<bf16*>(base + bk->plan.off[B_S]);
+  bf16* ctx = reinterpret_cast<bf16*>(base + bk->plan.off[B_CTX]);
+  bf16* y1 = reinterpret_cast<bf16*>(base + bk->plan.off[B_Y1]);
+  bf16* f = reinterpret_cast<bf16*>(base + bk->plan.off[B_F]);
+  bf16* y2 = reinterpret_cast<bf16*>(base + bk->plan.off[B_Y2]);
+  const int H = c->hidden, F = c->ffn, nh = c->n_heads, d = H / nh;
+  const int act = c->gelu == RM_GELU_TANH ? 2 : 1;
+  const bool dec = c->arch == RM_DEC_PRELN;
+  const float eps = c->ln_eps;
+  const bool prof_on = h->prof_every > 0 && (h->calls % h->prof_every) == 0;
+  ++h->calls;
+
+  // algorithmic work of each launch (unpadded tokens; attention entries that
+  // the mask admits: L*L per head, or L*(L+1)/2 when causal)
+  double att = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const double L = static_cast<double>(offsets[i + 1] - offsets[i]);
+    att += dec ? L * (L + 1) / 2 : L * L;
+  }
+  att *= nh;
+  const double Td = T, Hd = H, Fd = F;
+  auto gemm_flops = [&](double N, double K) { return 2.0 * Td * N * K; };
+  auto gemm_bytes = [&](double N, double K) { return 2.0 * (Td * K + N * K + Td * N); };
+  const double att_flops = 2.0 * att * d;            // one of the two contractions
+  const double sm_bytes = 4.0 * att;                 // bf16 read + write per admitted entry
+  const double ctx_bytes = 2.0 * att + 2.0 * Td * Hd * 2;   // P, V, ctx
+
+  RM_KERNEL(RM_K_EMBED, 0, 6.0 * Td * Hd + 4.0 * Td,
+            embed_launch(d_ids, d_off, n, T, h->emb_word, h->emb_pos, dec ? nullptr : h->ln_emb_g,
+                         dec ? nullptr : h->ln_emb_b, eps, c->vocab, c->max_pos, H, x,
+                         h->d_err + ERR_CLAMPED, st));
+  if (dec)
+    RM_KERNEL(RM_K_LAYERNORM, 0, 4.0 * Td * Hd,
+              res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps, 1, 2, st));
+  const double ln_bytes = (dec ? 8.0 : 6.0) * Td * Hd;
+  for (int l = 0; l < c->n_layers; ++l) {
+    const LayerW& L = h->layers[l];
+    RM_GEMM(gemm_flops(3 * Hd, Hd), gemm_bytes(3 * Hd, Hd),
+            gemm(h, bk->a_in, L.tm[0], T, 3 * H, H, L.b_qkv, qkv, 0, st));
+    RM_KERNEL(RM_K_SCORES, att_flops, 2.0 * Td * Hd * 2 + 2.0 * att,
+              attn_scores_launch(qkv, s, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
+    RM_KERNEL(RM_K_SOFTMAX, 0, sm_bytes,
+              softmax_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, st));
+    RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
+              attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
+    RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd),
+            gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st));
+    if (!dec) {
+      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
+                res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, 1, 0, st));
+      RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
+              gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
+      RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
+              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st));
+      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
+                res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, 1, 0, st));
+    } else {
+      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
+                res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, 1, 1, st));
+      RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
+              gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
+      RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
+              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st));
+      const bool last = l + 1 == c->n_layers;
+      const float* g = last ? h->lnf_g : h->layers[l + 1].ln1_g;
+      const float* b = last ? h->lnf_b : h->layers[l + 1].ln1_b;
+      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes, res_ln_launch(y2, x, z, g, b, T, H, eps, 1, 1, st));
+    }
+  }
+  RM_KERNEL(RM_K_HEAD, 2.0 * n * Hd, 2.0 * n * Hd + 4.0 * n,
+            head_launch(dec ? z : x, d_off, n, h->w_r, h->b_r, H, dec ? 1 : 0, d_out, st));
+  if (host_out != nullptr)
+    RM_CUDA(cudaMemcpyAsync(host_out, d_out, 4 * static_cast<size_t>(n), cudaMemcpyDeviceToHost, st));
+  h->last_stream = st;
+  return RM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rm_last_error(void) { return g_msg; }
+
+size_t rm_weights_bytes(const rm_config* cfg) {
+  const char* why = "";
+  if (validate_config(cfg, false, &why) != RM_OK) return 0;
+  int64_t total = 0;
+  for (const auto& s : segments(cfg)) total += s.elems;
+  return static_cast<size_t>(total) * (cfg->weight_dtype == RM_F32 ? 4 : 2);
+}
+
+int rm_create(const rm_config* cfg, const void* weights, size_t weights_bytes, rm_handle** out) {
+  g_msg[0] = '\0';
+  const char* why = "";
+  if (out == nullptr || weights == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  if (validate_config(cfg, false, &why) != RM_OK) return set_error(RM_E_INVAL, "%s", why);
+  const size_t need = rm_weights_bytes(cfg);
+  if (weights_bytes != need)
+    return set_error(RM_E_INVAL, "weights_bytes is %zu, the layout needs %zu", weights_bytes, need);
+  int dev = 0, ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0)
+    return set_error(RM_E_DEVICE, "no CUDA device");
+  RM_CUDA(cudaGetDevice(&dev));
+  cudaDeviceProp prop;
+  RM_CUDA(cudaGetDeviceProperties(&prop, dev));
+  if (prop.major != 10)
+    return set_error(RM_E_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                     prop.major, prop.minor);
+  rm_handle* h = new rm_handle();
+  h->cfg = *cfg;
+  h->cfg.sched_table = nullptr;   // the handle keeps its own copy in sched
+  h->sched = sched_cost_from(cfg);
+  h->device = dev;
+  h->num_sms = prop.multiProcessorCount;
+  int rc = upload_weights(h, weights);
+  if (rc == RM_OK) {
+    const int64_t T = cfg->max_tokens;
+    const int64_t Lp = align_up(cfg->max_len, 8);
+    const int64_t Smax = static_cast<int64_t>(cfg->n_heads) * T * Lp;
+    const MetaLayout ml(cfg->max_batch_seqs);
+    h->meta_bytes = align_up(ml.bytes, 256);
+    h->fixed_bytes = h->meta_bytes + align_up(4 * T, 256) + align_up(4 * cfg->max_batch_seqs, 256);
+    h->arena_bytes = h->fixed_bytes +
+                     arena_bound(cfg->arch, cfg->hidden, cfg->ffn, align_up(T, 128),
+                                 align_up(std::max<int64_t>(Smax, 1), 65536));
+    cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&h->d_err, ERR_WORDS * sizeof(int32_t));
+    if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, ERR_WORDS * sizeof(int32_t));
+    if (e == cudaSuccess)
+      e = cudaHostAlloc(&h->pinned, static_cast<size_t>(kSlots) * h->meta_bytes, cudaHostAllocDefault);
+    for (int k = 0; k < kSlots && e == cudaSuccess; ++k)
+      e = cudaEventCreateWithFlags(&h->ev[k], cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      rc = set_error(e == cudaErrorMemoryAllocation ? RM_E_NOMEM : RM_E_CUDA, "create: %s",
+                     cudaGetErrorString(e));
+    } else {
+      h->d_meta = h->arena;
+      h->d_ids = reinterpret_cast<int32_t*>(h->arena + h->meta_bytes);
+      h->d_scores = reinterpret_cast<float*>(h->arena + h->meta_bytes + align_up(4 * T, 256));
+      h->planned = h->arena + h->fixed_bytes;
+    }
+  }
+  if (rc != RM_OK) {
+    rm_destroy(h);
+    return rc;
+  }
+  *out = h;
+  return RM_OK;
+}
+
+int rm_score(rm_handle* h, const int32_t* packed_token_ids, const int32_t* seq_offsets,
+             int32_t n_seqs, float* out_scores, void* stream) {
+  if (h == nullptr || packed_token_ids == nullptr || seq_offsets == nullptr || out_scores == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  return score_impl(h, packed_token_ids, nullptr, seq_offsets, n_seqs, out_scores, nullptr,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int rm_score_host(rm_handle* h, const int32_t* host_token_ids, const int32_t* seq_offsets,
+                  int32_t n_seqs, float* host_scores, void* stream) {
+  if (h == nullptr || host_token_ids == nullptr || seq_offsets == nullptr || host_scores == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  return score_impl(h, nullptr, host_token_ids, seq_offsets, n_seqs, nullptr, host_scores,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int rm_schedule_cfg(const rm_config* cfg, const int32_t* lengths, int32_t n, int32_t* out_batches) {
+  const char* why = "";
+  if (validate_config(cfg, true, &why) != RM_OK) return set_error(RM_E_INVAL, "%s", why);
+  if (n < 0) return set_error(RM_E_INVAL, "n must be >= 0");
+  if (n > 0 && (lengths == nullptr || out_batches == nullptr))
+    return set_error(RM_E_INVAL, "NULL argument");
+  for (int32_t i = 0; i < n; ++i)
+    if (lengths[i] < 1 || lengths[i] > cfg->max_len)
+      return set_error(RM_E_RANGE, "length %d of request %d outside 1..max_len", lengths[i], i);
+  if (n == 0) return 0;
+  return schedule_dp(sched_cost_from(cfg), lengths, n, out_batches);
+}
+
+int rm_schedule(const rm_handle* h, const int32_t* lengths, int32_t n, int32_t* out_batches) {
+  if (h == nullptr) return set_error(RM_E_INVAL, "NULL handle");
+  if (n < 0) return set_error(RM_E_INVAL, "n must be >= 0");
+  if (n > 0 && (lengths == nullptr || out_batches == nullptr))
+    return set_error(RM_E_INVAL, "NULL argument");
+  for (int32_t i = 0; i < n; ++i)
+    if (lengths[i] < 1 || lengths[i] > h->cfg.max_len)
+      return set_error(RM_E_RANGE, "length %d of request %d outside 1..max_len", lengths[i], i);
+  if (n == 0) return 0;
+  return schedule_dp(h->sched, lengths, n, out_batches);
+}
+
+int rm_get_device_error(rm_handle* h, int32_t* out) {
+  if (h == nullptr || out == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  RM_CUDA(cudaStreamSynchronize(h->last_stream));
+  RM_CUDA(cudaMemcpy(out, h->d_err, ERR_WORDS * sizeof(int32_t), cudaMemcpyDeviceToHost));
+  return RM_OK;
+}
+
+int rm_profile(rm_handle* h, int32_t every) {
+  if (h == nullptr || every < 0) return set_error(RM_E_INVAL, "bad argument");
+  for (auto& r : h->prof) {
+    h->ev_pool.push_back(r.a);
+    h->ev_pool.push_back(r.b);
+  }
+  h->prof.clear();
+  h->prof_every = every;
+  h->calls = 0;
+  return RM_OK;
+}
+
+int rm_profile_read(rm_handle* h, double* out_ms, int64_t* out_launches, double* out_flops,
+                    double* out_bytes, int64_t* out_total_launches) {
+  if (h == nullptr || out_ms == nullptr || out_launches == nullptr || out_flops == nullptr ||
+      out_bytes == nullptr || out_total_launches == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  RM_CUDA(cudaStreamSynchronize(h->last_stream));
+  for (int k = 0; k < RM_K_CLASSES; ++k) {
+    out_ms[k] = 0;
+    out_launches[k] = 0;
+    out_flops[k] = 0;
+    out_bytes[k] = 0;
+  }
+  for (const auto& r : h->prof) {
+    float ms = 0;
+    RM_CUDA(cudaEventElapsedTime(&ms, r.a, r.b));
+    out_ms[r.cls] += ms;
+    out_launches[r.cls] += 1;
+    out_flops[r.cls] += r.flops;
+    out_bytes[r.cls] += r.bytes;
+  }
+  *out_total_launches = h->launches;
+  return RM_OK;
+}
+
+int rm_arena_stats(const rm_handle* h, int64_t* out) {
+  if (h == nullptr || out == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  out[0] = h->arena_bytes;
+  out[1] = h->fixed_bytes + h->max_peak;
+  out[2] = static_cast<int64_t>(h->buckets.size());
+  return RM_OK;
+}
+
+void rm_destroy(rm_handle* h) {
+  if (h == nullptr) return;
+  if (h->last_stream != nullptr || h->arena != nullptr) cudaStreamSynchronize(h->last_stream);
+  for (int k = 0; k < kSlots; ++k)
+    if (h->ev[k]) cudaEventDestroy(h->ev[k]);
+  for (auto& r : h->prof) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : h->ev_pool) cudaEventDestroy(e);
+  if (h->pinned) cudaFreeHost(h->pinned);
+  if (h->d_err) cudaFree(h->d_err);
+  if (h->arena) cudaFree(h->arena);
+  if (h->wbuf) cudaFree(h->wbuf);
+  delete h;
+}
+
+// ---------------------------------------------------------------------------
+// rm_ops.h
+// ---------------------------------------------------------------------------
+
+int rm_varlen_meta(const int32_t* offsets, int32_t n, int32_t n_heads, int32_t* rb_off,
+                   int64_t* s_off) {
+  if (offsets == nullptr || rb_off == nullptr || s_off == nullptr || n < 0 || n_heads < 1)
+    return set_error(RM_E_INVAL, "bad argument");
+  return host_varlen_meta(offsets, n, n_heads, rb_off, s_off, nullptr);
+}
+
+int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
+               int32_t M, int32_t N, int32_t K, int32_t act, void* stream) {
+  if (x == nullptr || w == nullptr || y == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  if (M < 1 || N < 8 || K < 8 || N % 8 != 0 || K % 8 != 0)
+    return set_error(RM_E_INVAL, "need M >= 1 and N, K positive multiples of 8");
+  if (act < 0 || act > 2 || (y_dtype != RM_F32 && y_dtype != RM_BF16))
+    return set_error(RM_E_INVAL, "bad act or y_dtype");
+  if ((reinterpret_cast<uintptr_t>(y) & 15) != 0) return set_error(RM_E_INVAL, "y must be 16-byte aligned");
+  int dev = 0, sms = 148;
+  RM_CUDA(cudaGetDevice(&dev));
+  RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  const int bn = gemm_pick_bn(M, N, sms);
+  CUtensorMap ta, tb;
+  const char* why = "";
+  if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, bn, &why))
+    return set_error(RM_E_INVAL, "tensor map: %s", why);
+  int32_t* err = nullptr;
+  RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
+  RM_LAUNCH(gemm_launch(ta, tb, bn, M, N, K, bias, y, y_dtype == RM_F32, act, err,
+                        static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_embed(const int32_t* ids, const int32_t* offsets, int32_t n_seqs, int32_t T,
+                const void* emb_word, const void* emb_pos, const float* ln_g, const float* ln_b,
+                float eps, int32_t V, int32_t P, int32_t H, void* x, int32_t* err_count,
+                void* stream) {
+  if (ids == nullptr || offsets == nullptr || emb_word == nullptr || emb_pos == nullptr || x == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || T < 0 || V < 1 || P < 1 || H < 8 || H % 8 != 0 || H > 4096)
+    return set_error(RM_E_INVAL, "bad sizes");
+  if ((ln_g == nullptr) != (ln_b == nullptr)) return set_error(RM_E_INVAL, "ln_g and ln_b go together");
+  RM_LAUNCH(embed_launch(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps, V, P, H, x,
+                         err_count, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_attn_scores(const void* qkv, void* S, const int32_t* offsets, const int32_t* rb_off,
+                      const int64_t* s_off, int32_t n_seqs, int32_t n_row_blocks,
+                      int32_t n_heads, int32_t head_dim, int32_t causal, void* stream) {
+  if (qkv == nullptr || S == nullptr || offsets == nullptr || rb_off == nullptr || s_off == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || n_row_blocks < 0 || n_heads < 1 || head_dim < 2 || head_dim % 2 || head_dim > 128)
+    return set_error(RM_E_INVAL, "bad sizes");
+  RM_LAUNCH(attn_scores_launch(qkv, S, offsets, rb_off, s_off, n_seqs, n_row_blocks, n_heads,
+                               head_dim, causal != 0, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_softmax(void* S, int32_t s_dtype, const int32_t* offsets, const int64_t* s_off,
+                  int32_t n_seqs, int32_t T, int32_t n_heads, int32_t max_len, int32_t causal,
+                  void* stream) {
+  if (S == nullptr || offsets == nullptr || s_off == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || T < 0 || n_heads < 1 || max_len < 1 || max_len > 1024 ||
+      (s_dtype != RM_F32 && s_dtype != RM_BF16))
+    return set_error(RM_E_INVAL, "bad sizes");
+  RM_LAUNCH(softmax_launch(S, s_dtype, offsets, s_off, n_seqs, T, n_heads, max_len, causal != 0,
+                           static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_attn_context(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
+                       const int32_t* rb_off, const int64_t* s_off, int32_t n_seqs,
+                       int32_t n_row_blocks, int32_t n_heads, int32_t head_dim, int32_t causal,
+                       void* stream) {
+  if (S == nullptr || qkv == nullptr || ctx == nullptr || offsets == nullptr || rb_off == nullptr ||
+      s_off == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || n_row_blocks < 0 || n_heads < 1 || head_dim < 2 || head_dim % 2 || head_dim > 128)
+    return set_error(RM_E_INVAL, "bad sizes");
+  RM_LAUNCH(attn_context_launch(S, qkv, ctx, offsets, rb_off, s_off, n_seqs, n_row_blocks, n_heads,
+                                head_dim, causal != 0, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_res_ln(const void* y, void* x, void* z, const float* g, const float* b, int32_t T,
+                 int32_t H, float eps, int32_t dtype, int32_t mode, void* stream) {
+  if (x == nullptr || g == nullptr || b == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  if (mode < 0 || mode > 2 || (mode != 2 && y == nullptr) || (mode != 0 && z == nullptr))
+    return set_error(RM_E_INVAL, "bad mode or missing y/z");
+  if (T < 0 || H < 8 || H % 8 != 0 || H > 4096 || (dtype != RM_F32 && dtype != RM_BF16))
+    return set_error(RM_E_INVAL, "bad sizes");
+  RM_LAUNCH(res_ln_launch(y, x, z, g, b, T, H, eps, dtype, mode, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_head(const void* x, const int32_t* offsets, int32_t n_seqs, const float* w_r, float b_r,
+               int32_t H, int32_t last_token, float* out, void* stream) {
+  if (x == nullptr || offsets == nullptr || w_r == nullptr || out == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 0 || H < 8 || H % 8 != 0) return set_error(RM_E_INVAL, "bad sizes");
+  RM_LAUNCH(head_launch(x, offsets, n_seqs, w_r, b_r, H, last_token != 0, out,
+                        static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_arena_plan(const void* cfgp, int32_t T, int32_t n_seqs, int64_t s_elems, int64_t* out_off,
+                  int64_t* out_bytes, int32_t* out_first, int32_t* out_last, int32_t max_bufs,
+                  int64_t* out_peak) {
+  (void)n_seqs;
+  const rm_config* cfg = static_cast<const rm_config*>(cfgp);
+  const char* why = "";
+  if (validate_config(cfg, false, &why) != RM_OK) return set_error(RM_E_INVAL, "%s", why);
+  if (T < 0 || s_elems < 0 || out_off == nullptr || out_bytes == nullptr || out_first == nullptr ||
+      out_last == nullptr || out_peak == nullptr)
+    return set_error(RM_E_INVAL, "bad argument");
+  const ArenaPlan p = plan_arena(cfg->arch, cfg->hidden, cfg->ffn, T, s_elems);
+  const int nb = std::min<int>(B_COUNT, max_bufs);
+  for (int k = 0; k < nb; ++k) {
+    out_off[k] = p.off[k];
+    out_bytes[k] = p.bytes[k];
+    out_first[k] = p.first[k];
+    out_last[k] = p.last[k];
+  }
+  *out_peak = p.peak;
+  return B_COUNT;
+}
+
+}  // extern "C"

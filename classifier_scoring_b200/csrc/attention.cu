@@ -1,0 +1,329 @@
+// Varlen multi-head attention in three kernels over the packed layout:
+//   scores   S = Q K^T / sqrt(d) for each sequence and head, only the valid
+//            L x L block (causal: the lower triangle);
+//   softmax  masked row softmax in place on S -- the Softmax batch reduction
+//            of the TurboTransformers abstract ("TurboTransformers: An
+//            Efficient GPU Serving System For Transformer Models");
+//   context  C = P V into the packed [T][H] context.
+// No token of one sequence ever meets a token of another: every CTA works
+// inside one sequence, located from the per-sequence offsets.
+//
+// The two small per-sequence contractions (L <= 1024, d <= 128) use warp-level
+// mma.sync m16n8k16 bf16 tiles with fp32 accumulation; together they are a few
+// percent of the scorer's FLOPs.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rmk {
+namespace {
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+struct BlockSeq {
+  int t0, L, Lp, row0;
+  long long sbase;
+};
+
+// CTA blockIdx.x -> (sequence, 64-row query block).
+__device__ __forceinline__ BlockSeq locate_block(const int32_t* offsets, const int32_t* rb_off,
+                                                 const int64_t* s_off, int n, int b) {
+  BlockSeq q;
+  const int i = upper_index(rb_off, n, b);
+  q.t0 = offsets[i];
+  q.L = offsets[i + 1] - q.t0;
+  q.Lp = (q.L + 7) & ~7;
+  q.row0 = (b - rb_off[i]) * 64;
+  q.sbase = s_off[i];
+  return q;
+}
+
+// 4 warps x 16 query rows; keys in blocks of 64 staged in shared memory.
+template <int DP>
+__global__ void __launch_bounds__(128)
+    attn_scores_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ S,
+                       const int32_t* __restrict__ offsets, const int32_t* __restrict__ rb_off,
+                       const int64_t* __restrict__ s_off, int n, int H, int d, float scale,
+                       int causal) {
+  __shared__ __align__(16) bf16 ks[64][DP + 8];
+  const BlockSeq q = locate_block(offsets, rb_off, s_off, n, blockIdx.x);
+  const int hd = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const size_t H3 = 3 * static_cast<size_t>(H);
+  const bf16* qb = qkv + static_cast<size_t>(q.t0) * H3 + hd * d;
+  const bf16* kbp = qkv + static_cast<size_t>(q.t0) * H3 + H + hd * d;
+  bf16* sb = S + q.sbase + static_cast<size_t>(hd) * q.L * q.Lp;
+  const int ra = q.row0 + warp * 16 + g, rb = ra + 8;
+
+  auto ld_pair = [&](const bf16* base, int r, int c) -> uint32_t {
+    return (r < q.L && c < d) ? *reinterpret_cast<const uint32_t*>(base + r * H3 + c) : 0u;
+  };
+  uint32_t qa[DP / 16][4];
+#pragma unroll
+  for (int s = 0; s < DP / 16; ++s) {
+    const int c0 = s * 16 + 2 * tq;
+    qa[s][0] = ld_pair(qb, ra, c0);
+    qa[s][1] = ld_pair(qb, rb, c0);
+    qa[s][2] = ld_pair(qb, ra, c0 + 8);
+    qa[s][3] = ld_pair(qb, rb, c0 + 8);
+  }
+  const int row_end = min(q.L, q.row0 + 64);
+  const int kend = causal ? row_end : q.L;
+  const int wrow0 = q.row0 + warp * 16;
+  const int wrow_last = min(wrow0 + 15, q.L - 1);
+  for (int kb = 0; kb < kend; kb += 64) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 64 * (DP / 2); idx += 128) {
+      const int r = idx / (DP / 2), cp = (idx % (DP / 2)) * 2;
+      *reinterpret_cast<uint32_t*>(&ks[r][cp]) = ld_pair(kbp, kb + r, cp);
+    }
+    __syncthreads();
+    if (wrow0 >= q.L) continue;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int key0 = kb + nt * 8;
+      if (key0 >= kend || (causal && key0 > wrow_last)) break;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < DP / 16; ++s) {
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&ks[nt * 8 + g][s * 16 + 2 * tq]);
+        const uint32_t b1 =
+            *reinterpret_cast<const uint32_t*>(&ks[nt * 8 + g][s * 16 + 8 + 2 * tq]);
+        mma_bf16_16816(acc, qa[s], b0, b1);
+      }
+      const int c = key0 + 2 * tq;
+      // the pair (c, c+1) stays inside the row's Lp (c even, Lp a multiple of 8)
+      if (ra < q.L && c < (causal ? ra + 1 : q.L))
+        *reinterpret_cast<uint32_t*>(sb + static_cast<size_t>(ra) * q.Lp + c) =
+            pack_bf16x2(acc[0] * scale, acc[1] * scale);
+      if (rb < q.L && c < (causal ? rb + 1 : q.L))
+        *reinterpret_cast<uint32_t*>(sb + static_cast<size_t>(rb) * q.Lp + c) =
+            pack_bf16x2(acc[2] * scale, acc[3] * scale);
+    }
+  }
+}
+
+// Masked softmax: G lanes per row, MAXC 8-element chunks per lane, 8 warps per CTA.
+template <typename T, int G, int MAXC>
+__global__ void __launch_bounds__(256)
+    softmax_kernel(T* __restrict__ S, const int32_t* __restrict__ offsets,
+                   const int64_t* __restrict__ s_off, int n, long long rows, int nh, int causal) {
+  const int lane = threadIdx.x & 31, sub = lane % G;
+  const long long R =
+      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * (32 / G) + lane / G;
+  const bool valid = R < rows;
+  int len = 0;
+  T* row = S;
+  if (valid) {
+    int lo = 0, hi = n - 1;   // largest i with nh * offsets[i] <= R
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (static_cast<long long>(nh) * offsets[mid] <= R) lo = mid; else hi = mid - 1;
+    }
+    const int L = offsets[lo + 1] - offsets[lo];
+    const int Lp = (L + 7) & ~7;
+    const long long rr = R - static_cast<long long>(nh) * offsets[lo];
+    const int r = static_cast<int>(rr % L);
+    len = causal ? r + 1 : L;
+    row = S + s_off[lo] + rr * Lp;
+  }
+  float v[MAXC][8];
+  float m = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int col = (c * G + sub) * 8;
+    if (col < len) {
+      Chunk8<T>::load(row + col, v[c]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (col + e >= len) v[c][e] = -INFINITY;
+        m = fmaxf(m, v[c][e]);
+      }
+    }
+  }
+  m = group_max<G>(m);
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int col = (c * G + sub) * 8;
+    if (col < len) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float p = (col + e < len) ? __expf(v[c][e] - m) : 0.f;
+        v[c][e] = p;
+        s += p;
+      }
+    }
+  }
+  s = group_sum<G>(s);
+  const float inv = 1.0f / s;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int col = (c * G + sub) * 8;
+    if (col < len) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[c][e] *= inv;
+      Chunk8<T>::store(row + col, v[c]);
+    }
+  }
+}
+
+template <int DP>
+__global__ void __launch_bounds__(128)
+    attn_context_kernel(const bf16* __restrict__ S, const bf16* __restrict__ qkv,
+                        bf16* __restrict__ ctx, const int32_t* __restrict__ offsets,
+                        const int32_t* __restrict__ rb_off, const int64_t* __restrict__ s_off,
+                        int n, int H, int d, int causal) {
+  __shared__ __align__(16) bf16 vt[DP][64 + 8];   // V block transposed: [dim][key]
+  const BlockSeq q = locate_block(offsets, rb_off, s_off, n, blockIdx.x);
+  const int hd = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const size_t H3 = 3 * static_cast<size_t>(H);
+  const bf16* vb = qkv + static_cast<size_t>(q.t0) * H3 + 2 * H + hd * d;
+  const bf16* pb = S + q.sbase + static_cast<size_t>(hd) * q.L * q.Lp;
+  const int ra = q.row0 + warp * 16 + g, rb = ra + 8;
+  const int lim_a = causal ? ra + 1 : q.L, lim_b = causal ? rb + 1 : q.L;
+
+  auto ld_p = [&](int r, int lim, int c) -> uint32_t {
+    if (r >= q.L || c >= lim) return 0u;
+    uint32_t v = *reinterpret_cast<const uint32_t*>(pb + static_cast<size_t>(r) * q.Lp + c);
+    return (c + 1 < lim) ? v : (v & 0xffffu);
+  };
+  float acc[DP / 8][4];
+#pragma unroll
+  for (int t = 0; t < DP / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+
+  const int row_end = min(q.L, q.row0 + 64);
+  const int kend = causal ? row_end : q.L;
+  const int wrow0 = q.row0 + warp * 16;
+  const int wrow_last = min(wrow0 + 15, q.L - 1);
+  for (int kb = 0; kb < kend; kb += 64) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 64 * (DP / 2); idx += 128) {
+      const int r = idx & 63, cp = (idx >> 6) * 2;
+      uint32_t v = 0u;
+      if (kb + r < q.L && cp < d) v = *reinterpret_cast<const uint32_t*>(vb + (kb + r) * H3 + cp);
+      *reinterpret_cast<uint16_t*>(&vt[cp][r]) = static_cast<uint16_t>(v & 0xffffu);
+      *reinterpret_cast<uint16_t*>(&vt[cp + 1][r]) = static_cast<uint16_t>(v >> 16);
+    }
+    __syncthreads();
+    if (wrow0 >= q.L) continue;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      const int key0 = kb + s * 16;
+      if (key0 >= kend || (causal && key0 > wrow_last)) break;
+      uint32_t a[4];
+      a[0] = ld_p(ra, lim_a, key0 + 2 * tq);
+      a[1] = ld_p(rb, lim_b, key0 + 2 * tq);
+      a[2] = ld_p(ra, lim_a, key0 + 8 + 2 * tq);
+      a[3] = ld_p(rb, lim_b, key0 + 8 + 2 * tq);
+#pragma unroll
+      for (int t = 0; t < DP / 8; ++t) {
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&vt[t * 8 + g][s * 16 + 2 * tq]);
+        const uint32_t b1 =
+            *reinterpret_cast<const uint32_t*>(&vt[t * 8 + g][s * 16 + 8 + 2 * tq]);
+        mma_bf16_16816(acc[t], a, b0, b1);
+      }
+    }
+  }
+  if (wrow0 >= q.L) return;
+  bf16* cb = ctx + static_cast<size_t>(q.t0) * H + hd * d;
+#pragma unroll
+  for (int t = 0; t < DP / 8; ++t) {
+    const int col = t * 8 + 2 * tq;
+    if (col < d) {
+      if (ra < q.L)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(ra) * H + col) =
+            pack_bf16x2(acc[t][0], acc[t][1]);
+      if (rb < q.L)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(rb) * H + col) =
+            pack_bf16x2(acc[t][2], acc[t][3]);
+    }
+  }
+}
+
+int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 : -1)); }
+
+template <typename T, int G, int MAXC>
+cudaError_t softmax_t(void* S, const int32_t* offsets, const int64_t* s_off, int n, long long rows,
+                      int nh, int causal, cudaStream_t st) {
+  const long long rows_per_cta = 8LL * (32 / G);
+  const long long blocks = (rows + rows_per_cta - 1) / rows_per_cta;
+  softmax_kernel<T, G, MAXC><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<T*>(S), offsets, s_off, n, rows, nh, causal);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t softmax_dispatch(void* S, const int32_t* offsets, const int64_t* s_off, int n,
+                             long long rows, int nh, int max_len, int causal, cudaStream_t st) {
+  const int chunks = ((max_len + 7) & ~7) / 8;
+  if (chunks <= 4) return softmax_t<T, 4, 1>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 8) return softmax_t<T, 8, 1>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 16) return softmax_t<T, 16, 1>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 32) return softmax_t<T, 32, 1>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 64) return softmax_t<T, 32, 2>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 96) return softmax_t<T, 32, 3>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 128) return softmax_t<T, 32, 4>(S, offsets, s_off, n, rows, nh, causal, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
+                               const int32_t* rb_off, const int64_t* s_off, int n_seqs,
+                               int n_row_blocks, int n_heads, int head_dim, int causal,
+                               cudaStream_t st) {
+  if (n_row_blocks == 0) return cudaSuccess;
+  const int H = n_heads * head_dim;
+  const float scale = 1.0f / sqrtf(static_cast<float>(head_dim));
+  dim3 grid(n_row_blocks, n_heads);
+  const bf16* q = static_cast<const bf16*>(qkv);
+  bf16* s = static_cast<bf16*>(S);
+  switch (pad_head_dim(head_dim)) {
+    case 32: attn_scores_kernel<32><<<grid, 128, 0, st>>>(q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
+    case 64: attn_scores_kernel<64><<<grid, 128, 0, st>>>(q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
+    case 128: attn_scores_kernel<128><<<grid, 128, 0, st>>>(q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const int64_t* s_off,
+                           int n_seqs, int T, int n_heads, int max_len, int causal,
+                           cudaStream_t st) {
+  const long long rows = static_cast<long long>(n_heads) * T;
+  if (rows == 0) return cudaSuccess;
+  if (s_dtype == 0)
+    return softmax_dispatch<float>(S, offsets, s_off, n_seqs, rows, n_heads, max_len, causal, st);
+  return softmax_dispatch<bf16>(S, offsets, s_off, n_seqs, rows, n_heads, max_len, causal, st);
+}
+
+cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
+                                const int32_t* rb_off, const int64_t* s_off, int n_seqs,
+                                int n_row_blocks, int n_heads, int head_dim, int causal,
+                                cudaStream_t st) {
+  if (n_row_blocks == 0) return cudaSuccess;
+  const int H = n_heads * head_dim;
+  dim3 grid(n_row_blocks, n_heads);
+  const bf16* s = static_cast<const bf16*>(S);
+  const bf16* q = static_cast<const bf16*>(qkv);
+  bf16* c = static_cast<bf16*>(ctx);
+  switch (pad_head_dim(head_dim)) {
+    case 32: attn_context_kernel<32><<<grid, 128, 0, st>>>(s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
+    case 64: attn_context_kernel<64><<<grid, 128, 0, st>>>(s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
+    case 128: attn_context_kernel<128><<<grid, 128, 0, st>>>(s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace rmk

@@ -1,0 +1,91 @@
+// Shared device/host helpers of the scorer's kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rmk {
+
+using bf16 = __nv_bfloat16;
+
+// ---------------------------------------------------------------------------
+// Element conversion.  fp32 -> bf16 rounds to nearest even (the intrinsic).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ float to_f32(float v) { return v; }
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);   // .x = lo (low half), .y = hi
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Eight consecutive elements ("a chunk"): 16 bytes of bf16 or 32 bytes of fp32.
+template <typename T> struct Chunk8;
+template <> struct Chunk8<bf16> {
+  static __device__ __forceinline__ void load(const bf16* p, float* f) {
+    uint4 v = *reinterpret_cast<const uint4*>(p);
+    f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+  }
+  static __device__ __forceinline__ void store(bf16* p, const float* f) {
+    uint4 v;
+    v.x = pack_bf16x2(f[0], f[1]); v.y = pack_bf16x2(f[2], f[3]);
+    v.z = pack_bf16x2(f[4], f[5]); v.w = pack_bf16x2(f[6], f[7]);
+    *reinterpret_cast<uint4*>(p) = v;
+  }
+};
+template <> struct Chunk8<float> {
+  static __device__ __forceinline__ void load(const float* p, float* f) {
+    float4 a = reinterpret_cast<const float4*>(p)[0];
+    float4 b = reinterpret_cast<const float4*>(p)[1];
+    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+  }
+  static __device__ __forceinline__ void store(float* p, const float* f) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(f[0], f[1], f[2], f[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+};
+
+__device__ __forceinline__ void load_f32x8(const float* p, float* f) { Chunk8<float>::load(p, f); }
+
+// Reductions over aligned groups of G lanes (G a power of two <= 32).
+template <int G> __device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+template <int G> __device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Largest i in [0, n) with a[i] <= key, for a non-decreasing a with a[0] <= key.
+template <typename I>
+__device__ __forceinline__ int upper_index(const I* a, int n, long long key) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if ((long long)a[mid] <= key) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// GELU: u * Phi(u) (erf form) or the tanh approximation; both call CUDA's
+// erff / tanhf.
+__device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.0f + erff(u * 0.70710678118654752f)); }
+__device__ __forceinline__ float gelu_tanh(float u) {
+  return 0.5f * u * (1.0f + tanhf(0.79788456080286536f * (u + 0.044715f * u * u * u)));
+}
+
+// Device error words (rm_get_device_error): [0] clamped token ids, [1] waits
+// that gave up.
+enum { ERR_CLAMPED = 0, ERR_TIMEOUT = 1, ERR_WORDS = 2 };
+
+}  // namespace rmk

@@ -1,0 +1,53 @@
+// Internal launchers of the scorer's kernels (host-callable, not exported).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rmk {
+
+// ---- tcgen05 GEMM (gemm_tc.cu) ----
+// Column-tile width for an M x N problem on num_sms SMs (256 or 128).
+int gemm_pick_bn(int M, int N, int num_sms);
+// a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, bn}.
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int M, int N, int K,
+                        const float* bias, void* y, bool out_f32, int act, int* err,
+                        cudaStream_t st);
+
+// ---- TMA descriptors (tma.cpp) ----
+// 2-D bf16 row-major [rows][cols] tensor, box {64 cols, box_rows}, 128-byte swizzle,
+// zero fill outside.  Returns false (message in *why) if the driver refuses it.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_rows, const char** why);
+
+// ---- row kernels (rowops.cu) ----
+cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs, int T,
+                         const void* emb_word, const void* emb_pos, const float* ln_g,
+                         const float* ln_b, float eps, int V, int P, int H, void* x,
+                         int32_t* err_count, cudaStream_t st);
+// dtype: 0 fp32, 1 bf16; mode 0 post, 1 pre, 2 plain (see rm_ops.h)
+cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
+                          int H, float eps, int dtype, int mode, cudaStream_t st);
+cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
+                        float b_r, int H, int last_token, float* out, cudaStream_t st);
+// weight conversion at create
+cudaError_t cvt_to_bf16_launch(const void* src, int src_dtype, void* dst, size_t n,
+                               cudaStream_t st);
+cudaError_t cvt_to_f32_launch(const void* src, int src_dtype, float* dst, size_t n,
+                              cudaStream_t st);
+
+// ---- attention (attention.cu) ----
+cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
+                               const int32_t* rb_off, const int64_t* s_off, int n_seqs,
+                               int n_row_blocks, int n_heads, int head_dim, int causal,
+                               cudaStream_t st);
+cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const int64_t* s_off,
+                           int n_seqs, int T, int n_heads, int max_len, int causal,
+                           cudaStream_t st);
+cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
+                                const int32_t* rb_off, const int64_t* s_off, int n_seqs,
+                                int n_row_blocks, int n_heads, int head_dim, int causal,
+                                cudaStream_t st);
+
+}  // namespace rmk

@@ -1,0 +1,297 @@
+// Row kernels of the scorer: embedding gather (+ embedding LayerNorm),
+// residual + LayerNorm, the scalar head, and weight conversion.
+//
+// LayerNorm is one of the two "batch reduction" hot spots named in the
+// TurboTransformers abstract ("TurboTransformers: An Efficient GPU Serving
+// System For Transformer Models"); its proposed-method section parallelises
+// it with the GPU memory hierarchy and thread-level parallelism in mind.
+// Here: one warp per row; each lane holds its 16-byte chunks of the row in
+// registers (a row is read from HBM exactly once), mean and biased variance
+// are two register passes reduced with warp shuffles, fp32 math throughout.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace rmk {
+namespace {
+
+constexpr int kWarps = 8;   // warps (rows) per CTA
+
+template <int MAXC>
+__device__ __forceinline__ void row_moments(const float (&v)[MAXC][8], int nch, int lane, int H,
+                                            float& mean, float& rstd, float eps) {
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c)
+    if (lane + 32 * c < nch) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[c][e];
+    }
+  mean = group_sum<32>(s) / static_cast<float>(H);
+  float q = 0.f;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c)
+    if (lane + 32 * c < nch) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[c][e] - mean;
+        q += d * d;
+      }
+    }
+  const float var = group_sum<32>(q) / static_cast<float>(H);
+  rstd = rsqrtf(var + eps);
+}
+
+template <int MAXC>
+__device__ __forceinline__ void normalize(float (&v)[MAXC][8], int nch, int lane, float mean,
+                                          float rstd, const float* __restrict__ g,
+                                          const float* __restrict__ b) {
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      float gg[8], bb[8];
+      load_f32x8(g + ch * 8, gg);
+      load_f32x8(b + ch * 8, bb);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[c][e] = (v[c][e] - mean) * rstd * gg[e] + bb[e];
+    }
+  }
+}
+
+template <int MAXC, bool LN>
+__global__ void __launch_bounds__(kWarps * 32)
+    embed_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ offsets, int n_seqs,
+                 int T, const bf16* __restrict__ ew, const bf16* __restrict__ ep,
+                 const float* __restrict__ g, const float* __restrict__ b, float eps, int V, int H,
+                 bf16* __restrict__ x, int32_t* __restrict__ err) {
+  const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const int i = upper_index(offsets, n_seqs, t);
+  const int pos = t - offsets[i];
+  int id = ids[t];
+  if (id < 0 || id >= V) {
+    if (lane == 0 && err != nullptr) atomicAdd(err, 1);
+    id = id < 0 ? 0 : V - 1;
+  }
+  const int nch = H >> 3;
+  const bf16* wr = ew + static_cast<size_t>(id) * H;
+  const bf16* pr = ep + static_cast<size_t>(pos) * H;
+  float v[MAXC][8];
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      float a[8], p[8];
+      Chunk8<bf16>::load(wr + ch * 8, a);
+      Chunk8<bf16>::load(pr + ch * 8, p);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[c][e] = a[e] + p[e];
+    }
+  }
+  if (LN) {
+    float mean, rstd;
+    row_moments<MAXC>(v, nch, lane, H, mean, rstd, eps);
+    normalize<MAXC>(v, nch, lane, mean, rstd, g, b);
+  }
+  bf16* xr = x + static_cast<size_t>(t) * H;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) Chunk8<bf16>::store(xr + ch * 8, v[c]);
+  }
+}
+
+// MODE 0: x = LN(y + x); MODE 1: x = y + x, z = LN(x); MODE 2: z = LN(x)
+template <typename T, int MAXC, int MODE>
+__global__ void __launch_bounds__(kWarps * 32)
+    res_ln_kernel(const T* __restrict__ y, T* __restrict__ x, T* __restrict__ z,
+                  const float* __restrict__ g, const float* __restrict__ b, int rows, int H,
+                  float eps) {
+  const int r = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const int nch = H >> 3;
+  const size_t base = static_cast<size_t>(r) * H;
+  float v[MAXC][8];
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) {
+      Chunk8<T>::load(x + base + ch * 8, v[c]);
+      if (MODE != 2) {
+        float u[8];
+        Chunk8<T>::load(y + base + ch * 8, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[c][e] += u[e];
+      }
+    }
+  }
+  if (MODE == 1) {
+    // the residual stream keeps the rounded sum, LN reads the same rounded values
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int ch = lane + 32 * c;
+      if (ch < nch) {
+        Chunk8<T>::store(x + base + ch * 8, v[c]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[c][e] = to_f32(from_f32<T>(v[c][e]));
+      }
+    }
+  }
+  float mean, rstd;
+  row_moments<MAXC>(v, nch, lane, H, mean, rstd, eps);
+  normalize<MAXC>(v, nch, lane, mean, rstd, g, b);
+  T* out = (MODE == 0 ? x : z) + base;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lane + 32 * c;
+    if (ch < nch) Chunk8<T>::store(out + ch * 8, v[c]);
+  }
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+    head_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ offsets, int n,
+                const float* __restrict__ w, float br, int H, int last, float* __restrict__ out) {
+  const int i = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (i >= n) return;
+  const int t = last ? offsets[i + 1] - 1 : offsets[i];
+  const bf16* xr = x + static_cast<size_t>(t) * H;
+  float acc = 0.f;
+  for (int ch = lane; ch < (H >> 3); ch += 32) {
+    float a[8], ww[8];
+    Chunk8<bf16>::load(xr + ch * 8, a);
+    load_f32x8(w + ch * 8, ww);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc = fmaf(a[e], ww[e], acc);
+  }
+  acc = group_sum<32>(acc);
+  if (lane == 0) out[i] = acc + br;
+}
+
+template <typename S>
+__global__ void cvt_bf16_kernel(const S* __restrict__ src, bf16* __restrict__ dst, size_t n) {
+  for (size_t k = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; k < n;
+       k += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[k] = from_f32<bf16>(to_f32(src[k]));
+}
+template <typename S>
+__global__ void cvt_f32_kernel(const S* __restrict__ src, float* __restrict__ dst, size_t n) {
+  for (size_t k = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; k < n;
+       k += static_cast<size_t>(gridDim.x) * blockDim.x)
+    dst[k] = to_f32(src[k]);
+}
+
+// Smallest supported chunks-per-lane count >= need (H <= 4096).
+int pick_maxc(int H) {
+  const int need = (H / 8 + 31) / 32;
+  for (int m : {1, 2, 3, 4, 6, 8, 12, 16})
+    if (m >= need) return m;
+  return -1;
+}
+
+template <int MAXC>
+cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, const void* ew,
+                    const void* ep, const float* g, const float* b, float eps, int V, int H,
+                    void* x, int32_t* err, cudaStream_t st) {
+  dim3 grid((T + kWarps - 1) / kWarps);
+  if (g != nullptr)
+    embed_kernel<MAXC, true><<<grid, kWarps * 32, 0, st>>>(
+        ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
+        V, H, static_cast<bf16*>(x), err);
+  else
+    embed_kernel<MAXC, false><<<grid, kWarps * 32, 0, st>>>(
+        ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
+        V, H, static_cast<bf16*>(x), err);
+  return cudaGetLastError();
+}
+
+template <typename T, int MAXC>
+cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const float* b, int rows,
+                     int H, float eps, int mode, cudaStream_t st) {
+  dim3 grid((rows + kWarps - 1) / kWarps);
+  const T* yy = static_cast<const T*>(y);
+  T* xx = static_cast<T*>(x);
+  T* zz = static_cast<T*>(z);
+  if (mode == 0)
+    res_ln_kernel<T, MAXC, 0><<<grid, kWarps * 32, 0, st>>>(yy, xx, zz, g, b, rows, H, eps);
+  else if (mode == 1)
+    res_ln_kernel<T, MAXC, 1><<<grid, kWarps * 32, 0, st>>>(yy, xx, zz, g, b, rows, H, eps);
+  else
+    res_ln_kernel<T, MAXC, 2><<<grid, kWarps * 32, 0, st>>>(yy, xx, zz, g, b, rows, H, eps);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+#define RMK_MAXC_SWITCH(maxc, CALL)      \
+  switch (maxc) {                        \
+    case 1: { constexpr int M_ = 1; return CALL; }  \
+    case 2: { constexpr int M_ = 2; return CALL; }  \
+    case 3: { constexpr int M_ = 3; return CALL; }  \
+    case 4: { constexpr int M_ = 4; return CALL; }  \
+    case 6: { constexpr int M_ = 6; return CALL; }  \
+    case 8: { constexpr int M_ = 8; return CALL; }  \
+    case 12: { constexpr int M_ = 12; return CALL; } \
+    case 16: { constexpr int M_ = 16; return CALL; } \
+    default: return cudaErrorInvalidValue;            \
+  }
+
+cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs, int T,
+                         const void* emb_word, const void* emb_pos, const float* ln_g,
+                         const float* ln_b, float eps, int V, int P, int H, void* x,
+                         int32_t* err_count, cudaStream_t st) {
+  (void)P;
+  if (T == 0) return cudaSuccess;
+  const int maxc = pick_maxc(H);
+  RMK_MAXC_SWITCH(maxc, (embed_t<M_>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps,
+                                     V, H, x, err_count, st)))
+}
+
+cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
+                          int H, float eps, int dtype, int mode, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  const int maxc = pick_maxc(H);
+  if (dtype == 0) {
+    RMK_MAXC_SWITCH(maxc, (res_ln_t<float, M_>(y, x, z, g, b, T, H, eps, mode, st)))
+  }
+  RMK_MAXC_SWITCH(maxc, (res_ln_t<bf16, M_>(y, x, z, g, b, T, H, eps, mode, st)))
+}
+
+cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
+                        float b_r, int H, int last_token, float* out, cudaStream_t st) {
+  if (n_seqs == 0) return cudaSuccess;
+  dim3 grid((n_seqs + kWarps - 1) / kWarps);
+  head_kernel<<<grid, kWarps * 32, 0, st>>>(static_cast<const bf16*>(x), offsets, n_seqs, w_r,
+                                            b_r, H, last_token, out);
+  return cudaGetLastError();
+}
+
+cudaError_t cvt_to_bf16_launch(const void* src, int src_dtype, void* dst, size_t n,
+                               cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 16));
+  if (src_dtype == 0)
+    cvt_bf16_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(src),
+                                                   static_cast<bf16*>(dst), n);
+  else
+    cvt_bf16_kernel<bf16><<<blocks, 256, 0, st>>>(static_cast<const bf16*>(src),
+                                                  static_cast<bf16*>(dst), n);
+  return cudaGetLastError();
+}
+
+cudaError_t cvt_to_f32_launch(const void* src, int src_dtype, float* dst, size_t n,
+                              cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 16));
+  if (src_dtype == 0)
+    cvt_f32_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(src), dst, n);
+  else
+    cvt_f32_kernel<bf16><<<blocks, 256, 0, st>>>(static_cast<const bf16*>(src), dst, n);
+  return cudaGetLastError();
+}
+
+}  // namespace rmk

@@ -1,0 +1,114 @@
+/*
+ * rm_ops.h -- one C entry point per step of the scoring hot path.
+ *
+ * rm_score (rm.h) chains exactly these launchers; they are exported so that
+ * each step can be checked on its own against the fp64 oracle.  All pointers
+ * are DEVICE pointers unless marked host; all work is asynchronous on stream
+ * (a cudaStream_t as void*).  Return RM_OK or a negative RM_E_* code (rm.h);
+ * arguments are validated on the host before anything is enqueued.
+ *
+ * Packed varlen layout shared by the steps (TurboTransformers review,
+ * "variable-length input" in the abstract; no padding to a fixed length):
+ *   offsets[n+1]  int32 token offsets, sequence i = rows offsets[i]..offsets[i+1]-1,
+ *                 L_i = offsets[i+1]-offsets[i] >= 1.
+ *   X[T][H]       activations, row-major.
+ *   QKV[T][3H]    Q in columns 0..H-1, K in H..2H-1, V in 2H..3H-1; head j
+ *                 uses columns j*d .. j*d+d-1 of each.
+ *   S             attention scores/probabilities.  With Lp_i = round_up(L_i, 8)
+ *                 the entry (sequence i, head j, query r, key c) is at
+ *                 S[s_off[i] + (j*L_i + r)*Lp_i + c], s_off[i] = sum_{k<i} h*L_k*Lp_k.
+ *                 Only c < L_i (causal: c <= r) is ever read or written.
+ *   rb_off[n+1]   prefix sums of ceil(L_i/64): the 64-query row blocks that
+ *                 the attention launches distribute over CTAs.
+ * dtype arguments: RM_F32 (0) or RM_BF16 (1) from rm.h.
+ */
+#ifndef RM_OPS_H_
+#define RM_OPS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host helper: rb_off[n+1] and s_off[n+1] for the layout above (host arrays).
+ * Returns RM_OK, RM_E_INVAL for a length < 1 or non-monotone offsets. */
+int rm_varlen_meta(const int32_t* offsets, int32_t n, int32_t n_heads,
+                   int32_t* rb_off, int64_t* s_off);
+
+/* Y[M][N] = act(X[M][K] . W[N][K]^T + bias[N]) -- the QKV, output and FFN
+ * projections (the "BLAS routines" of the TurboTransformers abstract; tensor
+ * cores per its proposed-method section).  bf16 operands, fp32 accumulation
+ * in tensor memory (tcgen05), bias/GELU in the epilogue.
+ *   x: bf16 [M][K] row-major; w: bf16 [N][K] row-major (nn.Linear layout);
+ *   bias: fp32 [N] or NULL; y: [M][N] row-major of y_dtype (RM_F32|RM_BF16).
+ *   act: 0 = none, 1 = GELU (erf), 2 = GELU (tanh).
+ * Requires M >= 1, N and K multiples of 8, 16-byte aligned x, w, y. */
+int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
+               int32_t M, int32_t N, int32_t K, int32_t act, void* stream);
+
+/* X[t] = E_word[clamp(ids[t])] + E_pos[t - offsets[i]] for each token t of
+ * sequence i, then (ln_g != NULL) the embedding LayerNorm.  ids out of 0..V-1
+ * are clamped and counted with atomicAdd into *err_count (may be NULL).
+ * E_word: bf16 [V][H]; E_pos: bf16 [P][H]; ln_g, ln_b: fp32 [H] or NULL;
+ * x: bf16 [T][H].  Requires every L_i <= P. */
+int rm_op_embed(const int32_t* ids, const int32_t* offsets, int32_t n_seqs, int32_t T,
+                const void* emb_word, const void* emb_pos, const float* ln_g, const float* ln_b,
+                float eps, int32_t V, int32_t P, int32_t H, void* x, int32_t* err_count,
+                void* stream);
+
+/* Attention scores S = (Q K^T)/sqrt(d) per sequence and head, only the valid
+ * L_i x L_i block (causal: keys c <= r).  qkv: bf16 [T][3H]; S: bf16.
+ * n_row_blocks = rb_off[n] (host value); head_dim even, <= 128. */
+int rm_op_attn_scores(const void* qkv, void* S, const int32_t* offsets, const int32_t* rb_off,
+                      const int64_t* s_off, int32_t n_seqs, int32_t n_row_blocks,
+                      int32_t n_heads, int32_t head_dim, int32_t causal, void* stream);
+
+/* Masked row softmax in place over every row of S: p_c = exp(s_c - max)/sum
+ * over keys c < L_i (causal: c <= r) -- the Softmax batch reduction of the
+ * TurboTransformers abstract.  fp32 math; s_dtype RM_BF16 or RM_F32.
+ * T = offsets[n] and max_len >= every L_i (host values). */
+int rm_op_softmax(void* S, int32_t s_dtype, const int32_t* offsets, const int64_t* s_off,
+                  int32_t n_seqs, int32_t T, int32_t n_heads, int32_t max_len, int32_t causal,
+                  void* stream);
+
+/* Context C = P V per sequence and head into ctx[T][H] (head j in columns
+ * j*d..j*d+d-1).  S holds P (bf16), qkv: bf16 [T][3H], ctx: bf16 [T][H]. */
+int rm_op_attn_context(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
+                       const int32_t* rb_off, const int64_t* s_off, int32_t n_seqs,
+                       int32_t n_row_blocks, int32_t n_heads, int32_t head_dim, int32_t causal,
+                       void* stream);
+
+/* Residual + LayerNorm over rows of length H (the LayerNorm batch reduction of
+ * the TurboTransformers abstract), fp32 math, rows of dtype (RM_BF16|RM_F32):
+ *   mode 0 (post-LN): x = LN(y + x)              (z unused, may be NULL)
+ *   mode 1 (pre-LN):  x = y + x;  z = LN(x)      (both written)
+ *   mode 2 (plain):   z = LN(x)                  (y unused, may be NULL)
+ * LN(u) = g * (u - mean)/sqrt(var + eps) + b with the biased variance.
+ * y, x, z: [T][H]; g, b: fp32 [H]. */
+int rm_op_res_ln(const void* y, void* x, void* z, const float* g, const float* b, int32_t T,
+                 int32_t H, float eps, int32_t dtype, int32_t mode, void* stream);
+
+/* Scalar head ("Learning to summarize from human feedback" summary, method
+ * section): out[i] = w_r . u_i + b_r where u_i = x[offsets[i]] (last_token =
+ * 0) or x[offsets[i+1]-1] (last_token = 1).  x: bf16 [T][H]; w_r: fp32 [H];
+ * out: fp32 [n]. */
+int rm_op_head(const void* x, const int32_t* offsets, int32_t n_seqs, const float* w_r,
+               float b_r, int32_t H, int32_t last_token, float* out, void* stream);
+
+/* Host only: the arena plan for one call of a handle created with cfg.
+ * Fills, for each intermediate buffer k < returned count (<= max_bufs):
+ * out_off[k], out_bytes[k] (byte offset/size in the arena), out_first[k],
+ * out_last[k] (first and last step that uses it; buffers whose step ranges
+ * overlap are live together and never share bytes).  *out_peak = arena bytes
+ * the plan needs.  T tokens, n_seqs sequences, s_elems score elements
+ * (s_off[n]).  Returns the buffer count or a negative RM_E_* code. */
+int rm_arena_plan(const void* cfg, int32_t T, int32_t n_seqs, int64_t s_elems,
+                  int64_t* out_off, int64_t* out_bytes, int32_t* out_first, int32_t* out_last,
+                  int32_t max_bufs, int64_t* out_peak);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RM_OPS_H_ */

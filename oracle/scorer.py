@@ -139,6 +139,12 @@ def softmax_masked(s: np.ndarray, allowed: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
+def linear(x: np.ndarray, w: np.ndarray, b) -> np.ndarray:
+    """x W^T + b with W stored [out][in] (b may be None)."""
+    y = x @ w.T
+    return y if b is None else y + b
+
+
 def gelu(u: np.ndarray, kind: int = GELU_ERF) -> np.ndarray:
     """GELU: u * Phi(u) with the normal CDF Phi (erf form), or the tanh approximation."""
     if kind == GELU_ERF:
@@ -179,19 +185,19 @@ def mha(x: np.ndarray, lw: Dict[str, np.ndarray], n_heads: int, causal: bool) ->
     """
     L, H = x.shape
     d = H // n_heads
-    qkv = x @ lw["w_qkv"].T + lw["b_qkv"]
+    qkv = linear(x, lw["w_qkv"], lw["b_qkv"])
     q, k, v = qkv[:, :H], qkv[:, H:2 * H], qkv[:, 2 * H:]
     o = np.empty((L, H))
     for j in range(n_heads):
         cols = slice(j * d, (j + 1) * d)
         pj = attention_probs(q[:, cols], k[:, cols], causal)
         o[:, cols] = pj @ v[:, cols]
-    return o @ lw["w_o"].T + lw["b_o"]
+    return linear(o, lw["w_o"], lw["b_o"])
 
 
 def ffn(x: np.ndarray, lw: Dict[str, np.ndarray], kind: int) -> np.ndarray:
     """W_2 GELU(W_1 x + b_1) + b_2, row-wise."""
-    return gelu(x @ lw["w_1"].T + lw["b_1"], kind) @ lw["w_2"].T + lw["b_2"]
+    return linear(gelu(linear(x, lw["w_1"], lw["b_1"]), kind), lw["w_2"], lw["b_2"])
 
 
 def encoder_layer(x, lw, m: OracleModel):

@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every declared symbol and validates
+configs on the host, all without a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import synth
+import classifier_scoring_b200 as rm
+from classifier_scoring_b200 import build
+from tests.helpers import config_for
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build.build()
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(rm_[a-z0-9_]+)\s*\(",
+                                text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 15, names
+    out = subprocess.run(["nm", "-D", "--defined-only", rm.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (rm_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    L = rm.lib()
+    for n in names:
+        assert hasattr(L, n)
+
+
+def test_library_links_no_cudart_shared_object():
+    out = subprocess.run(["ldd", rm.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcudart" not in out
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_weights_bytes_match_layout(name):
+    shape = synth.WORKLOADS[name].shape
+    esz = 4 if shape.weight_dtype == synth.W_F32 else 2
+    assert rm.weights_bytes(config_for(shape)) == synth.n_weight_elems(shape) * esz
+
+
+@pytest.mark.parametrize("field,value", [
+    ("arch", 2), ("n_layers", 0), ("hidden", 100), ("n_heads", 7), ("ffn", 12), ("vocab", 0),
+    ("max_pos", 10), ("weight_dtype", 3), ("gelu", 5), ("ln_eps", 0.0), ("max_batch_seqs", 0),
+    ("max_tokens", 0), ("max_len", 0), ("max_len", 2000), ("sched_max_batch", 0), ("sched_c0", -1),
+])
+def test_invalid_config_is_rejected_on_host(field, value):
+    cfg = config_for(synth.TINY, max_len=32)
+    setattr(cfg, field, value)
+    assert rm.weights_bytes(cfg) == 0
+    h = ctypes.c_void_p()
+    buf = np.zeros(16, dtype=np.uint8)
+    rc = rm.lib().rm_create(ctypes.byref(cfg), buf.ctypes.data, 16, ctypes.byref(h))
+    assert rc == rm.RM_E_INVAL
+    assert h.value is None
+    assert rm.lib().rm_last_error().decode()
+
+
+def test_head_dim_limits():
+    cfg = config_for(synth.TINY, max_len=32)
+    cfg.hidden, cfg.n_heads = 264, 1          # d = 264 > 128
+    assert rm.weights_bytes(cfg) == 0
+    cfg.hidden, cfg.n_heads = 120, 8          # d = 15, odd
+    assert rm.weights_bytes(cfg) == 0
+
+
+def test_create_checks_weight_size_before_the_device():
+    cfg = config_for(synth.TINY, max_len=32)
+    n = rm.weights_bytes(cfg)
+    buf = np.zeros(n - 4, dtype=np.uint8)
+    h = ctypes.c_void_p()
+    assert rm.lib().rm_create(ctypes.byref(cfg), buf.ctypes.data, n - 4, ctypes.byref(h)) == rm.RM_E_INVAL
+    assert "weights_bytes" in rm.lib().rm_last_error().decode()
+
+
+def test_null_arguments_are_errors_not_crashes():
+    L = rm.lib()
+    assert L.rm_score(None, None, None, 1, None, None) == rm.RM_E_INVAL
+    assert L.rm_score_host(None, None, None, 1, None, None) == rm.RM_E_INVAL
+    assert L.rm_schedule(None, None, 0, None) == rm.RM_E_INVAL
+    assert L.rm_get_device_error(None, None) == rm.RM_E_INVAL
+    assert L.rm_arena_stats(None, None) == rm.RM_E_INVAL
+    L.rm_destroy(None)
+    assert L.rm_op_gemm(None, None, None, None, 1, 1, 8, 8, 0, None) == rm.RM_E_INVAL
+    assert L.rm_op_res_ln(None, None, None, None, None, 1, 8, 1e-5, 1, 0, None) == rm.RM_E_INVAL
+
+
+def test_varlen_meta_layout():
+    lens = np.array([1, 7, 64, 65, 130, 8])
+    off = synth.offsets_from_lengths(lens)
+    rb, so = rm.ops.varlen_meta(off, 3)
+    Lp = (lens + 7) // 8 * 8
+    assert rb.tolist() == [0] + np.cumsum((lens + 63) // 64).tolist()
+    assert so.tolist() == [0] + np.cumsum(3 * lens * Lp).tolist()
+    bad = off.copy()
+    bad[2] = bad[1]
+    with pytest.raises(rm.RmError):
+        rm.ops.varlen_meta(bad, 3)

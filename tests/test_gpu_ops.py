@@ -1,0 +1,282 @@
+"""Step-level parity of the CUDA path against the fp64 oracle (one test per
+hot-path step, called through the C ABI of include/rm_ops.h)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import classifier_scoring_b200 as rm
+from oracle import scorer as O
+from tests.helpers import F32_RTOL
+
+pytestmark = pytest.mark.gpu
+BF16_REL = 2.0 ** -8      # one bf16 rounding of the output
+
+
+def dev(a, dtype):
+    return torch.as_tensor(np.ascontiguousarray(a)).to(dtype).cuda()
+
+
+def f64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    rm.lib()
+    torch.cuda.init()
+
+
+# --- GEMM (QKV / out-proj / FFN projections) -----------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 8), (130, 936, 312), (3264, 2304, 768), (257, 768, 3072),
+                                   (1000, 1200, 312), (128, 256, 64), (64, 128, 1200),
+                                   (555, 3072, 768), (26112 // 16, 6144, 2048)])
+@pytest.mark.parametrize("act", [0, 1, 2])
+def test_gemm_fp32_out(M, N, K, act):
+    g = torch.Generator().manual_seed(M * 7 + N + K + act)
+    x = (torch.randn(M, K, generator=g)).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    b = torch.randn(N, generator=g, dtype=torch.float32) * 0.1
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    xd, wd, bd = x.cuda(), w.cuda(), b.cuda()
+    rm.ops.gemm(xd, wd, bd, y, rm.F32, M, N, K, act)
+    torch.cuda.synchronize()
+    X, W, B = f64(x), f64(w), f64(b)
+    pre = O.linear(X, W, B)
+    ref = pre if act == 0 else O.gelu(pre, O.GELU_ERF if act == 1 else O.GELU_TANH)
+    scale = np.abs(X) @ np.abs(W).T + np.abs(B)          # sum_k |a_k b_k| + |bias|
+    err = np.abs(f64(y) - ref)
+    # GELU' <= 1.13; erff/tanhf add a few fp32 ulps of the output
+    bound = F32_RTOL * scale * (1.0 if act == 0 else 1.2) + (0 if act == 0 else 4e-7 * np.abs(ref))
+    assert np.all(err <= bound), float((err / bound).max())
+
+
+@pytest.mark.parametrize("M,N,K", [(3264, 2304, 768), (77, 936, 312)])
+def test_gemm_bf16_out_and_no_bias(M, N, K):
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    rm.ops.gemm(x.cuda(), w.cuda(), None, y, rm.BF16, M, N, K, 0)
+    torch.cuda.synchronize()
+    ref = O.linear(f64(x), f64(w), None)
+    scale = np.abs(f64(x)) @ np.abs(f64(w)).T
+    assert np.all(np.abs(f64(y) - ref) <= BF16_REL * np.abs(ref) + F32_RTOL * scale)
+
+
+def test_gemm_rejects_bad_shapes():
+    x = torch.zeros(16, 12, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rm.RmError):
+        rm.ops.gemm(x, x, None, x, rm.BF16, 16, 16, 12, 0)
+
+
+# --- residual + LayerNorm ---------------------------------------------------------
+
+@pytest.mark.parametrize("H", [128, 312, 768, 2048])
+@pytest.mark.parametrize("mode", [0, 1, 2])
+def test_res_ln_fp32(H, mode):
+    T = 777
+    rng = np.random.default_rng(H + mode)
+    y = rng.normal(0, 1, (T, H)).astype(np.float32)
+    x = rng.normal(0.5, 2, (T, H)).astype(np.float32)
+    gm = (1 + rng.normal(0, 0.2, H)).astype(np.float32)
+    bt = rng.normal(0, 0.2, H).astype(np.float32)
+    yd, xd, zd = dev(y, torch.float32), dev(x, torch.float32), torch.zeros(T, H, device="cuda")
+    rm.ops.res_ln(yd, xd, zd, dev(gm, torch.float32), dev(bt, torch.float32), T, H, 1e-5,
+                  rm.F32, mode)
+    torch.cuda.synchronize()
+    u = x.astype(np.float64) + (y.astype(np.float64) if mode != 2 else 0)
+    if mode == 1:
+        u = u.astype(np.float32).astype(np.float64)       # the stored residual is fp32
+    ref = O.layer_norm(u, gm.astype(np.float64), bt.astype(np.float64), 1e-5)
+    out = f64(xd) if mode == 0 else f64(zd)
+    assert np.all(np.abs(out - ref) <= F32_RTOL * (np.abs(ref) + np.abs(gm)))
+    if mode == 1:
+        assert np.array_equal(f64(xd), u)
+
+
+@pytest.mark.parametrize("H", [312, 768, 2048])
+def test_res_ln_bf16(H):
+    T = 3264
+    rng = np.random.default_rng(H)
+    y = rng.normal(0, 1, (T, H))
+    x = rng.normal(0, 1, (T, H))
+    gm = (1 + rng.normal(0, 0.02, H)).astype(np.float32)
+    bt = rng.normal(0, 0.02, H).astype(np.float32)
+    yd, xd = dev(y, torch.bfloat16), dev(x, torch.bfloat16)
+    u = f64(yd) + f64(xd)
+    rm.ops.res_ln(yd, xd, None, dev(gm, torch.float32), dev(bt, torch.float32), T, H, 1e-12,
+                  rm.BF16, 0)
+    torch.cuda.synchronize()
+    ref = O.layer_norm(u, gm.astype(np.float64), bt.astype(np.float64), 1e-12)
+    assert np.all(np.abs(f64(xd) - ref) <= BF16_REL * np.abs(ref) + 1e-4 * np.abs(gm))
+
+
+# --- softmax -------------------------------------------------------------------------
+
+def varlen_rows(lens, nh, rng, dtype):
+    off = synth.offsets_from_lengths(lens)
+    rb, so = rm.ops.varlen_meta(off, nh)
+    S = np.full(int(so[-1]), np.nan, dtype=np.float32)
+    for i, L in enumerate(lens):
+        Lp = (L + 7) // 8 * 8
+        blk = S[so[i]:so[i + 1]].reshape(nh, L, Lp)
+        blk[:, :, :L] = rng.normal(0, 3, (nh, L, L))
+    return off, rb, so, S
+
+
+@pytest.mark.parametrize("lens", [[1, 2, 3, 100, 57], [64, 128, 256], [513, 560, 7], [1024, 1000]],
+                         ids=["short", "tinybert", "long", "max"])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("dtype", [rm.F32, rm.BF16], ids=["f32", "bf16"])
+def test_softmax(lens, causal, dtype):
+    nh = 3
+    rng = np.random.default_rng(len(lens) + causal)
+    lens = np.array(lens)
+    off, rb, so, S = varlen_rows(lens, nh, rng, dtype)
+    tdt = torch.float32 if dtype == rm.F32 else torch.bfloat16
+    Sd = dev(S, tdt)
+    S_in = f64(Sd)
+    rm.ops.softmax(Sd, dtype, dev(off, torch.int32), dev(so, torch.int64), len(lens),
+                   int(off[-1]), nh, int(lens.max()), causal)
+    torch.cuda.synchronize()
+    P = f64(Sd)
+    for i, L in enumerate(lens):
+        Lp = (L + 7) // 8 * 8
+        got = P[so[i]:so[i + 1]].reshape(nh, L, Lp)
+        s_in = S_in[so[i]:so[i + 1]].reshape(nh, L, Lp)[:, :, :L]
+        allowed = np.tril(np.ones((L, L), bool)) if causal else np.ones((L, L), bool)
+        ref = O.softmax_masked(s_in, np.broadcast_to(allowed, (nh, L, L)))
+        g = got[:, :, :L]
+        ok = np.broadcast_to(allowed, g.shape)
+        tol = F32_RTOL if dtype == rm.F32 else BF16_REL
+        assert np.all(np.abs(g[ok] - ref[ok]) <= tol * ref[ok] + 1e-37)
+        # entries inside a written 8-wide chunk but outside the row are exactly 0
+        for r in (0, L - 1):
+            lim = r + 1 if causal else L
+            end = min(Lp, (lim + 7) // 8 * 8)
+            assert np.all(got[:, r, lim:end] == 0)
+
+
+# --- attention scores and context -----------------------------------------------------
+
+def qkv_for(T, H, rng):
+    return rng.normal(0, 1, (T, 3 * H))
+
+
+@pytest.mark.parametrize("nh,d", [(2, 64), (12, 26), (12, 64), (16, 128)])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_attention_scores(nh, d, causal):
+    H = nh * d
+    lens = np.array([1, 65, 130, 64, 9])
+    off = synth.offsets_from_lengths(lens)
+    rb, so = rm.ops.varlen_meta(off, nh)
+    rng = np.random.default_rng(nh + d + causal)
+    qkv = dev(qkv_for(int(off[-1]), H, rng), torch.bfloat16)
+    Q = f64(qkv)
+    S = torch.full((int(so[-1]),), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rm.ops.attn_scores(qkv, S, dev(off, torch.int32), dev(rb, torch.int32), dev(so, torch.int64),
+                       len(lens), int(rb[-1]), nh, d, causal)
+    torch.cuda.synchronize()
+    Sh = f64(S)
+    for i, L in enumerate(lens):
+        Lp = (L + 7) // 8 * 8
+        blk = Sh[so[i]:so[i + 1]].reshape(nh, L, Lp)
+        rows = Q[off[i]:off[i + 1]]
+        for j in range(nh):
+            q = rows[:, j * d:(j + 1) * d]
+            k = rows[:, H + j * d:H + (j + 1) * d]
+            ref = q @ k.T / np.sqrt(d)
+            scale = np.abs(q) @ np.abs(k).T / np.sqrt(d)
+            ok = np.tril(np.ones((L, L), bool)) if causal else np.ones((L, L), bool)
+            err = np.abs(blk[j][:, :L] - ref)
+            assert np.all(err[ok] <= BF16_REL * np.abs(ref[ok]) + F32_RTOL * scale[ok])
+
+
+@pytest.mark.parametrize("nh,d", [(2, 64), (12, 26), (16, 128)])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_attention_context(nh, d, causal):
+    H = nh * d
+    lens = np.array([1, 65, 130, 64, 9])
+    off = synth.offsets_from_lengths(lens)
+    rb, so = rm.ops.varlen_meta(off, nh)
+    rng = np.random.default_rng(nh * d + causal)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng), torch.bfloat16)
+    V = f64(qkv)
+    # probabilities with junk (NaN) outside the allowed keys: the kernel must not read them
+    P = np.full(int(so[-1]), np.nan, dtype=np.float32)
+    for i, L in enumerate(lens):
+        Lp = (L + 7) // 8 * 8
+        blk = P[so[i]:so[i + 1]].reshape(nh, L, Lp)
+        ok = np.tril(np.ones((L, L), bool)) if causal else np.ones((L, L), bool)
+        s = rng.normal(0, 2, (nh, L, L))
+        blk[:, :, :L] = np.where(ok, O.softmax_masked(s, np.broadcast_to(ok, s.shape)), np.nan)
+    Pd = dev(P, torch.bfloat16)
+    Ph = f64(Pd)
+    ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rm.ops.attn_context(Pd, qkv, ctx, dev(off, torch.int32), dev(rb, torch.int32),
+                        dev(so, torch.int64), len(lens), int(rb[-1]), nh, d, causal)
+    torch.cuda.synchronize()
+    C = f64(ctx)
+    for i, L in enumerate(lens):
+        Lp = (L + 7) // 8 * 8
+        blk = Ph[so[i]:so[i + 1]].reshape(nh, L, Lp)[:, :, :L]
+        rows = V[off[i]:off[i + 1]]
+        for j in range(nh):
+            p = np.nan_to_num(blk[j], nan=0.0)
+            v = rows[:, 2 * H + j * d:2 * H + (j + 1) * d]
+            ref = p @ v
+            scale = np.abs(p) @ np.abs(v)
+            got = C[off[i]:off[i + 1], j * d:(j + 1) * d]
+            assert np.all(np.abs(got - ref) <= BF16_REL * np.abs(ref) + F32_RTOL * scale)
+
+
+# --- embedding and head ----------------------------------------------------------------
+
+@pytest.mark.parametrize("H,ln", [(128, True), (312, True), (768, True), (2048, False)])
+def test_embed(H, ln):
+    V, P = 1000, 600
+    lens = np.array([1, 560, 33, 8])
+    off = synth.offsets_from_lengths(lens)
+    rng = np.random.default_rng(H)
+    ids = rng.integers(0, V, int(off[-1])).astype(np.int32)
+    ids[5] = V + 7            # out of range: clamped to V-1 and counted
+    ids[9] = -3               # clamped to 0
+    ew = dev(rng.normal(0, 0.5, (V, H)), torch.bfloat16)
+    ep = dev(rng.normal(0, 0.5, (P, H)), torch.bfloat16)
+    g = dev(1 + rng.normal(0, 0.1, H), torch.float32)
+    b = dev(rng.normal(0, 0.1, H), torch.float32)
+    x = torch.zeros(int(off[-1]), H, dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    rm.ops.embed(dev(ids, torch.int32), dev(off, torch.int32), len(lens), int(off[-1]), ew, ep,
+                 g if ln else None, b if ln else None, 1e-12, V, P, H, x, err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 2
+    EW, EP = f64(ew), f64(ep)
+    cid = np.clip(ids, 0, V - 1)
+    for i, L in enumerate(lens):
+        u = EW[cid[off[i]:off[i + 1]]] + EP[:L]
+        ref = O.layer_norm(u, f64(g), f64(b), 1e-12) if ln else u
+        got = f64(x)[off[i]:off[i + 1]]
+        assert np.all(np.abs(got - ref) <= BF16_REL * np.abs(ref) + 1e-5 * (1 + np.abs(ref)))
+
+
+@pytest.mark.parametrize("last", [0, 1])
+def test_head(last):
+    H = 768
+    lens = np.array([1, 17, 100, 2])
+    off = synth.offsets_from_lengths(lens)
+    rng = np.random.default_rng(last)
+    x = dev(rng.normal(0, 1, (int(off[-1]), H)), torch.bfloat16)
+    w = rng.normal(0, 0.05, H).astype(np.float32)
+    out = torch.zeros(len(lens), dtype=torch.float32, device="cuda")
+    rm.ops.head(x, dev(off, torch.int32), len(lens), dev(w, torch.float32), 0.25, H, last, out)
+    torch.cuda.synchronize()
+    X = f64(x)
+    rows = X[off[1:] - 1] if last else X[off[:-1]]
+    ref = rows @ w.astype(np.float64) + 0.25
+    assert np.all(np.abs(f64(out) - ref) <= F32_RTOL * (np.abs(rows) @ np.abs(w) + 0.25))

@@ -281,3 +281,13 @@ def test_scores_are_sensitive_to_every_layer_term():
         m.layers[0][name] = m.layers[0][name] * 0.5
         assert abs(O.score_one(m, ids) - base) > 1e-6, name
         m.layers[0][name] = saved
+
+
+def test_oracle_reproduces_stored_golden_scores():
+    import os
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    sys.path.insert(0, os.path.join(here, "golden"))
+    import make_golden
+    gold = np.loadtxt(os.path.join(here, "golden", "tiny_enc_scores.txt"))
+    assert np.max(np.abs(make_golden.tiny_enc_scores() - gold)) <= 1e-12
