@@ -47,7 +47,8 @@ UNIT = "sequences/s"
 # tokens; C0 stands for the fixed per-batch cost (launch sequence, weight
 # streaming) of about 20k token-steps.
 SCHED_C0, SCHED_C1 = 20000, 1
-KERNEL_NAMES = ("gemm", "attn_scores", "softmax", "attn_context", "layernorm", "embed", "head")
+KERNEL_NAMES = ("gemm", "attn_scores", "softmax", "attn_context", "layernorm", "embed", "head",
+                "attn_fused")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic per launch of the dominant kernel (tcgen05 GEMM) from one ncu
@@ -89,6 +90,10 @@ def workload_config(name):
             "parallelism": "replicas"}
 
 
+def lanes_note(n):
+    return f"{n} stream(s) per GPU, consecutive DP batches dealt round-robin"
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -101,7 +106,6 @@ class ClockSampler:
         self.proc = None
         self.path = out_path
         try:
-            self.f = open(out_path, "w") if out_path else subprocess.DEVNULL
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-i", str(gpu_index), "-lms", "200"],
@@ -149,25 +153,33 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
-def time_oracle(name: str, budget_s: float, min_requests: int = 4, start: int = 0):
-    """Score requests of the workload's stream with the fp64 oracle, one by one,
-    until budget_s has elapsed; returns (sequences/s, requests scored)."""
-    from oracle import scorer
-    w = synth.WORKLOADS[name]
-    s = w.shape
-    m = scorer.unpack_weights(synth.make_weights(s, w.seed), s.arch, s.n_layers, s.hidden,
-                              s.n_heads, s.ffn, s.vocab, s.max_pos, s.weight_dtype, s.gelu, s.ln_eps)
-    st = synth.make_stream(w)
-    t0 = time.perf_counter()
-    k = 0
-    while True:
-        i = (start + k) % len(st.lengths)
-        scorer.score_one(m, st.ids[st.starts[i]:st.starts[i] + st.lengths[i]])
-        k += 1
-        el = time.perf_counter() - t0
-        if (el >= budget_s and k >= min_requests) or k >= len(st.lengths):
-            break
-    return k / el, k, el
+class OracleTimer:
+    """The fp64 CPU oracle on the workload's seeded stream (loaded once)."""
+
+    def __init__(self, name: str):
+        from oracle import scorer
+        self.scorer = scorer
+        w = synth.WORKLOADS[name]
+        s = w.shape
+        self.m = scorer.unpack_weights(synth.make_weights(s, w.seed), s.arch, s.n_layers, s.hidden,
+                                       s.n_heads, s.ffn, s.vocab, s.max_pos, s.weight_dtype, s.gelu,
+                                       s.ln_eps)
+        self.st = synth.make_stream(w)
+
+    def run(self, budget_s: float, min_requests: int = 4, start: int = 0):
+        """Score requests one by one until budget_s has elapsed and at least
+        min_requests are done; returns (sequences/s, requests, seconds)."""
+        st = self.st
+        t0 = time.perf_counter()
+        k = 0
+        while True:
+            i = (start + k) % len(st.lengths)
+            self.scorer.score_one(self.m, st.ids[st.starts[i]:st.starts[i] + st.lengths[i]])
+            k += 1
+            el = time.perf_counter() - t0
+            if (el >= budget_s and k >= min_requests) or k >= len(st.lengths):
+                break
+        return k / el, k, el
 
 
 def reference_arm(args):
@@ -178,8 +190,9 @@ def reference_arm(args):
     w = synth.WORKLOADS[name]
     per_step = 8 if w.shape.hidden >= 768 else 64
     times, done = [], 0
+    timer = OracleTimer(name)
     for it in range(args.warmup + args.steps):
-        rate, k, el = time_oracle(name, 0.0, min_requests=per_step, start=it * per_step)
+        rate, k, el = timer.run(0.0, min_requests=per_step, start=it * per_step)
         if it >= args.warmup:
             times.append(el)
             done += k
@@ -233,12 +246,26 @@ def b200_arm(args):
                            sched_max_batch=w.max_batch, sched_c0=SCHED_C0, sched_c1=SCHED_C1)
     sc = rm.Scorer(cfg, flat)
     del flat
-    stream = torch.cuda.Stream()
+    # lanes: handles that share the weights, each on its own stream, so that
+    # consecutive batches overlap on the GPU
+    lanes = [sc] + [sc.shared() for _ in range(args.lanes - 1)]
+    streams = [torch.cuda.Stream() for _ in range(args.lanes)]
+    stream = streams[0]
 
     # the schedule is deterministic: pack the stream in batch order once, on the device
     batch = sc.schedule(st.lengths)
     nb = int(batch.max()) + 1
     groups = [np.nonzero(batch == b)[0] for b in range(nb)]
+    if args.batch_index is not None:
+        # one DP batch only (small profiling case): the step scores just this batch
+        keep = groups[args.batch_index % nb]
+        sub = np.zeros(len(st.lengths), dtype=bool)
+        sub[keep] = True
+        st = synth.Stream(lengths=st.lengths[keep], ids=st.ids, starts=st.starts[keep])
+        n_req = len(keep)
+        batch = np.zeros(n_req, dtype=np.int32)
+        nb = 1
+        groups = [np.arange(n_req)]
     order = np.concatenate(groups)
     packed_ids, _ = synth.pack(st, order)
     b_tok = np.zeros(nb + 1, dtype=np.int64)
@@ -253,14 +280,29 @@ def b200_arm(args):
     out_dev = torch.zeros(n_req, dtype=torch.float32, device="cuda")
     ev_batch = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
 
+    fork_ev = torch.cuda.Event()
+    join_ev = [torch.cuda.Event() for _ in streams]
+
+    def fork():
+        # every lane starts after what stream 0 has enqueued so far
+        fork_ev.record(stream)
+        for s2 in streams[1:]:
+            s2.wait_event(fork_ev)
+
+    def join():
+        for k, s2 in enumerate(streams[1:], 1):
+            join_ev[k].record(s2)
+            stream.wait_event(join_ev[k])
+
     def step(record=False):
         bt = sc.schedule(st.lengths)                          # S0 on the host
-        if record and not np.array_equal(bt, batch):
+        if record and args.batch_index is None and not np.array_equal(bt, batch):
             raise RuntimeError("schedule changed between steps")
         for b in range(nb):
-            sc.score(ids_dev[b_tok[b]:], b_off[b], out_dev[b_seq[b]:], stream)
+            k = b % len(lanes)
+            lanes[k].score(ids_dev[b_tok[b]:], b_off[b], out_dev[b_seq[b]:], streams[k])
             if record:
-                ev_batch[b].record(stream)
+                ev_batch[b].record(streams[k])
 
     def barrier():
         if dist is not None:
@@ -268,12 +310,16 @@ def b200_arm(args):
 
     # warm-up (plans every length bucket, compiles nothing: the kernels are prebuilt)
     for _ in range(args.warmup):
+        fork()
         step()
+        join()
     torch.cuda.synchronize()
 
-    sc.profile(args.profile_every)
-    launches0 = sc.profile_read()["total_launches"]
-    sc.profile(args.profile_every)
+    launches0 = 0
+    for h in lanes:
+        h.profile(args.profile_every)
+        launches0 += h.profile_read()["total_launches"]
+        h.profile(args.profile_every)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
     out_dir = os.path.join(ROOT, "gpurun_out")
@@ -286,17 +332,28 @@ def b200_arm(args):
     t_end = torch.cuda.Event(enable_timing=True)
     wall0 = time.perf_counter()
     t_start.record(stream)
+    fork()
     for k in range(args.steps):
         step(record=(k == args.steps - 1))
+    join()
     t_end.record(stream)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     barrier()
     clk = clocks.stop()
     elapsed_ms = t_start.elapsed_time(t_end)
-    prof = sc.profile_read()
+    prof = None
+    for h in lanes:
+        p1 = h.profile_read()
+        h.profile(0)
+        if prof is None:
+            prof = p1
+        else:
+            for kname in KERNEL_NAMES:
+                for f in ("ms", "launches", "flops", "bytes"):
+                    prof[kname][f] += p1[kname][f]
+            prof["total_launches"] += p1["total_launches"]
     launches = prof["total_launches"] - launches0
-    sc.profile(0)
     # latency in the last timed step: every request is queued at the step's start
     # and completes with its batch; the step's start is taken as the last
     # batch's completion minus the mean step time
@@ -313,19 +370,15 @@ def b200_arm(args):
     out_pin = torch.empty(n_req, dtype=torch.float32).pin_memory()
     ids_np = ids_pin.numpy()
     host_ids = st.ids
+    # position in the arrival-ordered id array of every packed token (batch order)
+    gather = np.concatenate([np.arange(st.starts[i], st.starts[i] + st.lengths[i]) for i in order])
 
     def e2e_step():
-        bt = sc.schedule(st.lengths)
-        pos = 0
-        for b in range(nb):                                   # S1: host gather into pinned memory
-            g = groups[b]
-            for i in g:
-                L = int(st.lengths[i])
-                ids_np[pos:pos + L] = host_ids[st.starts[i]:st.starts[i] + L]
-                pos += L
-        del bt
+        sc.schedule(st.lengths)                               # S0
+        np.take(host_ids, gather, out=ids_np)                 # S1: host gather into pinned memory
         for b in range(nb):
-            sc.score_host(ids_pin[b_tok[b]:], b_off[b], out_pin[b_seq[b]:], stream)
+            k = b % len(lanes)
+            lanes[k].score_host(ids_pin[b_tok[b]:], b_off[b], out_pin[b_seq[b]:], streams[k])
 
     e2e_step()
     torch.cuda.synchronize()
@@ -334,9 +387,11 @@ def b200_arm(args):
     e1 = torch.cuda.Event(enable_timing=True)
     ew0 = time.perf_counter()
     e0.record(stream)
+    fork()
     e_steps = max(1, args.steps)
     for _ in range(e_steps):
         e2e_step()
+    join()
     e1.record(stream)
     torch.cuda.synchronize()
     e_wall = time.perf_counter() - ew0
@@ -380,7 +435,7 @@ def b200_arm(args):
             continue
         e = {"launches_timed": d["launches"], "avg_us": 1000 * d["ms"] / d["launches"],
              "share_of_timed": d["ms"] / max(1e-9, sum(prof[x]["ms"] for x in KERNEL_NAMES))}
-        if d["flops"] and kname in ("gemm", "attn_scores", "attn_context"):
+        if d["flops"] and kname in ("gemm", "attn_scores", "attn_context", "attn_fused"):
             e["tflops"] = d["flops"] / (d["ms"] * 1e-3) / 1e12
         if d["bytes"]:
             e["gbs"] = d["bytes"] / (d["ms"] * 1e-3) / 1e9
@@ -391,7 +446,7 @@ def b200_arm(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(name),
+        "config": dict(workload_config(name), lanes=lanes_note(len(lanes))),
         "p50_latency_ms": p50, "p99_latency_ms": p99, "batches_per_step": nb,
         "tokens_per_step": int(b_tok[-1]),
         "roofline": roofline,
@@ -404,16 +459,89 @@ def b200_arm(args):
         "context": {"turbotransformers_req_s_len2_100": 402, "hardware": "not named on the page"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, k, el = time_oracle(name, args.cpu_budget)
+        rate, k, el = OracleTimer(name).run(args.cpu_budget)
         result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": oracle_threads(),
                                   "kind": "oracle",
                                   "sample": f"first {k} requests of the seeded stream scored one by "
                                             f"one by the fp64 numpy oracle ({el:.1f} s)"}
     if rank == 0:
         print(json.dumps(result), flush=True)
-    sc.close()
+    for h in lanes:
+        h.close()
     if dist is not None:
         dist.destroy_process_group()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# the two batch reductions alone, on working sets far larger than L2
+# ---------------------------------------------------------------------------
+def kernel_bench(args):
+    import torch
+    import classifier_scoring_b200 as rm
+    from classifier_scoring_b200 import build as rmbuild
+
+    rmbuild.build()
+    torch.cuda.set_device(0)
+    pk, pk_kind = peaks()
+    st = torch.cuda.Stream()
+    reps = max(3, args.steps)
+    out = {"metric": "HBM GB/s of the softmax and residual+LayerNorm kernels alone",
+           "unit": "GB/s", "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": f"hbm_gbs of {pk_kind}",
+           "kernels": {}}
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(reps):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    # softmax over the score blocks of sequences with lengths U[5, 500], 12 heads
+    rng = np.random.default_rng(7)
+    nh = 12
+    for label, lo, hi, causal in (("softmax_len5_500", 5, 500, 0), ("softmax_len256_560_causal", 256, 560, 1),
+                                  ("softmax_len2_100", 2, 100, 0)):
+        lens = []
+        tot = 0
+        while tot < 1.0e9:                       # about 2 GB of bf16 scores
+            L = int(rng.integers(lo, hi + 1))
+            lens.append(L)
+            tot += nh * L * ((L + 7) // 8 * 8)
+        lens = np.array(lens)
+        off = synth.offsets_from_lengths(lens)
+        rb, so = rm.ops.varlen_meta(off, nh)
+        S = torch.randn(int(so[-1]), dtype=torch.bfloat16, device="cuda")
+        d_off = torch.from_numpy(off).cuda()
+        d_so = torch.from_numpy(so).cuda()
+        n, T = len(lens), int(off[-1])
+        # the kernel's rows are independent, so a launch covers at most 2^31 rows: fine here
+        ms = timed(lambda: rm.ops.softmax(S, rm.BF16, d_off, d_so, n, T, nh, int(lens.max()), causal, st))
+        entries = nh * float(np.sum(lens * (lens + 1) / 2 if causal else lens * lens))
+        gb = 4.0 * entries / 1e9
+        out["kernels"][label] = {"ms": ms, "algorithmic_GB": gb, "gbs": gb / (ms * 1e-3),
+                                 "frac_of_measured": gb / (ms * 1e-3) / pk["hbm_gbs"],
+                                 "sequences": n, "heads": nh}
+        del S
+    for label, H, T, mode in (("res_ln_post_H768", 768, 1 << 20, 0), ("res_ln_pre_H2048", 2048, 1 << 18, 1)):
+        y = torch.randn(T, H, dtype=torch.bfloat16, device="cuda")
+        x = torch.randn(T, H, dtype=torch.bfloat16, device="cuda")
+        z = torch.empty_like(x) if mode == 1 else None
+        g = torch.ones(H, dtype=torch.float32, device="cuda")
+        b = torch.zeros(H, dtype=torch.float32, device="cuda")
+        ms = timed(lambda: rm.ops.res_ln(y, x, z, g, b, T, H, 1e-5, rm.BF16, mode, st))
+        gb = (6.0 if mode == 0 else 8.0) * H * T / 1e9
+        out["kernels"][label] = {"ms": ms, "algorithmic_GB": gb, "gbs": gb / (ms * 1e-3),
+                                 "frac_of_measured": gb / (ms * 1e-3) / pk["hbm_gbs"],
+                                 "rows": T, "hidden": H}
+        del y, x, z
+    print(json.dumps(out), flush=True)
     return 0
 
 
@@ -428,12 +556,20 @@ def main():
                     help="time the kernels of every n-th batch with CUDA events (0 = off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel-bench", action="store_true",
+                    help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
+    ap.add_argument("--lanes", type=int, default=1,
+                    help="handles sharing the weights, one stream each, batches dealt round-robin")
+    ap.add_argument("--batch-index", type=int, default=None,
+                    help="score only this DP batch of the stream per step (small profiling case)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "b200":
         print("note: at least 3 warm-up steps are required; using 3", file=sys.stderr)
         args.warmup = 3
     if args.impl == "reference":
         return reference_arm(args)
+    if args.kernel_bench:
+        return kernel_bench(args)
     return b200_arm(args)
 
 

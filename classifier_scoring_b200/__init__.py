@@ -20,6 +20,7 @@ __all__ = ["RmConfig", "RmError", "Scorer", "lib", "schedule", "weights_bytes", 
 ENC_POSTLN, DEC_PRELN = 0, 1
 F32, BF16 = 0, 1
 GELU_ERF, GELU_TANH = 0, 1
+ATTN_FUSED, ATTN_MATERIALIZED = 0, 1
 RM_OK, RM_E_INVAL, RM_E_NOMEM, RM_E_CUDA, RM_E_RANGE, RM_E_DEVICE = 0, -1, -2, -3, -4, -5
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmscore.so")
@@ -40,15 +41,17 @@ class RmConfig(ctypes.Structure):
         ("max_batch_seqs", ctypes.c_int32), ("max_tokens", ctypes.c_int32), ("max_len", ctypes.c_int32),
         ("sched_max_batch", ctypes.c_int32), ("sched_c0", ctypes.c_int64), ("sched_c1", ctypes.c_int64),
         ("sched_table", ctypes.POINTER(ctypes.c_int64)), ("sched_table_b", ctypes.c_int32),
-        ("sched_table_l", ctypes.c_int32),
+        ("sched_table_l", ctypes.c_int32), ("attn_impl", ctypes.c_int32),
     ]
 
     @classmethod
     def make(cls, *, arch, n_layers, hidden, n_heads, ffn, vocab, max_pos, weight_dtype,
              gelu=GELU_ERF, ln_eps=1e-12, max_batch_seqs=64, max_tokens=8192, max_len=512,
-             sched_max_batch=64, sched_c0=0, sched_c1=1, sched_table=None) -> "RmConfig":
+             sched_max_batch=64, sched_c0=0, sched_c1=1, sched_table=None,
+             attn_impl=0) -> "RmConfig":
         c = cls(arch, n_layers, hidden, n_heads, ffn, vocab, max_pos, weight_dtype, gelu, ln_eps,
-                max_batch_seqs, max_tokens, max_len, sched_max_batch, sched_c0, sched_c1, None, 0, 0)
+                max_batch_seqs, max_tokens, max_len, sched_max_batch, sched_c0, sched_c1, None, 0, 0,
+                attn_impl)
         if sched_table is not None:
             t = np.ascontiguousarray(sched_table, dtype=np.int64)
             c._table_keepalive = t
@@ -73,6 +76,7 @@ def lib() -> ctypes.CDLL:
     sig = {
         "rm_weights_bytes": (SZ, [cfgp]),
         "rm_create": (ctypes.c_int, [cfgp, P, SZ, ctypes.POINTER(P)]),
+        "rm_create_shared": (ctypes.c_int, [P, ctypes.POINTER(P)]),
         "rm_score": (ctypes.c_int, [P, P, P, I32, P, P]),
         "rm_score_host": (ctypes.c_int, [P, P, P, I32, P, P]),
         "rm_schedule": (ctypes.c_int, [P, P, I32, P]),
@@ -89,6 +93,7 @@ def lib() -> ctypes.CDLL:
         "rm_op_attn_scores": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_softmax": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attn_context": (ctypes.c_int, [P, P, P, P, P, P, I32, I32, I32, I32, I32, P]),
+        "rm_op_attn_fused": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_res_ln": (ctypes.c_int, [P, P, P, P, P, I32, I32, F, I32, I32, P]),
         "rm_op_head": (ctypes.c_int, [P, P, I32, P, F, I32, I32, P, P]),
         "rm_arena_plan": (ctypes.c_int, [cfgp, I32, I32, I64, P, P, P, P, I32, P]),
@@ -144,12 +149,20 @@ def schedule(cfg: RmConfig, lengths) -> np.ndarray:
 class Scorer:
     """A scorer handle (rm_create ... rm_destroy)."""
 
-    def __init__(self, cfg: RmConfig, weights: np.ndarray):
-        w = np.ascontiguousarray(weights)
+    def __init__(self, cfg: RmConfig, weights: np.ndarray = None, *, share: "Scorer" = None):
         h = ctypes.c_void_p()
-        _check(lib().rm_create(ctypes.byref(cfg), w.ctypes.data, w.nbytes, ctypes.byref(h)))
+        if share is not None:
+            _check(lib().rm_create_shared(share._h, ctypes.byref(h)))
+            cfg = share.cfg
+        else:
+            w = np.ascontiguousarray(weights)
+            _check(lib().rm_create(ctypes.byref(cfg), w.ctypes.data, w.nbytes, ctypes.byref(h)))
         self._h = h
         self.cfg = cfg
+
+    def shared(self) -> "Scorer":
+        """A new handle on the same weights with its own arena (rm_create_shared)."""
+        return Scorer(self.cfg, share=self)
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
@@ -191,7 +204,8 @@ class Scorer:
         _check(lib().rm_get_device_error(self._h, out.ctypes.data))
         return out
 
-    K_NAMES = ("gemm", "attn_scores", "softmax", "attn_context", "layernorm", "embed", "head")
+    K_NAMES = ("gemm", "attn_scores", "softmax", "attn_context", "layernorm", "embed", "head",
+               "attn_fused")
 
     def profile(self, every: int) -> None:
         """Time every-th call's launches with CUDA events (0 = off); restarts counters."""
@@ -258,6 +272,12 @@ class ops:
         _check(lib().rm_op_attn_context(_ptr(S), _ptr(qkv), _ptr(ctx), _ptr(offsets_dev),
                                         _ptr(rb_dev), _ptr(so_dev), n_seqs, n_row_blocks, n_heads,
                                         head_dim, int(causal), _stream(stream)))
+
+    @staticmethod
+    def attn_fused(qkv, ctx, offsets_dev, rb_dev, n_seqs, n_row_blocks, n_heads, head_dim, causal,
+                   stream=None):
+        _check(lib().rm_op_attn_fused(_ptr(qkv), _ptr(ctx), _ptr(offsets_dev), _ptr(rb_dev), n_seqs,
+                                      n_row_blocks, n_heads, head_dim, int(causal), _stream(stream)))
 
     @staticmethod
     def res_ln(y, x, z, g, b, T, H, eps, dtype, mode, stream=None):

@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <memory>
 #include <string>
 #include <utility>
 #include <vector>
@@ -72,6 +73,8 @@ int validate_config(const rm_config* c, bool sched_only, const char** why) {
   if (!(c->ln_eps > 0.0f) || !std::isfinite(c->ln_eps)) return bad("ln_eps must be > 0");
   if (c->max_batch_seqs < 1) return bad("max_batch_seqs must be >= 1");
   if (c->max_tokens < 1 || c->max_tokens > (1 << 24)) return bad("max_tokens must be in 1..2^24");
+  if (c->attn_impl != RM_ATTN_FUSED && c->attn_impl != RM_ATTN_MATERIALIZED)
+    return bad("attn_impl must be 0 or 1");
   return RM_OK;
 }
 
@@ -134,7 +137,7 @@ int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
 struct LayerW {
   bf16 *w_qkv, *w_o, *w_1, *w_2;
   float *b_qkv, *b_o, *ln1_g, *ln1_b, *b_1, *b_2, *ln2_g, *ln2_b;
-  CUtensorMap tm[4][2];   // [qkv, o, 1, 2][box rows 128, 256]
+  CUtensorMap tm[4][kGemmTileCount];   // [qkv, o, 1, 2][box rows of each tile width]
 };
 
 struct Bucket {
@@ -154,6 +157,7 @@ struct rm_handle {
   SchedCost sched;
   int device = 0, num_sms = 148;
   void* wbuf = nullptr;
+  std::shared_ptr<void> weights_owner;   // shared by handles made with rm_create_shared
   bf16 *emb_word = nullptr, *emb_pos = nullptr;
   float *ln_emb_g = nullptr, *ln_emb_b = nullptr, *lnf_g = nullptr, *lnf_b = nullptr,
         *w_r = nullptr;
@@ -291,9 +295,9 @@ int upload_weights(rm_handle* h, const void* weights) {
     const bf16* mats[4] = {L.w_qkv, L.w_o, L.w_1, L.w_2};
     const int64_t rows[4] = {3 * H, H, F, H}, cols[4] = {H, H, H, F};
     for (int m = 0; m < 4; ++m)
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < kGemmTileCount; ++b) {
         const char* why = "";
-        if (!make_tmap_bf16(&L.tm[m][b], mats[m], rows[m], cols[m], b ? 256 : 128, &why))
+        if (!make_tmap_bf16(&L.tm[m][b], mats[m], rows[m], cols[m], kGemmTileWidths[b], &why))
           return set_error(RM_E_CUDA, "weight tensor map: %s", why);
       }
   }
@@ -311,7 +315,7 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
   }
   const rm_config* c = &h->cfg;
   Bucket b;
-  b.plan = plan_arena(c->arch, c->hidden, c->ffn, Tb, Sb);
+  b.plan = plan_arena(c->arch, c->hidden, c->ffn, Tb, c->attn_impl == RM_ATTN_FUSED ? 0 : Sb);
   if (h->fixed_bytes + b.plan.peak > h->arena_bytes)
     return set_error(RM_E_RANGE, "arena plan (%lld bytes) exceeds the reservation",
                      (long long)b.plan.peak);
@@ -328,11 +332,11 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
   return RM_OK;
 }
 
-int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[2], int M, int N, int K,
-         const float* bias, void* y, int act, cudaStream_t st) {
+int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCount], int M, int N,
+         int K, const float* bias, void* y, int act, cudaStream_t st) {
   const int bn = gemm_pick_bn(M, N, h->num_sms);
-  cudaError_t e = gemm_launch(a, b[bn == 256 ? 1 : 0], bn, M, N, K, bias, y, false, act,
-                              h->d_err, st);
+  cudaError_t e = gemm_launch(a, b[gemm_tile_index(bn)], bn, M, N, K, bias, y, false, act,
+                              h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return RM_OK;
 }
@@ -457,6 +461,8 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   const float eps = c->ln_eps;
   const bool prof_on = h->prof_every > 0 && (h->calls % h->prof_every) == 0;
   ++h->calls;
+  // the launch sequence below overlaps each kernel's launch with its predecessor
+  PdlScope pdl(true);
 
   // algorithmic work of each launch (unpadded tokens; attention entries that
   // the mask admits: L*L per head, or L*(L+1)/2 when causal)
@@ -485,12 +491,17 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
     const LayerW& L = h->layers[l];
     RM_GEMM(gemm_flops(3 * Hd, Hd), gemm_bytes(3 * Hd, Hd),
             gemm(h, bk->a_in, L.tm[0], T, 3 * H, H, L.b_qkv, qkv, 0, st));
-    RM_KERNEL(RM_K_SCORES, att_flops, 2.0 * Td * Hd * 2 + 2.0 * att,
-              attn_scores_launch(qkv, s, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
-    RM_KERNEL(RM_K_SOFTMAX, 0, sm_bytes,
-              softmax_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, st));
-    RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
-              attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
+    if (c->attn_impl == RM_ATTN_FUSED) {
+      RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
+                attn_fused_launch(qkv, ctx, d_off, d_rb, n, nrb, nh, d, dec, st));
+    } else {
+      RM_KERNEL(RM_K_SCORES, att_flops, 2.0 * Td * Hd * 2 + 2.0 * att,
+                attn_scores_launch(qkv, s, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
+      RM_KERNEL(RM_K_SOFTMAX, 0, sm_bytes,
+                softmax_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, st));
+      RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
+                attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
+    }
     RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd),
             gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st));
     if (!dec) {
@@ -520,6 +531,36 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   if (host_out != nullptr)
     RM_CUDA(cudaMemcpyAsync(host_out, d_out, 4 * static_cast<size_t>(n), cudaMemcpyDeviceToHost, st));
   h->last_stream = st;
+  return RM_OK;
+}
+
+// Arena, error words, pinned metadata ring and its events of one handle.
+int alloc_runtime(rm_handle* h) {
+  const rm_config* cfg = &h->cfg;
+  const int64_t T = cfg->max_tokens;
+  const int64_t Lp = align_up(cfg->max_len, 8);
+  const int64_t Smax = static_cast<int64_t>(cfg->n_heads) * T * Lp;
+  const MetaLayout ml(cfg->max_batch_seqs);
+  h->meta_bytes = align_up(ml.bytes, 256);
+  h->fixed_bytes = h->meta_bytes + align_up(4 * T, 256) + align_up(4 * cfg->max_batch_seqs, 256);
+  const int64_t Sres =
+      cfg->attn_impl == RM_ATTN_FUSED ? 0 : align_up(std::max<int64_t>(Smax, 1), 65536);
+  h->arena_bytes =
+      h->fixed_bytes + arena_bound(cfg->arch, cfg->hidden, cfg->ffn, align_up(T, 128), Sres);
+  cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
+  if (e == cudaSuccess) e = cudaMalloc(&h->d_err, ERR_WORDS * sizeof(int32_t));
+  if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, ERR_WORDS * sizeof(int32_t));
+  if (e == cudaSuccess)
+    e = cudaHostAlloc(&h->pinned, static_cast<size_t>(kSlots) * h->meta_bytes, cudaHostAllocDefault);
+  for (int k = 0; k < kSlots && e == cudaSuccess; ++k)
+    e = cudaEventCreateWithFlags(&h->ev[k], cudaEventDisableTiming);
+  if (e != cudaSuccess)
+    return set_error(e == cudaErrorMemoryAllocation ? RM_E_NOMEM : RM_E_CUDA, "create: %s",
+                     cudaGetErrorString(e));
+  h->d_meta = h->arena;
+  h->d_ids = reinterpret_cast<int32_t*>(h->arena + h->meta_bytes);
+  h->d_scores = reinterpret_cast<float*>(h->arena + h->meta_bytes + align_up(4 * T, 256));
+  h->planned = h->arena + h->fixed_bytes;
   return RM_OK;
 }
 
@@ -561,33 +602,41 @@ int rm_create(const rm_config* cfg, const void* weights, size_t weights_bytes, r
   h->device = dev;
   h->num_sms = prop.multiProcessorCount;
   int rc = upload_weights(h, weights);
-  if (rc == RM_OK) {
-    const int64_t T = cfg->max_tokens;
-    const int64_t Lp = align_up(cfg->max_len, 8);
-    const int64_t Smax = static_cast<int64_t>(cfg->n_heads) * T * Lp;
-    const MetaLayout ml(cfg->max_batch_seqs);
-    h->meta_bytes = align_up(ml.bytes, 256);
-    h->fixed_bytes = h->meta_bytes + align_up(4 * T, 256) + align_up(4 * cfg->max_batch_seqs, 256);
-    h->arena_bytes = h->fixed_bytes +
-                     arena_bound(cfg->arch, cfg->hidden, cfg->ffn, align_up(T, 128),
-                                 align_up(std::max<int64_t>(Smax, 1), 65536));
-    cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
-    if (e == cudaSuccess) e = cudaMalloc(&h->d_err, ERR_WORDS * sizeof(int32_t));
-    if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, ERR_WORDS * sizeof(int32_t));
-    if (e == cudaSuccess)
-      e = cudaHostAlloc(&h->pinned, static_cast<size_t>(kSlots) * h->meta_bytes, cudaHostAllocDefault);
-    for (int k = 0; k < kSlots && e == cudaSuccess; ++k)
-      e = cudaEventCreateWithFlags(&h->ev[k], cudaEventDisableTiming);
-    if (e != cudaSuccess) {
-      rc = set_error(e == cudaErrorMemoryAllocation ? RM_E_NOMEM : RM_E_CUDA, "create: %s",
-                     cudaGetErrorString(e));
-    } else {
-      h->d_meta = h->arena;
-      h->d_ids = reinterpret_cast<int32_t*>(h->arena + h->meta_bytes);
-      h->d_scores = reinterpret_cast<float*>(h->arena + h->meta_bytes + align_up(4 * T, 256));
-      h->planned = h->arena + h->fixed_bytes;
-    }
+  if (h->wbuf != nullptr) h->weights_owner = std::shared_ptr<void>(h->wbuf, [](void* p) { cudaFree(p); });
+  if (rc == RM_OK) rc = alloc_runtime(h);
+  if (rc != RM_OK) {
+    rm_destroy(h);
+    return rc;
   }
+  *out = h;
+  return RM_OK;
+}
+
+int rm_create_shared(const rm_handle* base, rm_handle** out) {
+  g_msg[0] = '\0';
+  if (base == nullptr || out == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  int dev = 0;
+  RM_CUDA(cudaGetDevice(&dev));
+  if (dev != base->device)
+    return set_error(RM_E_INVAL, "the current device (%d) is not the base handle's (%d)", dev,
+                     base->device);
+  rm_handle* h = new rm_handle();
+  h->cfg = base->cfg;
+  h->sched = base->sched;
+  h->device = base->device;
+  h->num_sms = base->num_sms;
+  h->wbuf = base->wbuf;
+  h->weights_owner = base->weights_owner;
+  h->emb_word = base->emb_word;
+  h->emb_pos = base->emb_pos;
+  h->ln_emb_g = base->ln_emb_g;
+  h->ln_emb_b = base->ln_emb_b;
+  h->lnf_g = base->lnf_g;
+  h->lnf_b = base->lnf_b;
+  h->w_r = base->w_r;
+  h->b_r = base->b_r;
+  h->layers = base->layers;      // tensor maps of the same (shared) weight matrices
+  const int rc = alloc_runtime(h);
   if (rc != RM_OK) {
     rm_destroy(h);
     return rc;
@@ -701,8 +750,8 @@ void rm_destroy(rm_handle* h) {
   if (h->pinned) cudaFreeHost(h->pinned);
   if (h->d_err) cudaFree(h->d_err);
   if (h->arena) cudaFree(h->arena);
-  if (h->wbuf) cudaFree(h->wbuf);
-  delete h;
+  if (h->wbuf && !h->weights_owner) cudaFree(h->wbuf);   // upload failed before ownership
+  delete h;                                                // drops this handle's weight reference
 }
 
 // ---------------------------------------------------------------------------
@@ -723,7 +772,8 @@ int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t
     return set_error(RM_E_INVAL, "need M >= 1 and N, K positive multiples of 8");
   if (act < 0 || act > 2 || (y_dtype != RM_F32 && y_dtype != RM_BF16))
     return set_error(RM_E_INVAL, "bad act or y_dtype");
-  if ((reinterpret_cast<uintptr_t>(y) & 15) != 0) return set_error(RM_E_INVAL, "y must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (reinterpret_cast<uintptr_t>(bias) & 15) != 0)
+    return set_error(RM_E_INVAL, "y and bias must be 16-byte aligned");
   int dev = 0, sms = 148;
   RM_CUDA(cudaGetDevice(&dev));
   RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
@@ -734,7 +784,7 @@ int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t
     return set_error(RM_E_INVAL, "tensor map: %s", why);
   int32_t* err = nullptr;
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
-  RM_LAUNCH(gemm_launch(ta, tb, bn, M, N, K, bias, y, y_dtype == RM_F32, act, err,
+  RM_LAUNCH(gemm_launch(ta, tb, bn, M, N, K, bias, y, y_dtype == RM_F32, act, err, sms,
                         static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
@@ -788,6 +838,18 @@ int rm_op_attn_context(const void* S, const void* qkv, void* ctx, const int32_t*
     return set_error(RM_E_INVAL, "bad sizes");
   RM_LAUNCH(attn_context_launch(S, qkv, ctx, offsets, rb_off, s_off, n_seqs, n_row_blocks, n_heads,
                                 head_dim, causal != 0, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const int32_t* rb_off,
+                     int32_t n_seqs, int32_t n_row_blocks, int32_t n_heads, int32_t head_dim,
+                     int32_t causal, void* stream) {
+  if (qkv == nullptr || ctx == nullptr || offsets == nullptr || rb_off == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || n_row_blocks < 0 || n_heads < 1 || head_dim < 2 || head_dim % 2 || head_dim > 128)
+    return set_error(RM_E_INVAL, "bad sizes");
+  RM_LAUNCH(attn_fused_launch(qkv, ctx, offsets, rb_off, n_seqs, n_row_blocks, n_heads, head_dim,
+                              causal != 0, static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(128)
                        const int64_t* __restrict__ s_off, int n, int H, int d, float scale,
                        int causal) {
   __shared__ __align__(16) bf16 ks[64][DP + 8];
+  pdl_launch_dependents();
+  pdl_wait();
   const BlockSeq q = locate_block(offsets, rb_off, s_off, n, blockIdx.x);
   const int hd = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
@@ -116,6 +118,8 @@ template <typename T, int G, int MAXC>
 __global__ void __launch_bounds__(256)
     softmax_kernel(T* __restrict__ S, const int32_t* __restrict__ offsets,
                    const int64_t* __restrict__ s_off, int n, long long rows, int nh, int causal) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31, sub = lane % G;
   const long long R =
       (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * (32 / G) + lane / G;
@@ -183,6 +187,8 @@ __global__ void __launch_bounds__(128)
                         const int32_t* __restrict__ rb_off, const int64_t* __restrict__ s_off,
                         int n, int H, int d, int causal) {
   __shared__ __align__(16) bf16 vt[DP][64 + 8];   // V block transposed: [dim][key]
+  pdl_launch_dependents();
+  pdl_wait();
   const BlockSeq q = locate_block(offsets, rb_off, s_off, n, blockIdx.x);
   const int hd = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
@@ -250,6 +256,163 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Fused attention: scores, masked online softmax and P.V in one pass, the
+// probabilities never leave registers.  Same work decomposition as above: a
+// CTA per (sequence, 64-query block, head), 4 warps x 16 query rows, keys in
+// blocks of 64 staged in shared memory.  The running row maximum m and sum l
+// are rescaled per key block (the online softmax); P is rounded to bf16 for
+// the P.V tile exactly as the materialised path stores it.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+template <int DP>
+__global__ void __launch_bounds__(128)
+    attn_fused_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ ctx,
+                      const int32_t* __restrict__ offsets, const int32_t* __restrict__ rb_off,
+                      int n, int H, int d, float scale_log2, int causal) {
+  __shared__ __align__(16) bf16 ks[64][DP + 8];
+  __shared__ __align__(16) bf16 vs[64][DP + 8];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.x, hd = blockIdx.y;
+  const int i = upper_index(rb_off, n, b);
+  const int t0 = offsets[i];
+  const int L = offsets[i + 1] - t0;
+  const int row0 = (b - rb_off[i]) * 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const size_t H3 = 3 * static_cast<size_t>(H);
+  const bf16* qb = qkv + static_cast<size_t>(t0) * H3 + hd * d;
+  const bf16* kb_ = qkv + static_cast<size_t>(t0) * H3 + H + hd * d;
+  const bf16* vb = qkv + static_cast<size_t>(t0) * H3 + 2 * H + hd * d;
+  const int ra = row0 + warp * 16 + g, rb = ra + 8;
+
+  auto ld_pair = [&](const bf16* base, int r, int c) -> uint32_t {
+    return (r < L && c < d) ? *reinterpret_cast<const uint32_t*>(base + r * H3 + c) : 0u;
+  };
+  uint32_t qa[DP / 16][4];
+#pragma unroll
+  for (int s = 0; s < DP / 16; ++s) {
+    const int c0 = s * 16 + 2 * tq;
+    qa[s][0] = ld_pair(qb, ra, c0);
+    qa[s][1] = ld_pair(qb, rb, c0);
+    qa[s][2] = ld_pair(qb, ra, c0 + 8);
+    qa[s][3] = ld_pair(qb, rb, c0 + 8);
+  }
+  float o[DP / 8][4];
+#pragma unroll
+  for (int t = 0; t < DP / 8; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+
+  const int row_end = min(L, row0 + 64);
+  const int kend = causal ? row_end : L;
+  const int wrow0 = row0 + warp * 16;
+  const int wrow_last = min(wrow0 + 15, L - 1);
+  const uint32_t vs_base = static_cast<uint32_t>(__cvta_generic_to_shared(&vs[0][0]));
+  for (int kb = 0; kb < kend; kb += 64) {
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < 64 * (DP / 2); idx += 128) {
+      const int r = idx / (DP / 2), cp = (idx % (DP / 2)) * 2;
+      *reinterpret_cast<uint32_t*>(&ks[r][cp]) = ld_pair(kb_, kb + r, cp);
+      *reinterpret_cast<uint32_t*>(&vs[r][cp]) = ld_pair(vb, kb + r, cp);
+    }
+    __syncthreads();
+    if (wrow0 >= L || (causal && kb > wrow_last)) continue;
+    // S = Q K^T for this warp's 16 rows and 64 keys (8 tiles of 8 keys)
+    float sc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int s = 0; s < DP / 16; ++s) {
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&ks[nt * 8 + g][s * 16 + 2 * tq]);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&ks[nt * 8 + g][s * 16 + 8 + 2 * tq]);
+        mma_bf16_16816(sc[nt], qa[s], b0, b1);
+      }
+    }
+    // mask, scale (log2 domain), row maxima over this block
+    const int lim_a = causal ? min(ra + 1, L) : L, lim_b = causal ? min(rb + 1, L) : L;
+    float bm_a = -INFINITY, bm_b = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const int c = kb + nt * 8 + 2 * tq;
+      sc[nt][0] = (c < lim_a) ? sc[nt][0] * scale_log2 : -INFINITY;
+      sc[nt][1] = (c + 1 < lim_a) ? sc[nt][1] * scale_log2 : -INFINITY;
+      sc[nt][2] = (c < lim_b) ? sc[nt][2] * scale_log2 : -INFINITY;
+      sc[nt][3] = (c + 1 < lim_b) ? sc[nt][3] * scale_log2 : -INFINITY;
+      bm_a = fmaxf(bm_a, fmaxf(sc[nt][0], sc[nt][1]));
+      bm_b = fmaxf(bm_b, fmaxf(sc[nt][2], sc[nt][3]));
+    }
+    bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 1));
+    bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 2));
+    bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 1));
+    bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
+    const float mn_a = fmaxf(m_a, bm_a), mn_b = fmaxf(m_b, bm_b);
+    // rows whose keys are all masked so far keep m = -inf; use 0 as the shift then
+    const float sh_a = mn_a == -INFINITY ? 0.f : mn_a, sh_b = mn_b == -INFINITY ? 0.f : mn_b;
+    const float al_a = exp2f(m_a - sh_a), al_b = exp2f(m_b - sh_b);
+    m_a = mn_a;
+    m_b = mn_b;
+    float ps_a = 0.f, ps_b = 0.f;
+    uint32_t pa[4][4];   // P as the A operand of four k=16 steps
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const float p0 = exp2f(sc[nt][0] - sh_a), p1 = exp2f(sc[nt][1] - sh_a);
+      const float p2 = exp2f(sc[nt][2] - sh_b), p3 = exp2f(sc[nt][3] - sh_b);
+      ps_a += p0 + p1;
+      ps_b += p2 + p3;
+      pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+      pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+    }
+    l_a = l_a * al_a + ps_a;
+    l_b = l_b * al_b + ps_b;
+#pragma unroll
+    for (int t = 0; t < DP / 8; ++t) {
+      o[t][0] *= al_a;
+      o[t][1] *= al_a;
+      o[t][2] *= al_b;
+      o[t][3] *= al_b;
+    }
+    // O += P V: B operand (keys x dims) from row-major V via ldmatrix.trans;
+    // one x4 load gives the fragments of two 8-dim tiles for 16 keys
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+      for (int t = 0; t < DP / 8; t += 2) {
+        uint32_t bv[4];
+        const int key = s * 16 + (lane & 15);
+        const int dim = t * 8 + (lane >> 4) * 8;
+        ldmatrix_x4_trans(bv, vs_base + static_cast<uint32_t>((key * (DP + 8) + dim) * 2));
+        mma_bf16_16816(o[t], pa[s], bv[0], bv[1]);
+        mma_bf16_16816(o[t + 1], pa[s], bv[2], bv[3]);
+      }
+    }
+  }
+  if (wrow0 >= L) return;
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+  const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
+  bf16* cb = ctx + static_cast<size_t>(t0) * H + hd * d;
+#pragma unroll
+  for (int t = 0; t < DP / 8; ++t) {
+    const int col = t * 8 + 2 * tq;
+    if (col < d) {
+      if (ra < L)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(ra) * H + col) =
+            pack_bf16x2(o[t][0] * inv_a, o[t][1] * inv_a);
+      if (rb < L)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(rb) * H + col) =
+            pack_bf16x2(o[t][2] * inv_b, o[t][3] * inv_b);
+    }
+  }
+}
+
 int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 : -1)); }
 
 template <typename T, int G, int MAXC>
@@ -257,8 +420,8 @@ cudaError_t softmax_t(void* S, const int32_t* offsets, const int64_t* s_off, int
                       int nh, int causal, cudaStream_t st) {
   const long long rows_per_cta = 8LL * (32 / G);
   const long long blocks = (rows + rows_per_cta - 1) / rows_per_cta;
-  softmax_kernel<T, G, MAXC><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-      static_cast<T*>(S), offsets, s_off, n, rows, nh, causal);
+  launch_k(softmax_kernel<T, G, MAXC>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+           static_cast<T*>(S), offsets, s_off, n, rows, nh, causal);
   return cudaGetLastError();
 }
 
@@ -289,9 +452,9 @@ cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
   const bf16* q = static_cast<const bf16*>(qkv);
   bf16* s = static_cast<bf16*>(S);
   switch (pad_head_dim(head_dim)) {
-    case 32: attn_scores_kernel<32><<<grid, 128, 0, st>>>(q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
-    case 64: attn_scores_kernel<64><<<grid, 128, 0, st>>>(q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
-    case 128: attn_scores_kernel<128><<<grid, 128, 0, st>>>(q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
+    case 32: launch_k(attn_scores_kernel<32>, grid, 128, 0, st, q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
+    case 64: launch_k(attn_scores_kernel<64>, grid, 128, 0, st, q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
+    case 128: launch_k(attn_scores_kernel<128>, grid, 128, 0, st, q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
@@ -307,6 +470,24 @@ cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const i
   return softmax_dispatch<bf16>(S, offsets, s_off, n_seqs, rows, n_heads, max_len, causal, st);
 }
 
+cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                              const int32_t* rb_off, int n_seqs, int n_row_blocks, int n_heads,
+                              int head_dim, int causal, cudaStream_t st) {
+  if (n_row_blocks == 0) return cudaSuccess;
+  const int H = n_heads * head_dim;
+  const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(head_dim));
+  dim3 grid(n_row_blocks, n_heads);
+  const bf16* q = static_cast<const bf16*>(qkv);
+  bf16* c = static_cast<bf16*>(ctx);
+  switch (pad_head_dim(head_dim)) {
+    case 32: launch_k(attn_fused_kernel<32>, grid, 128, 0, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal); break;
+    case 64: launch_k(attn_fused_kernel<64>, grid, 128, 0, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal); break;
+    case 128: launch_k(attn_fused_kernel<128>, grid, 128, 0, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
                                 const int32_t* rb_off, const int64_t* s_off, int n_seqs,
                                 int n_row_blocks, int n_heads, int head_dim, int causal,
@@ -318,9 +499,9 @@ cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const
   const bf16* q = static_cast<const bf16*>(qkv);
   bf16* c = static_cast<bf16*>(ctx);
   switch (pad_head_dim(head_dim)) {
-    case 32: attn_context_kernel<32><<<grid, 128, 0, st>>>(s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
-    case 64: attn_context_kernel<64><<<grid, 128, 0, st>>>(s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
-    case 128: attn_context_kernel<128><<<grid, 128, 0, st>>>(s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
+    case 32: launch_k(attn_context_kernel<32>, grid, 128, 0, st, s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
+    case 64: launch_k(attn_context_kernel<64>, grid, 128, 0, st, s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
+    case 128: launch_k(attn_context_kernel<128>, grid, 128, 0, st, s, q, c, offsets, rb_off, s_off, n_seqs, H, head_dim, causal); break;
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();

@@ -84,8 +84,47 @@ __device__ __forceinline__ float gelu_tanh(float u) {
   return 0.5f * u * (1.0f + tanhf(0.79788456080286536f * (u + 0.044715f * u * u * u)));
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel on its stream finishes;
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible, and pdl_launch_dependents() lets the next kernel start launching.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Device error words (rm_get_device_error): [0] clamped token ids, [1] waits
 // that gave up.
 enum { ERR_CLAMPED = 0, ERR_TIMEOUT = 1, ERR_WORDS = 2 };
+
+}  // namespace rmk
+
+namespace rmk {
+
+// Launches with programmatic stream serialization while a PdlScope is alive
+// on this thread (rm_score's launch sequence); plain stream order otherwise.
+inline thread_local bool g_pdl = false;
+struct PdlScope {
+  bool saved;
+  explicit PdlScope(bool on) : saved(g_pdl) { g_pdl = on; }
+  ~PdlScope() { g_pdl = saved; }
+};
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 }  // namespace rmk

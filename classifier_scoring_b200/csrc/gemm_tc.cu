@@ -3,17 +3,23 @@
 // "BLAS routines" of the TurboTransformers abstract, on tensor cores as its
 // proposed-method section does; here bf16 in, fp32 accumulation).
 //
-// One CTA computes one 128 x BN output tile.  Four warps:
+// Persistent, warp-specialised kernel: one CTA per SM walks the 128 x BN
+// output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... (M fastest, so the
+// CTAs of one wave share a few weight column blocks in L2).  Six warps:
 //   warp 0, one lane : TMA producer -- K-major 128x64 (A) and BNx64 (B) bf16
-//                      boxes, 128-byte swizzle, into a STAGES-deep smem ring;
-//   warp 1, one lane : issues tcgen05.mma (M=128, N=BN, K=16) into a TMEM
-//                      accumulator, and tcgen05.commit to free each stage;
-//   all four warps   : epilogue -- tcgen05.ld 32 columns at a time (warp w
-//                      owns TMEM lanes 32w..32w+31 = tile rows), + bias,
-//                      optional GELU, store bf16 or fp32.
+//                      boxes, 128-byte swizzle, into a STAGES-deep smem ring
+//                      that runs on across tile boundaries;
+//   warp 1, one lane : issues tcgen05.mma (M=128, N=BN, K=16) into one of two
+//                      TMEM accumulators, tcgen05.commit frees each stage and
+//                      marks the accumulator full;
+//   warps 2..5       : epilogue -- tcgen05.ld 32 columns at a time (warp w
+//                      reads TMEM lanes 32*(w%4)..+31 = tile rows), + bias,
+//                      optional GELU, store bf16 or fp32, then release the
+//                      accumulator.  The epilogue of tile i overlaps the
+//                      mainloop of tile i+1.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that
-// gives up counts into err[ERR_TIMEOUT], the CTA skips its stores, frees its
-// TMEM and returns.
+// gives up counts into err[ERR_TIMEOUT] and the role leaves its loop; the CTA
+// then waits (bounded) for its own copies, frees its TMEM and returns.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -24,6 +30,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                      // 64 bf16 = one 128-byte swizzle row
+constexpr int kThreads = 192;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -36,6 +43,9 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
@@ -75,6 +85,11 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
 
 // Shared-memory matrix descriptor of a K-major operand tile written by TMA
 // with the 128-byte swizzle: rows of 128 B, 8-row (1024 B) swizzle atoms.
@@ -103,47 +118,70 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int BN, int STAGES>
+template <int BN>
+constexpr int stages_for() {
+  return BN <= 64 ? 8 : (BN <= 128 ? 6 : (BN <= 192 ? 5 : 4));
+}
+constexpr uint32_t tmem_cols_for(int bn) {
+  // two accumulators of bn fp32 columns, rounded up to a power of two >= 32
+  return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
+}
+
+template <int BN>
 struct GemmSmem {
+  static constexpr int kStages = stages_for<BN>();
   static constexpr int kA = BM * BK * 2;
   static constexpr int kB = BN * BK * 2;
-  static constexpr int kStage = kA + kB;
-  static constexpr int kBarOff = STAGES * kStage;                 // full[S], empty[S], done
-  static constexpr int kSlotOff = kBarOff + (2 * STAGES + 1) * 8;
-  static constexpr int kBiasOff = (kSlotOff + 16 + 15) & ~15;
-  static constexpr int kBytes = kBiasOff + BN * 4 + 1024;          // + alignment slack
+  static constexpr int kStage = kA + kB;     // multiple of 1024 for BN % 8 == 0
+  static constexpr int kBarOff = kStages * kStage;   // full[S], empty[S], accf[2], acce[2]
+  static constexpr int kSlotOff = kBarOff + (2 * kStages + 4) * 8;
+  static constexpr int kBytes = kSlotOff + 16 + 1024;   // + alignment slack
 };
 
-template <int BN, int STAGES, int ACT, bool OUT_F32>
-__global__ void __launch_bounds__(128, 1)
+template <int ACT>
+__device__ __forceinline__ float epilogue_act(float t) {
+  if (ACT == 1) return gelu_erf(t);
+  if (ACT == 2) return gelu_tanh(t);
+  return t;
+}
+
+template <int BN, int ACT, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
                         const float* __restrict__ bias, void* __restrict__ y,
                         int* __restrict__ err) {
-  using L = GemmSmem<BN, STAGES>;
-  constexpr uint32_t kTmemCols = BN;   // BN in {64, 128, 256}: a power of two >= 32
+  using L = GemmSmem<BN>;
+  constexpr int S = L::kStages;
+  constexpr uint32_t kTmemCols = tmem_cols_for(BN);
+  static_assert(L::kStage % 1024 == 0, "stage size keeps the 1024-byte swizzle alignment");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
-  float* sbias = reinterpret_cast<float*>(smem + L::kBiasOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM;
+  const int tiles_m = (M + BM - 1) / BM;
+  const int tiles = tiles_m * ((N + BN - 1) / BN);
   const int nk = (K + BK - 1) / BK;
-  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + STAGES),
-                 done = smem_u32(bars + 2 * STAGES);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S),
+                 accf0 = smem_u32(bars + 2 * S), acce0 = smem_u32(bars + 2 * S + 2);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(done, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf0 + 8 * a, 1);
+      mbar_init(acce0 + 8 * a, 4);   // one arrival per epilogue warp
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -154,105 +192,136 @@ __global__ void __launch_bounds__(128, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  for (int c = threadIdx.x; c < BN; c += blockDim.x)
-    sbias[c] = (bias != nullptr && n0 + c < N) ? bias[n0 + c] : 0.0f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // the prologue above overlaps the previous kernel; global memory waits for it
+  pdl_launch_dependents();
+  pdl_wait();
 
-  if (warp == 0 && lane == 0) {
-    // ---- TMA producer ----
-    int issued = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (kb >= STAGES && !mbar_wait(empty0 + 8 * s, ph ^ 1)) {
-        atomicAdd(err + ERR_TIMEOUT, 1);
-        break;
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer ----
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+        const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (it >= S && !mbar_wait(empty0 + 8 * s, ph ^ 1)) {
+            atomicAdd(err + ERR_TIMEOUT, 1);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full0 + 8 * s, L::kStage);
+          tma_load_2d(smem_u32(smem + s * L::kStage), &tmA, kb * BK, m0, full0 + 8 * s);
+          tma_load_2d(smem_u32(smem + s * L::kStage + L::kA), &tmB, kb * BK, n0, full0 + 8 * s);
+        }
       }
-      mbar_arrive_expect_tx(full0 + 8 * s, L::kStage);
-      tma_load_2d(smem_u32(smem + s * L::kStage), &tmA, kb * BK, m0, full0 + 8 * s);
-      tma_load_2d(smem_u32(smem + s * L::kStage + L::kA), &tmB, kb * BK, n0, full0 + 8 * s);
-      ++issued;
+      // copies in flight land before this CTA's shared memory is released
+      for (int j = it - 1; j >= 0 && j >= it - S; --j) mbar_wait(full0 + 8 * (j % S), (j / S) & 1);
     }
-    // Copies still in flight land before this CTA's shared memory is released:
-    // wait (bounded) for the last min(issued, STAGES) stages to fill.
-    for (int kb = issued - 1; kb >= 0 && kb >= issued - STAGES; --kb)
-      mbar_wait(full0 + 8 * (kb % STAGES), (kb / STAGES) & 1);
-  } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ----
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (kb / STAGES) & 1;
-      if (!mbar_wait(full0 + 8 * s, ph)) {
-        atomicAdd(err + ERR_TIMEOUT, 1);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1, use = local >> 1;
+        if (use > 0 && !mbar_wait(acce0 + 8 * acc, (use - 1) & 1)) {
+          atomicAdd(err + ERR_TIMEOUT, 1);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc) * (kTmemCols / 2);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (it / S) & 1;
+          if (!mbar_wait(full0 + 8 * s, ph)) {
+            atomicAdd(err + ERR_TIMEOUT, 1);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc_k_sw128(smem_u32(smem + s * L::kStage));
+          const uint64_t bd = smem_desc_k_sw128(smem_u32(smem + s * L::kStage + L::kA));
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // advance 16 elements = 32 bytes along K inside the swizzle atom
+            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+                "l"(ad + 2ull * k), "l"(bd + 2ull * k), "r"(idesc), "r"(accum)
+                : "memory");
+          }
+          tc_commit(empty0 + 8 * s);   // frees the stage once these MMAs are done
+        }
+        tc_commit(accf0 + 8 * acc);    // the accumulator is complete
+      }
+    }
+  } else {
+    // ---- epilogue: TMEM -> registers -> bias/GELU -> global ----
+    const int q = warp & 3;                      // TMEM lane quarter of this warp
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    int local = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+      const int acc = local & 1, use = local >> 1;
+      const bool ready = mbar_wait(accf0 + 8 * acc, use & 1);
+      if (!__all_sync(0xffffffffu, ready)) {
+        if (lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
         break;
       }
       tc_fence_after();
-      const uint64_t ad = smem_desc_k_sw128(smem_u32(smem + s * L::kStage));
-      const uint64_t bd = smem_desc_k_sw128(smem_u32(smem + s * L::kStage + L::kA));
-#pragma unroll
-      for (int k = 0; k < BK / 16; ++k) {
-        // advance 16 elements = 32 bytes along K inside the swizzle atom
-        const uint32_t acc = (kb > 0 || k > 0) ? 1u : 0u;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "setp.ne.b32 p, %4, 0;\n\t"
-            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem),
-            "l"(ad + 2ull * k), "l"(bd + 2ull * k), "r"(idesc), "r"(acc)
-            : "memory");
-      }
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              empty0 + 8 * s)
-          : "memory");
-    }
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(done)
-        : "memory");
-  }
-  __syncwarp();
-
-  // ---- epilogue: TMEM -> registers -> bias/GELU -> global ----
-  const bool ready = mbar_wait(done, 0);
-  tc_fence_after();
-  if (!ready && lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
-  const int row = m0 + warp * 32 + lane;
-  if (__all_sync(0xffffffffu, ready)) {
+      const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+      const int row = m0 + q * 32 + lane;
+      const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld_32cols(tmem + (static_cast<uint32_t>(warp * 32) << 16) + c, r);
-      if (row < M && n0 + c < N) {
-        float v[32];
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld_32cols(base + c, r);
+        tmem_wait_ld();
+        if (row < M && n0 + c < N) {
+          float v[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float t = __uint_as_float(r[j]) + sbias[c + j];
-          if (ACT == 1) t = gelu_erf(t);
-          if (ACT == 2) t = gelu_tanh(t);
-          v[j] = t;
-        }
+          for (int g = 0; g < 8; ++g) {
+            const int col = n0 + c + 4 * g;
+            float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (bias != nullptr && col < N) b4 = __ldg(reinterpret_cast<const float4*>(bias + col));
+            v[4 * g + 0] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 0]) + b4.x);
+            v[4 * g + 1] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 1]) + b4.y);
+            v[4 * g + 2] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 2]) + b4.z);
+            v[4 * g + 3] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 3]) + b4.w);
+          }
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int col = n0 + c + 8 * g;
-          if (col < N) {
-            if (OUT_F32) {
-              float* dst = static_cast<float*>(y) + static_cast<size_t>(row) * N + col;
-              Chunk8<float>::store(dst, v + 8 * g);
-            } else {
-              bf16* dst = static_cast<bf16*>(y) + static_cast<size_t>(row) * N + col;
-              Chunk8<bf16>::store(dst, v + 8 * g);
+          for (int g = 0; g < 4; ++g) {
+            const int col = n0 + c + 8 * g;
+            if (col < N) {
+              if (OUT_F32) {
+                Chunk8<float>::store(static_cast<float*>(y) + static_cast<size_t>(row) * N + col,
+                                     v + 8 * g);
+              } else {
+                Chunk8<bf16>::store(static_cast<bf16*>(y) + static_cast<size_t>(row) * N + col,
+                                    v + 8 * g);
+              }
             }
           }
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce0 + 8 * acc);   // accumulator free for tile local+2
     }
   }
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
+    tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(kTmemCols)
                  : "memory");
@@ -262,47 +331,53 @@ __global__ void __launch_bounds__(128, 1)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int BN, int STAGES, int ACT, bool OUT_F32>
+template <int BN, int ACT, bool OUT_F32>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
-                       const float* bias, void* y, int* err, cudaStream_t st) {
-  using L = GemmSmem<BN, STAGES>;
-  auto kern = gemm_bf16_tc_kernel<BN, STAGES, ACT, OUT_F32>;
-  static bool configured = false;   // per instantiation; attribute is per device function
+                       const float* bias, void* y, int* err, int num_sms, cudaStream_t st) {
+  using L = GemmSmem<BN>;
+  auto kern = gemm_bf16_tc_kernel<BN, ACT, OUT_F32>;
+  static bool configured = false;   // the attribute is per function; one device per process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM);
-  kern<<<grid, 128, L::kBytes, st>>>(a, b, M, N, K, bias, y, err);
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  launch_k(kern, dim3(grid), dim3(kThreads), L::kBytes, st, a, b, M, N, K, bias, y, err);
   return cudaGetLastError();
 }
 
-template <int BN, int STAGES>
+template <int BN>
 cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
-                       const float* bias, void* y, bool out_f32, int act, int* err,
+                       const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
                        cudaStream_t st) {
   if (out_f32) {
-    if (act == 1) return launch_one<BN, STAGES, 1, true>(a, b, M, N, K, bias, y, err, st);
-    if (act == 2) return launch_one<BN, STAGES, 2, true>(a, b, M, N, K, bias, y, err, st);
-    return launch_one<BN, STAGES, 0, true>(a, b, M, N, K, bias, y, err, st);
+    if (act == 1) return launch_one<BN, 1, true>(a, b, M, N, K, bias, y, err, num_sms, st);
+    if (act == 2) return launch_one<BN, 2, true>(a, b, M, N, K, bias, y, err, num_sms, st);
+    return launch_one<BN, 0, true>(a, b, M, N, K, bias, y, err, num_sms, st);
   }
-  if (act == 1) return launch_one<BN, STAGES, 1, false>(a, b, M, N, K, bias, y, err, st);
-  if (act == 2) return launch_one<BN, STAGES, 2, false>(a, b, M, N, K, bias, y, err, st);
-  return launch_one<BN, STAGES, 0, false>(a, b, M, N, K, bias, y, err, st);
+  if (act == 1) return launch_one<BN, 1, false>(a, b, M, N, K, bias, y, err, num_sms, st);
+  if (act == 2) return launch_one<BN, 2, false>(a, b, M, N, K, bias, y, err, num_sms, st);
+  return launch_one<BN, 0, false>(a, b, M, N, K, bias, y, err, num_sms, st);
 }
 
 }  // namespace
 
+const int kGemmTileWidths[kGemmTileCount] = {64, 128, 192, 256};
+
 int gemm_pick_bn(int M, int N, int num_sms) {
-  // Fewest waves first, then the larger tile (less B re-read, longer mainloop).
-  const int tm = (M + BM - 1) / BM;
+  // Makespan of the persistent grid: rounds of tiles times the tile's width
+  // (mainloop time grows with BN), plus a fixed cost per tile (pipeline fill,
+  // epilogue tail) worth about 48 columns.  Ties go to the wider tile.
+  const long long tm = (M + BM - 1) / BM;
   int best = 256;
   long long best_cost = -1;
-  for (int bn : {256, 128}) {
-    const long long tiles = static_cast<long long>(tm) * ((N + bn - 1) / bn);
-    const long long waves = (tiles + num_sms - 1) / num_sms;
-    const long long cost = waves * (bn + 64);   // per-tile time ~ bn, plus fixed overhead
+  for (int i = kGemmTileCount - 1; i >= 0; --i) {
+    const int bn = kGemmTileWidths[i];
+    const long long tiles = tm * ((N + bn - 1) / bn);
+    const long long rounds = (tiles + num_sms - 1) / num_sms;
+    const long long cost = rounds * (bn + 48);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = bn;
@@ -312,10 +387,15 @@ int gemm_pick_bn(int M, int N, int num_sms) {
 }
 
 cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int M, int N, int K,
-                        const float* bias, void* y, bool out_f32, int act, int* err,
+                        const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
                         cudaStream_t st) {
-  if (bn == 256) return launch_act<256, 4>(a, b, M, N, K, bias, y, out_f32, act, err, st);
-  return launch_act<128, 6>(a, b, M, N, K, bias, y, out_f32, act, err, st);
+  switch (bn) {
+    case 64: return launch_act<64>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 128: return launch_act<128>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 192: return launch_act<192>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 256: return launch_act<256>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace rmk

@@ -8,11 +8,15 @@
 namespace rmk {
 
 // ---- tcgen05 GEMM (gemm_tc.cu) ----
-// Column-tile width for an M x N problem on num_sms SMs (256 or 128).
+constexpr int kGemmTileCount = 4;
+extern const int kGemmTileWidths[kGemmTileCount];   // 64, 128, 192, 256
+// Column-tile width for an M x N problem on num_sms SMs (one of kGemmTileWidths).
 int gemm_pick_bn(int M, int N, int num_sms);
+inline int gemm_tile_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : bn == 192 ? 2 : 3; }
 // a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, bn}.
+// Persistent grid of min(tiles, num_sms) CTAs.
 cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int M, int N, int K,
-                        const float* bias, void* y, bool out_f32, int act, int* err,
+                        const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
                         cudaStream_t st);
 
 // ---- TMA descriptors (tma.cpp) ----
@@ -45,6 +49,10 @@ cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
 cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const int64_t* s_off,
                            int n_seqs, int T, int n_heads, int max_len, int causal,
                            cudaStream_t st);
+// scores + masked softmax + context in one kernel (probabilities stay in registers)
+cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                              const int32_t* rb_off, int n_seqs, int n_row_blocks, int n_heads,
+                              int head_dim, int causal, cudaStream_t st);
 cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
                                 const int32_t* rb_off, const int64_t* s_off, int n_seqs,
                                 int n_row_blocks, int n_heads, int head_dim, int causal,

@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                  int T, const bf16* __restrict__ ew, const bf16* __restrict__ ep,
                  const float* __restrict__ g, const float* __restrict__ b, float eps, int V, int H,
                  bf16* __restrict__ x, int32_t* __restrict__ err) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     res_ln_kernel(const T* __restrict__ y, T* __restrict__ x, T* __restrict__ z,
                   const float* __restrict__ g, const float* __restrict__ b, int rows, int H,
                   float eps) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int r = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
@@ -155,6 +159,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 __global__ void __launch_bounds__(kWarps * 32)
     head_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ offsets, int n,
                 const float* __restrict__ w, float br, int H, int last, float* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int i = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (i >= n) return;
@@ -199,11 +205,11 @@ cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, co
                     void* x, int32_t* err, cudaStream_t st) {
   dim3 grid((T + kWarps - 1) / kWarps);
   if (g != nullptr)
-    embed_kernel<MAXC, true><<<grid, kWarps * 32, 0, st>>>(
+    launch_k(embed_kernel<MAXC, true>, grid, kWarps * 32, 0, st, 
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
         V, H, static_cast<bf16*>(x), err);
   else
-    embed_kernel<MAXC, false><<<grid, kWarps * 32, 0, st>>>(
+    launch_k(embed_kernel<MAXC, false>, grid, kWarps * 32, 0, st, 
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
         V, H, static_cast<bf16*>(x), err);
   return cudaGetLastError();
@@ -217,11 +223,11 @@ cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const floa
   T* xx = static_cast<T*>(x);
   T* zz = static_cast<T*>(z);
   if (mode == 0)
-    res_ln_kernel<T, MAXC, 0><<<grid, kWarps * 32, 0, st>>>(yy, xx, zz, g, b, rows, H, eps);
+    launch_k(res_ln_kernel<T, MAXC, 0>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps);
   else if (mode == 1)
-    res_ln_kernel<T, MAXC, 1><<<grid, kWarps * 32, 0, st>>>(yy, xx, zz, g, b, rows, H, eps);
+    launch_k(res_ln_kernel<T, MAXC, 1>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps);
   else
-    res_ln_kernel<T, MAXC, 2><<<grid, kWarps * 32, 0, st>>>(yy, xx, zz, g, b, rows, H, eps);
+    launch_k(res_ln_kernel<T, MAXC, 2>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps);
   return cudaGetLastError();
 }
 
@@ -265,7 +271,7 @@ cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const
                         float b_r, int H, int last_token, float* out, cudaStream_t st) {
   if (n_seqs == 0) return cudaSuccess;
   dim3 grid((n_seqs + kWarps - 1) / kWarps);
-  head_kernel<<<grid, kWarps * 32, 0, st>>>(static_cast<const bf16*>(x), offsets, n_seqs, w_r,
+  launch_k(head_kernel, grid, kWarps * 32, 0, st, static_cast<const bf16*>(x), offsets, n_seqs, w_r,
                                             b_r, H, last_token, out);
   return cudaGetLastError();
 }
@@ -275,10 +281,10 @@ cudaError_t cvt_to_bf16_launch(const void* src, int src_dtype, void* dst, size_t
   if (n == 0) return cudaSuccess;
   const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 16));
   if (src_dtype == 0)
-    cvt_bf16_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(src),
+    launch_k(cvt_bf16_kernel<float>, blocks, 256, 0, st, static_cast<const float*>(src),
                                                    static_cast<bf16*>(dst), n);
   else
-    cvt_bf16_kernel<bf16><<<blocks, 256, 0, st>>>(static_cast<const bf16*>(src),
+    launch_k(cvt_bf16_kernel<bf16>, blocks, 256, 0, st, static_cast<const bf16*>(src),
                                                   static_cast<bf16*>(dst), n);
   return cudaGetLastError();
 }
@@ -288,9 +294,9 @@ cudaError_t cvt_to_f32_launch(const void* src, int src_dtype, float* dst, size_t
   if (n == 0) return cudaSuccess;
   const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, 148 * 16));
   if (src_dtype == 0)
-    cvt_f32_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(src), dst, n);
+    launch_k(cvt_f32_kernel<float>, blocks, 256, 0, st, static_cast<const float*>(src), dst, n);
   else
-    cvt_f32_kernel<bf16><<<blocks, 256, 0, st>>>(static_cast<const bf16*>(src), dst, n);
+    launch_k(cvt_f32_kernel<bf16>, blocks, 256, 0, st, static_cast<const bf16*>(src), dst, n);
   return cudaGetLastError();
 }
 

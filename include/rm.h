@@ -58,6 +58,14 @@ extern "C" {
 #define RM_GELU_ERF  0   /* u * Phi(u)                                              */
 #define RM_GELU_TANH 1   /* 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3)))         */
 
+/* rm_config.attn_impl: how the attention step runs inside rm_score.
+ * FUSED: scores, masked softmax and P.V in one kernel (rm_op_attn_fused);
+ * the probabilities stay in registers.  MATERIALIZED: the three kernels
+ * rm_op_attn_scores -> rm_op_softmax -> rm_op_attn_context with the score
+ * matrix in HBM.  Both compute the same values up to rounding order. */
+#define RM_ATTN_FUSED        0
+#define RM_ATTN_MATERIALIZED 1
+
 typedef struct rm_handle rm_handle;
 
 typedef struct rm_config {
@@ -81,6 +89,7 @@ typedef struct rm_config {
   const int64_t* sched_table;    /* optional host table T[b-1][L-1], row-major,       */
   int32_t sched_table_b;         /*   sched_table_b >= Bmax rows, sched_table_l >=    */
   int32_t sched_table_l;         /*   max_len columns, non-decreasing along L; copied */
+  int32_t attn_impl;             /* RM_ATTN_FUSED (default) | RM_ATTN_MATERIALIZED    */
 } rm_config;
 
 /* Number of bytes the flat weights buffer must hold for cfg.
@@ -101,6 +110,14 @@ size_t rm_weights_bytes(const rm_config* cfg);
  * Errors: RM_E_INVAL (cfg/size), RM_E_DEVICE (no sm_100 device), RM_E_NOMEM,
  * RM_E_CUDA.  *out is set only on success. */
 int rm_create(const rm_config* cfg, const void* weights, size_t weights_bytes, rm_handle** out);
+
+/* A second handle on the same device that shares base's device weights
+ * (no copy) but has its own arena, metadata staging and error words, so that
+ * two streams can each keep a batch in flight.  The weights stay alive until
+ * the last handle that shares them is destroyed; base may be destroyed first.
+ * Errors: RM_E_INVAL (NULL, or the current device is not base's), RM_E_NOMEM,
+ * RM_E_CUDA. */
+int rm_create_shared(const rm_handle* base, rm_handle** out);
 
 /* Score n_seqs packed sequences.
  *   packed_token_ids: device int32[T], T = seq_offsets[n_seqs]; sequence i is
@@ -155,7 +172,8 @@ int rm_arena_stats(const rm_handle* h, int64_t* out);
 #define RM_K_LAYERNORM 4   /* residual + LayerNorm                                   */
 #define RM_K_EMBED     5   /* embedding gather (+ LN)                                */
 #define RM_K_HEAD      6   /* scalar head                                            */
-#define RM_K_CLASSES   7
+#define RM_K_ATTN_FUSED 7  /* fused attention (scores + softmax + context)           */
+#define RM_K_CLASSES   8
 
 /* Opt-in kernel timing.  every >= 1: each every-th rm_score* call from now on
  * records CUDA events around each of its kernel launches on its stream

@@ -80,6 +80,14 @@ int rm_op_attn_context(const void* S, const void* qkv, void* ctx, const int32_t*
                        int32_t n_row_blocks, int32_t n_heads, int32_t head_dim, int32_t causal,
                        void* stream);
 
+/* The three attention steps above in one kernel: per sequence, head and
+ * 64-query block, S = QK^T/sqrt(d) over keys c < L_i (causal: c <= r) with an
+ * online (running max and sum) softmax, P rounded to bf16, C = P V written to
+ * ctx[T][H].  No score buffer.  qkv: bf16 [T][3H]; ctx: bf16 [T][H]. */
+int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const int32_t* rb_off,
+                     int32_t n_seqs, int32_t n_row_blocks, int32_t n_heads, int32_t head_dim,
+                     int32_t causal, void* stream);
+
 /* Residual + LayerNorm over rows of length H (the LayerNorm batch reduction of
  * the TurboTransformers abstract), fp32 math, rows of dtype (RM_BF16|RM_F32):
  *   mode 0 (post-LN): x = LN(y + x)              (z unused, may be NULL)

@@ -280,3 +280,35 @@ def test_head(last):
     rows = X[off[1:] - 1] if last else X[off[:-1]]
     ref = rows @ w.astype(np.float64) + 0.25
     assert np.all(np.abs(f64(out) - ref) <= F32_RTOL * (np.abs(rows) @ np.abs(w) + 0.25))
+
+
+@pytest.mark.parametrize("lens", [[1, 65, 130, 64, 9], [300, 7, 560], [100] * 8],
+                         ids=["ragged", "long", "uniform"])
+@pytest.mark.parametrize("nh,d", [(2, 64), (12, 26), (12, 64), (16, 128)])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_attention_fused(lens, nh, d, causal):
+    H = nh * d
+    lens = np.array(lens)
+    off = synth.offsets_from_lengths(lens)
+    rb, so = rm.ops.varlen_meta(off, nh)
+    rng = np.random.default_rng(nh * d + causal + len(lens))
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    X = f64(qkv)
+    ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rm.ops.attn_fused(qkv, ctx, dev(off, torch.int32), dev(rb, torch.int32), len(lens),
+                      int(rb[-1]), nh, d, causal)
+    torch.cuda.synchronize()
+    C = f64(ctx)
+    for i, L in enumerate(lens):
+        rows = X[off[i]:off[i + 1]]
+        for j in range(nh):
+            q = rows[:, j * d:(j + 1) * d]
+            k = rows[:, H + j * d:H + (j + 1) * d]
+            v = rows[:, 2 * H + j * d:2 * H + (j + 1) * d]
+            p = O.attention_probs(q, k, bool(causal))
+            ref = p @ v
+            # one bf16 rounding of the output and of every probability
+            tol = BF16_REL * np.abs(ref) + 2 * BF16_REL * (p @ np.abs(v)) + F32_RTOL
+            got = C[off[i]:off[i + 1], j * d:(j + 1) * d]
+            assert np.all(np.abs(got - ref) <= tol), float((np.abs(got - ref) / tol).max())

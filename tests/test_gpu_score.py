@@ -66,11 +66,13 @@ def oracle_scores(name, ids, off, sample):
     return np.array([O.score_one(m, ids[off[i]:off[i + 1]]) for i in sample])
 
 
-def test_tiny_encoder_all_sequences_match_golden_and_oracle():
+@pytest.mark.parametrize("attn", [rm.ATTN_FUSED, rm.ATTN_MATERIALIZED], ids=["fused", "materialized"])
+def test_tiny_encoder_all_sequences_match_golden_and_oracle(attn):
     w = synth.WORKLOADS["tiny-enc"]
     st = synth.make_stream(w)
     ids, off = synth.pack(st, np.arange(len(st.lengths)))
-    got = gpu_scores(scorer("tiny-enc", max_batch_seqs=8, max_tokens=256, max_len=64), ids, off)
+    got = gpu_scores(scorer("tiny-enc", max_batch_seqs=8, max_tokens=256, max_len=64,
+                            attn_impl=attn), ids, off)
     ref = oracle_scores("tiny-enc", ids, off, range(len(off) - 1))
     gold = np.loadtxt(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "tiny_enc_scores.txt"))
     assert np.max(np.abs(ref - gold)) <= 1e-12
@@ -94,17 +96,18 @@ def _dp_batches(name, n_req):
     return st, batch
 
 
-@pytest.mark.parametrize("name,n_req,which,n_sample", [
-    ("bert-base-len2-100", 2000, "last", 8), ("bert-base-len2-100", 2000, "first", 8),
-    ("bert-base-len5-500", 400, "last", 3)])
-def test_bert_base_dp_batch_sampled(name, n_req, which, n_sample):
+@pytest.mark.parametrize("name,n_req,which,n_sample,attn", [
+    ("bert-base-len2-100", 2000, "last", 8, 0), ("bert-base-len2-100", 2000, "first", 8, 0),
+    ("bert-base-len2-100", 2000, "last", 4, 1),
+    ("bert-base-len5-500", 400, "last", 3, 0), ("bert-base-len5-500", 400, "last", 2, 1)])
+def test_bert_base_dp_batch_sampled(name, n_req, which, n_sample, attn):
     w = synth.WORKLOADS[name]
     st, batch = _dp_batches(name, n_req)
     b = int(batch.max()) if which == "last" else 0
     idx = np.nonzero(batch == b)[0]
     ids, off = synth.pack(st, idx)
     sc = scorer(name, max_batch_seqs=w.max_batch, max_tokens=w.max_batch * w.len_hi,
-                max_len=512)
+                max_len=512, attn_impl=attn)
     got = gpu_scores(sc, ids, off)
     sample = np.linspace(0, len(idx) - 1, n_sample).astype(int)
     ref = oracle_scores(name, ids, off, sample)
@@ -112,24 +115,26 @@ def test_bert_base_dp_batch_sampled(name, n_req, which, n_sample):
     assert np.max(np.abs(got[sample] - ref)) <= SCORE_ATOL
 
 
-def test_bert_base_mixed_lengths_every_sequence():
+@pytest.mark.parametrize("attn", [rm.ATTN_FUSED, rm.ATTN_MATERIALIZED], ids=["fused", "materialized"])
+def test_bert_base_mixed_lengths_every_sequence(attn):
     """A ragged batch of every length class, all sequences checked."""
     name = "bert-base-len2-100"
     lens = np.array([1, 2, 3, 7, 8, 9, 63, 64, 65, 100, 127, 128, 129, 200, 511, 512])
     off = synth.offsets_from_lengths(lens)
     ids = synth.make_token_ids(int(off[-1]), 30522, 77)
-    sc = scorer(name, max_batch_seqs=64, max_tokens=6400, max_len=512)
+    sc = scorer(name, max_batch_seqs=64, max_tokens=6400, max_len=512, attn_impl=attn)
     got = gpu_scores(sc, ids, off)
     ref = oracle_scores(name, ids, off, range(len(lens)))
     assert np.max(np.abs(got - ref)) <= SCORE_ATOL
 
 
-def test_decoder_small_shape_every_sequence():
+@pytest.mark.parametrize("attn", [rm.ATTN_FUSED, rm.ATTN_MATERIALIZED], ids=["fused", "materialized"])
+def test_decoder_small_shape_every_sequence(attn):
     """The pre-LN causal path on a small decoder (fast oracle), all sequences."""
     shape = synth.ModelShape(synth.DEC_PRELN, 3, 256, 4, 1024, 5000, 600, synth.W_BF16,
                              synth.GELU_ERF, 1e-5)
     flat = synth.make_weights(shape, 9)
-    cfg = config_for(shape, max_batch_seqs=16, max_tokens=4096, max_len=600)
+    cfg = config_for(shape, max_batch_seqs=16, max_tokens=4096, max_len=600, attn_impl=attn)
     lens = np.array([1, 2, 65, 256, 300, 560, 17])
     off = synth.offsets_from_lengths(lens)
     ids = synth.make_token_ids(int(off[-1]), shape.vocab, 10)
@@ -235,3 +240,32 @@ def test_handle_schedule_matches_oracle():
     lengths = synth.make_stream(w).lengths
     ref, _ = OS.schedule_dp(lengths, 64, OS.linear_cost(0, 1))
     assert np.array_equal(sc.schedule(lengths), ref)
+
+
+def test_shared_handles_on_two_streams_match_one_handle():
+    name = "bert-base-len2-100"
+    w = synth.WORKLOADS[name]
+    st, batch = _dp_batches(name, 800)
+    base = rm.Scorer(config_for(w.shape, max_batch_seqs=64, max_tokens=6400, max_len=512),
+                     weights(name))
+    other = base.shared()
+    batches = [np.nonzero(batch == b)[0] for b in range(int(batch.max()) + 1)]
+    packed = [synth.pack(st, idx) for idx in batches]
+    ref = [gpu_scores(base, ids, off) for ids, off in packed]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    handles = [base, other]
+    outs = []
+    ids_d = [torch.from_numpy(ids).cuda() for ids, _ in packed]
+    torch.cuda.synchronize()
+    for k, (ids, off) in enumerate(packed):
+        o = torch.full((len(off) - 1,), float("nan"), dtype=torch.float32, device="cuda")
+        handles[k % 2].score(ids_d[k], off, o, streams[k % 2])
+        outs.append(o)
+    torch.cuda.synchronize()
+    for o, r in zip(outs, ref):
+        assert np.array_equal(o.cpu().numpy().astype(np.float64), r)
+    # the weights outlive the handle that uploaded them
+    base.close()
+    ids, off = packed[0]
+    assert np.array_equal(gpu_scores(other, ids, off), ref[0])
+    other.close()
