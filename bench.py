@@ -57,6 +57,27 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 GEMM_TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
 
 
+def replica_workload(w, rank: int):
+    """The workload a replica scores: the same model, its own seeded request stream."""
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def reduce_times(vals, dist, device):
+    """Max over ranks of per-rank timings (ms); plain values when single-process."""
+    vals = np.asarray(vals, dtype=np.float64)
+    if dist is None:
+        return vals
+    import torch
+    t = torch.tensor(vals, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().numpy()
+
+
+def whole_job_rate(world: int, per_rank_units: int, steps: int, max_ms: float) -> float:
+    """Units processed by all ranks per second of the slowest rank."""
+    return world * per_rank_units * steps / (max_ms / 1000.0)
+
+
 def rank_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
@@ -235,8 +256,7 @@ def b200_arm(args):
     w = synth.WORKLOADS[name]
     s = w.shape
     flat = synth.make_weights(s, w.seed)
-    wr = dataclasses.replace(w, seed=w.seed + 1000 * rank)       # each replica its own requests
-    st = synth.make_stream(wr)
+    st = synth.make_stream(replica_workload(w, rank))            # each replica its own requests
     n_req = len(st.lengths)
     max_len = min(s.max_pos, 1024, max(w.len_hi, int(st.lengths.max())))
     cfg = rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
@@ -404,16 +424,10 @@ def b200_arm(args):
     d2h = 4 * n_req
 
     # ---- reduce over ranks ----
-    vals = np.array([elapsed_ms, e_ms], dtype=np.float64)
-    if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor(vals, device="cuda")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        vals = t.cpu().numpy()
+    vals = reduce_times([elapsed_ms, e_ms], dist, "cuda")
     max_ms, max_e_ms = float(vals[0]), float(vals[1])
-    total_seqs = world * n_req * args.steps
-    value = total_seqs / (max_ms / 1000.0)
-    e2e_value = world * n_req * e_steps / (max_e_ms / 1000.0)
+    value = whole_job_rate(world, n_req, args.steps, max_ms)
+    e2e_value = whole_job_rate(world, n_req, e_steps, max_e_ms)
 
     pk, pk_kind = peaks()
     g = prof["gemm"]

@@ -113,69 +113,102 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-// Masked softmax: G lanes per row, MAXC 8-element chunks per lane, 8 warps per CTA.
-template <typename T, int G, int MAXC>
+// Masked softmax.  A group of G lanes owns U consecutive rows; each lane
+// holds MAXC 8-element chunks of each of them in registers.  All U*MAXC loads
+// of a lane are issued before the first reduction, so short rows still keep
+// enough bytes in flight to cover HBM latency.  The group finds the sequence
+// of its first row by binary search over the offsets and walks forward from
+// there (consecutive rows belong to the same sequence or the next ones).
+template <typename T, int G, int MAXC, int U>
 __global__ void __launch_bounds__(256)
     softmax_kernel(T* __restrict__ S, const int32_t* __restrict__ offsets,
                    const int64_t* __restrict__ s_off, int n, long long rows, int nh, int causal) {
   pdl_launch_dependents();
   pdl_wait();
   const int lane = threadIdx.x & 31, sub = lane % G;
-  const long long R =
-      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * (32 / G) + lane / G;
-  const bool valid = R < rows;
-  int len = 0;
-  T* row = S;
-  if (valid) {
-    int lo = 0, hi = n - 1;   // largest i with nh * offsets[i] <= R
+  const long long R0 =
+      ((static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * (32 / G) + lane / G) * U;
+  int len[U];
+  T* row[U];
+  if (R0 < rows) {
+    int lo = 0, hi = n - 1;   // largest i with nh * offsets[i] <= R0
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (static_cast<long long>(nh) * offsets[mid] <= R) lo = mid; else hi = mid - 1;
+      if (static_cast<long long>(nh) * offsets[mid] <= R0) lo = mid; else hi = mid - 1;
     }
-    const int L = offsets[lo + 1] - offsets[lo];
-    const int Lp = (L + 7) & ~7;
-    const long long rr = R - static_cast<long long>(nh) * offsets[lo];
-    const int r = static_cast<int>(rr % L);
-    len = causal ? r + 1 : L;
-    row = S + s_off[lo] + rr * Lp;
-  }
-  float v[MAXC][8];
-  float m = -INFINITY;
+    int i = lo;
+    long long seq_row0 = static_cast<long long>(nh) * offsets[i];
+    long long seq_row1 = static_cast<long long>(nh) * offsets[i + 1];
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int col = (c * G + sub) * 8;
-    if (col < len) {
-      Chunk8<T>::load(row + col, v[c]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (col + e >= len) v[c][e] = -INFINITY;
-        m = fmaxf(m, v[c][e]);
+    for (int u = 0; u < U; ++u) {
+      const long long R = R0 + u;
+      len[u] = 0;
+      row[u] = S;
+      if (R < rows) {
+        while (R >= seq_row1) {
+          ++i;
+          seq_row0 = seq_row1;
+          seq_row1 = static_cast<long long>(nh) * offsets[i + 1];
+        }
+        const int L = offsets[i + 1] - offsets[i];
+        const long long rr = R - seq_row0;
+        len[u] = causal ? static_cast<int>(rr % L) + 1 : L;
+        row[u] = S + s_off[i] + rr * ((L + 7) & ~7);
       }
     }
-  }
-  m = group_max<G>(m);
-  float s = 0.f;
+  } else {
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int col = (c * G + sub) * 8;
-    if (col < len) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float p = (col + e < len) ? __expf(v[c][e] - m) : 0.f;
-        v[c][e] = p;
-        s += p;
-      }
+    for (int u = 0; u < U; ++u) {
+      len[u] = 0;
+      row[u] = S;
     }
   }
-  s = group_sum<G>(s);
-  const float inv = 1.0f / s;
+  float v[U][MAXC][8];
 #pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int col = (c * G + sub) * 8;
-    if (col < len) {
+  for (int u = 0; u < U; ++u)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[c][e] *= inv;
-      Chunk8<T>::store(row + col, v[c]);
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) Chunk8<T>::load(row[u] + col, v[u][c]);
+    }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (col + e >= len[u]) v[u][c][e] = -INFINITY;
+          m = fmaxf(m, v[u][c][e]);
+        }
+      }
+    }
+    m = group_max<G>(m);
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float p = (col + e < len[u]) ? __expf(v[u][c][e] - m) : 0.f;
+          v[u][c][e] = p;
+          sum += p;
+        }
+      }
+    }
+    sum = group_sum<G>(sum);
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[u][c][e] *= inv;
+        Chunk8<T>::store(row[u] + col, v[u][c]);
+      }
     }
   }
 }
@@ -415,27 +448,30 @@ __global__ void __launch_bounds__(128)
 
 int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 : -1)); }
 
-template <typename T, int G, int MAXC>
+template <typename T, int G, int MAXC, int U>
 cudaError_t softmax_t(void* S, const int32_t* offsets, const int64_t* s_off, int n, long long rows,
                       int nh, int causal, cudaStream_t st) {
-  const long long rows_per_cta = 8LL * (32 / G);
+  const long long rows_per_cta = 8LL * (32 / G) * U;
   const long long blocks = (rows + rows_per_cta - 1) / rows_per_cta;
-  launch_k(softmax_kernel<T, G, MAXC>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+  launch_k(softmax_kernel<T, G, MAXC, U>, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
            static_cast<T*>(S), offsets, s_off, n, rows, nh, causal);
   return cudaGetLastError();
 }
 
+// Lanes per row G = the smallest power of two covering the longest row's
+// 8-element chunks (at most 32), and U rows per lane group so that a lane has
+// four chunks in flight.
 template <typename T>
 cudaError_t softmax_dispatch(void* S, const int32_t* offsets, const int64_t* s_off, int n,
                              long long rows, int nh, int max_len, int causal, cudaStream_t st) {
   const int chunks = ((max_len + 7) & ~7) / 8;
-  if (chunks <= 4) return softmax_t<T, 4, 1>(S, offsets, s_off, n, rows, nh, causal, st);
-  if (chunks <= 8) return softmax_t<T, 8, 1>(S, offsets, s_off, n, rows, nh, causal, st);
-  if (chunks <= 16) return softmax_t<T, 16, 1>(S, offsets, s_off, n, rows, nh, causal, st);
-  if (chunks <= 32) return softmax_t<T, 32, 1>(S, offsets, s_off, n, rows, nh, causal, st);
-  if (chunks <= 64) return softmax_t<T, 32, 2>(S, offsets, s_off, n, rows, nh, causal, st);
-  if (chunks <= 96) return softmax_t<T, 32, 3>(S, offsets, s_off, n, rows, nh, causal, st);
-  if (chunks <= 128) return softmax_t<T, 32, 4>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 4) return softmax_t<T, 4, 1, 4>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 8) return softmax_t<T, 8, 1, 4>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 16) return softmax_t<T, 16, 1, 4>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 32) return softmax_t<T, 32, 1, 4>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 64) return softmax_t<T, 32, 2, 2>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 96) return softmax_t<T, 32, 3, 1>(S, offsets, s_off, n, rows, nh, causal, st);
+  if (chunks <= 128) return softmax_t<T, 32, 4, 1>(S, offsets, s_off, n, rows, nh, causal, st);
   return cudaErrorInvalidValue;
 }
 

@@ -30,6 +30,7 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                      // 64 bf16 = one 128-byte swizzle row
+
 constexpr int kThreads = 192;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -138,14 +139,20 @@ struct GemmSmem {
   static constexpr int kA = BM * BK * 2;
   static constexpr int kB = BN * BK * 2;
   static constexpr int kStage = kA + kB;     // multiple of 1024 for BN % 8 == 0
-  static constexpr int kBarOff = kStages * kStage;   // full[S], empty[S], accf[2], acce[2]
+  // epilogue staging: per epilogue warp 32 rows x 128 B of output (64 bf16 or
+  // 32 fp32 columns), row pitch padded by 16 B so that both the row-wise
+  // writes and the line-wise reads touch every bank group evenly
+  static constexpr int kStagePitch = 128 + 16;
+  static constexpr int kStageWarpBytes = 32 * kStagePitch;
+  static constexpr int kEpiOff = kStages * kStage;
+  static constexpr int kBarOff = kEpiOff + 4 * kStageWarpBytes;   // full[S], empty[S], accf[2], acce[2]
   static constexpr int kSlotOff = kBarOff + (2 * kStages + 4) * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;   // + alignment slack
 };
 
 template <int ACT>
 __device__ __forceinline__ float epilogue_act(float t) {
-  if (ACT == 1) return gelu_erf(t);
+  if (ACT == 1) return gelu_erf_fast(t);
   if (ACT == 2) return gelu_tanh(t);
   return t;
 }
@@ -265,9 +272,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ---- epilogue: TMEM -> registers -> bias/GELU -> global ----
+    // ---- epilogue: TMEM -> registers -> bias/GELU -> smem staging -> global ----
+    // Each thread owns one tile row (its TMEM lane).  A round takes 128 B of
+    // that row (64 bf16 / 32 fp32 columns), writes it to the warp's staging
+    // rows, then the warp stores 4 full 128-byte row segments per instruction.
+    constexpr int ESZ = OUT_F32 ? 4 : 2;
+    constexpr int CPR = 128 / ESZ;               // columns per round
     const int q = warp & 3;                      // TMEM lane quarter of this warp
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    uint8_t* stg = smem + L::kEpiOff + (warp - 2) * L::kStageWarpBytes;
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int acc = local & 1, use = local >> 1;
@@ -278,37 +291,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
-      const int row = m0 + q * 32 + lane;
+      const int row0 = m0 + q * 32;
       const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld_32cols(base + c, r);
-        tmem_wait_ld();
-        if (row < M && n0 + c < N) {
-          float v[32];
+      for (int c = 0; c < BN; c += CPR) {
+        if (n0 + c >= N) break;                  // uniform across the warp
+        float v[CPR];
+        {
+          uint32_t r[32];
 #pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const int col = n0 + c + 4 * g;
-            float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (bias != nullptr && col < N) b4 = __ldg(reinterpret_cast<const float4*>(bias + col));
-            v[4 * g + 0] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 0]) + b4.x);
-            v[4 * g + 1] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 1]) + b4.y);
-            v[4 * g + 2] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 2]) + b4.z);
-            v[4 * g + 3] = epilogue_act<ACT>(__uint_as_float(r[4 * g + 3]) + b4.w);
+          for (int h = 0; h < CPR / 32; ++h) {
+            tmem_ld_32cols(base + c + 32 * h, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[32 * h + j] = __uint_as_float(r[j]);
           }
+        }
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = n0 + c + 8 * g;
-            if (col < N) {
-              if (OUT_F32) {
-                Chunk8<float>::store(static_cast<float*>(y) + static_cast<size_t>(row) * N + col,
-                                     v + 8 * g);
-              } else {
-                Chunk8<bf16>::store(static_cast<bf16*>(y) + static_cast<size_t>(row) * N + col,
-                                    v + 8 * g);
-              }
-            }
+        for (int g = 0; g < CPR / 4; ++g) {
+          const int col = n0 + c + 4 * g;
+          float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (bias != nullptr && col < N) b4 = __ldg(reinterpret_cast<const float4*>(bias + col));
+          v[4 * g + 0] = epilogue_act<ACT>(v[4 * g + 0] + b4.x);
+          v[4 * g + 1] = epilogue_act<ACT>(v[4 * g + 1] + b4.y);
+          v[4 * g + 2] = epilogue_act<ACT>(v[4 * g + 2] + b4.z);
+          v[4 * g + 3] = epilogue_act<ACT>(v[4 * g + 3] + b4.w);
+        }
+        __syncwarp();                            // the previous round's reads are done
+        uint8_t* my_row = stg + lane * L::kStagePitch;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint4 u;
+          if (OUT_F32) {
+            u = make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                           __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+          } else {
+            u = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                           pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+          }
+          *reinterpret_cast<uint4*>(my_row + 16 * j) = u;
+        }
+        __syncwarp();
+        const int ch = lane & 7;                 // 16-byte chunk of a 128-byte segment
+        const int gcol = n0 + c + ch * (16 / ESZ);
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int rr = it * 4 + (lane >> 3);
+          const int grow = row0 + rr;
+          if (grow < M && gcol < N) {
+            const uint4 u = *reinterpret_cast<const uint4*>(stg + rr * L::kStagePitch + ch * 16);
+            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(y) +
+                                      (static_cast<size_t>(grow) * N + gcol) * ESZ) = u;
           }
         }
       }
@@ -367,6 +400,9 @@ cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
 const int kGemmTileWidths[kGemmTileCount] = {64, 128, 192, 256};
 
 int gemm_pick_bn(int M, int N, int num_sms) {
+#ifdef RM_GEMM_FORCE_BN
+  return RM_GEMM_FORCE_BN;
+#endif
   // Makespan of the persistent grid: rounds of tiles times the tile's width
   // (mainloop time grows with BN), plus a fixed cost per tile (pipeline fill,
   // epilogue tail) worth about 48 columns.  Ties go to the wider tile.

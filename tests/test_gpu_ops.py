@@ -312,3 +312,21 @@ def test_attention_fused(lens, nh, d, causal):
             tol = BF16_REL * np.abs(ref) + 2 * BF16_REL * (p @ np.abs(v)) + F32_RTOL
             got = C[off[i]:off[i + 1], j * d:(j + 1) * d]
             assert np.all(np.abs(got - ref) <= tol), float((np.abs(got - ref) / tol).max())
+
+
+def test_gemm_gelu_epilogue_against_cuda_erf_and_oracle():
+    """GELU of the epilogue (Abramowitz & Stegun 7.1.26 erf) on a dense grid of
+    pre-activations: x = 0, W = 0, so y = GELU(bias)."""
+    N = 8192
+    u = torch.linspace(-12, 12, N, dtype=torch.float32)
+    x = torch.zeros(16, 64, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(N, 64, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(16, N, dtype=torch.float32, device="cuda")
+    rm.ops.gemm(x, w, u.cuda(), y, rm.F32, 16, N, 64, 1)
+    torch.cuda.synchronize()
+    got = f64(y[0])
+    cuda_erff = torch.nn.functional.gelu(u.cuda()).double().cpu().numpy()   # CUDA's erff
+    ref = O.gelu(u.double().numpy())
+    assert np.max(np.abs(got - ref)) <= 2e-6
+    assert np.max(np.abs(got - cuda_erff)) <= 2e-6
+    assert np.all(f64(y) == got[None, :])
