@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
         "rm_op_softmax": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attn_context": (ctypes.c_int, [P, P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attn_fused": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
+        "rm_op_attention_noalloc": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, P]),
         "rm_op_res_ln": (ctypes.c_int, [P, P, P, P, P, I32, I32, F, I32, I32, P]),
         "rm_op_head": (ctypes.c_int, [P, P, I32, P, F, I32, I32, P, P]),
         "rm_arena_plan": (ctypes.c_int, [cfgp, I32, I32, I64, P, P, P, P, I32, P]),
@@ -278,6 +279,13 @@ class ops:
                    stream=None):
         _check(lib().rm_op_attn_fused(_ptr(qkv), _ptr(ctx), _ptr(offsets_dev), _ptr(rb_dev), n_seqs,
                                       n_row_blocks, n_heads, head_dim, int(causal), _stream(stream)))
+
+    @staticmethod
+    def attention_noalloc(qkv, ctx, offsets, n_heads, head_dim, causal, stream=None):
+        """rm_op_attention_noalloc: host offsets; scratch in the library's static array."""
+        off = _i32(offsets)
+        _check(lib().rm_op_attention_noalloc(_ptr(qkv), _ptr(ctx), off.ctypes.data, len(off) - 1,
+                                             n_heads, head_dim, int(causal), _stream(stream)))
 
     @staticmethod
     def res_ln(y, x, z, g, b, T, H, eps, dtype, mode, stream=None):

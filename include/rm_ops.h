@@ -88,6 +88,28 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
                      int32_t n_seqs, int32_t n_row_blocks, int32_t n_heads, int32_t head_dim,
                      int32_t causal, void* stream);
 
+/* The materialised attention step (rm_op_attn_scores -> rm_op_softmax ->
+ * rm_op_attn_context) without any device allocation: the score matrix and the
+ * per-call metadata live in one file-scope device array of 8 MiB + 64 KiB that
+ * every device loading this library keeps until the process exits.  The pages
+ * have no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory where they run the step (a plugin inside another
+ * runtime that owns the device memory pool, or a path where cudaMalloc is not
+ * allowed because it may synchronize the device or fail under pressure).
+ *   qkv: bf16 [T][3H]; ctx: bf16 [T][H] (written); offsets: HOST int32[n+1].
+ * Limits: n_seqs <= 4096, every L_i <= 1024 and sum_i n_heads*L_i*round_up(L_i,8)
+ * <= 4 Mi score entries; larger calls return RM_E_RANGE (use the three
+ * caller-allocated entry points instead).  The first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture.  The call copies its metadata into the
+ * array on stream and calls no cudaMalloc or cudaFree.  Every call shares the
+ * array and it keeps the last call's contents (nothing in it needs to start at
+ * zero: each call writes every entry it reads), so calls that overlap on the
+ * GPU -- on different streams, or from different threads without ordering --
+ * race and give wrong results. */
+int rm_op_attention_noalloc(const void* qkv, void* ctx, const int32_t* offsets, int32_t n_seqs,
+                            int32_t n_heads, int32_t head_dim, int32_t causal, void* stream);
+
 /* Residual + LayerNorm over rows of length H (the LayerNorm batch reduction of
  * the TurboTransformers abstract), fp32 math, rows of dtype (RM_BF16|RM_F32):
  *   mode 0 (post-LN): x = LN(y + x)              (z unused, may be NULL)
