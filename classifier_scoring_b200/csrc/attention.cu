@@ -446,7 +446,220 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// 16-byte asynchronous copy global -> shared; src_size 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* gptr, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(gptr),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// The same fused attention for head dims that are a multiple of 8: Q, K and V
+// tiles arrive by 16-byte cp.async (zero-filled outside the sequence), Q, K0
+// and V0 all in flight at once, and K/V are double-buffered so the next key
+// block loads while the current one is multiplied.  Q fragments come from
+// shared memory through ldmatrix.
+template <int DP>
+struct FusedSmem {
+  static constexpr int kPitch = DP + 8;          // elements; 16-byte aligned rows
+  static constexpr int kTile = 64 * kPitch;      // elements per 64-row tile
+  static constexpr int kBytes = 5 * kTile * 2;   // Q, K x2, V x2
+};
+
+template <int DP>
+__global__ void __launch_bounds__(128)
+    attn_fused_async_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ ctx,
+                            const int32_t* __restrict__ offsets, const int32_t* __restrict__ rb_off,
+                            int n, int H, int d, float scale_log2, int causal) {
+  using FS = FusedSmem<DP>;
+  constexpr int P = FS::kPitch;
+  extern __shared__ __align__(16) uint8_t fsm_raw[];
+  bf16* qs = reinterpret_cast<bf16*>(fsm_raw);
+  bf16* kbuf = qs + FS::kTile;
+  bf16* vbuf = kbuf + 2 * FS::kTile;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int b = blockIdx.x, hd = blockIdx.y;
+  const int i = upper_index(rb_off, n, b);
+  const int t0 = offsets[i];
+  const int L = offsets[i + 1] - t0;
+  const int row0 = (b - rb_off[i]) * 64;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+  const size_t H3 = 3 * static_cast<size_t>(H);
+  const bf16* qb = qkv + static_cast<size_t>(t0) * H3 + hd * d;
+  const bf16* kb_ = qkv + static_cast<size_t>(t0) * H3 + H + hd * d;
+  const bf16* vb = qkv + static_cast<size_t>(t0) * H3 + 2 * H + hd * d;
+  const int ra = row0 + warp * 16 + g, rb = ra + 8;
+  const int row_end = min(L, row0 + 64);
+  const int kend = causal ? row_end : L;
+  const int nkb = (kend + 63) / 64;
+  const int wrow0 = row0 + warp * 16;
+  const int wrow_last = min(wrow0 + 15, L - 1);
+
+  auto issue = [&](bf16* dst, const bf16* src, int rbase) {
+#pragma unroll
+    for (int k = 0; k < (64 * (DP / 8)) / 128; ++k) {
+      const int idx = threadIdx.x + k * 128;
+      const int r = idx / (DP / 8), c = (idx % (DP / 8)) * 8;
+      const bool ok = (rbase + r < L) && (c < d);
+      const bf16* gsrc = ok ? src + static_cast<size_t>(rbase + r) * H3 + c : src;
+      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * P + c)), gsrc, ok);
+    }
+  };
+  issue(qs, qb, row0);
+  issue(kbuf, kb_, 0);
+  issue(vbuf, vb, 0);
+  cp_async_commit();                                   // group 0: Q, K0, V0
+  if (nkb > 1) {
+    issue(kbuf + FS::kTile, kb_, 64);
+    issue(vbuf + FS::kTile, vb, 64);
+  }
+  cp_async_commit();                                   // group 1: K1, V1 (may be empty)
+  cp_async_wait_1();
+  __syncthreads();
+
+  uint32_t qa[DP / 16][4];
+  {
+    const uint32_t qs_base = static_cast<uint32_t>(__cvta_generic_to_shared(qs));
+#pragma unroll
+    for (int s = 0; s < DP / 16; ++s) {
+      const int r = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int c = s * 16 + (lane >> 4) * 8;
+      ldmatrix_x4(qa[s], qs_base + static_cast<uint32_t>((r * P + c) * 2));
+    }
+  }
+  float o[DP / 8][4];
+#pragma unroll
+  for (int t = 0; t < DP / 8; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+
+  for (int j = 0; j < nkb; ++j) {
+    const int kb = j * 64;
+    const int buf = j & 1;
+    if (j > 0) {
+      cp_async_wait_1();                               // group j (K_j, V_j) has landed
+      __syncthreads();
+    }
+    const bf16* ks = kbuf + buf * FS::kTile;
+    const uint32_t vs_base = static_cast<uint32_t>(__cvta_generic_to_shared(vbuf + buf * FS::kTile));
+    if (!(wrow0 >= L || (causal && kb > wrow_last))) {
+      float sc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+        for (int s = 0; s < DP / 16; ++s) {
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(ks + (nt * 8 + g) * P + s * 16 + 2 * tq);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(ks + (nt * 8 + g) * P + s * 16 + 8 + 2 * tq);
+          mma_bf16_16816(sc[nt], qa[s], b0, b1);
+        }
+      }
+      const int lim_a = causal ? min(ra + 1, L) : L, lim_b = causal ? min(rb + 1, L) : L;
+      float bm_a = -INFINITY, bm_b = -INFINITY;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const int c = kb + nt * 8 + 2 * tq;
+        sc[nt][0] = (c < lim_a) ? sc[nt][0] * scale_log2 : -INFINITY;
+        sc[nt][1] = (c + 1 < lim_a) ? sc[nt][1] * scale_log2 : -INFINITY;
+        sc[nt][2] = (c < lim_b) ? sc[nt][2] * scale_log2 : -INFINITY;
+        sc[nt][3] = (c + 1 < lim_b) ? sc[nt][3] * scale_log2 : -INFINITY;
+        bm_a = fmaxf(bm_a, fmaxf(sc[nt][0], sc[nt][1]));
+        bm_b = fmaxf(bm_b, fmaxf(sc[nt][2], sc[nt][3]));
+      }
+      bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 1));
+      bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 2));
+      bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 1));
+      bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
+      const float mn_a = fmaxf(m_a, bm_a), mn_b = fmaxf(m_b, bm_b);
+      const float sh_a = mn_a == -INFINITY ? 0.f : mn_a, sh_b = mn_b == -INFINITY ? 0.f : mn_b;
+      const float al_a = exp2f(m_a - sh_a), al_b = exp2f(m_b - sh_b);
+      m_a = mn_a;
+      m_b = mn_b;
+      float ps_a = 0.f, ps_b = 0.f;
+      uint32_t pa[4][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        const float p0 = exp2f(sc[nt][0] - sh_a), p1 = exp2f(sc[nt][1] - sh_a);
+        const float p2 = exp2f(sc[nt][2] - sh_b), p3 = exp2f(sc[nt][3] - sh_b);
+        ps_a += p0 + p1;
+        ps_b += p2 + p3;
+        pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+        pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+      }
+      l_a = l_a * al_a + ps_a;
+      l_b = l_b * al_b + ps_b;
+#pragma unroll
+      for (int t = 0; t < DP / 8; ++t) {
+        o[t][0] *= al_a;
+        o[t][1] *= al_a;
+        o[t][2] *= al_b;
+        o[t][3] *= al_b;
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+#pragma unroll
+        for (int t = 0; t < DP / 8; t += 2) {
+          uint32_t bv[4];
+          const int key = s * 16 + (lane & 15);
+          const int dim = t * 8 + (lane >> 4) * 8;
+          ldmatrix_x4_trans(bv, vs_base + static_cast<uint32_t>((key * P + dim) * 2));
+          mma_bf16_16816(o[t], pa[s], bv[0], bv[1]);
+          mma_bf16_16816(o[t + 1], pa[s], bv[2], bv[3]);
+        }
+      }
+    }
+    __syncthreads();                                   // every warp is done with buffer buf
+    if (j + 2 < nkb) {
+      issue(kbuf + buf * FS::kTile, kb_, kb + 128);
+      issue(vbuf + buf * FS::kTile, vb, kb + 128);
+    }
+    cp_async_commit();                                 // group j+2 (may be empty)
+  }
+  if (wrow0 >= L) return;
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+  const float inv_a = 1.0f / l_a, inv_b = 1.0f / l_b;
+  bf16* cb = ctx + static_cast<size_t>(t0) * H + hd * d;
+#pragma unroll
+  for (int t = 0; t < DP / 8; ++t) {
+    const int col = t * 8 + 2 * tq;
+    if (col < d) {
+      if (ra < L)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(ra) * H + col) =
+            pack_bf16x2(o[t][0] * inv_a, o[t][1] * inv_a);
+      if (rb < L)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(rb) * H + col) =
+            pack_bf16x2(o[t][2] * inv_b, o[t][3] * inv_b);
+    }
+  }
+}
+
 int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 : -1)); }
+
+template <int DP>
+cudaError_t launch_fused_async(dim3 grid, cudaStream_t st, const bf16* q, bf16* c,
+                               const int32_t* offsets, const int32_t* rb_off, int n, int H, int d,
+                               float scale_log2, int causal) {
+  static bool configured = false;   // the attribute is per function; one device per process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fused_async_kernel<DP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         FusedSmem<DP>::kBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  launch_k(attn_fused_async_kernel<DP>, grid, dim3(128), FusedSmem<DP>::kBytes, st, q, c, offsets,
+           rb_off, n, H, d, scale_log2, causal);
+  return cudaGetLastError();
+}
 
 template <typename T, int G, int MAXC, int U>
 cudaError_t softmax_t(void* S, const int32_t* offsets, const int64_t* s_off, int n, long long rows,
@@ -515,6 +728,14 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
   dim3 grid(n_row_blocks, n_heads);
   const bf16* q = static_cast<const bf16*>(qkv);
   bf16* c = static_cast<bf16*>(ctx);
+  if (head_dim % 8 == 0) {
+    switch (pad_head_dim(head_dim)) {
+      case 32: return launch_fused_async<32>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal);
+      case 64: return launch_fused_async<64>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal);
+      case 128: return launch_fused_async<128>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (pad_head_dim(head_dim)) {
     case 32: launch_k(attn_fused_kernel<32>, grid, 128, 0, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal); break;
     case 64: launch_k(attn_fused_kernel<64>, grid, 128, 0, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal); break;
