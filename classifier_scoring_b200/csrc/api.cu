@@ -479,26 +479,46 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   const double sm_bytes = 4.0 * att;                 // bf16 read + write per admitted entry
   const double ctx_bytes = 2.0 * att + 2.0 * Td * Hd * 2;   // P, V, ctx
 
+  // weights of the next GEMMs to pull into L2 during the latency-bound kernels
+  // before them (skipped when they would crowd out the activations)
+  const unsigned long long pf_cap = 32ull << 20;
+  auto pf_of = [&](const void* a, unsigned long long na, const void* b, unsigned long long nb) {
+    L2Prefetch p;
+    if (na + nb > pf_cap) return p;
+    p.ptr[0] = a;
+    p.bytes[0] = na;
+    p.ptr[1] = b;
+    p.bytes[1] = nb;
+    return p;
+  };
+  const unsigned long long w_qkv_b = 2ull * 3 * H * H, w_o_b = 2ull * H * H, w_1_b = 2ull * F * H,
+                           w_2_b = 2ull * H * F;
+  const L2Prefetch pf_qkv0 = pf_of(h->layers[0].w_qkv, w_qkv_b, nullptr, 0);
   RM_KERNEL(RM_K_EMBED, 0, 6.0 * Td * Hd + 4.0 * Td,
             embed_launch(d_ids, d_off, n, T, h->emb_word, h->emb_pos, dec ? nullptr : h->ln_emb_g,
                          dec ? nullptr : h->ln_emb_b, eps, c->vocab, c->max_pos, H, x,
-                         h->d_err + ERR_CLAMPED, st));
+                         h->d_err + ERR_CLAMPED, st, dec ? L2Prefetch{} : pf_qkv0));
   if (dec)
     RM_KERNEL(RM_K_LAYERNORM, 0, 4.0 * Td * Hd,
-              res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps, 1, 2, st));
+              res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps, 1, 2, st,
+                            pf_qkv0));
   const double ln_bytes = (dec ? 8.0 : 6.0) * Td * Hd;
   for (int l = 0; l < c->n_layers; ++l) {
     const LayerW& L = h->layers[l];
+    const L2Prefetch pf_o = pf_of(L.w_o, w_o_b, nullptr, 0);
+    const L2Prefetch pf_ffn = pf_of(L.w_1, w_1_b, L.w_2, w_2_b);
+    const L2Prefetch pf_next =
+        l + 1 < c->n_layers ? pf_of(h->layers[l + 1].w_qkv, w_qkv_b, nullptr, 0) : L2Prefetch{};
     RM_GEMM(gemm_flops(3 * Hd, Hd), gemm_bytes(3 * Hd, Hd),
             gemm(h, bk->a_in, L.tm[0], T, 3 * H, H, L.b_qkv, qkv, 0, st));
     if (c->attn_impl == RM_ATTN_FUSED) {
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
-                attn_fused_launch(qkv, ctx, d_off, d_rb, n, nrb, nh, d, dec, st));
+                attn_fused_launch(qkv, ctx, d_off, d_rb, n, nrb, nh, d, dec, st, pf_o));
     } else {
       RM_KERNEL(RM_K_SCORES, att_flops, 2.0 * Td * Hd * 2 + 2.0 * att,
                 attn_scores_launch(qkv, s, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
       RM_KERNEL(RM_K_SOFTMAX, 0, sm_bytes,
-                softmax_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, st));
+                softmax_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, h->d_err, st));
       RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
                 attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
     }
@@ -506,16 +526,16 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
             gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st));
     if (!dec) {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, 1, 0, st));
+                res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, 1, 0, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
               gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
       RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
               gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st));
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, 1, 0, st));
+                res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, 1, 0, st, pf_next));
     } else {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, 1, 1, st));
+                res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, 1, 1, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
               gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
       RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
@@ -523,7 +543,7 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
       const bool last = l + 1 == c->n_layers;
       const float* g = last ? h->lnf_g : h->layers[l + 1].ln1_g;
       const float* b = last ? h->lnf_b : h->layers[l + 1].ln1_b;
-      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes, res_ln_launch(y2, x, z, g, b, T, H, eps, 1, 1, st));
+      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes, res_ln_launch(y2, x, z, g, b, T, H, eps, 1, 1, st, pf_next));
     }
   }
   RM_KERNEL(RM_K_HEAD, 2.0 * n * Hd, 2.0 * n * Hd + 4.0 * n,
@@ -823,7 +843,7 @@ int rm_op_softmax(void* S, int32_t s_dtype, const int32_t* offsets, const int64_
       (s_dtype != RM_F32 && s_dtype != RM_BF16))
     return set_error(RM_E_INVAL, "bad sizes");
   RM_LAUNCH(softmax_launch(S, s_dtype, offsets, s_off, n_seqs, T, n_heads, max_len, causal != 0,
-                           static_cast<cudaStream_t>(stream)));
+                           nullptr, static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

@@ -476,7 +476,7 @@ template <int DP>
 __global__ void __launch_bounds__(128)
     attn_fused_async_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ ctx,
                             const int32_t* __restrict__ offsets, const int32_t* __restrict__ rb_off,
-                            int n, int H, int d, float scale_log2, int causal) {
+                            int n, int H, int d, float scale_log2, int causal, L2PrefetchArgs pf) {
   using FS = FusedSmem<DP>;
   constexpr int P = FS::kPitch;
   extern __shared__ __align__(16) uint8_t fsm_raw[];
@@ -484,6 +484,7 @@ __global__ void __launch_bounds__(128)
   bf16* kbuf = qs + FS::kTile;
   bf16* vbuf = kbuf + 2 * FS::kTile;
   pdl_launch_dependents();
+  l2_prefetch_share(pf);
   pdl_wait();
   const int b = blockIdx.x, hd = blockIdx.y;
   const int i = upper_index(rb_off, n, b);
@@ -647,7 +648,12 @@ int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 
 template <int DP>
 cudaError_t launch_fused_async(dim3 grid, cudaStream_t st, const bf16* q, bf16* c,
                                const int32_t* offsets, const int32_t* rb_off, int n, int H, int d,
-                               float scale_log2, int causal) {
+                               float scale_log2, int causal, const L2Prefetch& pf) {
+  L2PrefetchArgs pa;
+  for (int k = 0; k < 2; ++k) {
+    pa.ptr[k] = pf.ptr[k];
+    pa.bytes[k] = pf.bytes[k];
+  }
   static bool configured = false;   // the attribute is per function; one device per process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_fused_async_kernel<DP>,
@@ -657,7 +663,7 @@ cudaError_t launch_fused_async(dim3 grid, cudaStream_t st, const bf16* q, bf16* 
     configured = true;
   }
   launch_k(attn_fused_async_kernel<DP>, grid, dim3(128), FusedSmem<DP>::kBytes, st, q, c, offsets,
-           rb_off, n, H, d, scale_log2, causal);
+           rb_off, n, H, d, scale_log2, causal, pa);
   return cudaGetLastError();
 }
 
@@ -710,10 +716,11 @@ cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
 }
 
 cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const int64_t* s_off,
-                           int n_seqs, int T, int n_heads, int max_len, int causal,
+                           int n_seqs, int T, int n_heads, int max_len, int causal, int* err,
                            cudaStream_t st) {
   const long long rows = static_cast<long long>(n_heads) * T;
   if (rows == 0) return cudaSuccess;
+  (void)err;   // the row kernel has no waits that could give up
   if (s_dtype == 0)
     return softmax_dispatch<float>(S, offsets, s_off, n_seqs, rows, n_heads, max_len, causal, st);
   return softmax_dispatch<bf16>(S, offsets, s_off, n_seqs, rows, n_heads, max_len, causal, st);
@@ -721,7 +728,7 @@ cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const i
 
 cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets,
                               const int32_t* rb_off, int n_seqs, int n_row_blocks, int n_heads,
-                              int head_dim, int causal, cudaStream_t st) {
+                              int head_dim, int causal, cudaStream_t st, const L2Prefetch& pf) {
   if (n_row_blocks == 0) return cudaSuccess;
   const int H = n_heads * head_dim;
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(head_dim));
@@ -730,9 +737,9 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
   bf16* c = static_cast<bf16*>(ctx);
   if (head_dim % 8 == 0) {
     switch (pad_head_dim(head_dim)) {
-      case 32: return launch_fused_async<32>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal);
-      case 64: return launch_fused_async<64>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal);
-      case 128: return launch_fused_async<128>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal);
+      case 32: return launch_fused_async<32>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
+      case 64: return launch_fused_async<64>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
+      case 128: return launch_fused_async<128>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
       default: return cudaErrorInvalidValue;
     }
   }

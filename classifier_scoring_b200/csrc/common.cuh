@@ -112,6 +112,31 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// This CTA's share of up to two byte ranges, pulled into L2 with bulk
+// prefetches (16-byte granules; no shared memory, no completion to wait for).
+struct L2PrefetchArgs {
+  const void* ptr[2];
+  unsigned long long bytes[2];
+};
+__device__ __forceinline__ void l2_prefetch_share(const L2PrefetchArgs& pf) {
+  if (threadIdx.x != 0) return;
+  for (int k = 0; k < 2; ++k) {
+    if (pf.ptr[k] == nullptr || pf.bytes[k] == 0) continue;
+    const unsigned long long granules = pf.bytes[k] / 16;
+    const unsigned long long per = (granules + gridDim.x - 1) / gridDim.x;
+    const unsigned long long g0 = per * blockIdx.x;
+    if (g0 >= granules) continue;
+    unsigned long long left = (granules - g0 < per ? granules - g0 : per) * 16;
+    const char* a = static_cast<const char*>(pf.ptr[k]) + g0 * 16;
+    while (left > 0) {
+      const unsigned int sz = left > 65536ull ? 65536u : static_cast<unsigned int>(left);
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a), "r"(sz) : "memory");
+      a += sz;
+      left -= sz;
+    }
+  }
+}
+
 // Device error words (rm_get_device_error): [0] clamped token ids, [1] waits
 // that gave up.
 enum { ERR_CLAMPED = 0, ERR_TIMEOUT = 1, ERR_WORDS = 2 };

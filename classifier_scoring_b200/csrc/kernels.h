@@ -25,14 +25,23 @@ cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows, const char** why);
 
+// Weights of the next GEMMs to pull into L2 while a latency-bound kernel runs
+// (the whole model does not stay in L2, so a GEMM would otherwise start on
+// cold weights).  Each CTA issues bulk L2 prefetches for its slice.
+struct L2Prefetch {
+  const void* ptr[2] = {nullptr, nullptr};
+  unsigned long long bytes[2] = {0, 0};
+};
+
 // ---- row kernels (rowops.cu) ----
 cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs, int T,
                          const void* emb_word, const void* emb_pos, const float* ln_g,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
-                         int32_t* err_count, cudaStream_t st);
+                         int32_t* err_count, cudaStream_t st, const L2Prefetch& pf = {});
 // dtype: 0 fp32, 1 bf16; mode 0 post, 1 pre, 2 plain (see rm_ops.h)
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
-                          int H, float eps, int dtype, int mode, cudaStream_t st);
+                          int H, float eps, int dtype, int mode, cudaStream_t st,
+                          const L2Prefetch& pf = {});
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
                         float b_r, int H, int last_token, float* out, cudaStream_t st);
 // weight conversion at create
@@ -46,13 +55,15 @@ cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
                                const int32_t* rb_off, const int64_t* s_off, int n_seqs,
                                int n_row_blocks, int n_heads, int head_dim, int causal,
                                cudaStream_t st);
+// err: device error words (ERR_TIMEOUT counts waits that gave up) or NULL
 cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const int64_t* s_off,
-                           int n_seqs, int T, int n_heads, int max_len, int causal,
+                           int n_seqs, int T, int n_heads, int max_len, int causal, int* err,
                            cudaStream_t st);
 // scores + masked softmax + context in one kernel (probabilities stay in registers)
 cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets,
                               const int32_t* rb_off, int n_seqs, int n_row_blocks, int n_heads,
-                              int head_dim, int causal, cudaStream_t st);
+                              int head_dim, int causal, cudaStream_t st,
+                              const L2Prefetch& pf = {});
 cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
                                 const int32_t* rb_off, const int64_t* s_off, int n_seqs,
                                 int n_row_blocks, int n_heads, int head_dim, int causal,

@@ -116,7 +116,7 @@ extern "C" int rm_op_attention_noalloc(const void* qkv, void* ctx, const int32_t
                                      head_dim, causal != 0, st);
   if (e == cudaSuccess)
     e = softmax_launch(d_s, RM_BF16, d_off, d_so, n_seqs, offsets[n_seqs], n_heads, max_len,
-                       causal != 0, st);
+                       causal != 0, nullptr, st);
   if (e == cudaSuccess)
     e = attn_context_launch(d_s, qkv, ctx, d_off, d_rb, d_so, n_seqs, n_row_blocks, n_heads,
                             head_dim, causal != 0, st);

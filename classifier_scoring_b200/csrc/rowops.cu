@@ -65,8 +65,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     embed_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ offsets, int n_seqs,
                  int T, const bf16* __restrict__ ew, const bf16* __restrict__ ep,
                  const float* __restrict__ g, const float* __restrict__ b, float eps, int V, int H,
-                 bf16* __restrict__ x, int32_t* __restrict__ err) {
+                 bf16* __restrict__ x, int32_t* __restrict__ err, L2PrefetchArgs pf) {
   pdl_launch_dependents();
+  l2_prefetch_share(pf);   // static weights: no need to wait for the previous kernel
   pdl_wait();
   const int t = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -111,8 +112,9 @@ template <typename T, int MAXC, int MODE>
 __global__ void __launch_bounds__(kWarps * 32)
     res_ln_kernel(const T* __restrict__ y, T* __restrict__ x, T* __restrict__ z,
                   const float* __restrict__ g, const float* __restrict__ b, int rows, int H,
-                  float eps) {
+                  float eps, L2PrefetchArgs pf) {
   pdl_launch_dependents();
+  l2_prefetch_share(pf);
   pdl_wait();
   const int r = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -191,6 +193,15 @@ __global__ void cvt_f32_kernel(const S* __restrict__ src, float* __restrict__ ds
     dst[k] = to_f32(src[k]);
 }
 
+L2PrefetchArgs pf_args(const L2Prefetch& pf) {
+  L2PrefetchArgs a;
+  for (int k = 0; k < 2; ++k) {
+    a.ptr[k] = pf.ptr[k];
+    a.bytes[k] = pf.bytes[k];
+  }
+  return a;
+}
+
 // Smallest supported chunks-per-lane count >= need (H <= 4096).
 int pick_maxc(int H) {
   const int need = (H / 8 + 31) / 32;
@@ -202,32 +213,35 @@ int pick_maxc(int H) {
 template <int MAXC>
 cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, const void* ew,
                     const void* ep, const float* g, const float* b, float eps, int V, int H,
-                    void* x, int32_t* err, cudaStream_t st) {
+                    void* x, int32_t* err, cudaStream_t st, const L2Prefetch& pf) {
   dim3 grid((T + kWarps - 1) / kWarps);
   if (g != nullptr)
     launch_k(embed_kernel<MAXC, true>, grid, kWarps * 32, 0, st, 
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<bf16*>(x), err);
+        V, H, static_cast<bf16*>(x), err, pf_args(pf));
   else
     launch_k(embed_kernel<MAXC, false>, grid, kWarps * 32, 0, st, 
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<bf16*>(x), err);
+        V, H, static_cast<bf16*>(x), err, pf_args(pf));
   return cudaGetLastError();
 }
 
 template <typename T, int MAXC>
 cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const float* b, int rows,
-                     int H, float eps, int mode, cudaStream_t st) {
+                     int H, float eps, int mode, cudaStream_t st, const L2Prefetch& pf) {
   dim3 grid((rows + kWarps - 1) / kWarps);
   const T* yy = static_cast<const T*>(y);
   T* xx = static_cast<T*>(x);
   T* zz = static_cast<T*>(z);
   if (mode == 0)
-    launch_k(res_ln_kernel<T, MAXC, 0>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps);
+    launch_k(res_ln_kernel<T, MAXC, 0>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps,
+             pf_args(pf));
   else if (mode == 1)
-    launch_k(res_ln_kernel<T, MAXC, 1>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps);
+    launch_k(res_ln_kernel<T, MAXC, 1>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps,
+             pf_args(pf));
   else
-    launch_k(res_ln_kernel<T, MAXC, 2>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps);
+    launch_k(res_ln_kernel<T, MAXC, 2>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps,
+             pf_args(pf));
   return cudaGetLastError();
 }
 
@@ -249,22 +263,23 @@ cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const floa
 cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs, int T,
                          const void* emb_word, const void* emb_pos, const float* ln_g,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
-                         int32_t* err_count, cudaStream_t st) {
+                         int32_t* err_count, cudaStream_t st, const L2Prefetch& pf) {
   (void)P;
   if (T == 0) return cudaSuccess;
   const int maxc = pick_maxc(H);
   RMK_MAXC_SWITCH(maxc, (embed_t<M_>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps,
-                                     V, H, x, err_count, st)))
+                                     V, H, x, err_count, st, pf)))
 }
 
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
-                          int H, float eps, int dtype, int mode, cudaStream_t st) {
+                          int H, float eps, int dtype, int mode, cudaStream_t st,
+                          const L2Prefetch& pf) {
   if (T == 0) return cudaSuccess;
   const int maxc = pick_maxc(H);
   if (dtype == 0) {
-    RMK_MAXC_SWITCH(maxc, (res_ln_t<float, M_>(y, x, z, g, b, T, H, eps, mode, st)))
+    RMK_MAXC_SWITCH(maxc, (res_ln_t<float, M_>(y, x, z, g, b, T, H, eps, mode, st, pf)))
   }
-  RMK_MAXC_SWITCH(maxc, (res_ln_t<bf16, M_>(y, x, z, g, b, T, H, eps, mode, st)))
+  RMK_MAXC_SWITCH(maxc, (res_ln_t<bf16, M_>(y, x, z, g, b, T, H, eps, mode, st, pf)))
 }
 
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
