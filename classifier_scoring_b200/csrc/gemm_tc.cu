@@ -126,7 +126,8 @@ __device__ __forceinline__ void tmem_wait_ld() {
 
 template <int BN>
 constexpr int stages_for() {
-  return BN <= 64 ? 8 : (BN <= 128 ? 6 : (BN <= 192 ? 5 : 4));
+  // as many 64-deep K stages as fit beside the epilogue staging (<= 227 KB)
+  return BN <= 64 ? 8 : (BN <= 96 ? 7 : (BN <= 128 ? 6 : (BN <= 192 ? 5 : 4)));
 }
 constexpr uint32_t tmem_cols_for(int bn) {
   // two accumulators of bn fp32 columns, rounded up to a power of two >= 32
@@ -145,7 +146,9 @@ struct GemmSmem {
   static constexpr int kStagePitch = 128 + 16;
   static constexpr int kStageWarpBytes = 32 * kStagePitch;
   static constexpr int kEpiOff = kStages * kStage;
-  static constexpr int kBarOff = kEpiOff + 4 * kStageWarpBytes;   // full[S], empty[S], accf[2], acce[2]
+  // bias of the tile, per epilogue warp and accumulator (no cross-warp barrier)
+  static constexpr int kBiasOff = kEpiOff + 4 * kStageWarpBytes;
+  static constexpr int kBarOff = kBiasOff + 4 * 2 * BN * 4;       // full[S], empty[S], accf[2], acce[2]
   static constexpr int kSlotOff = kBarOff + (2 * kStages + 4) * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;   // + alignment slack
 };
@@ -281,9 +284,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;                      // TMEM lane quarter of this warp
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     uint8_t* stg = smem + L::kEpiOff + (warp - 2) * L::kStageWarpBytes;
+    float* sbias_warp = reinterpret_cast<float*>(smem + L::kBiasOff) + (warp - 2) * 2 * BN;
     int local = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
       const int acc = local & 1, use = local >> 1;
+      // stage this tile's bias while the mainloop still runs (this warp's
+      // buffer for the accumulator was last read two tiles ago)
+      float* sbias = sbias_warp + acc * BN;
+      {
+        const int nb0 = (t / tiles_m) * BN;
+        for (int j = lane; j < BN; j += 32)
+          sbias[j] = (bias != nullptr && nb0 + j < N) ? __ldg(bias + nb0 + j) : 0.0f;
+        __syncwarp();
+      }
       const bool ready = mbar_wait(accf0 + 8 * acc, use & 1);
       if (!__all_sync(0xffffffffu, ready)) {
         if (lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
@@ -309,9 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int g = 0; g < CPR / 4; ++g) {
-          const int col = n0 + c + 4 * g;
-          float4 b4 = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (bias != nullptr && col < N) b4 = __ldg(reinterpret_cast<const float4*>(bias + col));
+          // c + 4g < BN except in a partial last round, whose columns are not stored
+          const float4 b4 = (c + 4 * g < BN) ? *reinterpret_cast<const float4*>(sbias + c + 4 * g)
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
           v[4 * g + 0] = epilogue_act<ACT>(v[4 * g + 0] + b4.x);
           v[4 * g + 1] = epilogue_act<ACT>(v[4 * g + 1] + b4.y);
           v[4 * g + 2] = epilogue_act<ACT>(v[4 * g + 2] + b4.z);
@@ -333,12 +346,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
         const int ch = lane & 7;                 // 16-byte chunk of a 128-byte segment
-        const int gcol = n0 + c + ch * (16 / ESZ);
+        const int tcol = c + ch * (16 / ESZ);    // column inside the tile
+        const int gcol = n0 + tcol;
+        // a round can run past the tile (BN not a multiple of the round width):
+        // those columns belong to the next tile and are not stored
+        const bool col_ok = tcol < BN && gcol < N;
 #pragma unroll
         for (int it = 0; it < 8; ++it) {
           const int rr = it * 4 + (lane >> 3);
           const int grow = row0 + rr;
-          if (grow < M && gcol < N) {
+          if (grow < M && col_ok) {
             const uint4 u = *reinterpret_cast<const uint4*>(stg + rr * L::kStagePitch + ch * 16);
             *reinterpret_cast<uint4*>(static_cast<uint8_t*>(y) +
                                       (static_cast<size_t>(grow) * N + gcol) * ESZ) = u;
@@ -397,7 +414,7 @@ cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
 
 }  // namespace
 
-const int kGemmTileWidths[kGemmTileCount] = {64, 128, 192, 256};
+const int kGemmTileWidths[kGemmTileCount] = {64, 96, 128, 160, 192, 224, 256};
 
 int gemm_pick_bn(int M, int N, int num_sms) {
 #ifdef RM_GEMM_FORCE_BN
@@ -427,8 +444,11 @@ cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int 
                         cudaStream_t st) {
   switch (bn) {
     case 64: return launch_act<64>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 96: return launch_act<96>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
     case 128: return launch_act<128>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 160: return launch_act<160>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
     case 192: return launch_act<192>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 224: return launch_act<224>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
     case 256: return launch_act<256>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
     default: return cudaErrorInvalidValue;
   }

@@ -8,11 +8,11 @@
 namespace rmk {
 
 // ---- tcgen05 GEMM (gemm_tc.cu) ----
-constexpr int kGemmTileCount = 4;
-extern const int kGemmTileWidths[kGemmTileCount];   // 64, 128, 192, 256
+constexpr int kGemmTileCount = 7;
+extern const int kGemmTileWidths[kGemmTileCount];   // 64, 96, 128, 160, 192, 224, 256
 // Column-tile width for an M x N problem on num_sms SMs (one of kGemmTileWidths).
 int gemm_pick_bn(int M, int N, int num_sms);
-inline int gemm_tile_index(int bn) { return bn == 64 ? 0 : bn == 128 ? 1 : bn == 192 ? 2 : 3; }
+inline int gemm_tile_index(int bn) { return (bn - 64) / 32; }
 // a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, bn}.
 // Persistent grid of min(tiles, num_sms) CTAs.
 cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int M, int N, int K,
