@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         "rm_last_error": (ctypes.c_char_p, []),
         "rm_varlen_meta": (ctypes.c_int, [P, I32, I32, P, P]),
         "rm_op_gemm": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
+        "rm_op_gemm_tiled": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P]),
+        "rm_gemm_tile": (ctypes.c_int, [I32, I32, I32, I32, P]),
         "rm_op_embed": (ctypes.c_int, [P, P, I32, I32, P, P, P, P, F, I32, I32, I32, P, P, P]),
         "rm_op_attn_scores": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_softmax": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P]),
@@ -247,6 +249,17 @@ class ops:
     def gemm(x, w, bias, y, y_dtype, M, N, K, act=0, stream=None):
         _check(lib().rm_op_gemm(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), y_dtype, M, N, K, act,
                                 _stream(stream)))
+
+    @staticmethod
+    def gemm_tiled(x, w, bias, y, y_dtype, M, N, K, act=0, cg=0, bn=0, stream=None):
+        _check(lib().rm_op_gemm_tiled(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), y_dtype, M, N, K,
+                                      act, cg, bn, _stream(stream)))
+
+    @staticmethod
+    def gemm_tile(M, N, K, num_sms):
+        out = np.zeros(2, dtype=np.int32)
+        _check(lib().rm_gemm_tile(M, N, K, num_sms, out.ctypes.data))
+        return int(out[0]), int(out[1])
 
     @staticmethod
     def embed(ids, offsets_dev, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps, V, P, H, x,

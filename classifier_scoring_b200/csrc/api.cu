@@ -334,9 +334,9 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
 
 int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCount], int M, int N,
          int K, const float* bias, void* y, int act, cudaStream_t st) {
-  const int bn = gemm_pick_bn(M, N, h->num_sms);
-  cudaError_t e = gemm_launch(a, b[gemm_tile_index(bn)], bn, M, N, K, bias, y, false, act,
-                              h->d_err, h->num_sms, st);
+  const GemmTile tile = gemm_pick(M, N, K, h->num_sms);
+  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], tile, M, N, K, bias, y, false,
+                              act, h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return RM_OK;
 }
@@ -787,6 +787,12 @@ int rm_varlen_meta(const int32_t* offsets, int32_t n, int32_t n_heads, int32_t* 
 
 int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
                int32_t M, int32_t N, int32_t K, int32_t act, void* stream) {
+  return rm_op_gemm_tiled(x, w, bias, y, y_dtype, M, N, K, act, 0, 0, stream);
+}
+
+int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
+                     int32_t M, int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn,
+                     void* stream) {
   if (x == nullptr || w == nullptr || y == nullptr) return set_error(RM_E_INVAL, "NULL argument");
   if (M < 1 || N < 8 || K < 8 || N % 8 != 0 || K % 8 != 0)
     return set_error(RM_E_INVAL, "need M >= 1 and N, K positive multiples of 8");
@@ -794,18 +800,34 @@ int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t
     return set_error(RM_E_INVAL, "bad act or y_dtype");
   if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (reinterpret_cast<uintptr_t>(bias) & 15) != 0)
     return set_error(RM_E_INVAL, "y and bias must be 16-byte aligned");
+  if (cg != 0) {
+    bool known = false;
+    if (cg == 1)
+      for (int i = 0; i < kGemmTileCount; ++i) known = known || kGemmTileWidths[i] == bn;
+    if (cg == 2) known = bn == 128 || bn == 192 || bn == 256;
+    if (!known) return set_error(RM_E_INVAL, "no %d-CTA tile of width %d", cg, bn);
+  }
   int dev = 0, sms = 148;
   RM_CUDA(cudaGetDevice(&dev));
   RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const int bn = gemm_pick_bn(M, N, sms);
+  const GemmTile tile = cg != 0 ? GemmTile{cg, bn} : gemm_pick(M, N, K, sms);
   CUtensorMap ta, tb;
   const char* why = "";
-  if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, bn, &why))
+  if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, tile.b_box(), &why))
     return set_error(RM_E_INVAL, "tensor map: %s", why);
   int32_t* err = nullptr;
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
-  RM_LAUNCH(gemm_launch(ta, tb, bn, M, N, K, bias, y, y_dtype == RM_F32, act, err, sms,
+  RM_LAUNCH(gemm_launch(ta, tb, tile, M, N, K, bias, y, y_dtype == RM_F32, act, err, sms,
                         static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_gemm_tile(int32_t M, int32_t N, int32_t K, int32_t num_sms, int32_t* out) {
+  if (out == nullptr || M < 1 || N < 1 || K < 1 || num_sms < 1)
+    return set_error(RM_E_INVAL, "bad arguments");
+  const GemmTile t = gemm_pick(M, N, K, num_sms);
+  out[0] = t.cg;
+  out[1] = t.bn;
   return RM_OK;
 }
 

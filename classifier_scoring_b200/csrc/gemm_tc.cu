@@ -3,9 +3,15 @@
 // "BLAS routines" of the TurboTransformers abstract, on tensor cores as its
 // proposed-method section does; here bf16 in, fp32 accumulation).
 //
-// Persistent, warp-specialised kernel: one CTA per SM walks the 128 x BN
-// output tiles t = blockIdx.x, blockIdx.x + gridDim.x, ... (M fastest, so the
-// CTAs of one wave share a few weight column blocks in L2).  Six warps:
+// Persistent, warp-specialised kernel: one CTA per SM (CG = 1) or one CTA pair
+// per two SMs (CG = 2) walks the (128*CG) x BN output tiles t = unit,
+// unit + units, ... (M fastest, so the CTAs of one wave share a few weight
+// column blocks in L2).  With CG = 2 the pair is a cluster of two CTAs and the
+// MMA is tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 rows of
+// A and half of the BN rows of B, the leader CTA issues the MMAs for both, and
+// each CTA's TMEM receives its own 128 rows of the accumulator.  Per SM this
+// moves half of B through shared memory, which keeps the operand ring ahead of
+// the tensor core.  No load uses multicast.  Six warps:
 //   warp 0, one lane : TMA producer -- K-major 128x64 (A) and BNx64 (B) bf16
 //                      boxes, 128-byte swizzle, into a STAGES-deep smem ring
 //                      that runs on across tile boundaries;
@@ -32,6 +38,13 @@ constexpr int BM = 128;
 constexpr int BK = 64;                      // 64 bf16 = one 128-byte swizzle row
 
 constexpr int kThreads = 192;
+// Time per column of a CTA-pair tile relative to a single-CTA tile, and the
+// smallest products for which pairs are considered (measured on B200: a pair
+// round took ~0.8x a single-CTA round of the same width at M = 26112,
+// K = 2048, but ~1.1x at M = 3328, K = 768, and lost at M = 3328, K = 3072).
+constexpr double kPairColumnCost = 0.8;
+constexpr int kPairMinM = 8192;
+constexpr int kPairMinK = 2048;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -80,16 +93,50 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t leader_bar) {
+  // both CTAs of the pair complete their bytes on the leader's barrier
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(leader_bar)
+      : "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+template <int CG>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
+  if (CG == 1)
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
+  else
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     bar)
+                 : "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major operand tile written by TMA
@@ -124,33 +171,34 @@ __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-template <int BN>
-constexpr int stages_for() {
-  // as many 64-deep K stages as fit beside the epilogue staging (<= 227 KB)
-  return BN <= 64 ? 8 : (BN <= 96 ? 7 : (BN <= 128 ? 6 : (BN <= 192 ? 5 : 4)));
-}
 constexpr uint32_t tmem_cols_for(int bn) {
   // two accumulators of bn fp32 columns, rounded up to a power of two >= 32
   return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
 }
 
-template <int BN>
+template <int BN, int CG>
 struct GemmSmem {
-  static constexpr int kStages = stages_for<BN>();
   static constexpr int kA = BM * BK * 2;
-  static constexpr int kB = BN * BK * 2;
-  static constexpr int kStage = kA + kB;     // multiple of 1024 for BN % 8 == 0
+  static constexpr int kB = (BN / CG) * BK * 2;   // this CTA's share of the B tile
+  static constexpr int kStage = kA + kB;          // multiple of 1024 for BN/CG % 8 == 0
   // epilogue staging: per epilogue warp 32 rows x 128 B of output (64 bf16 or
   // 32 fp32 columns), row pitch padded by 16 B so that both the row-wise
   // writes and the line-wise reads touch every bank group evenly
   static constexpr int kStagePitch = 128 + 16;
   static constexpr int kStageWarpBytes = 32 * kStagePitch;
-  static constexpr int kEpiOff = kStages * kStage;
   // bias of the tile, per epilogue warp and accumulator (no cross-warp barrier)
+  static constexpr int kBiasBytes = 4 * 2 * BN * 4;
+  // as many 64-deep K stages as fit beside the rest (227 KB per CTA), at most 8
+  static constexpr int kFixed = 4 * kStageWarpBytes + kBiasBytes + 20 * 8 + 16 + 1024;
+  static constexpr int kStagesFit = (232448 - kFixed) / kStage;
+  static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
+  static constexpr int kEpiOff = kStages * kStage;
   static constexpr int kBiasOff = kEpiOff + 4 * kStageWarpBytes;
-  static constexpr int kBarOff = kBiasOff + 4 * 2 * BN * 4;       // full[S], empty[S], accf[2], acce[2]
+  static constexpr int kBarOff = kBiasOff + kBiasBytes;   // full[S], empty[S], accf[2], acce[2]
   static constexpr int kSlotOff = kBarOff + (2 * kStages + 4) * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;   // + alignment slack
+  static_assert(kStages >= 3, "at least three stages");
+  static_assert(kBytes <= 232448, "fits one CTA's shared memory");
 };
 
 template <int ACT>
@@ -160,13 +208,13 @@ __device__ __forceinline__ float epilogue_act(float t) {
   return t;
 }
 
-template <int BN, int ACT, bool OUT_F32>
+template <int BN, int CG, int ACT, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
                         const float* __restrict__ bias, void* __restrict__ y,
                         int* __restrict__ err) {
-  using L = GemmSmem<BN>;
+  using L = GemmSmem<BN, CG>;
   constexpr int S = L::kStages;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
   static_assert(L::kStage % 1024 == 0, "stage size keeps the 1024-byte swizzle alignment");
@@ -177,7 +225,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kSlotOff);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_m = (M + BM - 1) / BM;
+  const uint32_t rank = CG == 2 ? cluster_rank() : 0u;   // 0 = leader of the pair
+  const int unit = blockIdx.x / CG, units = gridDim.x / CG;
+  const int tiles_m = (M + BM * CG - 1) / (BM * CG);
   const int tiles = tiles_m * ((N + BN - 1) / BN);
   const int nk = (K + BK - 1) / BK;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S),
@@ -190,20 +240,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
-      mbar_init(acce0 + 8 * a, 4);   // one arrival per epilogue warp
+      mbar_init(acce0 + 8 * a, 4 * CG);   // one arrival per epilogue warp of the pair
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if (CG == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(tmem_slot)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync_all();   // both CTAs' barriers exist before any remote signal
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // the prologue above overlaps the previous kernel; global memory waits for it
@@ -215,8 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- TMA producer ----
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-        const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+      for (int t = unit; t < tiles && ok; t += units) {
+        const int m0 = (t % tiles_m) * BM * CG + static_cast<int>(rank) * BM;
+        const int nb0 = (t / tiles_m) * BN + static_cast<int>(rank) * (BN / CG);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -225,21 +285,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full0 + 8 * s, L::kStage);
-          tma_load_2d(smem_u32(smem + s * L::kStage), &tmA, kb * BK, m0, full0 + 8 * s);
-          tma_load_2d(smem_u32(smem + s * L::kStage + L::kA), &tmB, kb * BK, n0, full0 + 8 * s);
+          const uint32_t dA = smem_u32(smem + s * L::kStage), dB = dA + L::kA;
+          if (CG == 1) {
+            mbar_arrive_expect_tx(full0 + 8 * s, L::kStage);
+            tma_load_2d(dA, &tmA, kb * BK, m0, full0 + 8 * s);
+            tma_load_2d(dB, &tmB, kb * BK, nb0, full0 + 8 * s);
+          } else {
+            // the leader expects the bytes of both CTAs on its own barrier
+            if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * L::kStage);
+            const uint32_t lbar = map_to_rank(full0 + 8 * s, 0);
+            tma_load_2d_pair(dA, &tmA, kb * BK, m0, lbar);
+            tma_load_2d_pair(dB, &tmB, kb * BK, nb0, lbar);
+          }
         }
       }
-      // copies in flight land before this CTA's shared memory is released
-      for (int j = it - 1; j >= 0 && j >= it - S; --j) mbar_wait(full0 + 8 * (j % S), (j / S) & 1);
+      // Before shared memory is released: the copies in flight have landed
+      // (the leader's full barriers count both CTAs' bytes) and the MMA
+      // completions that arrive on this CTA's empty barriers (from the
+      // leader, with a pair) have arrived.  Bounded; gives up at the first
+      // wait that runs out.
+      bool drained = true;
+      if (rank == 0)
+        for (int j = it - 1; drained && j >= 0 && j >= it - S; --j)
+          drained = mbar_wait(full0 + 8 * (j % S), (j / S) & 1);
+      if (ok)
+        for (int j = it - 1; drained && j >= 0 && j >= it - S; --j)
+          drained = mbar_wait(empty0 + 8 * (j % S), (j / S) & 1);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---- MMA issuer ----
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+    if (lane == 0 && rank == 0) {
+      // ---- MMA issuer (the leader issues for the pair) ----
+      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, BN);
       int it = 0, local = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++local) {
+      for (int t = unit; t < tiles && ok; t += units, ++local) {
         const int acc = local & 1, use = local >> 1;
         if (use > 0 && !mbar_wait(acce0 + 8 * acc, (use - 1) & 1)) {
           atomicAdd(err + ERR_TIMEOUT, 1);
@@ -262,16 +341,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < BK / 16; ++k) {
             // advance 16 elements = 32 bytes along K inside the swizzle atom
             const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-            asm volatile(
-                "{\n\t.reg .pred p;\n\t"
-                "setp.ne.b32 p, %4, 0;\n\t"
-                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
-                "l"(ad + 2ull * k), "l"(bd + 2ull * k), "r"(idesc), "r"(accum)
-                : "memory");
+            if (CG == 1)
+              asm volatile(
+                  "{\n\t.reg .pred p;\n\t"
+                  "setp.ne.b32 p, %4, 0;\n\t"
+                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+                  "l"(ad + 2ull * k), "l"(bd + 2ull * k), "r"(idesc), "r"(accum)
+                  : "memory");
+            else
+              asm volatile(
+                  "{\n\t.reg .pred p;\n\t"
+                  "setp.ne.b32 p, %4, 0;\n\t"
+                  "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d),
+                  "l"(ad + 2ull * k), "l"(bd + 2ull * k), "r"(idesc), "r"(accum)
+                  : "memory");
           }
-          tc_commit(empty0 + 8 * s);   // frees the stage once these MMAs are done
+          // frees the stage (in both CTAs of a pair) once these MMAs are done
+          tc_commit<CG>(empty0 + 8 * s);
+          if (CG == 2) tc_commit<CG>(map_to_rank(empty0 + 8 * s, 1));
         }
-        tc_commit(accf0 + 8 * acc);    // the accumulator is complete
+        tc_commit<CG>(accf0 + 8 * acc);    // the accumulator is complete
+        if (CG == 2) tc_commit<CG>(map_to_rank(accf0 + 8 * acc, 1));
       }
     }
   } else {
@@ -286,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* stg = smem + L::kEpiOff + (warp - 2) * L::kStageWarpBytes;
     float* sbias_warp = reinterpret_cast<float*>(smem + L::kBiasOff) + (warp - 2) * 2 * BN;
     int local = 0;
-    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++local) {
+    for (int t = unit; t < tiles; t += units, ++local) {
       const int acc = local & 1, use = local >> 1;
       // stage this tile's bias while the mainloop still runs (this warp's
       // buffer for the accumulator was last read two tiles ago)
@@ -303,7 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+      const int m0 = (t % tiles_m) * BM * CG + static_cast<int>(rank) * BM;
+      const int n0 = (t / tiles_m) * BN;
       const int row0 = m0 + q * 32;
       const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
 #pragma unroll 1
@@ -364,92 +455,151 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce0 + 8 * acc);   // accumulator free for tile local+2
+      // accumulator free for tile local+2 (the leader's barrier counts both CTAs)
+      if (lane == 0) {
+        if (CG == 1 || rank == 0) mbar_arrive(acce0 + 8 * acc);
+        else mbar_arrive_cluster(map_to_rank(acce0 + 8 * acc, 0));
+      }
     }
   }
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  if (CG == 2) cluster_sync_all();   // no remote signal or copy can outlive either CTA
+  else __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols)
-                 : "memory");
+    if (CG == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                   "r"(kTmemCols)
+                   : "memory");
   }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int BN, int ACT, bool OUT_F32>
+template <int BN, int CG, int ACT, bool OUT_F32>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
                        const float* bias, void* y, int* err, int num_sms, cudaStream_t st) {
-  using L = GemmSmem<BN>;
-  auto kern = gemm_bf16_tc_kernel<BN, ACT, OUT_F32>;
-  static bool configured = false;   // the attribute is per function; one device per process
+  using L = GemmSmem<BN, CG>;
+  auto kern = gemm_bf16_tc_kernel<BN, CG, ACT, OUT_F32>;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (CG == 2) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 2;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  // The attribute is per function and the co-resident pair count per device
+  // model; one device model per process.
+  static bool configured = false;
+  static int resident_units = 0;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
     if (e != cudaSuccess) return e;
+    if (CG == 2) {
+      // pairs must sit on the two SMs of one cluster slot: ask how many fit at once
+      cfg.gridDim = dim3(2 * (num_sms / 2));
+      cfg.attrs = attr;
+      cfg.numAttrs = na;
+      int clusters = 0;
+      e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
+      if (e != cudaSuccess) return e;
+      resident_units = clusters;
+    }
     configured = true;
   }
-  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  launch_k(kern, dim3(grid), dim3(kThreads), L::kBytes, st, a, b, M, N, K, bias, y, err);
-  return cudaGetLastError();
+  const int tiles = ((M + BM * CG - 1) / (BM * CG)) * ((N + BN - 1) / BN);
+  int max_units = num_sms / CG;
+  if (CG == 2 && resident_units > 0 && resident_units < max_units) max_units = resident_units;
+  cfg.gridDim = dim3(CG * (tiles < max_units ? tiles : max_units));
+  if (g_pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  return cudaLaunchKernelEx(&cfg, kern, a, b, M, N, K, bias, y, err);
 }
 
-template <int BN>
+template <int BN, int CG>
 cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
                        const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
                        cudaStream_t st) {
   if (out_f32) {
-    if (act == 1) return launch_one<BN, 1, true>(a, b, M, N, K, bias, y, err, num_sms, st);
-    if (act == 2) return launch_one<BN, 2, true>(a, b, M, N, K, bias, y, err, num_sms, st);
-    return launch_one<BN, 0, true>(a, b, M, N, K, bias, y, err, num_sms, st);
+    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, M, N, K, bias, y, err, num_sms, st);
+    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, M, N, K, bias, y, err, num_sms, st);
+    return launch_one<BN, CG, 0, true>(a, b, M, N, K, bias, y, err, num_sms, st);
   }
-  if (act == 1) return launch_one<BN, 1, false>(a, b, M, N, K, bias, y, err, num_sms, st);
-  if (act == 2) return launch_one<BN, 2, false>(a, b, M, N, K, bias, y, err, num_sms, st);
-  return launch_one<BN, 0, false>(a, b, M, N, K, bias, y, err, num_sms, st);
+  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, M, N, K, bias, y, err, num_sms, st);
+  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, M, N, K, bias, y, err, num_sms, st);
+  return launch_one<BN, CG, 0, false>(a, b, M, N, K, bias, y, err, num_sms, st);
 }
 
 }  // namespace
 
 const int kGemmTileWidths[kGemmTileCount] = {64, 96, 128, 160, 192, 224, 256};
 
-int gemm_pick_bn(int M, int N, int num_sms) {
-#ifdef RM_GEMM_FORCE_BN
-  return RM_GEMM_FORCE_BN;
+GemmTile gemm_pick(int M, int N, int K, int num_sms) {
+#if defined(RM_GEMM_FORCE_BN) && defined(RM_GEMM_FORCE_CG)
+  return GemmTile{RM_GEMM_FORCE_CG, RM_GEMM_FORCE_BN};
 #endif
-  // Makespan of the persistent grid: rounds of tiles times the tile's width
-  // (mainloop time grows with BN), plus a fixed cost per tile (pipeline fill,
-  // epilogue tail) worth about 48 columns.  Ties go to the wider tile.
-  const long long tm = (M + BM - 1) / BM;
-  int best = 256;
-  long long best_cost = -1;
-  for (int i = kGemmTileCount - 1; i >= 0; --i) {
-    const int bn = kGemmTileWidths[i];
+  // Makespan of the persistent grid: rounds of tiles times the per-SM time of
+  // one tile, modelled as proportional to BN plus a fixed cost per tile
+  // (pipeline fill, epilogue tail) worth about 48 columns.  A CTA pair moves
+  // half of the weight tile per SM, so its mainloop runs faster per column,
+  // but on B200 it only paid off on large products (M >= kPairMinM rows and
+  // K >= kPairMinK): on the short projections of small batches a pair ran
+  // slower than one CTA of the same width.
+  GemmTile best{1, 256};
+  double best_cost = -1;
+  auto consider = [&](int cg, int bn, double per_col) {
+    const long long tm = (M + 128LL * cg - 1) / (128LL * cg);
     const long long tiles = tm * ((N + bn - 1) / bn);
-    const long long rounds = (tiles + num_sms - 1) / num_sms;
-    const long long cost = rounds * (bn + 48);
+    const long long units = num_sms / cg;
+    const long long rounds = (tiles + units - 1) / units;
+    const double cost = static_cast<double>(rounds) * (bn * per_col + 48.0);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
-      best = bn;
+      best = GemmTile{cg, bn};
     }
-  }
+  };
+  for (int i = kGemmTileCount - 1; i >= 0; --i) consider(1, kGemmTileWidths[i], 1.0);
+  if (num_sms >= 2 && M >= kPairMinM && K >= kPairMinK)
+    for (int bn : {256, 192, 128}) consider(2, bn, kPairColumnCost);
   return best;
 }
 
-cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int M, int N, int K,
-                        const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
-                        cudaStream_t st) {
-  switch (bn) {
-    case 64: return launch_act<64>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 96: return launch_act<96>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 128: return launch_act<128>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 160: return launch_act<160>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 192: return launch_act<192>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 224: return launch_act<224>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 256: return launch_act<256>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, GemmTile tile, int M, int N,
+                        int K, const float* bias, void* y, bool out_f32, int act, int* err,
+                        int num_sms, cudaStream_t st) {
+  if (tile.cg == 2) {
+    switch (tile.bn) {
+      case 128: return launch_act<128, 2>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+      case 192: return launch_act<192, 2>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+      case 256: return launch_act<256, 2>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  switch (tile.bn) {
+    case 64: return launch_act<64, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 96: return launch_act<96, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 128: return launch_act<128, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 160: return launch_act<160, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 192: return launch_act<192, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 224: return launch_act<224, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    case 256: return launch_act<256, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
     default: return cudaErrorInvalidValue;
   }
 }

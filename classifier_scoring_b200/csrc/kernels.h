@@ -10,14 +10,20 @@ namespace rmk {
 // ---- tcgen05 GEMM (gemm_tc.cu) ----
 constexpr int kGemmTileCount = 7;
 extern const int kGemmTileWidths[kGemmTileCount];   // 64, 96, 128, 160, 192, 224, 256
-// Column-tile width for an M x N problem on num_sms SMs (one of kGemmTileWidths).
-int gemm_pick_bn(int M, int N, int num_sms);
-inline int gemm_tile_index(int bn) { return (bn - 64) / 32; }
-// a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, bn}.
-// Persistent grid of min(tiles, num_sms) CTAs.
-cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, int bn, int M, int N, int K,
-                        const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
-                        cudaStream_t st);
+// Output tile: cg = 1 (one CTA, 128 x bn) or 2 (a CTA pair, 256 x bn, each CTA
+// loading bn/2 rows of the weights).
+struct GemmTile {
+  int cg;
+  int bn;
+  int b_box() const { return bn / cg; }   // weight rows per TMA box
+};
+GemmTile gemm_pick(int M, int N, int K, int num_sms);
+inline int gemm_tile_index(int box_rows) { return (box_rows - 64) / 32; }
+// a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, tile.b_box()}.
+// Persistent grid of min(tiles, num_sms / cg) units of cg CTAs.
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, GemmTile tile, int M, int N,
+                        int K, const float* bias, void* y, bool out_f32, int act, int* err,
+                        int num_sms, cudaStream_t st);
 
 // ---- TMA descriptors (tma.cpp) ----
 // 2-D bf16 row-major [rows][cols] tensor, box {64 cols, box_rows}, 128-byte swizzle,

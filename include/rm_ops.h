@@ -48,6 +48,20 @@ int rm_varlen_meta(const int32_t* offsets, int32_t n, int32_t n_heads,
 int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
                int32_t M, int32_t N, int32_t K, int32_t act, void* stream);
 
+/* rm_op_gemm with an explicit output tile: cg = 1 (one CTA per 128 x bn tile,
+ * bn in {64, 96, 128, 160, 192, 224, 256}) or cg = 2 (a cluster of two CTAs
+ * per 256 x bn tile on the pair MMA, bn in {128, 192, 256}); cg = 0 takes the
+ * tile rm_gemm_tile picks (what rm_op_gemm does).  Same arguments and
+ * requirements as rm_op_gemm; RM_E_INVAL for a tile outside these sets. */
+int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
+                     int32_t M, int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn,
+                     void* stream);
+
+/* Host only: the output tile the projections use for an M x N x K product on
+ * a device with num_sms SMs.  out[0] = cg (1 or 2), out[1] = bn.  RM_E_INVAL
+ * for M, N, K or num_sms < 1 or out == NULL. */
+int rm_gemm_tile(int32_t M, int32_t N, int32_t K, int32_t num_sms, int32_t* out);
+
 /* X[t] = E_word[clamp(ids[t])] + E_pos[t - offsets[i]] for each token t of
  * sequence i, then (ln_g != NULL) the embedding LayerNorm.  ids out of 0..V-1
  * are clamped and counted with atomicAdd into *err_count (may be NULL).

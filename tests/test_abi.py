@@ -114,3 +114,26 @@ def test_varlen_meta_layout():
     bad[2] = bad[1]
     with pytest.raises(rm.RmError):
         rm.ops.varlen_meta(bad, 3)
+
+
+def test_gemm_tile_pick_is_a_known_tile():
+    tiles = {(1, bn) for bn in (64, 96, 128, 160, 192, 224, 256)} | {(2, bn) for bn in (128, 192, 256)}
+    for M in (1, 77, 128, 300, 3328, 26112):
+        for N in (8, 312, 768, 2304, 3072, 8192):
+            for K in (8, 768, 2048, 8192):
+                for sms in (1, 2, 148):
+                    t = rm.ops.gemm_tile(M, N, K, sms)
+                    assert t in tiles, (M, N, K, sms, t)
+                    if sms == 1:
+                        assert t[0] == 1            # a pair needs two SMs
+    with pytest.raises(rm.RmError):
+        rm.ops.gemm_tile(0, 8, 8, 148)
+
+
+def test_gemm_tiled_rejects_unknown_tiles_on_host():
+    # rejected before any device call: the pointers are never dereferenced
+    fake = 1 << 20
+    for cg, bn in [(2, 64), (2, 96), (1, 72), (3, 128), (-1, 128)]:
+        rc = rm.lib().rm_op_gemm_tiled(fake, fake, None, fake, rm.F32, 128, 128, 64, 0, cg, bn, None)
+        assert rc == -1, (cg, bn, rc)
+        assert b"tile" in rm.lib().rm_last_error()

@@ -72,6 +72,39 @@ def test_gemm_bf16_out_and_no_bias(M, N, K):
     assert np.all(np.abs(f64(y) - ref) <= BF16_REL * np.abs(ref) + F32_RTOL * scale)
 
 
+# Every output tile forced, on a ragged problem (partial last row and column
+# tiles -- with a CTA pair the second CTA's rows or weight half can lie wholly
+# outside -- and a partial last K block) and on a multi-round projection shape.
+GEMM_TILES = [(1, bn) for bn in (64, 96, 128, 160, 192, 224, 256)] + [(2, bn) for bn in (128, 192, 256)]
+
+
+@pytest.mark.parametrize("cg,bn", GEMM_TILES, ids=[f"cg{c}-bn{b}" for c, b in GEMM_TILES])
+@pytest.mark.parametrize("shape", ["ragged", "proj"])
+@pytest.mark.parametrize("out", ["f32-gelu", "bf16"])
+def test_gemm_every_tile(cg, bn, shape, out):
+    M, N, K = (555, 2 * bn + 40, 200) if shape == "ragged" else (3328, 2304, 768)
+    g = torch.Generator().manual_seed(cg * 1000 + bn + M)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    b = torch.randn(N, generator=g, dtype=torch.float32) * 0.1
+    X, W, B = f64(x), f64(w), f64(b)
+    scale = np.abs(X) @ np.abs(W).T + np.abs(B)
+    if out == "f32-gelu":
+        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+        rm.ops.gemm_tiled(x.cuda(), w.cuda(), b.cuda(), y, rm.F32, M, N, K, 1, cg, bn)
+        torch.cuda.synchronize()
+        ref = O.gelu(O.linear(X, W, B), O.GELU_ERF)
+        bound = F32_RTOL * scale * 1.2 + 4e-7 * np.abs(ref)
+    else:
+        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        rm.ops.gemm_tiled(x.cuda(), w.cuda(), b.cuda(), y, rm.BF16, M, N, K, 0, cg, bn)
+        torch.cuda.synchronize()
+        ref = O.linear(X, W, B)
+        bound = BF16_REL * np.abs(ref) + F32_RTOL * scale
+    err = np.abs(f64(y) - ref)
+    assert np.all(err <= bound), float(np.nanmax(err / bound))
+
+
 def test_gemm_rejects_bad_shapes():
     x = torch.zeros(16, 12, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(rm.RmError):
