@@ -53,8 +53,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the dominant kernel (tcgen05 GEMM) from one ncu
 # capture; valid only for the source it was taken on (sha256 prefix of
-# gemm_tc.cu).  See profiles/gemm_bf16_tc_bert_base_T3264.txt.
-GEMM_TRAFFIC = {"src_sha": None, "bytes_per_launch": None}
+# gemm_tc.cu).  Mean of the 48 projections of one T = 3328 batch (the step's
+# batches average T = 3243).
+GEMM_TRAFFIC = {"src_sha": "ad2c53e8a0c1ec30", "bytes_per_launch": 12518923}
 
 
 def replica_workload(w, rank: int):
