@@ -13,6 +13,8 @@ Contents:
                model, per sequence (padding-free) and padded-with-mask.
   schedule  -- the dynamic-programming batch scheduler and an exhaustive
                search over all set partitions for small queues.
+  best_of_n -- best-of-N / pairwise scoring of candidates that share a
+               prefix, each scored as its own concatenated sequence.
 
 Every function cites the page passage it follows.  Pins (tests that check
 this package against something other than itself) live in
