@@ -204,10 +204,48 @@ class OracleTimer:
         return k / el, k, el
 
 
+def reference_arm_prefix(args):
+    """The oracle on the best-of-N workload: each step scores one candidate
+    as its own prefix + candidate sequence (a bounded sample)."""
+    from oracle import best_of_n as OB
+    from oracle import scorer as O
+    w = synth.PREFIX_WORKLOADS[args.workload]
+    s = w.shape
+    ids, prefix_len, n_cand, cand_len = synth.make_prefix_groups(w)
+    m = O.unpack_weights(synth.make_weights(s, w.weight_seed), s.arch, s.n_layers, s.hidden,
+                         s.n_heads, s.ffn, s.vocab, s.max_pos, s.weight_dtype, s.gelu, s.ln_eps)
+    groups = OB.split_groups(ids, prefix_len, n_cand, cand_len)
+    seqs = [np.concatenate([p, c]) for p, cs in groups for c in cs]
+    times = []
+    for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        OB.score_candidates(m, seqs[it % len(seqs)], [0], [1], [len(seqs[it % len(seqs)])])
+        if it >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = args.steps / total
+    cores = oracle_threads()
+    sample = (f"one prefix + candidate sequence per step (candidates 0..{args.steps - 1} after "
+              f"{args.warmup} warm-up), fp64 numpy oracle, {total:.1f} s")
+    line = {"impl": "reference",
+            "metric": "candidate sequences scored/sec at 1 B200 (best-of-8 over shared prefixes, GPT-1.3B shape)",
+            "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def reference_arm(args):
     rank, world, _ = rank_env()
     if rank != 0:
         return 0
+    if args.workload in synth.PREFIX_WORKLOADS:
+        return reference_arm_prefix(args)
     name = args.workload
     w = synth.WORKLOADS[name]
     per_step = 8 if w.shape.hidden >= 768 else 64
@@ -582,13 +620,178 @@ def kernel_bench(args):
     return 0
 
 
+def prefix_bench(args):
+    """Best-of-N over shared prefixes (rm_score_prefix) on the GPT-1.3B shape.
+    A step scores every candidate of every group and selects each group's best;
+    the same candidates scored as independent concatenations through rm_score
+    are timed beside it.  Replicas under torchrun: each rank its own groups."""
+    import torch
+    import classifier_scoring_b200 as rm
+    from classifier_scoring_b200 import build as rmbuild
+
+    rank, world, local = rank_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the scorer has no CPU path)")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    rmbuild.build()
+    w = synth.PREFIX_WORKLOADS[args.workload]
+    s = w.shape
+    ids, prefix_len, n_cand, cand_len = synth.make_prefix_groups(w, 1000 * rank)
+    n_c, n_g = int(n_cand.sum()), len(n_cand)
+    # the unshared comparison: every prefix + candidate as its own sequence
+    cat, lens, pos, k = [], [], 0, 0
+    for g in range(n_g):
+        pre = ids[pos:pos + prefix_len[g]]
+        pos += int(prefix_len[g])
+        for _ in range(int(n_cand[g])):
+            c = ids[pos:pos + cand_len[k]]
+            pos += int(cand_len[k])
+            k += 1
+            cat.append(np.concatenate([pre, c]))
+            lens.append(len(cat[-1]))
+    cat_ids = np.concatenate(cat).astype(np.int32)
+    cat_off = synth.offsets_from_lengths(np.array(lens))
+    max_len = int(max(lens))
+    cfg = rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
+                           ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos, weight_dtype=s.weight_dtype,
+                           gelu=s.gelu, ln_eps=s.ln_eps, max_batch_seqs=n_g + n_c,
+                           max_tokens=int(cat_off[-1]), max_len=max_len,
+                           sched_max_batch=n_c, sched_c0=SCHED_C0, sched_c1=SCHED_C1)
+    flat = synth.make_weights(s, w.weight_seed)
+    sc = rm.Scorer(cfg, flat)
+    del flat
+    stream = torch.cuda.Stream()
+    ids_dev = torch.from_numpy(ids).cuda()
+    cat_dev = torch.from_numpy(cat_ids).cuda()
+    out = torch.zeros(n_c, device="cuda")
+    best = torch.zeros(n_g, dtype=torch.int32, device="cuda")
+    lo = torch.zeros(n_g, device="cuda")
+    out_cat = torch.zeros(n_c, device="cuda")
+
+    def shared():
+        sc.score_prefix(ids_dev, prefix_len, n_cand, cand_len, out, best, lo, stream)
+
+    def unshared():
+        sc.score(cat_dev, cat_off, out_cat, stream)
+
+    def timed(fn, steps):
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
+
+    for _ in range(args.warmup):
+        shared()
+        unshared()
+    torch.cuda.synchronize()
+    if np.max(np.abs(out.cpu().numpy() - out_cat.cpu().numpy())) > 2e-3:
+        raise RuntimeError("shared-prefix and unshared scores disagree")
+    l0 = sc.profile_read()["total_launches"]
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    out_dir = os.path.join(ROOT, "gpurun_out")
+    clocks = ClockSampler(gpu_index, os.path.join(out_dir, f"clocks_prefix_rank{rank}.csv")
+                          if os.path.isdir(out_dir) else None)
+    time.sleep(0.3)
+    ms_shared = timed(shared, args.steps)
+    clk = clocks.stop()
+    launches = sc.profile_read()["total_launches"] - l0
+    ms_unshared = timed(unshared, args.steps)
+    # end to end: ids from pinned host memory, scores and choices back to the host
+    ids_pin = torch.from_numpy(ids).pin_memory()
+    res_pin = torch.empty(n_c + 2 * n_g, dtype=torch.float32).pin_memory()
+    best_pin = torch.empty(n_g, dtype=torch.int32).pin_memory()
+
+    def e2e():
+        with torch.cuda.stream(stream):
+            ids_dev.copy_(ids_pin, non_blocking=True)
+            shared()
+            res_pin[:n_c].copy_(out, non_blocking=True)
+            res_pin[n_c:n_c + n_g].copy_(lo, non_blocking=True)
+            best_pin.copy_(best, non_blocking=True)
+
+    ms_e2e = timed(e2e, args.steps)
+    # kernel shares and the GEMM roofline from one profiled step
+    sc.profile(1)
+    shared()
+    torch.cuda.synchronize()
+    prof = sc.profile_read()
+    sc.profile(0)
+    vals = reduce_times([ms_shared, ms_unshared, ms_e2e], dist, "cuda")
+    value = whole_job_rate(world, n_c, args.steps, float(vals[0]))
+    pk, pk_kind = peaks()
+    g = prof["gemm"]
+    gemm_tflops = g["flops"] / (g["ms"] * 1e-3) / 1e12 if g["ms"] > 0 else None
+    total_ms = max(1e-9, sum(prof[x]["ms"] for x in KERNEL_NAMES))
+    result = {
+        "metric": "candidate sequences scored/sec at 1 B200 (best-of-8 over shared prefixes, GPT-1.3B shape)",
+        "value": value, "unit": "sequences/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": float(vals[0]) / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "model": "GPT-style 1.3B-shape causal reward model",
+                   "groups": n_g, "candidates_per_group": w.n_cand,
+                   "prefix_lengths": f"uniform {w.prefix_lo}..{w.prefix_hi}",
+                   "candidate_lengths": f"uniform {w.cand_lo}..{w.cand_hi}",
+                   "tokens_shared": int(len(ids)), "tokens_unshared": int(cat_off[-1]),
+                   "l2": "inputs larger than L2: every step streams all weights (2.6 GB)",
+                   "parallelism": "replicas"},
+        "unshared": {"value": whole_job_rate(world, n_c, args.steps, float(vals[1])),
+                     "ms_per_step": float(vals[1]) / args.steps,
+                     "api": "rm_score on the prefix + candidate concatenations"},
+        "roofline": {"kernel": "gemm_bf16_tc_kernel (QKV, output and FFN projections)",
+                     "measured_on": "one profiled step after the timed region",
+                     "bound": "tensor", "achieved": gemm_tflops, "peak": pk["bf16_tflops_sustained"],
+                     "unit": "TFLOP/s",
+                     "frac": gemm_tflops / pk["bf16_tflops_sustained"] if gemm_tflops else None,
+                     "peak_source": f"bf16_tflops_sustained of {pk_kind}", "traffic": None},
+        "kernels": {k: {"launches": prof[k]["launches"], "share": prof[k]["ms"] / total_ms}
+                    for k in KERNEL_NAMES if prof[k]["launches"]},
+        "e2e": {"value": whole_job_rate(world, n_c, args.steps, float(vals[2])), "unit": "sequences/s",
+                "h2d_bytes_per_step": 4 * int(len(ids)) + 4 * (3 * n_g + 2 * n_c + 2),
+                "d2h_bytes_per_step": 4 * n_c + 8 * n_g,
+                "api": "rm_score_prefix, ids from pinned host memory, scores and best/log-odds back"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import best_of_n as OB
+        from oracle import scorer as O
+        m = O.unpack_weights(synth.make_weights(s, w.weight_seed), s.arch, s.n_layers, s.hidden,
+                             s.n_heads, s.ffn, s.vocab, s.max_pos, s.weight_dtype, s.gelu, s.ln_eps)
+        t0 = time.perf_counter()
+        OB.score_candidates(m, cat[0], [0], [1], [len(cat[0])])
+        el = time.perf_counter() - t0
+        result["cpu_baseline"] = {"value": 1.0 / el, "unit": "sequences/s", "cores": oracle_threads(),
+                                  "kind": "oracle",
+                                  "sample": f"candidate 0 of group 0 ({len(cat[0])} tokens) scored "
+                                            f"as its own sequence by the fp64 numpy oracle ({el:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
-    ap.add_argument("--workload", default="bert-base-len2-100", choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default="bert-base-len2-100",
+                    choices=list(synth.WORKLOADS) + list(synth.PREFIX_WORKLOADS))
     ap.add_argument("--profile-every", type=int, default=8,
                     help="time the kernels of every n-th batch with CUDA events (0 = off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
@@ -607,6 +810,8 @@ def main():
         return reference_arm(args)
     if args.kernel_bench:
         return kernel_bench(args)
+    if args.workload in synth.PREFIX_WORKLOADS:
+        return prefix_bench(args)
     return b200_arm(args)
 
 

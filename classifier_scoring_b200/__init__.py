@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
         "rm_create": (ctypes.c_int, [cfgp, P, SZ, ctypes.POINTER(P)]),
         "rm_create_shared": (ctypes.c_int, [P, ctypes.POINTER(P)]),
         "rm_score": (ctypes.c_int, [P, P, P, I32, P, P]),
+        "rm_score_prefix": (ctypes.c_int, [P, P, P, P, P, I32, P, P, P, P]),
         "rm_score_host": (ctypes.c_int, [P, P, P, I32, P, P]),
         "rm_schedule": (ctypes.c_int, [P, P, I32, P]),
         "rm_schedule_cfg": (ctypes.c_int, [cfgp, P, I32, P]),
@@ -189,6 +190,14 @@ class Scorer:
         off = _i32(offsets)
         _check(lib().rm_score(self._h, _ptr(ids_dev), off.ctypes.data, len(off) - 1, _ptr(out_dev),
                               _stream(stream)))
+
+    def score_prefix(self, ids_dev, prefix_len, n_cand, cand_len, out_dev, best_dev=None,
+                     logodds_dev=None, stream=None) -> None:
+        """rm_score_prefix: candidates sharing a prefix; host group layout, device ids/outputs."""
+        pl, nc, cl = _i32(prefix_len), _i32(n_cand), _i32(cand_len)
+        _check(lib().rm_score_prefix(self._h, _ptr(ids_dev), pl.ctypes.data, nc.ctypes.data,
+                                     cl.ctypes.data, len(pl), _ptr(out_dev), _ptr(best_dev),
+                                     _ptr(logodds_dev), _stream(stream)))
 
     def score_host(self, ids_host, offsets, out_host, stream=None) -> None:
         """rm_score_host: host ids/out (pinned for asynchronous copies)."""

@@ -182,19 +182,40 @@ struct rm_handle {
   struct ProfRec { int cls; double flops, bytes; cudaEvent_t a, b; };
   std::vector<ProfRec> prof;
   std::vector<cudaEvent_t> ev_pool;
+  // host scratch of rm_score_prefix's segment list (reused across calls)
+  std::vector<int32_t> px_off, px_start, px_len, px_out, px_goff;
 };
 
 namespace {
 
 // Metadata of one call in a staging slot / the device meta region:
-// offsets int32[n+1] | rb_off int32[n+1] | s_off int64[n+1]  (16-byte aligned parts)
+// offsets int32[n+1] | rb_off int32[n+1] | s_off int64[n+1]  (16-byte aligned
+// parts), then for shared-prefix calls pre_start int32[n] | pre_len int32[n] |
+// out_index int32[n] | group_off int32[n+1].  `base` bytes are copied for a
+// plain call, `bytes` for a shared-prefix call.
 struct MetaLayout {
-  int64_t rb, so, bytes;
+  int64_t rb, so, base, pst, pln, oix, gof, bytes;
   explicit MetaLayout(int64_t n) {
     rb = align_up(4 * (n + 1), 16);
     so = rb + align_up(4 * (n + 1), 16);
-    bytes = so + align_up(8 * (n + 1), 16);
+    base = so + align_up(8 * (n + 1), 16);
+    pst = base;
+    pln = pst + align_up(4 * n, 16);
+    oix = pln + align_up(4 * n, 16);
+    gof = oix + align_up(4 * n, 16);
+    bytes = gof + align_up(4 * (n + 1), 16);
   }
+};
+
+// Segments of a shared-prefix call (rm_score_prefix), host arrays.
+struct PrefixSpec {
+  const int32_t* pre_start;   // [n] packed row of the prefix a segment continues
+  const int32_t* pre_len;     // [n] its length (0 for a prefix or a plain segment)
+  const int32_t* out_index;   // [n] output slot of the segment's score, -1 for none
+  const int32_t* group_off;   // [n_groups + 1] candidate slots of each group
+  int32_t n_groups;
+  int32_t* d_best;            // device [n_groups] or NULL
+  float* d_logodds;           // device [n_groups] or NULL
 };
 
 int host_varlen_meta(const int32_t* off, int32_t n, int32_t nh, int32_t* rb, int64_t* so,
@@ -403,7 +424,8 @@ struct ProfScope {
 // host_ids != NULL: copy the ids host->device (into the arena) once the call
 // has been validated, and the scores back into host_out at the end.
 int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, const int32_t* offsets,
-               int32_t n, float* d_out, float* host_out, cudaStream_t st) {
+               int32_t n, float* d_out, float* host_out, cudaStream_t st,
+               const PrefixSpec* px = nullptr) {
   const rm_config* c = &h->cfg;
   if (n < 1) return set_error(RM_E_INVAL, "n_seqs must be >= 1");
   if (n > c->max_batch_seqs)
@@ -419,7 +441,7 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   int64_t* p_so = reinterpret_cast<int64_t*>(ps + ml.so);
   if (offsets[0] != 0) return set_error(RM_E_INVAL, "seq_offsets[0] must be 0");
   for (int32_t i = 0; i < n; ++i) {
-    const int64_t L = static_cast<int64_t>(offsets[i + 1]) - offsets[i];
+    const int64_t L = static_cast<int64_t>(offsets[i + 1]) - offsets[i] + (px ? px->pre_len[i] : 0);
     if (L < 1) return set_error(RM_E_INVAL, "sequence %d has length %lld (< 1)", i, (long long)L);
     if (L > c->max_len)
       return set_error(RM_E_RANGE, "sequence %d has length %lld > max_len %d", i, (long long)L,
@@ -438,11 +460,21 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
     d_ids = h->d_ids;
     d_out = h->d_scores;
   }
-  RM_CUDA(cudaMemcpyAsync(h->d_meta, ps, ml.bytes, cudaMemcpyHostToDevice, st));
+  if (px != nullptr) {
+    std::memcpy(ps + ml.pst, px->pre_start, 4 * static_cast<size_t>(n));
+    std::memcpy(ps + ml.pln, px->pre_len, 4 * static_cast<size_t>(n));
+    std::memcpy(ps + ml.oix, px->out_index, 4 * static_cast<size_t>(n));
+    std::memcpy(ps + ml.gof, px->group_off, 4 * static_cast<size_t>(px->n_groups + 1));
+  }
+  RM_CUDA(cudaMemcpyAsync(h->d_meta, ps, px != nullptr ? ml.bytes : ml.base, cudaMemcpyHostToDevice, st));
   RM_CUDA(cudaEventRecord(h->ev[slot], st));
   const int32_t* d_off = reinterpret_cast<const int32_t*>(h->d_meta);
   const int32_t* d_rb = reinterpret_cast<const int32_t*>(h->d_meta + ml.rb);
   const int64_t* d_so = reinterpret_cast<const int64_t*>(h->d_meta + ml.so);
+  const int32_t* d_pst = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.pst) : nullptr;
+  const int32_t* d_pln = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.pln) : nullptr;
+  const int32_t* d_oix = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.oix) : nullptr;
+  const int32_t* d_gof = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.gof) : nullptr;
 
   Bucket* bk = nullptr;
   RM_TRY(get_bucket(h, T, S, &bk));
@@ -469,7 +501,8 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   double att = 0;
   for (int32_t i = 0; i < n; ++i) {
     const double L = static_cast<double>(offsets[i + 1] - offsets[i]);
-    att += dec ? L * (L + 1) / 2 : L * L;
+    const double P0 = px ? px->pre_len[i] : 0;   // shared-prefix keys every row sees
+    att += dec ? L * P0 + L * (L + 1) / 2 : L * L;
   }
   att *= nh;
   const double Td = T, Hd = H, Fd = F;
@@ -497,7 +530,7 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   RM_KERNEL(RM_K_EMBED, 0, 6.0 * Td * Hd + 4.0 * Td,
             embed_launch(d_ids, d_off, n, T, h->emb_word, h->emb_pos, dec ? nullptr : h->ln_emb_g,
                          dec ? nullptr : h->ln_emb_b, eps, c->vocab, c->max_pos, H, x,
-                         h->d_err + ERR_CLAMPED, st, dec ? L2Prefetch{} : pf_qkv0));
+                         h->d_err + ERR_CLAMPED, st, dec ? L2Prefetch{} : pf_qkv0, d_pln));
   if (dec)
     RM_KERNEL(RM_K_LAYERNORM, 0, 4.0 * Td * Hd,
               res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps, 1, 2, st,
@@ -511,7 +544,10 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
         l + 1 < c->n_layers ? pf_of(h->layers[l + 1].w_qkv, w_qkv_b, nullptr, 0) : L2Prefetch{};
     RM_GEMM(gemm_flops(3 * Hd, Hd), gemm_bytes(3 * Hd, Hd),
             gemm(h, bk->a_in, L.tm[0], T, 3 * H, H, L.b_qkv, qkv, 0, st));
-    if (c->attn_impl == RM_ATTN_FUSED) {
+    if (px != nullptr) {
+      RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
+                attn_fused_prefix_launch(qkv, ctx, d_off, d_rb, d_pst, d_pln, n, nrb, nh, d, st, pf_o));
+    } else if (c->attn_impl == RM_ATTN_FUSED) {
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
                 attn_fused_launch(qkv, ctx, d_off, d_rb, n, nrb, nh, d, dec, st, pf_o));
     } else {
@@ -547,7 +583,10 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
     }
   }
   RM_KERNEL(RM_K_HEAD, 2.0 * n * Hd, 2.0 * n * Hd + 4.0 * n,
-            head_launch(dec ? z : x, d_off, n, h->w_r, h->b_r, H, dec ? 1 : 0, d_out, st));
+            head_launch(dec ? z : x, d_off, n, h->w_r, h->b_r, H, dec ? 1 : 0, d_out, st, d_oix));
+  if (px != nullptr && (px->d_best != nullptr || px->d_logodds != nullptr))
+    RM_KERNEL(RM_K_HEAD, 0, 4.0 * px->group_off[px->n_groups] + 8.0 * px->n_groups,
+              best_of_n_launch(d_out, d_gof, px->n_groups, px->d_best, px->d_logodds, st));
   if (host_out != nullptr)
     RM_CUDA(cudaMemcpyAsync(host_out, d_out, 4 * static_cast<size_t>(n), cudaMemcpyDeviceToHost, st));
   h->last_stream = st;
@@ -671,6 +710,61 @@ int rm_score(rm_handle* h, const int32_t* packed_token_ids, const int32_t* seq_o
     return set_error(RM_E_INVAL, "NULL argument");
   return score_impl(h, packed_token_ids, nullptr, seq_offsets, n_seqs, out_scores, nullptr,
                     static_cast<cudaStream_t>(stream));
+}
+
+int rm_score_prefix(rm_handle* h, const int32_t* packed_token_ids, const int32_t* prefix_len,
+                    const int32_t* n_cand, const int32_t* cand_len, int32_t n_groups,
+                    float* out_scores, int32_t* out_best, float* out_logodds, void* stream) {
+  if (h == nullptr || packed_token_ids == nullptr || prefix_len == nullptr || n_cand == nullptr ||
+      cand_len == nullptr || out_scores == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  const rm_config* c = &h->cfg;
+  if (c->arch != RM_DEC_PRELN)
+    return set_error(RM_E_INVAL, "prefix sharing needs the causal decoder: an encoder's prefix "
+                                 "tokens attend to the candidate");
+  if ((c->hidden / c->n_heads) % 8 != 0)
+    return set_error(RM_E_INVAL, "prefix sharing needs head_dim %% 8 == 0");
+  if (n_groups < 1) return set_error(RM_E_INVAL, "n_groups must be >= 1");
+  h->px_off.assign(1, 0);
+  h->px_start.clear();
+  h->px_len.clear();
+  h->px_out.clear();
+  h->px_goff.assign(1, 0);
+  int64_t tok = 0;
+  int32_t slot = 0, k = 0;
+  for (int32_t g = 0; g < n_groups; ++g) {
+    const int32_t P = prefix_len[g];
+    if (P < 0 || n_cand[g] < 1)
+      return set_error(RM_E_INVAL, "group %d: prefix length %d, %d candidates", g, P, n_cand[g]);
+    const int64_t pstart = tok;
+    if (P > 0) {   // the prefix itself: one causal segment, not scored
+      tok += P;
+      h->px_off.push_back(static_cast<int32_t>(std::min<int64_t>(tok, INT32_MAX)));
+      h->px_start.push_back(0);
+      h->px_len.push_back(0);
+      h->px_out.push_back(-1);
+    }
+    for (int32_t j = 0; j < n_cand[g]; ++j, ++k) {
+      const int32_t l = cand_len[k];
+      if (l < 1) return set_error(RM_E_INVAL, "candidate %d of group %d has length %d", j, g, l);
+      if (static_cast<int64_t>(P) + l > c->max_pos)
+        return set_error(RM_E_RANGE, "group %d candidate %d: %lld positions exceed max_pos %d", g,
+                         j, (long long)P + l, c->max_pos);
+      tok += l;
+      h->px_off.push_back(static_cast<int32_t>(std::min<int64_t>(tok, INT32_MAX)));
+      h->px_start.push_back(static_cast<int32_t>(pstart));
+      h->px_len.push_back(P);
+      h->px_out.push_back(slot++);
+    }
+    h->px_goff.push_back(slot);
+    if (tok > c->max_tokens) return set_error(RM_E_RANGE, "%lld tokens exceed max_tokens %d",
+                                              (long long)tok, c->max_tokens);
+  }
+  const int32_t n = static_cast<int32_t>(h->px_start.size());
+  PrefixSpec px{h->px_start.data(), h->px_len.data(), h->px_out.data(), h->px_goff.data(),
+                n_groups, out_best, out_logodds};
+  return score_impl(h, packed_token_ids, nullptr, h->px_off.data(), n, out_scores, nullptr,
+                    static_cast<cudaStream_t>(stream), &px);
 }
 
 int rm_score_host(rm_handle* h, const int32_t* host_token_ids, const int32_t* seq_offsets,

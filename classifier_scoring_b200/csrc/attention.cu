@@ -472,11 +472,17 @@ struct FusedSmem {
   static constexpr int kBytes = 5 * kTile * 2;   // Q, K x2, V x2
 };
 
-template <int DP>
+//
+// With PFX, segment i continues a shared prefix: its keys are the pre_len[i]
+// rows that start at packed row pre_start[i] (all visible), followed by its
+// own rows (causal), so query row r sees virtual keys 0 .. pre_len[i] + r.
+template <int DP, bool PFX>
 __global__ void __launch_bounds__(128)
     attn_fused_async_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ ctx,
                             const int32_t* __restrict__ offsets, const int32_t* __restrict__ rb_off,
-                            int n, int H, int d, float scale_log2, int causal, L2PrefetchArgs pf) {
+                            int n, int H, int d, float scale_log2, int causal, L2PrefetchArgs pf,
+                            const int32_t* __restrict__ pre_start,
+                            const int32_t* __restrict__ pre_len) {
   using FS = FusedSmem<DP>;
   constexpr int P = FS::kPitch;
   extern __shared__ __align__(16) uint8_t fsm_raw[];
@@ -490,15 +496,17 @@ __global__ void __launch_bounds__(128)
   const int i = upper_index(rb_off, n, b);
   const int t0 = offsets[i];
   const int L = offsets[i + 1] - t0;
+  const int P0 = PFX ? pre_len[i] : 0;                 // shared-prefix keys before the own rows
+  const int ps = PFX ? pre_start[i] : 0;
+  const int Lk = P0 + L;                               // keys of the segment
   const int row0 = (b - rb_off[i]) * 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const size_t H3 = 3 * static_cast<size_t>(H);
   const bf16* qb = qkv + static_cast<size_t>(t0) * H3 + hd * d;
-  const bf16* kb_ = qkv + static_cast<size_t>(t0) * H3 + H + hd * d;
-  const bf16* vb = qkv + static_cast<size_t>(t0) * H3 + 2 * H + hd * d;
+  const bf16* colb = qkv + hd * d;                     // head column base of row 0
   const int ra = row0 + warp * 16 + g, rb = ra + 8;
   const int row_end = min(L, row0 + 64);
-  const int kend = causal ? row_end : L;
+  const int kend = causal ? P0 + row_end : Lk;
   const int nkb = (kend + 63) / 64;
   const int wrow0 = row0 + warp * 16;
   const int wrow_last = min(wrow0 + 15, L - 1);
@@ -513,13 +521,26 @@ __global__ void __launch_bounds__(128)
       cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * P + c)), gsrc, ok);
     }
   };
+  // key/value rows kbase.. of the segment's key sequence (prefix rows first)
+  auto issue_kv = [&](bf16* dst, int coff, int kbase) {
+#pragma unroll
+    for (int k = 0; k < (64 * (DP / 8)) / 128; ++k) {
+      const int idx = threadIdx.x + k * 128;
+      const int r = idx / (DP / 8), c = (idx % (DP / 8)) * 8;
+      const int vr = kbase + r;
+      const bool ok = (vr < Lk) && (c < d);
+      const int grow = vr < P0 ? ps + vr : t0 + vr - P0;
+      const bf16* gsrc = ok ? colb + static_cast<size_t>(grow) * H3 + coff + c : colb;
+      cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * P + c)), gsrc, ok);
+    }
+  };
   issue(qs, qb, row0);
-  issue(kbuf, kb_, 0);
-  issue(vbuf, vb, 0);
+  issue_kv(kbuf, H, 0);
+  issue_kv(vbuf, 2 * H, 0);
   cp_async_commit();                                   // group 0: Q, K0, V0
   if (nkb > 1) {
-    issue(kbuf + FS::kTile, kb_, 64);
-    issue(vbuf + FS::kTile, vb, 64);
+    issue_kv(kbuf + FS::kTile, H, 64);
+    issue_kv(vbuf + FS::kTile, 2 * H, 64);
   }
   cp_async_commit();                                   // group 1: K1, V1 (may be empty)
   cp_async_wait_1();
@@ -549,7 +570,7 @@ __global__ void __launch_bounds__(128)
     }
     const bf16* ks = kbuf + buf * FS::kTile;
     const uint32_t vs_base = static_cast<uint32_t>(__cvta_generic_to_shared(vbuf + buf * FS::kTile));
-    if (!(wrow0 >= L || (causal && kb > wrow_last))) {
+    if (!(wrow0 >= L || (causal && kb > P0 + wrow_last))) {
       float sc[8][4];
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
@@ -561,7 +582,7 @@ __global__ void __launch_bounds__(128)
           mma_bf16_16816(sc[nt], qa[s], b0, b1);
         }
       }
-      const int lim_a = causal ? min(ra + 1, L) : L, lim_b = causal ? min(rb + 1, L) : L;
+      const int lim_a = causal ? min(P0 + ra + 1, Lk) : Lk, lim_b = causal ? min(P0 + rb + 1, Lk) : Lk;
       float bm_a = -INFINITY, bm_b = -INFINITY;
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
@@ -617,8 +638,8 @@ __global__ void __launch_bounds__(128)
     }
     __syncthreads();                                   // every warp is done with buffer buf
     if (j + 2 < nkb) {
-      issue(kbuf + buf * FS::kTile, kb_, kb + 128);
-      issue(vbuf + buf * FS::kTile, vb, kb + 128);
+      issue_kv(kbuf + buf * FS::kTile, H, kb + 128);
+      issue_kv(vbuf + buf * FS::kTile, 2 * H, kb + 128);
     }
     cp_async_commit();                                 // group j+2 (may be empty)
   }
@@ -645,10 +666,11 @@ __global__ void __launch_bounds__(128)
 
 int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 : -1)); }
 
-template <int DP>
+template <int DP, bool PFX>
 cudaError_t launch_fused_async(dim3 grid, cudaStream_t st, const bf16* q, bf16* c,
                                const int32_t* offsets, const int32_t* rb_off, int n, int H, int d,
-                               float scale_log2, int causal, const L2Prefetch& pf) {
+                               float scale_log2, int causal, const L2Prefetch& pf,
+                               const int32_t* pre_start = nullptr, const int32_t* pre_len = nullptr) {
   L2PrefetchArgs pa;
   for (int k = 0; k < 2; ++k) {
     pa.ptr[k] = pf.ptr[k];
@@ -656,14 +678,14 @@ cudaError_t launch_fused_async(dim3 grid, cudaStream_t st, const bf16* q, bf16* 
   }
   static bool configured = false;   // the attribute is per function; one device per process
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fused_async_kernel<DP>,
+    cudaError_t e = cudaFuncSetAttribute(attn_fused_async_kernel<DP, PFX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          FusedSmem<DP>::kBytes);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  launch_k(attn_fused_async_kernel<DP>, grid, dim3(128), FusedSmem<DP>::kBytes, st, q, c, offsets,
-           rb_off, n, H, d, scale_log2, causal, pa);
+  launch_k(attn_fused_async_kernel<DP, PFX>, grid, dim3(128), FusedSmem<DP>::kBytes, st, q, c,
+           offsets, rb_off, n, H, d, scale_log2, causal, pa, pre_start, pre_len);
   return cudaGetLastError();
 }
 
@@ -737,9 +759,9 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
   bf16* c = static_cast<bf16*>(ctx);
   if (head_dim % 8 == 0) {
     switch (pad_head_dim(head_dim)) {
-      case 32: return launch_fused_async<32>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
-      case 64: return launch_fused_async<64>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
-      case 128: return launch_fused_async<128>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
+      case 32: return launch_fused_async<32, false>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
+      case 64: return launch_fused_async<64, false>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
+      case 128: return launch_fused_async<128, false>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, causal, pf);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -750,6 +772,26 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+cudaError_t attn_fused_prefix_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                                     const int32_t* rb_off, const int32_t* pre_start,
+                                     const int32_t* pre_len, int n_seqs, int n_row_blocks,
+                                     int n_heads, int head_dim, cudaStream_t st,
+                                     const L2Prefetch& pf) {
+  if (n_row_blocks == 0) return cudaSuccess;
+  if (head_dim % 8 != 0) return cudaErrorInvalidValue;
+  const int H = n_heads * head_dim;
+  const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(head_dim));
+  dim3 grid(n_row_blocks, n_heads);
+  const bf16* q = static_cast<const bf16*>(qkv);
+  bf16* c = static_cast<bf16*>(ctx);
+  switch (pad_head_dim(head_dim)) {
+    case 32: return launch_fused_async<32, true>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, 1, pf, pre_start, pre_len);
+    case 64: return launch_fused_async<64, true>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, 1, pf, pre_start, pre_len);
+    case 128: return launch_fused_async<128, true>(grid, st, q, c, offsets, rb_off, n_seqs, H, head_dim, scale_log2, 1, pf, pre_start, pre_len);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,

@@ -43,13 +43,19 @@ struct L2Prefetch {
 cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs, int T,
                          const void* emb_word, const void* emb_pos, const float* ln_g,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
-                         int32_t* err_count, cudaStream_t st, const L2Prefetch& pf = {});
+                         int32_t* err_count, cudaStream_t st, const L2Prefetch& pf = {},
+                         const int32_t* pos_base = nullptr);
 // dtype: 0 fp32, 1 bf16; mode 0 post, 1 pre, 2 plain (see rm_ops.h)
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
                           int H, float eps, int dtype, int mode, cudaStream_t st,
                           const L2Prefetch& pf = {});
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
-                        float b_r, int H, int last_token, float* out, cudaStream_t st);
+                        float b_r, int H, int last_token, float* out, cudaStream_t st,
+                        const int32_t* out_index = nullptr);
+// per group g (candidates group_off[g]..group_off[g+1]-1 of scores): the
+// first highest score's index and r_1 - r_0
+cudaError_t best_of_n_launch(const float* scores, const int32_t* group_off, int n_groups,
+                             int32_t* best, float* logodds, cudaStream_t st);
 // weight conversion at create
 cudaError_t cvt_to_bf16_launch(const void* src, int src_dtype, void* dst, size_t n,
                                cudaStream_t st);
@@ -70,6 +76,15 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
                               const int32_t* rb_off, int n_seqs, int n_row_blocks, int n_heads,
                               int head_dim, int causal, cudaStream_t st,
                               const L2Prefetch& pf = {});
+// Causal fused attention over segments that may continue a shared prefix:
+// query row r of segment i attends to the pre_len[i] rows starting at packed
+// row pre_start[i] (all of them) and to rows 0..r of its own segment.
+// head_dim % 8 == 0, <= 128.
+cudaError_t attn_fused_prefix_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                                     const int32_t* rb_off, const int32_t* pre_start,
+                                     const int32_t* pre_len, int n_seqs, int n_row_blocks,
+                                     int n_heads, int head_dim, cudaStream_t st,
+                                     const L2Prefetch& pf = {});
 cudaError_t attn_context_launch(const void* S, const void* qkv, void* ctx, const int32_t* offsets,
                                 const int32_t* rb_off, const int64_t* s_off, int n_seqs,
                                 int n_row_blocks, int n_heads, int head_dim, int causal,

@@ -65,7 +65,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     embed_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ offsets, int n_seqs,
                  int T, const bf16* __restrict__ ew, const bf16* __restrict__ ep,
                  const float* __restrict__ g, const float* __restrict__ b, float eps, int V, int H,
-                 bf16* __restrict__ x, int32_t* __restrict__ err, L2PrefetchArgs pf) {
+                 bf16* __restrict__ x, int32_t* __restrict__ err, L2PrefetchArgs pf,
+                 const int32_t* __restrict__ pos_base) {
   pdl_launch_dependents();
   l2_prefetch_share(pf);   // static weights: no need to wait for the previous kernel
   pdl_wait();
@@ -73,7 +74,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
   const int i = upper_index(offsets, n_seqs, t);
-  const int pos = t - offsets[i];
+  // a segment that continues a shared prefix starts at position pos_base[i]
+  const int pos = t - offsets[i] + (pos_base != nullptr ? pos_base[i] : 0);
   int id = ids[t];
   if (id < 0 || id >= V) {
     if (lane == 0 && err != nullptr) atomicAdd(err, 1);
@@ -160,12 +162,16 @@ __global__ void __launch_bounds__(kWarps * 32)
 
 __global__ void __launch_bounds__(kWarps * 32)
     head_kernel(const bf16* __restrict__ x, const int32_t* __restrict__ offsets, int n,
-                const float* __restrict__ w, float br, int H, int last, float* __restrict__ out) {
+                const float* __restrict__ w, float br, int H, int last, float* __restrict__ out,
+                const int32_t* __restrict__ out_index) {
   pdl_launch_dependents();
   pdl_wait();
   const int i = blockIdx.x * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (i >= n) return;
+  // out_index maps segments to output slots; a negative slot is not scored
+  const int slot = out_index != nullptr ? out_index[i] : i;
+  if (slot < 0) return;
   const int t = last ? offsets[i + 1] - 1 : offsets[i];
   const bf16* xr = x + static_cast<size_t>(t) * H;
   float acc = 0.f;
@@ -177,7 +183,32 @@ __global__ void __launch_bounds__(kWarps * 32)
     for (int e = 0; e < 8; ++e) acc = fmaf(a[e], ww[e], acc);
   }
   acc = group_sum<32>(acc);
-  if (lane == 0) out[i] = acc + br;
+  if (lane == 0) out[slot] = acc + br;
+}
+
+// Best-of-N selection per group of candidates: best[g] = the index (within
+// the group) of the highest score, the first one on ties; logodds[g] =
+// r_1 - r_0, the log-odds that candidate 1 is preferred over candidate 0
+// under the reward model's pairwise comparison (0 for a single candidate).
+__global__ void __launch_bounds__(128)
+    best_of_n_kernel(const float* __restrict__ scores, const int32_t* __restrict__ group_off,
+                     int n_groups, int32_t* __restrict__ best, float* __restrict__ logodds) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int g = blockIdx.x * blockDim.x + threadIdx.x;
+  if (g >= n_groups) return;
+  const int a = group_off[g], e = group_off[g + 1];
+  int arg = 0;
+  float top = scores[a];
+  for (int k = a + 1; k < e; ++k) {
+    const float v = scores[k];
+    if (v > top) {
+      top = v;
+      arg = k - a;
+    }
+  }
+  if (best != nullptr) best[g] = arg;
+  if (logodds != nullptr) logodds[g] = e - a >= 2 ? scores[a + 1] - scores[a] : 0.0f;
 }
 
 template <typename S>
@@ -213,16 +244,17 @@ int pick_maxc(int H) {
 template <int MAXC>
 cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, const void* ew,
                     const void* ep, const float* g, const float* b, float eps, int V, int H,
-                    void* x, int32_t* err, cudaStream_t st, const L2Prefetch& pf) {
+                    void* x, int32_t* err, cudaStream_t st, const L2Prefetch& pf,
+                    const int32_t* pos_base) {
   dim3 grid((T + kWarps - 1) / kWarps);
   if (g != nullptr)
-    launch_k(embed_kernel<MAXC, true>, grid, kWarps * 32, 0, st, 
+    launch_k(embed_kernel<MAXC, true>, grid, kWarps * 32, 0, st,
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<bf16*>(x), err, pf_args(pf));
+        V, H, static_cast<bf16*>(x), err, pf_args(pf), pos_base);
   else
-    launch_k(embed_kernel<MAXC, false>, grid, kWarps * 32, 0, st, 
+    launch_k(embed_kernel<MAXC, false>, grid, kWarps * 32, 0, st,
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<bf16*>(x), err, pf_args(pf));
+        V, H, static_cast<bf16*>(x), err, pf_args(pf), pos_base);
   return cudaGetLastError();
 }
 
@@ -263,12 +295,13 @@ cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const floa
 cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs, int T,
                          const void* emb_word, const void* emb_pos, const float* ln_g,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
-                         int32_t* err_count, cudaStream_t st, const L2Prefetch& pf) {
+                         int32_t* err_count, cudaStream_t st, const L2Prefetch& pf,
+                         const int32_t* pos_base) {
   (void)P;
   if (T == 0) return cudaSuccess;
   const int maxc = pick_maxc(H);
   RMK_MAXC_SWITCH(maxc, (embed_t<M_>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps,
-                                     V, H, x, err_count, st, pf)))
+                                     V, H, x, err_count, st, pf, pos_base)))
 }
 
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
@@ -283,11 +316,20 @@ cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const
 }
 
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
-                        float b_r, int H, int last_token, float* out, cudaStream_t st) {
+                        float b_r, int H, int last_token, float* out, cudaStream_t st,
+                        const int32_t* out_index) {
   if (n_seqs == 0) return cudaSuccess;
   dim3 grid((n_seqs + kWarps - 1) / kWarps);
   launch_k(head_kernel, grid, kWarps * 32, 0, st, static_cast<const bf16*>(x), offsets, n_seqs, w_r,
-                                            b_r, H, last_token, out);
+           b_r, H, last_token, out, out_index);
+  return cudaGetLastError();
+}
+
+cudaError_t best_of_n_launch(const float* scores, const int32_t* group_off, int n_groups,
+                             int32_t* best, float* logodds, cudaStream_t st) {
+  if (n_groups == 0) return cudaSuccess;
+  launch_k(best_of_n_kernel, dim3((n_groups + 127) / 128), dim3(128), 0, st, scores, group_off,
+           n_groups, best, logodds);
   return cudaGetLastError();
 }
 

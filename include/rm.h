@@ -133,6 +133,34 @@ int rm_create_shared(const rm_handle* base, rm_handle** out);
 int rm_score(rm_handle* h, const int32_t* packed_token_ids, const int32_t* seq_offsets,
              int32_t n_seqs, float* out_scores, void* stream);
 
+/* Best-of-N / pairwise scoring of candidates that share a prefix, for the
+ * causal decoder (arch RM_DEC_PRELN): the reward model scores each summary
+ * of a post as the sequence post + summary, and the best-of-N policy keeps the
+ * highest-scoring one ("Learning to summarize from human feedback": reward
+ * model and best-of-N sections; the reward model's pairwise loss compares
+ * r_1 - r_0).  Because the decoder is causal, the prefix's hidden states do not
+ * depend on what follows, so each prefix is computed once and every candidate
+ * attends to its keys and values: the result equals rm_score on the N
+ * concatenations, with the prefix's work done once instead of N times.
+ *   packed_token_ids: device int32, per group g: the prefix (prefix_len[g]
+ *                     tokens, may be 0) then its n_cand[g] candidates in order.
+ *   prefix_len, n_cand: HOST int32[n_groups]; cand_len: HOST int32[sum n_cand],
+ *                     candidates of group 0 first; every prefix_len + cand_len
+ *                     in 1..max_len and <= max_pos.
+ *   out_scores:       device float[sum n_cand], score of each prefix + candidate.
+ *   out_best:         device int32[n_groups] or NULL: index within the group of
+ *                     the highest score (the first on ties).
+ *   out_logodds:      device float[n_groups] or NULL: r_1 - r_0 of the group's
+ *                     first two candidates (the log-odds that candidate 1 is
+ *                     preferred), 0 for a single candidate.
+ * The prefix and each candidate count as one sequence against max_batch_seqs.
+ * RM_E_INVAL for an encoder config, head_dim % 8 != 0, null pointers,
+ * n_groups < 1, a negative prefix length or an empty group or candidate;
+ * RM_E_RANGE for the limits above.  Asynchronous on stream; no allocation. */
+int rm_score_prefix(rm_handle* h, const int32_t* packed_token_ids, const int32_t* prefix_len,
+                    const int32_t* n_cand, const int32_t* cand_len, int32_t n_groups,
+                    float* out_scores, int32_t* out_best, float* out_logodds, void* stream);
+
 /* As rm_score, but token ids and scores are HOST buffers.  The ids are copied
  * host->device and the scores device->host on stream inside the call's
  * enqueued work; both host buffers should be pinned (cudaHostAlloc /

@@ -78,6 +78,42 @@ WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class PrefixWorkload:
+    """Best-of-N scoring: n_groups prefixes (posts), each followed by n_cand
+    candidates (summaries), lengths uniform on the stated integer ranges."""
+    name: str
+    shape: ModelShape
+    seed: int
+    n_groups: int
+    n_cand: int
+    prefix_lo: int
+    prefix_hi: int
+    cand_lo: int
+    cand_hi: int
+    weight_seed: int
+
+
+# TL;DR-shaped best-of-8: posts + summaries of at most 48 tokens, totals within
+# the 256..560 range of the gpt-1.3b-rm stream
+PREFIX_WORKLOADS = {
+    # the same weights as gpt-1.3b-rm (seed 4), its own requests (seed 5)
+    "gpt-1.3b-best-of-8": PrefixWorkload("gpt-1.3b-best-of-8", GPT_1P3B, 5, 8, 8, 208, 512, 24, 48, 4),
+}
+
+
+def make_prefix_groups(w: PrefixWorkload, seed_offset: int = 0):
+    """(ids, prefix_len, n_cand, cand_len) in the packed shared-prefix layout:
+    per group its prefix, then its candidates."""
+    seed = w.seed + seed_offset
+    prefix_len = make_lengths(w.n_groups, w.prefix_lo, w.prefix_hi, seed)
+    cand_len = make_lengths(w.n_groups * w.n_cand, w.cand_lo, w.cand_hi, seed + 7919)
+    n_cand = np.full(w.n_groups, w.n_cand, dtype=np.int32)
+    total = int(prefix_len.astype(np.int64).sum() + cand_len.astype(np.int64).sum())
+    ids = make_token_ids(total, w.shape.vocab, seed)
+    return ids, prefix_len, n_cand, cand_len
+
+
 def weight_segments(s: ModelShape) -> List[Tuple[str, Tuple[int, ...], str]]:
     """(name, shape, kind) of every tensor in flat-buffer order.
 

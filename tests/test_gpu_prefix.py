@@ -1,0 +1,117 @@
+"""Shared-prefix best-of-N / pairwise scoring (rm_score_prefix) against the
+oracle, which scores every prefix + candidate as its own sequence, and
+against rm_score on the same concatenations."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import classifier_scoring_b200 as rm
+from oracle import best_of_n as B
+from tests.helpers import SCORE_ATOL, config_for, oracle_model
+
+pytestmark = pytest.mark.gpu
+
+DEC = synth.ModelShape(synth.DEC_PRELN, 3, 256, 4, 1024, 5000, 600, synth.W_BF16, synth.GELU_ERF, 1e-5)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.init()
+
+
+@pytest.fixture(scope="module")
+def flat():
+    return synth.make_weights(DEC, 9)
+
+
+@pytest.fixture(scope="module")
+def scorer(flat):
+    cfg = config_for(DEC, max_batch_seqs=32, max_tokens=4096, max_len=600)
+    with rm.Scorer(cfg, flat) as sc:
+        yield sc
+
+
+def layout(prefix_len, n_cand, seed):
+    rng = np.random.default_rng(seed)
+    cand_len = rng.integers(1, 90, int(np.sum(n_cand)))
+    T = int(np.sum(prefix_len) + cand_len.sum())
+    ids = synth.make_token_ids(T, DEC.vocab, seed + 1)
+    return ids, cand_len
+
+
+def run_prefix(sc, ids, prefix_len, n_cand, cand_len):
+    nc, ng = int(np.sum(n_cand)), len(n_cand)
+    ids_d = torch.from_numpy(ids.astype(np.int32)).cuda()
+    out = torch.full((nc,), float("nan"), device="cuda")
+    best = torch.full((ng,), -7, dtype=torch.int32, device="cuda")
+    lo = torch.full((ng,), float("nan"), device="cuda")
+    sc.score_prefix(ids_d, prefix_len, n_cand, cand_len, out, best, lo)
+    torch.cuda.synchronize()
+    return (out.cpu().numpy().astype(np.float64), best.cpu().numpy(),
+            lo.cpu().numpy().astype(np.float64))
+
+
+def concatenations(ids, prefix_len, n_cand, cand_len):
+    seqs = [np.concatenate([p, c]) for p, cs in B.split_groups(ids, prefix_len, n_cand, cand_len)
+            for c in cs]
+    return np.concatenate(seqs).astype(np.int32), synth.offsets_from_lengths([len(s) for s in seqs])
+
+
+# prefixes across 64-row blocks, a group without prefix, single-candidate groups,
+# candidates longer than one 64-row block
+CASES = {
+    "mixed": ([37, 0, 64, 130, 1], [3, 1, 2, 4, 2]),
+    "pairs": ([200, 90, 5], [2, 2, 2]),
+    "long-prefix": ([500], [5]),
+}
+
+
+@pytest.mark.parametrize("case", list(CASES))
+def test_prefix_scores_match_oracle_and_unshared_path(scorer, flat, case):
+    prefix_len, n_cand = CASES[case]
+    ids, cand_len = layout(prefix_len, n_cand, 31 + len(case))
+    if case == "long-prefix":
+        cand_len = np.minimum(cand_len, 100)
+        ids = ids[:int(np.sum(prefix_len) + cand_len.sum())]
+    got, best, lo = run_prefix(scorer, ids, prefix_len, n_cand, cand_len)
+    ref = B.score_candidates(oracle_model(DEC, flat), ids, prefix_len, n_cand, cand_len)
+    assert np.max(np.abs(got - ref)) <= SCORE_ATOL
+    # the same concatenations through rm_score: same arithmetic, prefix recomputed per candidate
+    cat_ids, cat_off = concatenations(ids, prefix_len, n_cand, cand_len)
+    plain = torch.full((len(cat_off) - 1,), float("nan"), device="cuda")
+    scorer.score(torch.from_numpy(cat_ids).cuda(), cat_off, plain)
+    torch.cuda.synchronize()
+    assert np.max(np.abs(got - plain.cpu().numpy())) <= 2e-3
+    # selection on the kernel's own fp32 scores: the oracle's rule, same decision
+    b_ref, lo_ref = B.select(got, n_cand)
+    assert best.tolist() == b_ref.tolist()
+    assert np.allclose(lo, lo_ref, rtol=1e-6, atol=1e-6)
+
+
+def test_best_and_logodds_are_optional(scorer):
+    prefix_len, n_cand = [10, 20], [2, 3]
+    ids, cand_len = layout(prefix_len, n_cand, 41)
+    ids_d = torch.from_numpy(ids.astype(np.int32)).cuda()
+    out = torch.empty(5, device="cuda")
+    scorer.score_prefix(ids_d, prefix_len, n_cand, cand_len, out)
+    torch.cuda.synchronize()
+    full, _, _ = run_prefix(scorer, ids, prefix_len, n_cand, cand_len)
+    assert np.array_equal(out.cpu().numpy().astype(np.float64), full)
+
+
+def test_invalid_prefix_calls(scorer, flat):
+    ids_d = torch.zeros(64, dtype=torch.int32, device="cuda")
+    out = torch.empty(4, device="cuda")
+    with pytest.raises(rm.RmError):                       # an empty candidate
+        scorer.score_prefix(ids_d, [3], [2], [0, 2], out)
+    with pytest.raises(rm.RmError):                       # a group without candidates
+        scorer.score_prefix(ids_d, [3], [0], [], out)
+    with pytest.raises(rm.RmError):                       # prefix + candidate beyond max_len
+        scorer.score_prefix(ids_d, [590], [1], [20], out)
+    enc = synth.TINY
+    with rm.Scorer(config_for(enc), synth.make_weights(enc, 0)) as e:
+        with pytest.raises(rm.RmError):                   # the encoder's prefix sees the candidate
+            e.score_prefix(ids_d, [3], [1], [2], out)
