@@ -90,3 +90,59 @@ def test_stable_sort_breaks_length_ties_by_index():
 def test_empty_queue():
     batch, c = S.schedule_dp(np.array([], dtype=np.int32), 4, S.linear_cost(1, 1))
     assert batch.size == 0 and c == 0
+
+
+# --- latency-aware variants -------------------------------------------------------
+
+def test_compositions_count():
+    assert [len(list(S.compositions(n))) for n in range(1, 8)] == [2 ** (n - 1) for n in range(1, 8)]
+
+
+def test_latency_and_cap_worked_example():
+    """Four requests of length 5, T(b, L) = 2 + b*L, Bmax 4.  By hand:
+    throughput puts all four in one batch (cost 22); summed completion times
+    of the eight batchings of the sorted queue are [4] 88, [3,1] 75, [1,3] 79,
+    [2,2] 72, [2,1,1] 69, [1,2,1] 71, [1,1,2] 73, [1,1,1,1] 70, so the latency
+    objective takes [2,1,1]; a cap of 15 forbids 22 and 17, so throughput
+    takes [2,2] (24)."""
+    lens = np.array([5, 5, 5, 5])
+    cost = S.linear_cost(2, 1)
+    b, c = S.schedule_dp(lens, 4, cost)
+    assert b.tolist() == [0, 0, 0, 0] and c == 22
+    b, c = S.schedule_dp(lens, 4, cost, objective=S.LATENCY)
+    assert b.tolist() == [0, 0, 1, 2] and c == 69
+    assert S.latency_cost(lens, b, cost) == 69
+    b, c = S.schedule_dp(lens, 4, cost, max_cost=15)
+    assert b.tolist() == [0, 0, 1, 1] and c == 24
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_latency_dp_equals_enumeration_of_sorted_batchings(seed):
+    rng = np.random.default_rng(100 + seed)
+    n = int(rng.integers(1, 11))
+    lens = rng.integers(1, 30, n)
+    bmax = int(rng.integers(1, n + 1))
+    cost = S.linear_cost(int(rng.integers(0, 60)), int(rng.integers(0, 4)))
+    cap = int(rng.integers(0, 120)) if seed % 2 else 0
+    b, c = S.schedule_dp(lens, bmax, cost, objective=S.LATENCY, max_cost=cap)
+    assert c == S.brute_force_sorted(lens, bmax, cost, S.LATENCY, cap)
+    assert c == S.latency_cost(lens, b, cost)
+    # the batches are consecutive runs of the sorted queue, numbered in order
+    order = S.sorted_order(lens)
+    assert np.all(np.diff(b[order]) >= 0) and np.all(np.diff(b[order]) <= 1)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_capped_throughput_dp_equals_exhaustive_search(seed):
+    rng = np.random.default_rng(200 + seed)
+    n = int(rng.integers(1, 9))
+    lens = rng.integers(1, 12, n)
+    bmax = int(rng.integers(1, n + 1))
+    cost = S.linear_cost(int(rng.integers(0, 30)), int(rng.integers(1, 4)))
+    cap = int(rng.integers(1, 80))
+    b, c = S.schedule_dp(lens, bmax, cost, max_cost=cap)
+    assert c == S.brute_force_cost(lens, bmax, cost, max_cost=cap)
+    assert c == S.schedule_cost(lens, b, cost)
+    for k in np.unique(b):
+        members = lens[b == k]
+        assert len(members) == 1 or cost(len(members), int(members.max())) <= cap
