@@ -784,6 +784,127 @@ def prefix_bench(args):
     return 0
 
 
+def serve_bench(args):
+    """Open-loop serving of the request stream with Poisson arrivals at
+    fractions of the saturation rate: whenever the GPU is idle, the host takes
+    every queued request, schedules the queue with the DP (throughput or
+    latency objective) and launches its batches through rm_score_host (ids
+    from pinned host memory, scores back).  Latency = batch completion (CUDA
+    event) - arrival.  One GPU; the saturation rate is measured first with
+    every request queued at t = 0."""
+    import torch
+    import classifier_scoring_b200 as rm
+    from classifier_scoring_b200 import build as rmbuild
+
+    rank, world, local = rank_env()
+    if world > 1:
+        raise SystemExit("--serve runs on one GPU")
+    torch.cuda.set_device(local)
+    rmbuild.build()
+    w = synth.WORKLOADS[args.workload]
+    s = w.shape
+    st = synth.make_stream(w)
+    n = len(st.lengths)
+    max_len = min(s.max_pos, 1024, max(w.len_hi, int(st.lengths.max())))
+    flat = synth.make_weights(s, w.seed)
+
+    def make_cfg(objective, cap):
+        return rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
+                                ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos,
+                                weight_dtype=s.weight_dtype, gelu=s.gelu, ln_eps=s.ln_eps,
+                                max_batch_seqs=w.max_batch, max_tokens=w.max_batch * max_len,
+                                max_len=max_len, sched_max_batch=w.max_batch, sched_c0=SCHED_C0,
+                                sched_c1=SCHED_C1, sched_objective=objective, sched_max_cost=cap)
+    # schedulers: the handle's own DP with each objective (host-only configs)
+    sched_cfgs = {"throughput": make_cfg(rm.SCHED_THROUGHPUT, 0),
+                  "latency": make_cfg(rm.SCHED_LATENCY, 0)}
+    sc = rm.Scorer(make_cfg(rm.SCHED_THROUGHPUT, 0), flat)
+    del flat
+    stream = torch.cuda.Stream()
+    total_tok = int(st.lengths.astype(np.int64).sum())
+    ids_pin = torch.empty(total_tok, dtype=torch.int32).pin_memory()
+    out_pin = torch.empty(n, dtype=torch.float32).pin_memory()
+    ids_np = ids_pin.numpy()
+
+    def run(arrivals, sched_name, warm=False):
+        cfg = sched_cfgs[sched_name]
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        nxt, queue, last_ev = 0, [], None
+        log = []                                     # (event, request indices)
+        windows = 0
+        while nxt < n or queue:
+            now = time.perf_counter() - t0
+            while nxt < n and arrivals[nxt] <= now:
+                queue.append(nxt)
+                nxt += 1
+            idle = last_ev is None or last_ev.query()
+            if queue and idle:
+                q = np.array(queue, dtype=np.int64)
+                queue = []
+                windows += 1
+                batch = rm.schedule(cfg, st.lengths[q])
+                tok, oc = 0, 0
+                for b in range(int(batch.max()) + 1):
+                    members = q[batch == b]
+                    lens = st.lengths[members]
+                    off = synth.offsets_from_lengths(lens)
+                    k = int(off[-1])
+                    np.concatenate([st.ids[st.starts[i]:st.starts[i] + st.lengths[i]] for i in members],
+                                   out=ids_np[tok:tok + k])
+                    sc.score_host(ids_pin[tok:], off, out_pin[oc:], stream)
+                    oc += len(members)
+                    ev = torch.cuda.Event(enable_timing=True)
+                    ev.record(stream)
+                    log.append((ev, members))
+                    tok += k
+                last_ev = log[-1][0]
+            elif not queue and nxt < n and idle:
+                time.sleep(max(0.0, min(arrivals[nxt] - now, 2e-4)))
+        torch.cuda.synchronize()
+        lat = np.empty(n)
+        done = np.empty(n)
+        for ev, members in log:
+            t_done = ev0.elapsed_time(ev) / 1000.0
+            done[members] = t_done
+            lat[members] = t_done - arrivals[members]
+        span = float(done.max() - arrivals.min())
+        return {"completed_per_s": n / span, "p50_ms": 1000 * float(np.median(lat)),
+                "p99_ms": 1000 * float(np.percentile(lat, 99)), "mean_ms": 1000 * float(lat.mean()),
+                "max_ms": 1000 * float(lat.max()), "windows": windows, "batches": len(log)}
+
+    zero = np.zeros(n)
+    for _ in range(args.warmup):
+        run(zero, "throughput")
+    sat = run(zero, "throughput")
+    sat_rate = sat["completed_per_s"]
+    results = []
+    for frac in (0.5, 0.9):
+        arrivals = synth.make_arrivals(n, frac * sat_rate, w.seed)
+        arrivals -= arrivals[0]
+        for name in ("throughput", "latency"):
+            r = run(arrivals, name)
+            r.update({"rate_frac": frac, "rate_req_s": frac * sat_rate, "objective": name})
+            results.append(r)
+    head = next(r for r in results if r["rate_frac"] == 0.9 and r["objective"] == "latency")
+    line = {"metric": "p99 latency at 0.9x of the saturation rate, Poisson arrivals (BERT-base, len 2-100)",
+            "value": head["p99_ms"], "unit": "ms", "n_gpus": 1, "steps": 1, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "requests": n, "arrivals": "Poisson (exponential gaps)",
+                       "policy": "when the GPU is idle, schedule every queued request with the DP and "
+                                 "launch its batches (rm_score_host, pinned host ids)",
+                       "scheduler_cost": f"T(b,L) = {SCHED_C0} + {SCHED_C1}*b*L"},
+            "saturation": {"completed_per_s": sat_rate, "p50_ms": sat["p50_ms"], "p99_ms": sat["p99_ms"],
+                           "batches": sat["batches"]},
+            "serving": results,
+            "context": {"turbotransformers_mean_latency_ms_at_402_req_s": 7.49}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -800,6 +921,9 @@ def main():
                     help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
     ap.add_argument("--lanes", type=int, default=2,
                     help="handles sharing the weights, one stream each, batches dealt round-robin")
+    ap.add_argument("--serve", action="store_true",
+                    help="open-loop Poisson serving at 0.5x and 0.9x of the saturation rate, "
+                         "throughput vs latency DP objective (p50/p99)")
     ap.add_argument("--batch-index", type=int, default=None,
                     help="score only this DP batch of the stream per step (small profiling case)")
     args = ap.parse_args()
@@ -812,6 +936,8 @@ def main():
         return kernel_bench(args)
     if args.workload in synth.PREFIX_WORKLOADS:
         return prefix_bench(args)
+    if args.serve:
+        return serve_bench(args)
     return b200_arm(args)
 
 

@@ -22,6 +22,7 @@ F32, BF16 = 0, 1
 GELU_ERF, GELU_TANH = 0, 1
 ATTN_FUSED, ATTN_MATERIALIZED = 0, 1
 RM_OK, RM_E_INVAL, RM_E_NOMEM, RM_E_CUDA, RM_E_RANGE, RM_E_DEVICE = 0, -1, -2, -3, -4, -5
+SCHED_THROUGHPUT, SCHED_LATENCY = 0, 1
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmscore.so")
 
@@ -42,16 +43,17 @@ class RmConfig(ctypes.Structure):
         ("sched_max_batch", ctypes.c_int32), ("sched_c0", ctypes.c_int64), ("sched_c1", ctypes.c_int64),
         ("sched_table", ctypes.POINTER(ctypes.c_int64)), ("sched_table_b", ctypes.c_int32),
         ("sched_table_l", ctypes.c_int32), ("attn_impl", ctypes.c_int32),
+        ("sched_objective", ctypes.c_int32), ("sched_max_cost", ctypes.c_int64),
     ]
 
     @classmethod
     def make(cls, *, arch, n_layers, hidden, n_heads, ffn, vocab, max_pos, weight_dtype,
              gelu=GELU_ERF, ln_eps=1e-12, max_batch_seqs=64, max_tokens=8192, max_len=512,
              sched_max_batch=64, sched_c0=0, sched_c1=1, sched_table=None,
-             attn_impl=0) -> "RmConfig":
+             attn_impl=0, sched_objective=0, sched_max_cost=0) -> "RmConfig":
         c = cls(arch, n_layers, hidden, n_heads, ffn, vocab, max_pos, weight_dtype, gelu, ln_eps,
                 max_batch_seqs, max_tokens, max_len, sched_max_batch, sched_c0, sched_c1, None, 0, 0,
-                attn_impl)
+                attn_impl, sched_objective, sched_max_cost)
         if sched_table is not None:
             t = np.ascontiguousarray(sched_table, dtype=np.int64)
             c._table_keepalive = t

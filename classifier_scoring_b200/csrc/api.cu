@@ -46,6 +46,9 @@ int validate_config(const rm_config* c, bool sched_only, const char** why) {
   if (c->sched_max_batch < 1) return bad("sched_max_batch must be >= 1");
   if (c->sched_c0 < 0 || c->sched_c1 < 0 || c->sched_c0 > (1LL << 40) || c->sched_c1 > (1LL << 40))
     return bad("sched_c0 and sched_c1 must be in 0..2^40");
+  if (c->sched_objective != RM_SCHED_THROUGHPUT && c->sched_objective != RM_SCHED_LATENCY)
+    return bad("sched_objective must be 0 or 1");
+  if (c->sched_max_cost < 0) return bad("sched_max_cost must be >= 0");
   if (c->sched_table != nullptr) {
     if (c->sched_table_b < c->sched_max_batch || c->sched_table_l < c->max_len)
       return bad("sched_table must have >= sched_max_batch rows and >= max_len columns");
@@ -81,6 +84,8 @@ int validate_config(const rm_config* c, bool sched_only, const char** why) {
 SchedCost sched_cost_from(const rm_config* c) {
   SchedCost s;
   s.bmax = c->sched_max_batch;
+  s.objective = c->sched_objective;
+  s.max_cost = c->sched_max_cost;
   s.c0 = c->sched_c0;
   s.c1 = c->sched_c1;
   if (c->sched_table != nullptr) {

@@ -12,6 +12,8 @@ namespace rmk {
 // ---- DP scheduler cost model ----
 struct SchedCost {
   int32_t bmax = 1;
+  int32_t objective = 0;        // RM_SCHED_THROUGHPUT | RM_SCHED_LATENCY
+  int64_t max_cost = 0;         // 0 = no cap on a batch of >= 2 requests
   int64_t c0 = 0, c1 = 0;
   std::vector<int64_t> table;   // [tb][tl] row-major, empty = linear model
   int32_t tb = 0, tl = 0;

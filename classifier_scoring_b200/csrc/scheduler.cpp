@@ -10,6 +10,12 @@
 //   non-decreasing in L); best[i] = min over the last batch (j, i] of
 //   best[j] + T(i - j, l_i) with i - j <= Bmax, ties to the smallest j;
 //   batches are numbered in execution order (ascending longest length).
+// Latency-aware variants (the review's main results report the scheduler's
+// mean latency at its serving rate): with objective RM_SCHED_LATENCY a batch
+// that starts at sorted position j is charged T * (n - j), the delay it adds
+// to every request from j on, so the DP minimises the sum of completion times
+// of batches run back to back in ascending longest length; with max_cost > 0
+// no batch of two or more requests may cost more than max_cost.
 // Costs are summed in 128-bit integers so no queue can overflow them.
 #include "host.h"
 
@@ -33,7 +39,12 @@ int schedule_dp(const SchedCost& cost, const int32_t* lengths, int32_t n, int32_
     __int128 b = -1;
     int32_t arg = j0;
     for (int32_t j = j0; j < i; ++j) {
-      const __int128 c = best[j] + static_cast<__int128>(cost.eval(i - j, longest));
+      const int64_t t = cost.eval(i - j, longest);
+      if (cost.max_cost > 0 && i - j >= 2 && t > cost.max_cost) continue;
+      const __int128 w = cost.objective == RM_SCHED_LATENCY
+                             ? static_cast<__int128>(t) * (n - j)
+                             : static_cast<__int128>(t);
+      const __int128 c = best[j] + w;
       if (b < 0 || c < b) {
         b = c;
         arg = j;

@@ -66,6 +66,16 @@ extern "C" {
 #define RM_ATTN_FUSED        0
 #define RM_ATTN_MATERIALIZED 1
 
+/* rm_config.sched_objective.  THROUGHPUT minimises the total time of the
+ * queue's batches.  LATENCY minimises the sum of the queued requests'
+ * completion times when the batches run back to back in ascending longest
+ * length: a batch that starts at sorted position j delays the n - j requests
+ * from j on, so dp[i] = min_j dp[j] + T(i-j, l_i) * (n - j).  The
+ * TurboTransformers review's main results report the scheduler's mean
+ * latency at its serving rate; this objective targets that figure directly. */
+#define RM_SCHED_THROUGHPUT 0
+#define RM_SCHED_LATENCY    1
+
 typedef struct rm_handle rm_handle;
 
 typedef struct rm_config {
@@ -90,6 +100,10 @@ typedef struct rm_config {
   int32_t sched_table_b;         /*   sched_table_b >= Bmax rows, sched_table_l >=    */
   int32_t sched_table_l;         /*   max_len columns, non-decreasing along L; copied */
   int32_t attn_impl;             /* RM_ATTN_FUSED (default) | RM_ATTN_MATERIALIZED    */
+  /* latency-aware scheduling (rm_schedule) */
+  int32_t sched_objective;       /* RM_SCHED_THROUGHPUT (default) | RM_SCHED_LATENCY  */
+  int64_t sched_max_cost;        /* 0 = no cap; else every batch of >= 2 requests     */
+                                 /*   costs at most this (single requests always ok) */
 } rm_config;
 
 /* Number of bytes the flat weights buffer must hold for cfg.

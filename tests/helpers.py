@@ -11,7 +11,7 @@ F32_RTOL = 1e-5
 
 def config_for(shape: synth.ModelShape, *, max_batch_seqs=64, max_tokens=8192, max_len=None,
                sched_max_batch=64, sched_c0=0, sched_c1=1, sched_table=None,
-               attn_impl=0) -> RmConfig:
+               attn_impl=0, sched_objective=0, sched_max_cost=0) -> RmConfig:
     if max_len is None:
         max_len = min(shape.max_pos, 1024)
     return RmConfig.make(arch=shape.arch, n_layers=shape.n_layers, hidden=shape.hidden,
@@ -19,7 +19,8 @@ def config_for(shape: synth.ModelShape, *, max_batch_seqs=64, max_tokens=8192, m
                          max_pos=shape.max_pos, weight_dtype=shape.weight_dtype, gelu=shape.gelu,
                          ln_eps=shape.ln_eps, max_batch_seqs=max_batch_seqs, max_tokens=max_tokens,
                          max_len=max_len, sched_max_batch=sched_max_batch, sched_c0=sched_c0,
-                         sched_c1=sched_c1, sched_table=sched_table, attn_impl=attn_impl)
+                         sched_c1=sched_c1, sched_table=sched_table, attn_impl=attn_impl,
+                         sched_objective=sched_objective, sched_max_cost=sched_max_cost)
 
 
 def oracle_model(shape: synth.ModelShape, flat):

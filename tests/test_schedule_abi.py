@@ -14,9 +14,10 @@ def built():
     build.build()
 
 
-def sched_cfg(bmax, c0, c1, max_len, table=None):
+def sched_cfg(bmax, c0, c1, max_len, table=None, objective=0, max_cost=0):
     return config_for(synth.BERT_BASE, max_len=max_len, sched_max_batch=bmax, sched_c0=c0,
-                      sched_c1=c1, sched_table=table)
+                      sched_c1=c1, sched_table=table, sched_objective=objective,
+                      sched_max_cost=max_cost)
 
 
 @pytest.mark.parametrize("name", ["bert-base-len2-100", "bert-base-len5-500"])
@@ -64,3 +65,35 @@ def test_empty_queue_and_errors():
     bad = np.tile(np.arange(100, 0, -1, dtype=np.int64), (4, 1))     # decreasing along L
     with pytest.raises(rm.RmError):
         rm.schedule(sched_cfg(4, 0, 0, 100, bad), [3])
+
+
+@pytest.mark.parametrize("objective", [S.THROUGHPUT, S.LATENCY], ids=["throughput", "latency"])
+@pytest.mark.parametrize("cap", [0, 30000, 120000])
+def test_latency_objective_and_cap_bit_exact_on_the_stream(objective, cap):
+    w = synth.WORKLOADS["bert-base-len2-100"]
+    lengths = synth.make_stream(w, 3000).lengths
+    ours = rm.schedule(sched_cfg(64, 20000, 1, 512, objective=objective, max_cost=cap), lengths)
+    ref, _ = S.schedule_dp(lengths, 64, S.linear_cost(20000, 1), objective=objective, max_cost=cap)
+    assert np.array_equal(ours, ref)
+
+
+def test_latency_objective_small_queues_bit_exact():
+    rng = np.random.default_rng(5)
+    for n in range(1, 10):
+        for _ in range(4):
+            lengths = rng.integers(1, 6, size=n)
+            bmax = int(rng.integers(1, n + 1))
+            c0, c1 = int(rng.integers(0, 20)), int(rng.integers(0, 4))
+            cap = int(rng.integers(0, 40))
+            cost = S.linear_cost(c0, c1)
+            for objective in (S.THROUGHPUT, S.LATENCY):
+                ours = rm.schedule(sched_cfg(bmax, c0, c1, 8, objective=objective, max_cost=cap), lengths)
+                ref, c = S.schedule_dp(lengths, bmax, cost, objective=objective, max_cost=cap)
+                assert np.array_equal(ours, ref)
+
+
+def test_latency_knobs_are_validated():
+    with pytest.raises(rm.RmError):
+        rm.schedule(sched_cfg(4, 1, 1, 100, objective=2), [3])
+    with pytest.raises(rm.RmError):
+        rm.schedule(sched_cfg(4, 1, 1, 100, max_cost=-1), [3])
