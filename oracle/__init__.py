@@ -15,6 +15,8 @@ Contents:
                search over all set partitions for small queues.
   best_of_n -- best-of-N / pairwise scoring of candidates that share a
                prefix, each scored as its own concatenated sequence.
+  ensemble  -- majority vote of scorer replicas ("experts") on the binary
+               class of their scores.
 
 Every function cites the page passage it follows.  Pins (tests that check
 this package against something other than itself) live in
