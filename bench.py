@@ -905,6 +905,112 @@ def serve_bench(args):
     return 0
 
 
+def ensemble_bench(args):
+    """Batch-1 latency of one expert and of a K-expert ensemble with majority
+    vote on one GPU (the experts run on their own streams at once), per
+    input length, over 1000 requests after 50 warm-up requests.  Each request
+    is timed from an idle GPU to its decision (CUDA events, synchronised per
+    request), so host launch time counts."""
+    import torch
+    import classifier_scoring_b200 as rm
+    from classifier_scoring_b200 import build as rmbuild
+    from classifier_scoring_b200.ensemble import Ensemble
+
+    rank, world, local = rank_env()
+    if world > 1:
+        raise SystemExit("--ensemble runs on one GPU")
+    torch.cuda.set_device(local)
+    rmbuild.build()
+    w = synth.WORKLOADS[args.workload]
+    s = w.shape
+    K = args.ensemble
+    lengths = list(w.fixed_lengths) or [int(w.len_lo), int(w.len_hi)]
+    max_len = max(lengths)
+    cfg = rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
+                           ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos, weight_dtype=s.weight_dtype,
+                           gelu=s.gelu, ln_eps=s.ln_eps, max_batch_seqs=1, max_tokens=max_len,
+                           max_len=max_len, sched_max_batch=1)
+    experts = [rm.Scorer(cfg, synth.make_weights(s, w.seed + 1000 * k)) for k in range(K)]
+    ens = Ensemble(experts)
+    main = torch.cuda.Stream()
+    scores = torch.zeros(K, 1, device="cuda")
+    dec = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n_warm, n_req = 50, 1000
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def lat_of(fn):
+        out = np.empty(n_req)
+        for r in range(n_warm + n_req):
+            torch.cuda.synchronize()
+            a.record(main)
+            fn()
+            b.record(main)
+            b.synchronize()
+            if r >= n_warm:
+                out[r - n_warm] = a.elapsed_time(b)
+        return out
+
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    out_dir = os.path.join(ROOT, "gpurun_out")
+    clocks = ClockSampler(gpu_index, os.path.join(out_dir, "clocks_ensemble.csv")
+                          if os.path.isdir(out_dir) else None)
+    time.sleep(0.3)
+    l0 = sum(e.profile_read()["total_launches"] for e in experts)
+    rows = []
+    for L in lengths:
+        ids = torch.from_numpy(synth.make_token_ids(L, s.vocab, w.seed + L)).cuda()
+        off = np.array([0, L], dtype=np.int32)
+        one = lat_of(lambda: experts[0].score(ids, off, scores[0], main))
+        many = lat_of(lambda: ens.score_and_vote(ids, off, scores, dec, stream=main))
+        # the same two calls captured once into CUDA graphs (rm_plan: kernels only)
+        plans = ens.plan(off)
+        plans[0].score(ids, scores[0], main)
+        ens.score_and_vote(ids, off, scores, dec, stream=main, plans=plans)
+        torch.cuda.synchronize()
+        g_one, g_many = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_one, stream=main):
+            plans[0].score(ids, scores[0], main)
+        with torch.cuda.graph(g_many, stream=main):
+            ens.score_and_vote(ids, off, scores, dec, stream=main, plans=plans)
+        def replay_on_main(g):
+            def fn():
+                with torch.cuda.stream(main):       # a graph replays on the current stream
+                    g.replay()
+            return fn
+        one_g = lat_of(replay_on_main(g_one))
+        many_g = lat_of(replay_on_main(g_many))
+        del g_one, g_many
+        for p in plans:
+            p.close()
+        rows.append({"len": L, "one_expert_p50_ms": float(np.median(one)),
+                     "one_expert_p99_ms": float(np.percentile(one, 99)),
+                     "ensemble_p50_ms": float(np.median(many)),
+                     "ensemble_p99_ms": float(np.percentile(many, 99)),
+                     "graph_one_expert_p50_ms": float(np.median(one_g)),
+                     "graph_one_expert_p99_ms": float(np.percentile(one_g, 99)),
+                     "graph_ensemble_p50_ms": float(np.median(many_g)),
+                     "graph_ensemble_p99_ms": float(np.percentile(many_g, 99))})
+    clk = clocks.stop()
+    launches = sum(e.profile_read()["total_launches"] for e in experts) - l0
+    head = rows[len(rows) // 2]
+    line = {"metric": f"batch-1 p50 latency of a {K}-expert ensemble with majority vote, one B200, "
+                      f"CUDA-graph replay ({s.n_layers}-layer H{s.hidden} encoder, length {head['len']})",
+            "value": head["graph_ensemble_p50_ms"], "unit": "ms", "n_gpus": 1, "steps": n_req,
+            "warmup": n_warm, "ms_per_step": head["graph_ensemble_p50_ms"], "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "experts": K,
+                       "weights": f"expert k: random N(0,0.02), seed {w.seed} + 1000k",
+                       "vote": "majority of [score > 0], even split by the summed margins",
+                       "timing": "per request from an idle GPU to the decision, CUDA events; "
+                                 "eager launches and CUDA-graph replay of the same calls"},
+            "latency": rows, "gpu_launches": int(launches), "clocks": clk}
+    print(json.dumps(line), flush=True)
+    for e in experts:
+        e.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -921,6 +1027,8 @@ def main():
                     help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
     ap.add_argument("--lanes", type=int, default=2,
                     help="handles sharing the weights, one stream each, batches dealt round-robin")
+    ap.add_argument("--ensemble", type=int, default=0,
+                    help="batch-1 latency of one expert vs this many experts voting (one GPU)")
     ap.add_argument("--serve", action="store_true",
                     help="open-loop Poisson serving at 0.5x and 0.9x of the saturation rate, "
                          "throughput vs latency DP objective (p50/p99)")
@@ -938,6 +1046,8 @@ def main():
         return prefix_bench(args)
     if args.serve:
         return serve_bench(args)
+    if args.ensemble > 0:
+        return ensemble_bench(args)
     return b200_arm(args)
 
 

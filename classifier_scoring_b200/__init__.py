@@ -81,6 +81,9 @@ def lib() -> ctypes.CDLL:
         "rm_create_shared": (ctypes.c_int, [P, ctypes.POINTER(P)]),
         "rm_score": (ctypes.c_int, [P, P, P, I32, P, P]),
         "rm_score_prefix": (ctypes.c_int, [P, P, P, P, P, I32, P, P, P, P]),
+        "rm_plan_create": (ctypes.c_int, [P, P, I32, P]),
+        "rm_score_plan": (ctypes.c_int, [P, P, P, P]),
+        "rm_plan_destroy": (None, [P]),
         "rm_score_host": (ctypes.c_int, [P, P, P, I32, P, P]),
         "rm_schedule": (ctypes.c_int, [P, P, I32, P]),
         "rm_schedule_cfg": (ctypes.c_int, [cfgp, P, I32, P]),
@@ -94,6 +97,7 @@ def lib() -> ctypes.CDLL:
         "rm_op_gemm": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_gemm_tiled": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P]),
         "rm_gemm_tile": (ctypes.c_int, [I32, I32, I32, I32, P]),
+        "rm_op_vote": (ctypes.c_int, [P, I32, I32, F, P, P, P]),
         "rm_op_embed": (ctypes.c_int, [P, P, I32, I32, P, P, P, P, F, I32, I32, I32, P, P, P]),
         "rm_op_attn_scores": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_softmax": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P]),
@@ -201,6 +205,10 @@ class Scorer:
                                      cl.ctypes.data, len(pl), _ptr(out_dev), _ptr(best_dev),
                                      _ptr(logodds_dev), _stream(stream)))
 
+    def plan(self, offsets) -> "Plan":
+        """rm_plan_create: a prepared batch shape for launch-only scoring."""
+        return Plan(self, offsets)
+
     def score_host(self, ids_host, offsets, out_host, stream=None) -> None:
         """rm_score_host: host ids/out (pinned for asynchronous copies)."""
         off = _i32(offsets)
@@ -265,6 +273,11 @@ class ops:
     def gemm_tiled(x, w, bias, y, y_dtype, M, N, K, act=0, cg=0, bn=0, stream=None):
         _check(lib().rm_op_gemm_tiled(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), y_dtype, M, N, K,
                                       act, cg, bn, _stream(stream)))
+
+    @staticmethod
+    def vote(scores, K, n, threshold=0.0, decision=None, votes=None, stream=None):
+        _check(lib().rm_op_vote(_ptr(scores), K, n, threshold, _ptr(decision), _ptr(votes),
+                                _stream(stream)))
 
     @staticmethod
     def gemm_tile(M, N, K, num_sms):
@@ -332,3 +345,30 @@ class ops:
                                        nb.ctypes.data, first.ctypes.data, last.ctypes.data,
                                        max_bufs, peak.ctypes.data))
         return off[:k], nb[:k], first[:k], last[:k], int(peak[0])
+
+
+class Plan:
+    """rm_plan: the batch shape of repeated calls, prepared once; score() only
+    enqueues kernels (capturable in a CUDA graph)."""
+
+    def __init__(self, scorer: "Scorer", offsets):
+        self._scorer = scorer                  # keeps the handle alive
+        off = _i32(offsets)
+        h = ctypes.c_void_p()
+        _check(lib().rm_plan_create(scorer._h, off.ctypes.data, len(off) - 1, ctypes.byref(h)))
+        self._p = h
+        self.n = len(off) - 1
+
+    def score(self, ids_dev, out_dev, stream=None) -> None:
+        _check(lib().rm_score_plan(self._p, _ptr(ids_dev), _ptr(out_dev), _stream(stream)))
+
+    def close(self):
+        if self._p:
+            lib().rm_plan_destroy(self._p)
+            self._p = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -426,6 +426,35 @@ struct ProfScope {
     ps_.done(RM_K_GEMM, flops, bytes);               \
   } while (0)
 
+// What the launch sequence of one call needs to know on the host.
+struct CallInfo {
+  int32_t n = 0, T = 0, nrb = 0, Lmax = 0;
+  int64_t S = 0;
+  double att = 0;   // attention entries the mask admits, summed over heads
+  const int32_t* d_off = nullptr;
+  const int32_t* d_rb = nullptr;
+  const int64_t* d_so = nullptr;
+  const int32_t *d_pst = nullptr, *d_pln = nullptr, *d_oix = nullptr, *d_gof = nullptr;
+  const PrefixSpec* px = nullptr;
+};
+
+// Attention entries the mask admits: L*L per head, L*(L+1)/2 when causal,
+// plus L*P for a segment that continues a shared prefix of P tokens.
+double attention_entries(const rm_config* c, const int32_t* offsets, int32_t n,
+                         const PrefixSpec* px) {
+  const bool dec = c->arch == RM_DEC_PRELN;
+  double att = 0;
+  for (int32_t i = 0; i < n; ++i) {
+    const double L = static_cast<double>(offsets[i + 1] - offsets[i]);
+    const double P0 = px ? px->pre_len[i] : 0;
+    att += dec ? L * P0 + L * (L + 1) / 2 : L * L;
+  }
+  return att * c->n_heads;
+}
+
+int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, float* d_out,
+                    cudaStream_t st);
+
 // host_ids != NULL: copy the ids host->device (into the arena) once the call
 // has been validated, and the scores back into host_out at the end.
 int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, const int32_t* offsets,
@@ -480,7 +509,39 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   const int32_t* d_pln = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.pln) : nullptr;
   const int32_t* d_oix = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.oix) : nullptr;
   const int32_t* d_gof = px ? reinterpret_cast<const int32_t*>(h->d_meta + ml.gof) : nullptr;
+  CallInfo ci;
+  ci.n = n;
+  ci.T = T;
+  ci.nrb = nrb;
+  ci.Lmax = Lmax;
+  ci.S = S;
+  ci.att = attention_entries(c, offsets, n, px);
+  ci.d_off = d_off;
+  ci.d_rb = d_rb;
+  ci.d_so = d_so;
+  ci.d_pst = d_pst;
+  ci.d_pln = d_pln;
+  ci.d_oix = d_oix;
+  ci.d_gof = d_gof;
+  ci.px = px;
+  RM_TRY(enqueue_forward(h, ci, d_ids, d_out, st));
+  if (host_out != nullptr)
+    RM_CUDA(cudaMemcpyAsync(host_out, d_out, 4 * static_cast<size_t>(n), cudaMemcpyDeviceToHost, st));
+  return RM_OK;
+}
 
+// The launch sequence of one call whose metadata is already on the device:
+// kernels only (no host synchronisation, no copies), so a caller may capture
+// it into a CUDA graph (rm_score_plan).
+int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, float* d_out,
+                    cudaStream_t st) {
+  const rm_config* c = &h->cfg;
+  const int32_t n = ci.n, T = ci.T, nrb = ci.nrb, Lmax = ci.Lmax;
+  const int64_t S = ci.S;
+  const int32_t *d_off = ci.d_off, *d_rb = ci.d_rb, *d_pst = ci.d_pst, *d_pln = ci.d_pln,
+                *d_oix = ci.d_oix, *d_gof = ci.d_gof;
+  const int64_t* d_so = ci.d_so;
+  const PrefixSpec* px = ci.px;
   Bucket* bk = nullptr;
   RM_TRY(get_bucket(h, T, S, &bk));
   uint8_t* base = h->planned;
@@ -503,13 +564,7 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
 
   // algorithmic work of each launch (unpadded tokens; attention entries that
   // the mask admits: L*L per head, or L*(L+1)/2 when causal)
-  double att = 0;
-  for (int32_t i = 0; i < n; ++i) {
-    const double L = static_cast<double>(offsets[i + 1] - offsets[i]);
-    const double P0 = px ? px->pre_len[i] : 0;   // shared-prefix keys every row sees
-    att += dec ? L * P0 + L * (L + 1) / 2 : L * L;
-  }
-  att *= nh;
+  const double att = ci.att;
   const double Td = T, Hd = H, Fd = F;
   auto gemm_flops = [&](double N, double K) { return 2.0 * Td * N * K; };
   auto gemm_bytes = [&](double N, double K) { return 2.0 * (Td * K + N * K + Td * N); };
@@ -592,8 +647,6 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   if (px != nullptr && (px->d_best != nullptr || px->d_logodds != nullptr))
     RM_KERNEL(RM_K_HEAD, 0, 4.0 * px->group_off[px->n_groups] + 8.0 * px->n_groups,
               best_of_n_launch(d_out, d_gof, px->n_groups, px->d_best, px->d_logodds, st));
-  if (host_out != nullptr)
-    RM_CUDA(cudaMemcpyAsync(host_out, d_out, 4 * static_cast<size_t>(n), cudaMemcpyDeviceToHost, st));
   h->last_stream = st;
   return RM_OK;
 }
@@ -772,6 +825,77 @@ int rm_score_prefix(rm_handle* h, const int32_t* packed_token_ids, const int32_t
                     static_cast<cudaStream_t>(stream), &px);
 }
 
+struct rm_plan {
+  rm_handle* h = nullptr;
+  CallInfo ci;
+  uint8_t* d_meta = nullptr;
+};
+
+int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_plan** out) {
+  if (h == nullptr || seq_offsets == nullptr || out == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  const rm_config* c = &h->cfg;
+  const int32_t n = n_seqs;
+  if (n < 1) return set_error(RM_E_INVAL, "n_seqs must be >= 1");
+  if (n > c->max_batch_seqs)
+    return set_error(RM_E_RANGE, "n_seqs %d exceeds max_batch_seqs %d", n, c->max_batch_seqs);
+  if (seq_offsets[0] != 0) return set_error(RM_E_INVAL, "seq_offsets[0] must be 0");
+  for (int32_t i = 0; i < n; ++i) {
+    const int64_t L = static_cast<int64_t>(seq_offsets[i + 1]) - seq_offsets[i];
+    if (L < 1) return set_error(RM_E_INVAL, "sequence %d has length %lld (< 1)", i, (long long)L);
+    if (L > c->max_len)
+      return set_error(RM_E_RANGE, "sequence %d has length %lld > max_len %d", i, (long long)L,
+                       c->max_len);
+  }
+  const int32_t T = seq_offsets[n];
+  if (T > c->max_tokens)
+    return set_error(RM_E_RANGE, "%d tokens exceed max_tokens %d", T, c->max_tokens);
+  const MetaLayout ml(n);
+  std::vector<uint8_t> meta(static_cast<size_t>(ml.base));
+  int32_t* p_off = reinterpret_cast<int32_t*>(meta.data());
+  int32_t* p_rb = reinterpret_cast<int32_t*>(meta.data() + ml.rb);
+  int64_t* p_so = reinterpret_cast<int64_t*>(meta.data() + ml.so);
+  std::memcpy(p_off, seq_offsets, 4 * static_cast<size_t>(n + 1));
+  int32_t Lmax = 0;
+  RM_TRY(host_varlen_meta(seq_offsets, n, c->n_heads, p_rb, p_so, &Lmax));
+  Bucket* bk = nullptr;
+  RM_TRY(get_bucket(h, T, p_so[n], &bk));   // the arena placement and tensor maps, made now
+  rm_plan* p = new rm_plan();
+  p->h = h;
+  cudaError_t e = cudaMalloc(&p->d_meta, ml.base);
+  if (e == cudaSuccess) e = cudaMemcpy(p->d_meta, meta.data(), ml.base, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(p->d_meta);
+    delete p;
+    return set_error(e == cudaErrorMemoryAllocation ? RM_E_NOMEM : RM_E_CUDA, "plan: %s",
+                     cudaGetErrorString(e));
+  }
+  CallInfo& ci = p->ci;
+  ci.n = n;
+  ci.T = T;
+  ci.nrb = p_rb[n];
+  ci.Lmax = Lmax;
+  ci.S = p_so[n];
+  ci.att = attention_entries(c, seq_offsets, n, nullptr);
+  ci.d_off = reinterpret_cast<const int32_t*>(p->d_meta);
+  ci.d_rb = reinterpret_cast<const int32_t*>(p->d_meta + ml.rb);
+  ci.d_so = reinterpret_cast<const int64_t*>(p->d_meta + ml.so);
+  *out = p;
+  return RM_OK;
+}
+
+int rm_score_plan(rm_plan* p, const int32_t* packed_token_ids, float* out_scores, void* stream) {
+  if (p == nullptr || packed_token_ids == nullptr || out_scores == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  return enqueue_forward(p->h, p->ci, packed_token_ids, out_scores, static_cast<cudaStream_t>(stream));
+}
+
+void rm_plan_destroy(rm_plan* p) {
+  if (p == nullptr) return;
+  cudaFree(p->d_meta);
+  delete p;
+}
+
 int rm_score_host(rm_handle* h, const int32_t* host_token_ids, const int32_t* seq_offsets,
                   int32_t n_seqs, float* host_scores, void* stream) {
   if (h == nullptr || host_token_ids == nullptr || seq_offsets == nullptr || host_scores == nullptr)
@@ -918,6 +1042,13 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
   RM_LAUNCH(gemm_launch(ta, tb, tile, M, N, K, bias, y, y_dtype == RM_F32, act, err, sms,
                         static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_op_vote(const float* scores, int32_t K, int32_t n, float threshold, int32_t* decision,
+               int32_t* votes, void* stream) {
+  if (scores == nullptr || K < 1 || n < 0) return set_error(RM_E_INVAL, "bad arguments");
+  RM_LAUNCH(vote_launch(scores, K, n, threshold, decision, votes, static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

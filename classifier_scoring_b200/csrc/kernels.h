@@ -52,6 +52,9 @@ cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
                         float b_r, int H, int last_token, float* out, cudaStream_t st,
                         const int32_t* out_index = nullptr);
+// majority vote of K experts' scores [K][n]
+cudaError_t vote_launch(const float* scores, int K, int n, float threshold, int32_t* decision,
+                        int32_t* votes, cudaStream_t st);
 // per group g (candidates group_off[g]..group_off[g+1]-1 of scores): the
 // first highest score's index and r_1 - r_0
 cudaError_t best_of_n_launch(const float* scores, const int32_t* group_off, int n_groups,

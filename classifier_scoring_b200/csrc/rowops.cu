@@ -186,6 +186,28 @@ __global__ void __launch_bounds__(kWarps * 32)
   if (lane == 0) out[slot] = acc + br;
 }
 
+// Majority vote of K experts per input i (scores [K][n], expert-major): an
+// expert answers [s > threshold]; the ensemble answers 1 with more than half
+// of the votes, 0 with fewer, and on an even split the sign of the margins
+// summed in expert order decides.
+__global__ void __launch_bounds__(128)
+    vote_kernel(const float* __restrict__ scores, int K, int n, float thr,
+                int32_t* __restrict__ decision, int32_t* __restrict__ votes) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  int v = 0;
+  float margin = 0.0f;
+  for (int k = 0; k < K; ++k) {
+    const float s = scores[static_cast<size_t>(k) * n + i];
+    v += s > thr ? 1 : 0;
+    margin = __fadd_rn(margin, __fsub_rn(s, thr));   // no contraction: the oracle's order and rounding
+  }
+  if (votes != nullptr) votes[i] = v;
+  if (decision != nullptr) decision[i] = 2 * v > K ? 1 : (2 * v < K ? 0 : (margin > 0.0f ? 1 : 0));
+}
+
 // Best-of-N selection per group of candidates: best[g] = the index (within
 // the group) of the highest score, the first one on ties; logodds[g] =
 // r_1 - r_0, the log-odds that candidate 1 is preferred over candidate 0
@@ -322,6 +344,14 @@ cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const
   dim3 grid((n_seqs + kWarps - 1) / kWarps);
   launch_k(head_kernel, grid, kWarps * 32, 0, st, static_cast<const bf16*>(x), offsets, n_seqs, w_r,
            b_r, H, last_token, out, out_index);
+  return cudaGetLastError();
+}
+
+cudaError_t vote_launch(const float* scores, int K, int n, float threshold, int32_t* decision,
+                        int32_t* votes, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  launch_k(vote_kernel, dim3((n + 127) / 128), dim3(128), 0, st, scores, K, n, threshold, decision,
+           votes);
   return cudaGetLastError();
 }
 

@@ -175,6 +175,21 @@ int rm_score_prefix(rm_handle* h, const int32_t* packed_token_ids, const int32_t
                     const int32_t* n_cand, const int32_t* cand_len, int32_t n_groups,
                     float* out_scores, int32_t* out_best, float* out_logodds, void* stream);
 
+/* A plan: the batch shape (seq_offsets) of repeated rm_score calls, prepared
+ * once.  rm_plan_create validates the offsets as rm_score does, builds the
+ * per-call metadata, allocates a small device block for it (the only
+ * allocation; synchronous) and fixes the arena placement.  rm_score_plan then
+ * enqueues the kernels alone -- no host synchronisation and no copies -- so it
+ * may be captured into a CUDA graph and replayed; each replay scores whatever
+ * ids are in packed_token_ids at that time.  A plan uses its handle's arena:
+ * it must not run concurrently with other calls on the same handle, and it is
+ * destroyed before its handle.  Errors as rm_score; RM_E_NOMEM / RM_E_CUDA
+ * when the metadata block cannot be made. */
+typedef struct rm_plan rm_plan;
+int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_plan** out);
+int rm_score_plan(rm_plan* plan, const int32_t* packed_token_ids, float* out_scores, void* stream);
+void rm_plan_destroy(rm_plan* plan);
+
 /* As rm_score, but token ids and scores are HOST buffers.  The ids are copied
  * host->device and the scores device->host on stream inside the call's
  * enqueued work; both host buffers should be pinned (cudaHostAlloc /

@@ -57,6 +57,17 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
                      int32_t M, int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn,
                      void* stream);
 
+/* Majority vote of an ensemble of K scorer replicas ("experts"), the SambaNova
+ * blog's accuracy section (Figs. 4-5: several TinyBERT instances vote on each
+ * input).  scores: device float[K][n], expert k's score of input i at
+ * scores[k*n + i].  Expert k answers [score > threshold]; decision[i] = 1 when
+ * more than K/2 experts answer 1, 0 when fewer, and on an even split 1 iff the
+ * margins sum_k (score - threshold), added in expert order in fp32, are > 0.
+ * decision, votes: device int32[n], either may be NULL.  RM_E_INVAL for
+ * K < 1, n < 0 or NULL scores.  Asynchronous on stream. */
+int rm_op_vote(const float* scores, int32_t K, int32_t n, float threshold, int32_t* decision,
+               int32_t* votes, void* stream);
+
 /* Host only: the output tile the projections use for an M x N x K product on
  * a device with num_sms SMs.  out[0] = cg (1 or 2), out[1] = bn.  RM_E_INVAL
  * for M, N, K or num_sms < 1 or out == NULL. */

@@ -63,3 +63,41 @@ def test_single_process_reduction_and_rate():
     assert bench.whole_job_rate(2, 10000, 5, 1000.0) == 100000.0
     w = synth.WORKLOADS["bert-base-len2-100"]
     assert bench.replica_workload(w, 0) == w
+
+
+def _ensemble_worker(rank, world, port, q):
+    """Each rank is one expert: its scores of the same inputs are gathered in
+    rank order and every rank reaches the same vote."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        from classifier_scoring_b200.ensemble import gather_scores
+        from oracle import ensemble as E
+        rng = np.random.default_rng(7 + rank)
+        local = torch.from_numpy(rng.normal(size=40).astype(np.float32))
+        allv = gather_scores(local)
+        d, v = E.majority_vote(allv.numpy())
+        q.put((rank, local.numpy().tolist(), allv.numpy().tolist(), d.tolist(), v.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ensemble_scores_gather_in_rank_order_and_vote_alike():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = 3
+    procs = [ctx.Process(target=_ensemble_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = {}
+    for _ in range(world):
+        r, local, allv, d, v = q.get(timeout=120)
+        out[r] = (local, allv, d, v)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for r in range(world):
+        assert out[r][1] == [out[k][0] for k in range(world)]     # row k = rank k's expert
+        assert out[r][2:] == out[0][2:]                            # the same decisions everywhere
