@@ -53,9 +53,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the dominant kernel (tcgen05 GEMM) from one ncu
 # capture; valid only for the source it was taken on (sha256 prefix of
-# gemm_tc.cu).  Mean of the 48 projections of one T = 3328 batch (the step's
-# batches average T = 3243).
-GEMM_TRAFFIC = {"src_sha": "ad2c53e8a0c1ec30", "bytes_per_launch": 12518923}
+# gemm_tc.cu).  Mean of the 48 projections of one fused call of two DP batches,
+# T = 6702 (the default step's fused calls average T = 6445).
+GEMM_TRAFFIC = {"src_sha": "ad2c53e8a0c1ec30", "bytes_per_launch": 21834549}
 
 
 def replica_workload(w, rank: int):
@@ -300,8 +300,8 @@ def b200_arm(args):
     max_len = min(s.max_pos, 1024, max(w.len_hi, int(st.lengths.max())))
     cfg = rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
                            ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos, weight_dtype=s.weight_dtype,
-                           gelu=s.gelu, ln_eps=s.ln_eps, max_batch_seqs=w.max_batch,
-                           max_tokens=w.max_batch * max_len, max_len=max_len,
+                           gelu=s.gelu, ln_eps=s.ln_eps, max_batch_seqs=args.fuse * w.max_batch,
+                           max_tokens=args.fuse * w.max_batch * max_len, max_len=max_len,
                            sched_max_batch=w.max_batch, sched_c0=SCHED_C0, sched_c1=SCHED_C1)
     sc = rm.Scorer(cfg, flat)
     del flat
@@ -315,9 +315,11 @@ def b200_arm(args):
     batch = sc.schedule(st.lengths)
     nb = int(batch.max()) + 1
     groups = [np.nonzero(batch == b)[0] for b in range(nb)]
+    n_dp_batches = nb
     if args.batch_index is not None:
-        # one DP batch only (small profiling case): the step scores just this batch
-        keep = groups[args.batch_index % nb]
+        # one call only (small profiling case): the step scores just this DP
+        # batch, or the `fuse` consecutive batches starting with it
+        keep = np.concatenate(groups[args.batch_index % nb:args.batch_index % nb + args.fuse])
         sub = np.zeros(len(st.lengths), dtype=bool)
         sub[keep] = True
         st = synth.Stream(lengths=st.lengths[keep], ids=st.ids, starts=st.starts[keep])
@@ -325,6 +327,12 @@ def b200_arm(args):
         batch = np.zeros(n_req, dtype=np.int32)
         nb = 1
         groups = [np.arange(n_req)]
+        n_dp_batches = min(args.fuse, n_dp_batches)
+    elif args.fuse > 1:
+        # executor: consecutive DP batches run as one forward pass (packed, so
+        # the result of every request is the same; the projections get more rows)
+        groups = [np.concatenate(groups[k:k + args.fuse]) for k in range(0, nb, args.fuse)]
+        nb = len(groups)
     order = np.concatenate(groups)
     packed_ids, _ = synth.pack(st, order)
     b_tok = np.zeros(nb + 1, dtype=np.int64)
@@ -520,8 +528,11 @@ def b200_arm(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(name), lanes=lanes_note(len(lanes))),
-        "p50_latency_ms": p50, "p99_latency_ms": p99, "batches_per_step": nb,
+        "config": dict(workload_config(name), lanes=lanes_note(len(lanes)),
+                       **({"fuse": f"{args.fuse} consecutive DP batches per rm_score call"}
+                          if args.fuse > 1 else {})),
+        "p50_latency_ms": p50, "p99_latency_ms": p99, "batches_per_step": n_dp_batches,
+        "calls_per_step": nb,
         "tokens_per_step": int(b_tok[-1]),
         "roofline": roofline,
         "kernels": kernels,
@@ -1025,6 +1036,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel-bench", action="store_true",
                     help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
+    ap.add_argument("--fuse", type=int, default=2,
+                    help="consecutive DP batches scored per rm_score call (executor batch fusion)")
     ap.add_argument("--lanes", type=int, default=2,
                     help="handles sharing the weights, one stream each, batches dealt round-robin")
     ap.add_argument("--ensemble", type=int, default=0,
