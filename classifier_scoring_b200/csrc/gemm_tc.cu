@@ -39,12 +39,13 @@ constexpr int BK = 64;                      // 64 bf16 = one 128-byte swizzle ro
 
 constexpr int kThreads = 192;
 // Time per column of a CTA-pair tile relative to a single-CTA tile, and the
-// smallest products for which pairs are considered (measured on B200: a pair
-// round took ~0.8x a single-CTA round of the same width at M = 26112,
-// K = 2048, but ~1.1x at M = 3328, K = 768, and lost at M = 3328, K = 3072).
+// smallest products for which pairs are considered (measured on B200 with
+// N-fastest tile order: pairs won by 12-16% on the M = 26112 projections and
+// by up to 3.5% at M = 13556 with N >= 2304, and lost at M <= 10048 or
+// N = 768).
 constexpr double kPairColumnCost = 0.8;
-constexpr int kPairMinM = 8192;
-constexpr int kPairMinK = 2048;
+constexpr int kPairMinM = 12288;
+constexpr int kPairMinN = 2048;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
                         const float* __restrict__ bias, void* __restrict__ y,
-                        int* __restrict__ err) {
+                        int* __restrict__ err, int n_fastest) {
   using L = GemmSmem<BN, CG>;
   constexpr int S = L::kStages;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
@@ -228,7 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = CG == 2 ? cluster_rank() : 0u;   // 0 = leader of the pair
   const int unit = blockIdx.x / CG, units = gridDim.x / CG;
   const int tiles_m = (M + BM * CG - 1) / (BM * CG);
-  const int tiles = tiles_m * ((N + BN - 1) / BN);
+  const int tiles_n = (N + BN - 1) / BN;
+  const int tiles = tiles_m * tiles_n;
+  // tile t -> (row block, column block).  N fastest: the CTAs running at the
+  // same time share a few A row panels and sweep all of B, so each A panel
+  // leaves DRAM once (the activations outgrow L2 well before the weights do);
+  // M fastest: they share a few B column panels.
+  auto m_blk = [&](int t) { return n_fastest ? t / tiles_n : t % tiles_m; };
+  auto n_blk = [&](int t) { return n_fastest ? t % tiles_n : t / tiles_m; };
   const int nk = (K + BK - 1) / BK;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S),
                  accf0 = smem_u32(bars + 2 * S), acce0 = smem_u32(bars + 2 * S + 2);
@@ -275,8 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int t = unit; t < tiles && ok; t += units) {
-        const int m0 = (t % tiles_m) * BM * CG + static_cast<int>(rank) * BM;
-        const int nb0 = (t / tiles_m) * BN + static_cast<int>(rank) * (BN / CG);
+        const int m0 = m_blk(t) * BM * CG + static_cast<int>(rank) * BM;
+        const int nb0 = n_blk(t) * BN + static_cast<int>(rank) * (BN / CG);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -382,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // buffer for the accumulator was last read two tiles ago)
       float* sbias = sbias_warp + acc * BN;
       {
-        const int nb0 = (t / tiles_m) * BN;
+        const int nb0 = n_blk(t) * BN;
         for (int j = lane; j < BN; j += 32)
           sbias[j] = (bias != nullptr && nb0 + j < N) ? __ldg(bias + nb0 + j) : 0.0f;
         __syncwarp();
@@ -393,8 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m0 = (t % tiles_m) * BM * CG + static_cast<int>(rank) * BM;
-      const int n0 = (t / tiles_m) * BN;
+      const int m0 = m_blk(t) * BM * CG + static_cast<int>(rank) * BM;
+      const int n0 = n_blk(t) * BN;
       const int row0 = m0 + q * 32;
       const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
 #pragma unroll 1
@@ -530,7 +538,9 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, a, b, M, N, K, bias, y, err);
+  // the activations (A, M rows) are at least as large as the weights (B, N rows)
+  const int n_fastest = M >= N ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, a, b, M, N, K, bias, y, err, n_fastest);
 }
 
 template <int BN, int CG>
@@ -556,11 +566,12 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms) {
   return GemmTile{RM_GEMM_FORCE_CG, RM_GEMM_FORCE_BN};
 #endif
   // Makespan of the persistent grid: rounds of tiles times the per-SM time of
-  // one tile, modelled as proportional to BN plus a fixed cost per tile
-  // (pipeline fill, epilogue tail) worth about 48 columns.  A CTA pair moves
+  // one tile, modelled as proportional to BN plus a fixed part worth about 160
+  // columns (pipeline fill, epilogue tail, and the A panel each tile reads
+  // whatever its width; fitted to B200 sweeps of the BERT projections).  A CTA pair moves
   // half of the weight tile per SM, so its mainloop runs faster per column,
   // but on B200 it only paid off on large products (M >= kPairMinM rows and
-  // K >= kPairMinK): on the short projections of small batches a pair ran
+  // N >= kPairMinN columns): on smaller or narrower projections a pair ran
   // slower than one CTA of the same width.
   GemmTile best{1, 256};
   double best_cost = -1;
@@ -569,14 +580,15 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms) {
     const long long tiles = tm * ((N + bn - 1) / bn);
     const long long units = num_sms / cg;
     const long long rounds = (tiles + units - 1) / units;
-    const double cost = static_cast<double>(rounds) * (bn * per_col + 48.0);
+    const double cost = static_cast<double>(rounds) * (bn * per_col + 160.0);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = GemmTile{cg, bn};
     }
   };
   for (int i = kGemmTileCount - 1; i >= 0; --i) consider(1, kGemmTileWidths[i], 1.0);
-  if (num_sms >= 2 && M >= kPairMinM && K >= kPairMinK)
+  (void)K;
+  if (num_sms >= 2 && M >= kPairMinM && N >= kPairMinN)
     for (int bn : {256, 192, 128}) consider(2, bn, kPairColumnCost);
   return best;
 }
