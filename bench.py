@@ -53,9 +53,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the dominant kernel (tcgen05 GEMM) from one ncu
 # capture; valid only for the source it was taken on (sha256 prefix of
-# gemm_tc.cu).  Mean of the 48 projections of one fused call of two DP batches,
-# T = 6702 (the default step's fused calls average T = 6445).
-GEMM_TRAFFIC = {"src_sha": "ad2c53e8a0c1ec30", "bytes_per_launch": 21834549}
+# gemm_tc.cu).  Mean of the 48 projections of one fused call of four DP batches,
+# T = 13556 (the default step's calls average T = 12728).
+GEMM_TRAFFIC = {"src_sha": "e4e7a50d168cf670", "bytes_per_launch": 47744672}
 
 
 def replica_workload(w, rank: int):
