@@ -110,7 +110,11 @@ __global__ void __launch_bounds__(kWarps * 32)
 }
 
 // MODE 0: x = LN(y + x); MODE 1: x = y + x, z = LN(x); MODE 2: z = LN(x)
-template <typename T, int MAXC, int MODE>
+// Wide rows (H > 1024) are split over WPR warps, so that a lane holds at most
+// four chunks: at H = 2048 one warp per row needs ~100 registers, which caps
+// an SM at 16 resident warps, too few to keep HBM busy.  The WPR partial sums
+// meet in shared memory (two CTA barriers per row pass).
+template <typename T, int MAXC, int MODE, int WPR>
 __global__ void __launch_bounds__(kWarps * 32)
     res_ln_kernel(const T* __restrict__ y, T* __restrict__ x, T* __restrict__ z,
                   const float* __restrict__ g, const float* __restrict__ b, int rows, int H,
@@ -118,16 +122,20 @@ __global__ void __launch_bounds__(kWarps * 32)
   pdl_launch_dependents();
   l2_prefetch_share(pf);
   pdl_wait();
-  const int r = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= rows) return;
+  constexpr int LPR = 32 * WPR;                        // lanes per row
+  __shared__ float part[kWarps];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * (kWarps / WPR) + warp / WPR;
+  const int lr = (warp % WPR) * 32 + lane;             // lane within the row
+  const bool live = r < rows;
+  if (WPR == 1 && !live) return;
   const int nch = H >> 3;
-  const size_t base = static_cast<size_t>(r) * H;
+  const size_t base = static_cast<size_t>(live ? r : 0) * H;
   float v[MAXC][8];
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
-    const int ch = lane + 32 * c;
-    if (ch < nch) {
+    const int ch = lr + LPR * c;
+    if (live && ch < nch) {
       Chunk8<T>::load(x + base + ch * 8, v[c]);
       if (MODE != 2) {
         float u[8];
@@ -141,8 +149,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     // the residual stream keeps the rounded sum, LN reads the same rounded values
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
-      const int ch = lane + 32 * c;
-      if (ch < nch) {
+      const int ch = lr + LPR * c;
+      if (live && ch < nch) {
         Chunk8<T>::store(x + base + ch * 8, v[c]);
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[c][e] = to_f32(from_f32<T>(v[c][e]));
@@ -150,12 +158,59 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
   }
   float mean, rstd;
-  row_moments<MAXC>(v, nch, lane, H, mean, rstd, eps);
-  normalize<MAXC>(v, nch, lane, mean, rstd, g, b);
+  if (WPR == 1) {
+    row_moments<MAXC>(v, nch, lr, H, mean, rstd, eps);
+  } else {
+    // the same two passes, each warp's share reduced across the row's warps
+    float s = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+      if (live && lr + LPR * c < nch) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += v[c][e];
+      }
+    s = group_sum<32>(s);
+    if (lane == 0) part[warp] = s;
+    __syncthreads();
+    float tot = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPR; ++w) tot += part[(warp / WPR) * WPR + w];
+    mean = tot / static_cast<float>(H);
+    float q = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+      if (live && lr + LPR * c < nch) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float d = v[c][e] - mean;
+          q += d * d;
+        }
+      }
+    q = group_sum<32>(q);
+    __syncthreads();                                   // every warp has read the sums
+    if (lane == 0) part[warp] = q;
+    __syncthreads();
+    float qt = 0.f;
+#pragma unroll
+    for (int w = 0; w < WPR; ++w) qt += part[(warp / WPR) * WPR + w];
+    rstd = rsqrtf(qt / static_cast<float>(H) + eps);
+  }
+  if (!live) return;
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int ch = lr + LPR * c;
+    if (ch < nch) {
+      float gg[8], bb[8];
+      load_f32x8(g + ch * 8, gg);
+      load_f32x8(b + ch * 8, bb);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[c][e] = (v[c][e] - mean) * rstd * gg[e] + bb[e];
+    }
+  }
   T* out = (MODE == 0 ? x : z) + base;
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
-    const int ch = lane + 32 * c;
+    const int ch = lr + LPR * c;
     if (ch < nch) Chunk8<T>::store(out + ch * 8, v[c]);
   }
 }
@@ -280,23 +335,38 @@ cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, co
   return cudaGetLastError();
 }
 
-template <typename T, int MAXC>
+template <typename T, int MAXC, int WPR>
 cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const float* b, int rows,
                      int H, float eps, int mode, cudaStream_t st, const L2Prefetch& pf) {
-  dim3 grid((rows + kWarps - 1) / kWarps);
+  dim3 grid((rows + kWarps / WPR - 1) / (kWarps / WPR));
   const T* yy = static_cast<const T*>(y);
   T* xx = static_cast<T*>(x);
   T* zz = static_cast<T*>(z);
   if (mode == 0)
-    launch_k(res_ln_kernel<T, MAXC, 0>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps,
-             pf_args(pf));
+    launch_k(res_ln_kernel<T, MAXC, 0, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H,
+             eps, pf_args(pf));
   else if (mode == 1)
-    launch_k(res_ln_kernel<T, MAXC, 1>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps,
-             pf_args(pf));
+    launch_k(res_ln_kernel<T, MAXC, 1, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H,
+             eps, pf_args(pf));
   else
-    launch_k(res_ln_kernel<T, MAXC, 2>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H, eps,
-             pf_args(pf));
+    launch_k(res_ln_kernel<T, MAXC, 2, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H,
+             eps, pf_args(pf));
   return cudaGetLastError();
+}
+
+// One warp per row up to H = 1024 (at most 4 chunks a lane); 2 warps per row
+// up to 2048 and 4 up to 4096.
+template <typename T>
+cudaError_t res_ln_dispatch(const void* y, void* x, void* z, const float* g, const float* b,
+                            int rows, int H, float eps, int mode, cudaStream_t st,
+                            const L2Prefetch& pf) {
+  const int chunks = H / 8;
+  if (chunks > 256) return res_ln_t<T, 4, 4>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 128) return res_ln_t<T, 4, 2>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 96) return res_ln_t<T, 4, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 64) return res_ln_t<T, 3, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 32) return res_ln_t<T, 2, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  return res_ln_t<T, 1, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
 }
 
 }  // namespace
@@ -330,11 +400,9 @@ cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const
                           int H, float eps, int dtype, int mode, cudaStream_t st,
                           const L2Prefetch& pf) {
   if (T == 0) return cudaSuccess;
-  const int maxc = pick_maxc(H);
-  if (dtype == 0) {
-    RMK_MAXC_SWITCH(maxc, (res_ln_t<float, M_>(y, x, z, g, b, T, H, eps, mode, st, pf)))
-  }
-  RMK_MAXC_SWITCH(maxc, (res_ln_t<bf16, M_>(y, x, z, g, b, T, H, eps, mode, st, pf)))
+  if (H % 8 != 0 || H > 4096) return cudaErrorInvalidValue;
+  if (dtype == 0) return res_ln_dispatch<float>(y, x, z, g, b, T, H, eps, mode, st, pf);
+  return res_ln_dispatch<bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
 }
 
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,
