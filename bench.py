@@ -125,6 +125,11 @@ def workload_config(name):
             "parallelism": "replicas"}
 
 
+def clocks_log(args, name):
+    """Where the raw nvidia-smi clock samples go (--clocks-dir), or None."""
+    return os.path.join(args.clocks_dir, name) if args.clocks_dir else None
+
+
 def lanes_note(n):
     return f"{n} stream(s) per GPU, consecutive DP batches dealt round-robin"
 
@@ -409,9 +414,7 @@ def b200_arm(args):
         h.profile(args.profile_every)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
-    out_dir = os.path.join(ROOT, "gpurun_out")
-    clocks = ClockSampler(gpu_index, os.path.join(out_dir, f"clocks_rank{rank}.csv")
-                          if os.path.isdir(out_dir) else None)
+    clocks = ClockSampler(gpu_index, clocks_log(args, f"clocks_rank{rank}.csv"))
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
@@ -731,9 +734,7 @@ def prefix_bench(args):
     l0 = sc.profile_read()["total_launches"]
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
-    out_dir = os.path.join(ROOT, "gpurun_out")
-    clocks = ClockSampler(gpu_index, os.path.join(out_dir, f"clocks_prefix_rank{rank}.csv")
-                          if os.path.isdir(out_dir) else None)
+    clocks = ClockSampler(gpu_index, clocks_log(args, f"clocks_prefix_rank{rank}.csv"))
     time.sleep(0.3)
     ms_shared = timed(shared, args.steps)
     clk = clocks.stop()
@@ -983,9 +984,7 @@ def ensemble_bench(args):
 
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
-    out_dir = os.path.join(ROOT, "gpurun_out")
-    clocks = ClockSampler(gpu_index, os.path.join(out_dir, "clocks_ensemble.csv")
-                          if os.path.isdir(out_dir) else None)
+    clocks = ClockSampler(gpu_index, clocks_log(args, "clocks_ensemble.csv"))
     time.sleep(0.3)
     l0 = sum(e.profile_read()["total_launches"] for e in experts)
     rows = []
@@ -1054,6 +1053,8 @@ def main():
                     help="time the kernels of every n-th batch with CUDA events (0 = off)")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="also write the raw clock samples of the timed region as CSV here")
     ap.add_argument("--kernel-bench", action="store_true",
                     help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
     ap.add_argument("--fuse", type=int, default=4,
