@@ -476,8 +476,11 @@ struct FusedSmem {
 // With PFX, segment i continues a shared prefix: its keys are the pre_len[i]
 // rows that start at packed row pre_start[i] (all visible), followed by its
 // own rows (causal), so query row r sees virtual keys 0 .. pre_len[i] + r.
+// Head dims up to 64 are held to 128 registers so that four CTAs share an SM
+// (137 registers allowed only three; 16 bytes of spill cost less than the
+// occupancy bought: 45.7 -> 42.0 us per BERT-base launch of 13k tokens).
 template <int DP, bool PFX>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, (DP <= 64 ? 4 : 1))
     attn_fused_async_kernel(const bf16* __restrict__ qkv, bf16* __restrict__ ctx,
                             const int32_t* __restrict__ offsets, const int32_t* __restrict__ rb_off,
                             int n, int H, int d, float scale_log2, int causal, L2PrefetchArgs pf,
