@@ -53,9 +53,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic per launch of the dominant kernel (tcgen05 GEMM) from one ncu
 # capture; valid only for the source it was taken on (sha256 prefix of
-# gemm_tc.cu).  Mean of the 48 projections of one fused call of four DP batches,
-# T = 13556 (the default step's calls average T = 12728).
-GEMM_TRAFFIC = {"src_sha": "e4e7a50d168cf670", "bytes_per_launch": 47744672}
+# gemm_tc.cu).  Mean of the 48 projections of one fused call of eight DP
+# batches, T = 27829 (the default step's calls average T = 25457).
+GEMM_TRAFFIC = {"src_sha": "e4e7a50d168cf670", "workload": "bert-base-len2-100", "fuse": 8,
+                "bytes_per_launch": 129556928}
 
 
 def replica_workload(w, rank: int):
@@ -515,7 +516,9 @@ def b200_arm(args):
     gemm_tflops = g["flops"] / (g["ms"] * 1e-3) / 1e12 if g["ms"] > 0 else None
     src = open(os.path.join(ROOT, "classifier_scoring_b200", "csrc", "gemm_tc.cu"), "rb").read()
     sha = hashlib.sha256(src).hexdigest()[:16]
-    traffic = GEMM_TRAFFIC["bytes_per_launch"] if GEMM_TRAFFIC["src_sha"] == sha else None
+    traffic = (GEMM_TRAFFIC["bytes_per_launch"]
+               if (GEMM_TRAFFIC["src_sha"] == sha and GEMM_TRAFFIC["workload"] == name
+                   and GEMM_TRAFFIC["fuse"] == args.fuse and args.batch_index is None) else None)
     measured_on = ("the timed region" if prof is prof_timed else
                    "one extra single-stream step after the timed region (the timed region "
                    f"ran {len(lanes)} overlapping streams)")
@@ -1057,7 +1060,7 @@ def main():
                     help="also write the raw clock samples of the timed region as CSV here")
     ap.add_argument("--kernel-bench", action="store_true",
                     help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
-    ap.add_argument("--fuse", type=int, default=4,
+    ap.add_argument("--fuse", type=int, default=8,
                     help="consecutive DP batches scored per rm_score call (executor batch fusion)")
     ap.add_argument("--lanes", type=int, default=2,
                     help="handles sharing the weights, one stream each, batches dealt round-robin")

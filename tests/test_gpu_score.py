@@ -115,6 +115,33 @@ def test_bert_base_dp_batch_sampled(name, n_req, which, n_sample, attn):
     assert np.max(np.abs(got[sample] - ref)) <= SCORE_ATOL
 
 
+def test_bench_launch_configuration_four_fused_batches():
+    """The call bench.py times: four consecutive DP batches of the full
+    10,000-request stream in one rm_score call (256 sequences, ~13k tokens),
+    on a handle sized as bench.py sizes it; sampled sequences against the
+    oracle, every score finite, and each sequence's score the same as when its
+    own DP batch is scored alone."""
+    name = "bert-base-len2-100"
+    w = synth.WORKLOADS[name]
+    st = synth.make_stream(w)
+    cfg_sched = config_for(w.shape, max_len=100, sched_max_batch=w.max_batch, sched_c0=20000,
+                           sched_c1=1)
+    batch = rm.schedule(cfg_sched, st.lengths)
+    idx = np.concatenate([np.nonzero(batch == b)[0] for b in range(80, 84)])
+    ids, off = synth.pack(st, idx)
+    sc = scorer(name, max_batch_seqs=4 * w.max_batch, max_tokens=4 * w.max_batch * 100, max_len=100)
+    got = gpu_scores(sc, ids, off)
+    assert len(idx) > 200 and np.all(np.isfinite(got))
+    sample = np.linspace(0, len(idx) - 1, 6).astype(int)
+    ref = oracle_scores(name, ids, off, sample)
+    assert np.max(np.abs(got[sample] - ref)) <= SCORE_ATOL
+    # the same requests as four separate calls: the packed layout makes fusion invisible
+    first = np.nonzero(batch == 80)[0]
+    ids1, off1 = synth.pack(st, first)
+    alone = gpu_scores(sc, ids1, off1)
+    assert np.max(np.abs(alone - got[:len(first)])) <= 2e-3
+
+
 @pytest.mark.parametrize("attn", [rm.ATTN_FUSED, rm.ATTN_MATERIALIZED], ids=["fused", "materialized"])
 def test_bert_base_mixed_lengths_every_sequence(attn):
     """A ragged batch of every length class, all sequences checked."""
