@@ -115,9 +115,9 @@ def test_bert_base_dp_batch_sampled(name, n_req, which, n_sample, attn):
     assert np.max(np.abs(got[sample] - ref)) <= SCORE_ATOL
 
 
-def test_bench_launch_configuration_four_fused_batches():
-    """The call bench.py times: four consecutive DP batches of the full
-    10,000-request stream in one rm_score call (256 sequences, ~13k tokens),
+def test_bench_launch_configuration_eight_fused_batches():
+    """The call bench.py times: eight consecutive DP batches of the full
+    10,000-request stream in one rm_score call (512 sequences, ~28k tokens),
     on a handle sized as bench.py sizes it; sampled sequences against the
     oracle, every score finite, and each sequence's score the same as when its
     own DP batch is scored alone."""
@@ -127,15 +127,15 @@ def test_bench_launch_configuration_four_fused_batches():
     cfg_sched = config_for(w.shape, max_len=100, sched_max_batch=w.max_batch, sched_c0=20000,
                            sched_c1=1)
     batch = rm.schedule(cfg_sched, st.lengths)
-    idx = np.concatenate([np.nonzero(batch == b)[0] for b in range(80, 84)])
+    idx = np.concatenate([np.nonzero(batch == b)[0] for b in range(80, 88)])
     ids, off = synth.pack(st, idx)
-    sc = scorer(name, max_batch_seqs=4 * w.max_batch, max_tokens=4 * w.max_batch * 100, max_len=100)
+    sc = scorer(name, max_batch_seqs=8 * w.max_batch, max_tokens=8 * w.max_batch * 100, max_len=100)
     got = gpu_scores(sc, ids, off)
-    assert len(idx) > 200 and np.all(np.isfinite(got))
+    assert len(idx) > 400 and np.all(np.isfinite(got))
     sample = np.linspace(0, len(idx) - 1, 6).astype(int)
     ref = oracle_scores(name, ids, off, sample)
     assert np.max(np.abs(got[sample] - ref)) <= SCORE_ATOL
-    # the same requests as four separate calls: the packed layout makes fusion invisible
+    # the same requests as separate calls: the packed layout makes fusion invisible
     first = np.nonzero(batch == 80)[0]
     ids1, off1 = synth.pack(st, first)
     alone = gpu_scores(sc, ids1, off1)
