@@ -360,7 +360,7 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
 
 int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCount], int M, int N,
          int K, const float* bias, void* y, int act, cudaStream_t st) {
-  const GemmTile tile = gemm_pick(M, N, K, h->num_sms);
+  const GemmTile tile = gemm_pick(M, N, K, h->num_sms, act);
   cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], tile, M, N, K, bias, y, false,
                               act, h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
@@ -1033,7 +1033,7 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
   int dev = 0, sms = 148;
   RM_CUDA(cudaGetDevice(&dev));
   RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-  const GemmTile tile = cg != 0 ? GemmTile{cg, bn} : gemm_pick(M, N, K, sms);
+  const GemmTile tile = cg != 0 ? GemmTile{cg, bn} : gemm_pick(M, N, K, sms, act);
   CUtensorMap ta, tb;
   const char* why = "";
   if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, tile.b_box(), &why))

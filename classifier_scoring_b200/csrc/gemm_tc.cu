@@ -37,7 +37,11 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;                      // 64 bf16 = one 128-byte swizzle row
 
-constexpr int kThreads = 192;
+// Epilogue warps: four (one per TMEM lane quarter) for a plain epilogue; eight
+// (two per quarter, alternating over the column rounds) when the epilogue
+// applies GELU, whose arithmetic otherwise outlasts a short mainloop.
+constexpr int epi_warps(int act) { return act != 0 ? 8 : 4; }
+constexpr int gemm_threads(int act) { return 64 + 32 * epi_warps(act); }
 // Time per column of a CTA-pair tile relative to a single-CTA tile, and the
 // smallest products for which pairs are considered (measured on B200 with
 // N-fastest tile order: pairs won by 12-16% on the M = 26112 projections and
@@ -168,6 +172,15 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -177,24 +190,28 @@ constexpr uint32_t tmem_cols_for(int bn) {
   return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
 }
 
-template <int BN, int CG>
+template <int BN, int CG, int EW>
 struct GemmSmem {
   static constexpr int kA = BM * BK * 2;
   static constexpr int kB = (BN / CG) * BK * 2;   // this CTA's share of the B tile
   static constexpr int kStage = kA + kB;          // multiple of 1024 for BN/CG % 8 == 0
-  // epilogue staging: per epilogue warp 32 rows x 128 B of output (64 bf16 or
-  // 32 fp32 columns), row pitch padded by 16 B so that both the row-wise
-  // writes and the line-wise reads touch every bank group evenly
-  static constexpr int kStagePitch = 128 + 16;
+  // epilogue staging: per epilogue warp 32 rows x one round of output (128 B
+  // with four epilogue warps, 64 B with eight), row pitch padded by 16 B so
+  // that both the row-wise writes and the segment-wise reads spread over the
+  // bank groups
+  static constexpr int kRoundBytes = EW == 4 ? 128 : 64;
+  static constexpr int kStagePitch = kRoundBytes + 16;
   static constexpr int kStageWarpBytes = 32 * kStagePitch;
-  // bias of the tile, per epilogue warp and accumulator (no cross-warp barrier)
-  static constexpr int kBiasBytes = 4 * 2 * BN * 4;
+  // bias of the tile per epilogue warp (no cross-warp barrier): two buffers
+  // (one per accumulator) with four warps, one with eight
+  static constexpr int kBiasFloatsPerWarp = EW == 4 ? 2 * BN : BN;
+  static constexpr int kBiasBytes = EW * kBiasFloatsPerWarp * 4;
   // as many 64-deep K stages as fit beside the rest (227 KB per CTA), at most 8
-  static constexpr int kFixed = 4 * kStageWarpBytes + kBiasBytes + 20 * 8 + 16 + 1024;
+  static constexpr int kFixed = EW * kStageWarpBytes + kBiasBytes + 20 * 8 + 16 + 1024;
   static constexpr int kStagesFit = (232448 - kFixed) / kStage;
   static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
   static constexpr int kEpiOff = kStages * kStage;
-  static constexpr int kBiasOff = kEpiOff + 4 * kStageWarpBytes;
+  static constexpr int kBiasOff = kEpiOff + EW * kStageWarpBytes;
   static constexpr int kBarOff = kBiasOff + kBiasBytes;   // full[S], empty[S], accf[2], acce[2]
   static constexpr int kSlotOff = kBarOff + (2 * kStages + 4) * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;   // + alignment slack
@@ -210,12 +227,13 @@ __device__ __forceinline__ float epilogue_act(float t) {
 }
 
 template <int BN, int CG, int ACT, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(ACT), 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
                         const float* __restrict__ bias, void* __restrict__ y,
                         int* __restrict__ err, int n_fastest) {
-  using L = GemmSmem<BN, CG>;
+  constexpr int EW = epi_warps(ACT);
+  using L = GemmSmem<BN, CG, EW>;
   constexpr int S = L::kStages;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
   static_assert(L::kStage % 1024 == 0, "stage size keeps the 1024-byte swizzle alignment");
@@ -248,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf0 + 8 * a, 1);
-      mbar_init(acce0 + 8 * a, 4 * CG);   // one arrival per epilogue warp of the pair
+      mbar_init(acce0 + 8 * a, EW * CG);   // one arrival per epilogue warp of the pair
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -374,21 +392,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---- epilogue: TMEM -> registers -> bias/GELU -> smem staging -> global ----
-    // Each thread owns one tile row (its TMEM lane).  A round takes 128 B of
-    // that row (64 bf16 / 32 fp32 columns), writes it to the warp's staging
-    // rows, then the warp stores 4 full 128-byte row segments per instruction.
+    // Each thread owns one tile row (its TMEM lane).  A round takes
+    // kRoundBytes of that row, writes it to the warp's staging rows, then the
+    // warp stores whole row segments.  With eight warps the two warps of a
+    // lane quarter take alternate rounds.
     constexpr int ESZ = OUT_F32 ? 4 : 2;
-    constexpr int CPR = 128 / ESZ;               // columns per round
+    constexpr int RB = L::kRoundBytes;
+    constexpr int CPR = RB / ESZ;                // columns per round
+    constexpr int NH = EW / 4;                   // warps per TMEM lane quarter
+    const int ew = warp - 2;
     const int q = warp & 3;                      // TMEM lane quarter of this warp
+    const int h0 = ew >> 2;                      // this warp's first round
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    uint8_t* stg = smem + L::kEpiOff + (warp - 2) * L::kStageWarpBytes;
-    float* sbias_warp = reinterpret_cast<float*>(smem + L::kBiasOff) + (warp - 2) * 2 * BN;
+    uint8_t* stg = smem + L::kEpiOff + ew * L::kStageWarpBytes;
+    float* sbias_warp = reinterpret_cast<float*>(smem + L::kBiasOff) + ew * L::kBiasFloatsPerWarp;
     int local = 0;
     for (int t = unit; t < tiles; t += units, ++local) {
       const int acc = local & 1, use = local >> 1;
-      // stage this tile's bias while the mainloop still runs (this warp's
-      // buffer for the accumulator was last read two tiles ago)
-      float* sbias = sbias_warp + acc * BN;
+      // stage this tile's bias while the mainloop still runs (with two
+      // buffers, the one for this accumulator was last read two tiles ago;
+      // with one, this warp's reads of the previous tile ended before its
+      // arrival below)
+      float* sbias = sbias_warp + (EW == 4 ? acc * BN : 0);
       {
         const int nb0 = n_blk(t) * BN;
         for (int j = lane; j < BN; j += 32)
@@ -406,10 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row0 = m0 + q * 32;
       const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += CPR) {
+      for (int c = h0 * CPR; c < BN; c += NH * CPR) {
         if (n0 + c >= N) break;                  // uniform across the warp
         float v[CPR];
-        {
+        if (CPR >= 32) {
           uint32_t r[32];
 #pragma unroll
           for (int h = 0; h < CPR / 32; ++h) {
@@ -418,6 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[32 * h + j] = __uint_as_float(r[j]);
           }
+        } else {
+          uint32_t r[16];
+          tmem_ld_16cols(base + c, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
         }
 #pragma unroll
         for (int g = 0; g < CPR / 4; ++g) {
@@ -432,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();                            // the previous round's reads are done
         uint8_t* my_row = stg + lane * L::kStagePitch;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < RB / 16; ++j) {
           uint4 u;
           if (OUT_F32) {
             u = make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
@@ -444,15 +475,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(my_row + 16 * j) = u;
         }
         __syncwarp();
-        const int ch = lane & 7;                 // 16-byte chunk of a 128-byte segment
+        // RB/16 16-byte chunks per row; a store instruction covers 32/(RB/16)
+        // rows (128-byte rows: 4, lanes along the row; 64-byte rows: 8, lanes
+        // down the rows, which keeps the 80-byte pitch free of bank conflicts)
+        constexpr int CH = RB / 16;
+        constexpr int RPI = 32 / CH;
+        const int ch = RB == 128 ? (lane & 7) : (lane >> 3);
+        const int rsub = RB == 128 ? (lane >> 3) : (lane & 7);
         const int tcol = c + ch * (16 / ESZ);    // column inside the tile
         const int gcol = n0 + tcol;
         // a round can run past the tile (BN not a multiple of the round width):
         // those columns belong to the next tile and are not stored
         const bool col_ok = tcol < BN && gcol < N;
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int rr = it * 4 + (lane >> 3);
+        for (int it = 0; it < 32 / RPI; ++it) {
+          const int rr = it * RPI + rsub;
           const int grow = row0 + rr;
           if (grow < M && col_ok) {
             const uint4 u = *reinterpret_cast<const uint4*>(stg + rr * L::kStagePitch + ch * 16);
@@ -493,10 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int CG, int ACT, bool OUT_F32>
 cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
                        const float* bias, void* y, int* err, int num_sms, cudaStream_t st) {
-  using L = GemmSmem<BN, CG>;
+  using L = GemmSmem<BN, CG, epi_warps(ACT)>;
   auto kern = gemm_bf16_tc_kernel<BN, CG, ACT, OUT_F32>;
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(gemm_threads(ACT));
   cfg.dynamicSmemBytes = L::kBytes;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -561,7 +598,7 @@ cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
 
 const int kGemmTileWidths[kGemmTileCount] = {64, 96, 128, 160, 192, 224, 256};
 
-GemmTile gemm_pick(int M, int N, int K, int num_sms) {
+GemmTile gemm_pick(int M, int N, int K, int num_sms, int act) {
 #if defined(RM_GEMM_FORCE_BN) && defined(RM_GEMM_FORCE_CG)
   return GemmTile{RM_GEMM_FORCE_CG, RM_GEMM_FORCE_BN};
 #endif
@@ -587,8 +624,10 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms) {
     }
   };
   for (int i = kGemmTileCount - 1; i >= 0; --i) consider(1, kGemmTileWidths[i], 1.0);
-  (void)K;
-  if (num_sms >= 2 && M >= kPairMinM && N >= kPairMinN)
+  // With a GELU epilogue and a short K the epilogue, not the mainloop, sets
+  // the pace, and single-CTA tiles measured 5-6% faster than pairs there.
+  const bool pair_ok = act == 0 || K >= 2048;
+  if (num_sms >= 2 && M >= kPairMinM && N >= kPairMinN && pair_ok)
     for (int bn : {256, 192, 128}) consider(2, bn, kPairColumnCost);
   return best;
 }

@@ -17,7 +17,7 @@ struct GemmTile {
   int bn;
   int b_box() const { return bn / cg; }   // weight rows per TMA box
 };
-GemmTile gemm_pick(int M, int N, int K, int num_sms);
+GemmTile gemm_pick(int M, int N, int K, int num_sms, int act = 0);
 inline int gemm_tile_index(int box_rows) { return (box_rows - 64) / 32; }
 // a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, tile.b_box()}.
 // Persistent grid of min(tiles, num_sms / cg) units of cg CTAs.

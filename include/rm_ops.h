@@ -68,9 +68,10 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
 int rm_op_vote(const float* scores, int32_t K, int32_t n, float threshold, int32_t* decision,
                int32_t* votes, void* stream);
 
-/* Host only: the output tile the projections use for an M x N x K product on
- * a device with num_sms SMs.  out[0] = cg (1 or 2), out[1] = bn.  RM_E_INVAL
- * for M, N, K or num_sms < 1 or out == NULL. */
+/* Host only: the output tile the projections without an activation use for
+ * an M x N x K product on a device with num_sms SMs (a GELU epilogue may take
+ * a single-CTA tile where this returns a pair).  out[0] = cg (1 or 2),
+ * out[1] = bn.  RM_E_INVAL for M, N, K or num_sms < 1 or out == NULL. */
 int rm_gemm_tile(int32_t M, int32_t N, int32_t K, int32_t num_sms, int32_t* out);
 
 /* X[t] = E_word[clamp(ids[t])] + E_pos[t - offsets[i]] for each token t of

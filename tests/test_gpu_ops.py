@@ -353,7 +353,7 @@ def test_attention_fused(lens, nh, d, causal):
 
 
 def test_gemm_gelu_epilogue_against_cuda_erf_and_oracle():
-    """GELU of the epilogue (Abramowitz & Stegun 7.1.26 erf) on a dense grid of
+    """GELU of the epilogue (Abramowitz & Stegun 7.1.28 erf) on a dense grid of
     pre-activations: x = 0, W = 0, so y = GELU(bias)."""
     N = 8192
     u = torch.linspace(-12, 12, N, dtype=torch.float32)
