@@ -55,8 +55,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # capture; valid only for the source it was taken on (sha256 prefix of
 # gemm_tc.cu).  Mean of the 48 projections of one fused call of eight DP
 # batches, T = 27829 (the default step's calls average T = 25457).
-GEMM_TRAFFIC = {"src_sha": "e4e7a50d168cf670", "workload": "bert-base-len2-100", "fuse": 8,
-                "bytes_per_launch": 129556928}
+GEMM_TRAFFIC = {"src_sha": "632d3288c2bd66bd", "workload": "bert-base-len2-100", "fuse": 8,
+                "bytes_per_launch": 130000480}
 
 
 def replica_workload(w, rank: int):
