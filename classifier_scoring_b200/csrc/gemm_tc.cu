@@ -5,24 +5,26 @@
 //
 // Persistent, warp-specialised kernel: one CTA per SM (CG = 1) or one CTA pair
 // per two SMs (CG = 2) walks the (128*CG) x BN output tiles t = unit,
-// unit + units, ... (M fastest, so the CTAs of one wave share a few weight
-// column blocks in L2).  With CG = 2 the pair is a cluster of two CTAs and the
-// MMA is tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 rows of
-// A and half of the BN rows of B, the leader CTA issues the MMAs for both, and
-// each CTA's TMEM receives its own 128 rows of the accumulator.  Per SM this
-// moves half of B through shared memory, which keeps the operand ring ahead of
-// the tensor core.  No load uses multicast.  Six warps:
+// unit + units, ...  Tiles run N fastest when the activations (A) are at least
+// as large as the weights (B): the CTAs of one wave then share a few A row
+// panels, so each panel leaves DRAM once while B stays in L2; otherwise M
+// fastest.  With CG = 2 the pair is a cluster of two CTAs and the MMA is
+// tcgen05.mma.cta_group::2 (M = 256): each CTA loads its own 128 rows of A and
+// half of the BN rows of B, the leader CTA issues the MMAs for both, and each
+// CTA's TMEM receives its own 128 rows of the accumulator.  Per SM this moves
+// half of B through shared memory.  No load uses multicast.  Warps:
 //   warp 0, one lane : TMA producer -- K-major 128x64 (A) and BNx64 (B) bf16
 //                      boxes, 128-byte swizzle, into a STAGES-deep smem ring
 //                      that runs on across tile boundaries;
-//   warp 1, one lane : issues tcgen05.mma (M=128, N=BN, K=16) into one of two
-//                      TMEM accumulators, tcgen05.commit frees each stage and
-//                      marks the accumulator full;
-//   warps 2..5       : epilogue -- tcgen05.ld 32 columns at a time (warp w
-//                      reads TMEM lanes 32*(w%4)..+31 = tile rows), + bias,
-//                      optional GELU, store bf16 or fp32, then release the
-//                      accumulator.  The epilogue of tile i overlaps the
-//                      mainloop of tile i+1.
+//   warp 1, one lane : issues tcgen05.mma (M=128*CG, N=BN, K=16) into one of
+//                      two TMEM accumulators, tcgen05.commit frees each stage
+//                      and marks the accumulator full;
+//   warps 2..        : epilogue (four warps, or eight when the epilogue applies
+//                      GELU) -- tcgen05.ld (warp w reads TMEM lanes
+//                      32*(w%4)..+31 = tile rows), + bias, optional GELU,
+//                      staged through shared memory into whole row segments of
+//                      bf16 or fp32, then release the accumulator.  The
+//                      epilogue of tile i overlaps the mainloop of tile i+1.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that
 // gives up counts into err[ERR_TIMEOUT] and the role leaves its loop; the CTA
 // then waits (bounded) for its own copies, frees its TMEM and returns.
