@@ -601,9 +601,6 @@ cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
 const int kGemmTileWidths[kGemmTileCount] = {64, 96, 128, 160, 192, 224, 256};
 
 GemmTile gemm_pick(int M, int N, int K, int num_sms, int act) {
-#if defined(RM_GEMM_FORCE_BN) && defined(RM_GEMM_FORCE_CG)
-  return GemmTile{RM_GEMM_FORCE_CG, RM_GEMM_FORCE_BN};
-#endif
   // Makespan of the persistent grid: rounds of tiles times the per-SM time of
   // one tile, modelled as proportional to BN plus a fixed part worth about 160
   // columns (pipeline fill, epilogue tail, and the A panel each tile reads
