@@ -679,14 +679,11 @@ cudaError_t launch_fused_async(dim3 grid, cudaStream_t st, const bf16* q, bf16* 
     pa.ptr[k] = pf.ptr[k];
     pa.bytes[k] = pf.bytes[k];
   }
-  static bool configured = false;   // the attribute is per function; one device per process
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fused_async_kernel<DP, PFX>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         FusedSmem<DP>::kBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  // the attribute is per function: set once (thread-safe static initialisation)
+  static const cudaError_t attr_err = cudaFuncSetAttribute(
+      attn_fused_async_kernel<DP, PFX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      FusedSmem<DP>::kBytes);
+  if (attr_err != cudaSuccess) return attr_err;
   launch_k(attn_fused_async_kernel<DP, PFX>, grid, dim3(128), FusedSmem<DP>::kBytes, st, q, c,
            offsets, rb_off, n, H, d, scale_log2, causal, pa, pre_start, pre_len);
   return cudaGetLastError();

@@ -547,28 +547,30 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
     attr[na].val.clusterDim.z = 1;
     ++na;
   }
-  // The attribute is per function and the co-resident pair count per device
-  // model; one device model per process.
-  static bool configured = false;
-  static int resident_units = 0;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
-    if (e != cudaSuccess) return e;
-    if (CG == 2) {
+  // Once per instantiation (thread-safe static initialisation): the shared
+  // memory attribute, per function, and for pairs the number of clusters
+  // that fit at once, per device model; one device model per process.
+  struct Setup {
+    cudaError_t err;
+    int resident_units;
+  };
+  static const Setup setup = [&]() {
+    Setup r{cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes), 0};
+    if (r.err == cudaSuccess && CG == 2) {
       // pairs must sit on the two SMs of one cluster slot: ask how many fit at once
-      cfg.gridDim = dim3(2 * (num_sms / 2));
-      cfg.attrs = attr;
-      cfg.numAttrs = na;
-      int clusters = 0;
-      e = cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg);
-      if (e != cudaSuccess) return e;
-      resident_units = clusters;
+      cudaLaunchConfig_t q = cfg;
+      q.gridDim = dim3(2 * (num_sms / 2));
+      q.attrs = attr;
+      q.numAttrs = na;
+      r.err = cudaOccupancyMaxActiveClusters(&r.resident_units, kern, &q);
     }
-    configured = true;
-  }
+    return r;
+  }();
+  if (setup.err != cudaSuccess) return setup.err;
   const int tiles = ((M + BM * CG - 1) / (BM * CG)) * ((N + BN - 1) / BN);
   int max_units = num_sms / CG;
-  if (CG == 2 && resident_units > 0 && resident_units < max_units) max_units = resident_units;
+  if (CG == 2 && setup.resident_units > 0 && setup.resident_units < max_units)
+    max_units = setup.resident_units;
   cfg.gridDim = dim3(CG * (tiles < max_units ? tiles : max_units));
   if (g_pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
