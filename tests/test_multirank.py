@@ -101,3 +101,16 @@ def test_ensemble_scores_gather_in_rank_order_and_vote_alike():
     for r in range(world):
         assert out[r][1] == [out[k][0] for k in range(world)]     # row k = rank k's expert
         assert out[r][2:] == out[0][2:]                            # the same decisions everywhere
+
+
+def test_code_hash_ignores_comments_and_metric_names(tmp_path):
+    import bench
+    a = tmp_path / "a.cu"
+    b = tmp_path / "b.cu"
+    a.write_text("int f() {  // one\n  return 1;\n}\n")
+    b.write_text("// header\nint f() {\n\n  return 1;   // two\n}\n")
+    assert bench.code_sha(str(a)) == bench.code_sha(str(b))
+    b.write_text("int f() {\n  return 2;\n}\n")
+    assert bench.code_sha(str(a)) != bench.code_sha(str(b))
+    assert bench.metric_for("bert-base-len2-100") == bench.METRIC
+    assert "len 5" in bench.metric_for("bert-base-len5-500")
