@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import weakref
 from typing import Optional
 
 import numpy as np
@@ -169,12 +170,16 @@ class Scorer:
             _check(lib().rm_create(ctypes.byref(cfg), w.ctypes.data, w.nbytes, ctypes.byref(h)))
         self._h = h
         self.cfg = cfg
+        self._plans = weakref.WeakSet()          # plans on this handle, closed with it
 
     def shared(self) -> "Scorer":
         """A new handle on the same weights with its own arena (rm_create_shared)."""
         return Scorer(self.cfg, share=self)
 
     def close(self):
+        # a plan uses its handle's arena: plans go first (rm_plan_destroy before rm_destroy)
+        for p in list(getattr(self, "_plans", ())):
+            p.close()
         if getattr(self, "_h", None) is not None and self._h.value:
             lib().rm_destroy(self._h)
             self._h = ctypes.c_void_p()
@@ -207,7 +212,9 @@ class Scorer:
 
     def plan(self, offsets) -> "Plan":
         """rm_plan_create: a prepared batch shape for launch-only scoring."""
-        return Plan(self, offsets)
+        p = Plan(self, offsets)
+        self._plans.add(p)
+        return p
 
     def score_host(self, ids_host, offsets, out_host, stream=None) -> None:
         """rm_score_host: host ids/out (pinned for asynchronous copies)."""
@@ -360,6 +367,8 @@ class Plan:
         self.n = len(off) - 1
 
     def score(self, ids_dev, out_dev, stream=None) -> None:
+        if not self._p:
+            raise RmError(RM_E_INVAL, "the plan (or its scorer) has been closed")
         _check(lib().rm_score_plan(self._p, _ptr(ids_dev), _ptr(out_dev), _stream(stream)))
 
     def close(self):
