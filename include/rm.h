@@ -176,7 +176,9 @@ int rm_score_prefix(rm_handle* h, const int32_t* packed_token_ids, const int32_t
                     float* out_scores, int32_t* out_best, float* out_logodds, void* stream);
 
 /* A plan: the batch shape (seq_offsets) of repeated rm_score calls, prepared
- * once.  rm_plan_create validates the offsets as rm_score does, builds the
+ * once.  The pages have no counterpart to this entry point; it exists so that
+ * a fixed-shape call (batch-1 latency, an ensemble of experts) can be captured
+ * into a CUDA graph and replayed without the host launching each kernel.  rm_plan_create validates the offsets as rm_score does, builds the
  * per-call metadata, allocates a small device block for it (the only
  * allocation; synchronous) and fixes the arena placement.  rm_score_plan then
  * enqueues the kernels alone -- no host synchronisation and no copies -- so it

@@ -48,7 +48,9 @@ int rm_varlen_meta(const int32_t* offsets, int32_t n, int32_t n_heads,
 int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
                int32_t M, int32_t N, int32_t K, int32_t act, void* stream);
 
-/* rm_op_gemm with an explicit output tile: cg = 1 (one CTA per 128 x bn tile,
+/* rm_op_gemm with an explicit output tile (the projections of rm_op_gemm; the
+ * tile choice itself has no counterpart in the pages and is exposed for
+ * testing every tile and for tuning): cg = 1 (one CTA per 128 x bn tile,
  * bn in {64, 96, 128, 160, 192, 224, 256}) or cg = 2 (a cluster of two CTAs
  * per 256 x bn tile on the pair MMA, bn in {128, 192, 256}); cg = 0 takes the
  * tile rm_gemm_tile picks (what rm_op_gemm does).  Same arguments and
@@ -68,8 +70,9 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
 int rm_op_vote(const float* scores, int32_t K, int32_t n, float threshold, int32_t* decision,
                int32_t* votes, void* stream);
 
-/* Host only: the output tile the projections without an activation use for
- * an M x N x K product on a device with num_sms SMs (a GELU epilogue may take
+/* Host only (no counterpart in the pages): the output tile the projections
+ * without an activation use for an M x N x K product on a device with num_sms
+ * SMs (a GELU epilogue may take
  * a single-CTA tile where this returns a pair).  out[0] = cg (1 or 2),
  * out[1] = bn.  RM_E_INVAL for M, N, K or num_sms < 1 or out == NULL. */
 int rm_gemm_tile(int32_t M, int32_t N, int32_t K, int32_t num_sms, int32_t* out);
