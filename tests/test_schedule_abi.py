@@ -97,3 +97,15 @@ def test_latency_knobs_are_validated():
         rm.schedule(sched_cfg(4, 1, 1, 100, objective=2), [3])
     with pytest.raises(rm.RmError):
         rm.schedule(sched_cfg(4, 1, 1, 100, max_cost=-1), [3])
+
+
+def test_default_stream_schedule_matches_the_oracle_and_batch_count():
+    """The schedule bench.py runs: the 10,000-request lengths-2..100 stream,
+    T(b, L) = 20000 + b*L, Bmax 64 -- bit-exact with the oracle, 157 batches."""
+    w = synth.WORKLOADS["bert-base-len2-100"]
+    lengths = synth.make_stream(w).lengths
+    ours = rm.schedule(sched_cfg(64, 20000, 1, 512), lengths)
+    ref, _ = S.schedule_dp(lengths, 64, S.linear_cost(20000, 1))
+    assert np.array_equal(ours, ref)
+    assert int(ours.max()) + 1 == 157
+    assert np.bincount(ours).max() <= 64
