@@ -137,3 +137,20 @@ def test_gemm_tiled_rejects_unknown_tiles_on_host():
         rc = rm.lib().rm_op_gemm_tiled(fake, fake, None, fake, rm.F32, 128, 128, 64, 0, cg, bn, None)
         assert rc == -1, (cg, bn, rc)
         assert b"tile" in rm.lib().rm_last_error()
+
+
+def test_headers_compile_as_c_and_host_calls_run_without_a_gpu(tmp_path):
+    """include/*.h as plain C11 (-Wall -Werror), linked against the library;
+    the host-only calls run here.  The latency objective on four equal
+    requests with T = 2 + b*L takes batches [2, 1, 1] (a worked example of the
+    oracle's pins)."""
+    exe = tmp_path / "abi_from_c"
+    src = os.path.join(ROOT, "tests", "c", "abi_from_c.c")
+    libdir = os.path.join(ROOT, "classifier_scoring_b200")
+    subprocess.run(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    src, "-o", str(exe), "-L", libdir, "-lrmscore", f"-Wl,-rpath,{libdir}"],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    cfg = config_for(synth.TINY)
+    assert int(out[0]) == rm.lib().rm_weights_bytes(ctypes.byref(cfg))
+    assert out[1:] == ["3", "0", "0", "1", "2"]
