@@ -90,6 +90,7 @@ def lib() -> ctypes.CDLL:
         "rm_schedule_cfg": (ctypes.c_int, [cfgp, P, I32, P]),
         "rm_get_device_error": (ctypes.c_int, [P, P]),
         "rm_arena_stats": (ctypes.c_int, [P, P]),
+        "rm_selftest_bounded_wait": (ctypes.c_int, [I64, P, P]),
         "rm_destroy": (None, [P]),
         "rm_profile": (ctypes.c_int, [P, I32]),
         "rm_profile_read": (ctypes.c_int, [P, P, P, P, P, P]),
@@ -381,3 +382,11 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def selftest_bounded_wait(limit_ns: int):
+    """rm_selftest_bounded_wait: (timed_out, elapsed_ns) of a wait that nothing ends."""
+    flag = ctypes.c_int32()
+    ns = ctypes.c_int64()
+    _check(lib().rm_selftest_bounded_wait(int(limit_ns), ctypes.byref(flag), ctypes.byref(ns)))
+    return int(flag.value), int(ns.value)

@@ -972,6 +972,30 @@ int rm_profile_read(rm_handle* h, double* out_ms, int64_t* out_launches, double*
   return RM_OK;
 }
 
+int rm_selftest_bounded_wait(int64_t limit_ns, int32_t* out_timed_out, int64_t* out_elapsed_ns) {
+  if (out_timed_out == nullptr || out_elapsed_ns == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (limit_ns < 1000 || limit_ns > 10000000000LL)
+    return set_error(RM_E_INVAL, "limit_ns must be in 1e3 .. 1e10");
+  void* d = nullptr;
+  RM_CUDA(cudaMalloc(&d, 16));
+  int* d_flag = static_cast<int*>(d);
+  unsigned long long* d_ns = reinterpret_cast<unsigned long long*>(static_cast<char*>(d) + 8);
+  cudaError_t e = cudaMemset(d, 0, 16);
+  if (e == cudaSuccess)
+    e = bounded_wait_selftest(static_cast<unsigned long long>(limit_ns), d_flag, d_ns, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  int flag = 0;
+  unsigned long long ns = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&flag, d_flag, sizeof flag, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(&ns, d_ns, sizeof ns, cudaMemcpyDeviceToHost);
+  cudaFree(d);
+  if (e != cudaSuccess) return set_error(RM_E_CUDA, "self-test: %s", cudaGetErrorString(e));
+  *out_timed_out = flag;
+  *out_elapsed_ns = static_cast<int64_t>(ns);
+  return RM_OK;
+}
+
 int rm_arena_stats(const rm_handle* h, int64_t* out) {
   if (h == nullptr || out == nullptr) return set_error(RM_E_INVAL, "NULL argument");
   out[0] = h->arena_bytes;

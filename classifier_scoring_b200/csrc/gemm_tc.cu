@@ -83,14 +83,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase of the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// Bounded wait for the phase of the given parity to complete; false once
+// limit_ns have passed without it.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity,
+                                              unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
   }
   return true;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
                                             uint32_t bar) {
@@ -654,6 +659,28 @@ cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, GemmTile til
     case 256: return launch_act<256, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+// Failure detection without a fault: one thread waits on an mbarrier that
+// nothing completes, through the same bounded wait the GEMM's roles use, and
+// records whether the wait gave up and how long it took.
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns, int* timed_out,
+                                             unsigned long long* elapsed_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  mbar_init(b, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const unsigned long long t0 = globaltimer_ns();
+  const bool ok = mbar_wait_for(b, 0, limit_ns);   // phase 0 never completes: no arrival
+  *elapsed_ns = globaltimer_ns() - t0;
+  *timed_out = ok ? 0 : 1;
+}
+
+cudaError_t bounded_wait_selftest(unsigned long long limit_ns, int* d_timed_out,
+                                  unsigned long long* d_elapsed_ns, cudaStream_t st) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, d_timed_out, d_elapsed_ns);
+  return cudaGetLastError();
 }
 
 }  // namespace rmk

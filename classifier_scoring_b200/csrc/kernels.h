@@ -18,6 +18,11 @@ struct GemmTile {
   int b_box() const { return bn / cg; }   // weight rows per TMA box
 };
 GemmTile gemm_pick(int M, int N, int K, int num_sms, int act = 0);
+// One thread waits on an mbarrier that nothing completes, with the GEMM's
+// bounded wait and the given limit; writes 1 to *d_timed_out when the wait
+// gave up, and the time it took.
+cudaError_t bounded_wait_selftest(unsigned long long limit_ns, int* d_timed_out,
+                                  unsigned long long* d_elapsed_ns, cudaStream_t st);
 inline int gemm_tile_index(int box_rows) { return (box_rows - 64) / 32; }
 // a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, tile.b_box()}.
 // Persistent grid of min(tiles, num_sms / cg) units of cg CTAs.

@@ -217,6 +217,16 @@ int rm_schedule_cfg(const rm_config* cfg, const int32_t* lengths, int32_t n, int
  * are invalid).  out: host int32[2]. */
 int rm_get_device_error(rm_handle* h, int32_t* out);
 
+/* Failure detection without a fault (the pages have no counterpart): runs on
+ * the current device one thread that waits, through the same bounded
+ * mbarrier wait as the GEMM's producer, MMA and epilogue roles, on a barrier
+ * that nothing completes, giving up after limit_ns (1e3 .. 1e10).  Writes
+ * *out_timed_out = 1 if the wait gave up (the expected result) and the
+ * nanoseconds it waited.  Synchronous; allocates (and frees) 16 bytes of
+ * device memory.  The CUDA context stays usable afterwards.  RM_E_INVAL for
+ * NULL outputs or a limit out of range, RM_E_CUDA on a CUDA error. */
+int rm_selftest_bounded_wait(int64_t limit_ns, int32_t* out_timed_out, int64_t* out_elapsed_ns);
+
 /* Arena figures: out[0] = bytes reserved at create, out[1] = largest plan used
  * by any call so far, out[2] = number of distinct length buckets planned.
  * out: host int64[3]. */
