@@ -305,6 +305,232 @@ def reference_arm(args):
 # ---------------------------------------------------------------------------
 # B200 arm
 # ---------------------------------------------------------------------------
+def stat_summary(vals):
+    """Median and a 95% t-interval of the mean of repeated measurements."""
+    v = np.asarray(vals, dtype=np.float64)
+    n = len(v)
+    mean = float(v.mean())
+    # two-sided 97.5% quantiles of Student's t for n - 1 = 1..9 degrees of freedom
+    tq = {1: 12.706, 2: 4.303, 3: 3.182, 4: 2.776, 5: 2.571, 6: 2.447, 7: 2.365, 8: 2.306, 9: 2.262}
+    half = tq.get(n - 1, 1.96) * float(v.std(ddof=1)) / np.sqrt(n) if n > 1 else 0.0
+    return {"n": n, "values": [float(x) for x in v], "median": float(np.median(v)), "mean": mean,
+            "ci95": [mean - half, mean + half], "min": float(v.min()), "max": float(v.max())}
+
+
+class StreamExecutor:
+    """Scores a request stream as rm_score calls, one per group of request
+    indices (a DP batch, or consecutive DP batches fused), dealt round-robin
+    to lanes (handles that share the weights, one stream each).  Every step
+    re-runs the DP scheduler on the host (S0) and checks it is unchanged."""
+
+    def __init__(self, torch, lanes, streams, st, groups, schedule):
+        self.torch = torch
+        self.lanes, self.streams, self.stream = lanes, streams, streams[0]
+        self.st, self.groups, self.schedule = st, groups, schedule
+        self.nb = len(groups)
+        self.n_req = int(sum(len(g) for g in groups))
+        order = np.concatenate(groups)
+        self.order = order
+        packed_ids, _ = synth.pack(st, order)
+        self.b_tok = np.zeros(self.nb + 1, dtype=np.int64)
+        self.b_seq = np.zeros(self.nb + 1, dtype=np.int64)
+        self.b_off = []
+        for b, g in enumerate(groups):
+            lens = st.lengths[g]
+            self.b_off.append(synth.offsets_from_lengths(lens))
+            self.b_tok[b + 1] = self.b_tok[b] + int(lens.sum())
+            self.b_seq[b + 1] = self.b_seq[b] + len(g)
+        self.ids_dev = torch.from_numpy(packed_ids).cuda()
+        self.out_dev = torch.zeros(self.n_req, dtype=torch.float32, device="cuda")
+        self.ev_batch = [torch.cuda.Event(enable_timing=True) for _ in range(self.nb)]
+        self.fork_ev = torch.cuda.Event()
+        self.join_ev = [torch.cuda.Event() for _ in streams]
+
+    def fork(self):
+        # every lane starts after what stream 0 has enqueued so far
+        self.fork_ev.record(self.stream)
+        for s2 in self.streams[1:]:
+            s2.wait_event(self.fork_ev)
+
+    def join(self):
+        for k, s2 in enumerate(self.streams[1:], 1):
+            self.join_ev[k].record(s2)
+            self.stream.wait_event(self.join_ev[k])
+
+    def step(self, record=False):
+        bt = self.lanes[0].schedule(self.st.lengths)                  # S0 on the host
+        if self.schedule is not None and record and not np.array_equal(bt, self.schedule):
+            raise RuntimeError("schedule changed between steps")
+        for b in range(self.nb):
+            k = b % len(self.lanes)
+            self.lanes[k].score(self.ids_dev[self.b_tok[b]:], self.b_off[b],
+                                self.out_dev[self.b_seq[b]:], self.streams[k])
+            if record:
+                self.ev_batch[b].record(self.streams[k])
+
+    def warm(self, n):
+        for _ in range(n):
+            self.fork()
+            self.step()
+            self.join()
+        self.torch.cuda.synchronize()
+
+    def timed(self, steps, barrier, record_last=False):
+        """CUDA-event milliseconds of `steps` steps on stream 0 (all lanes joined)."""
+        torch = self.torch
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(self.stream)
+        self.fork()
+        for k in range(steps):
+            self.step(record=record_last and k == steps - 1)
+        self.join()
+        b.record(self.stream)
+        torch.cuda.synchronize()
+        barrier()
+        return a.elapsed_time(b)
+
+    def latency(self, ms_per_step):
+        """p50 / p99 request latency in the last recorded step: every request is
+        queued at the step's start and completes with its call; the step's start
+        is the last call's completion minus the mean step time."""
+        per_batch = np.array([self.ev_batch[0].elapsed_time(e) for e in self.ev_batch])
+        first_done = ms_per_step - per_batch[-1]
+        lat = np.empty(self.n_req)
+        for b in range(self.nb):
+            lat[self.b_seq[b]:self.b_seq[b + 1]] = per_batch[b] + first_done
+        return float(np.median(lat)), float(np.percentile(lat, 99))
+
+    def profiled_step(self, sc):
+        """One step on a single stream with per-launch CUDA events (after timing)."""
+        sc.profile(1)
+        for b in range(self.nb):
+            sc.score(self.ids_dev[self.b_tok[b]:], self.b_off[b], self.out_dev[self.b_seq[b]:],
+                     self.stream)
+        self.torch.cuda.synchronize()
+        prof = sc.profile_read()
+        sc.profile(0)
+        return prof
+
+
+def launches_of(lanes):
+    return sum(h.profile_read()["total_launches"] for h in lanes)
+
+
+def arena_line(sc, note):
+    reserved, peak, nbuckets = (int(x) for x in sc.arena_stats())
+    return {"reserved_bytes": reserved, "peak_planned_bytes": peak, "buckets": nbuckets, "sized_for": note}
+
+
+def scorer_cfg(rm, s, w, fuse, max_len):
+    return rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
+                            ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos,
+                            weight_dtype=s.weight_dtype, gelu=s.gelu, ln_eps=s.ln_eps,
+                            max_batch_seqs=fuse * w.max_batch,
+                            max_tokens=fuse * w.max_batch * max_len, max_len=max_len,
+                            sched_max_batch=w.max_batch, sched_c0=SCHED_C0, sched_c1=SCHED_C1)
+
+
+def fused_groups(groups, fuse):
+    return [np.concatenate(groups[k:k + fuse]) for k in range(0, len(groups), fuse)]
+
+
+def secondary_workloads(args, torch, rm):
+    """The pages' other workloads, each on its own handle, one GPU, timed with
+    CUDA events after warm-up (reported beside the headline, not in it)."""
+    out = {}
+    stream = torch.cuda.Stream()
+    # lengths 5..500 (TurboTransformers review, main results: 144 req/s on its hardware)
+    name = "bert-base-len5-500"
+    w = synth.WORKLOADS[name]
+    s = w.shape
+    st = synth.make_stream(w)
+    max_len = min(s.max_pos, 1024, w.len_hi)
+    sc = rm.Scorer(scorer_cfg(rm, s, w, args.fuse, max_len), synth.make_weights(s, w.seed))
+    lanes = [sc] + [sc.shared() for _ in range(args.lanes - 1)]
+    streams = [stream] + [torch.cuda.Stream() for _ in range(args.lanes - 1)]
+    batch = sc.schedule(st.lengths)
+    groups = [np.nonzero(batch == b)[0] for b in range(int(batch.max()) + 1)]
+    row = {"metric": metric_for(name), "unit": UNIT, "config": workload_config(name)}
+    for label, gr in (("value", fused_groups(groups, args.fuse)), ("value_unfused", groups)):
+        ex = StreamExecutor(torch, lanes, streams, st, gr, batch)
+        ex.warm(2)
+        l0 = launches_of(lanes)
+        ms = ex.timed(args.extra_steps, lambda: None)
+        row[label] = ex.n_req * args.extra_steps / (ms / 1000.0)
+        row["ms_per_step" if label == "value" else "ms_per_step_unfused"] = ms / args.extra_steps
+        if label == "value":
+            row["gpu_launches"] = launches_of(lanes) - l0
+        del ex
+    row["steps"], row["warmup"] = args.extra_steps, 2
+    row["executor"] = {"lanes": len(lanes), "fuse": args.fuse, "unfused": "one DP batch (<= 32) per call"}
+    row["arena"] = arena_line(sc, f"{args.fuse} x {w.max_batch} sequences x {max_len} tokens")
+    for h in lanes:
+        h.close()
+    out[name] = row
+    torch.cuda.empty_cache()
+
+    # GPT-style 1.3B-shape reward model, batches of 64 sequences of 256..560 tokens
+    name = "gpt-1.3b-rm"
+    w = synth.WORKLOADS[name]
+    s = w.shape
+    st = synth.make_stream(w)
+    sc = rm.Scorer(scorer_cfg(rm, s, w, 1, w.len_hi), synth.make_weights(s, w.seed))
+    ex = StreamExecutor(torch, [sc], [stream], st, [np.arange(w.max_batch)], None)
+    ex.warm(2)
+    l0 = launches_of([sc])
+    ms = ex.timed(args.extra_steps, lambda: None)
+    n_launch = launches_of([sc]) - l0
+    prof = ex.profiled_step(sc)
+    pk, pk_kind = peaks()
+    g = prof["gemm"]
+    tf = g["flops"] / (g["ms"] * 1e-3) / 1e12 if g["ms"] > 0 else None
+    out[name] = {"metric": metric_for(name), "unit": UNIT, "value": w.max_batch * args.extra_steps / (ms / 1000.0),
+                 "ms_per_step": ms / args.extra_steps, "steps": args.extra_steps, "warmup": 2,
+                 "gpu_launches": n_launch,
+                 "config": workload_config(name),
+                 "gemm_tflops": tf, "gemm_frac_of_sustained": tf / pk["bf16_tflops_sustained"] if tf else None,
+                 "arena": arena_line(sc, f"{w.max_batch} sequences x {w.len_hi} tokens")}
+    sc.close()
+    del ex
+    torch.cuda.empty_cache()
+
+    # TinyBERT shape at batch 1, lengths 64 / 128 / 256 (SambaNova blog, Fig. 3)
+    name = "tinybert-b1"
+    w = synth.WORKLOADS[name]
+    s = w.shape
+    Lmax = max(w.fixed_lengths)
+    cfg = rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
+                           ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos, weight_dtype=s.weight_dtype,
+                           gelu=s.gelu, ln_eps=s.ln_eps, max_batch_seqs=1, max_tokens=Lmax,
+                           max_len=Lmax, sched_max_batch=1)
+    sc = rm.Scorer(cfg, synth.make_weights(s, w.seed))
+    o = torch.zeros(1, device="cuda")
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lat = {}
+    for L in w.fixed_lengths:
+        ids = torch.from_numpy(synth.make_token_ids(L, s.vocab, w.seed + L)).cuda()
+        off = np.array([0, L], dtype=np.int32)
+        vals = []
+        for r in range(20 + args.extra_requests):
+            torch.cuda.synchronize()
+            a.record(stream)
+            sc.score(ids, off, o, stream)
+            b.record(stream)
+            b.synchronize()
+            if r >= 20:
+                vals.append(a.elapsed_time(b))
+        lat[str(L)] = {"p50_ms": float(np.median(vals)), "p99_ms": float(np.percentile(vals, 99))}
+    out[name] = {"metric": "batch-1 p50 latency, TinyBERT shape (4 layers, H 312), eager rm_score from an idle GPU",
+                 "unit": "ms", "higher_is_better": False, "requests_per_length": args.extra_requests,
+                 "warmup": 20, "latency": lat, "value": lat[str(w.fixed_lengths[1])]["p50_ms"],
+                 "value_is": f"p50 at length {w.fixed_lengths[1]}",
+                 "arena": arena_line(sc, f"1 sequence x {Lmax} tokens")}
+    sc.close()
+    return out
+
+
 def b200_arm(args):
     import torch
     import classifier_scoring_b200 as rm
@@ -321,175 +547,89 @@ def b200_arm(args):
                                 device_id=torch.device("cuda", local))
     rmbuild.build()
 
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
     name = args.workload
     w = synth.WORKLOADS[name]
     s = w.shape
     flat = synth.make_weights(s, w.seed)
     st = synth.make_stream(replica_workload(w, rank))            # each replica its own requests
-    n_req = len(st.lengths)
     max_len = min(s.max_pos, 1024, max(w.len_hi, int(st.lengths.max())))
 
-    def make_cfg(fuse):
-        return rm.RmConfig.make(arch=s.arch, n_layers=s.n_layers, hidden=s.hidden, n_heads=s.n_heads,
-                                ffn=s.ffn, vocab=s.vocab, max_pos=s.max_pos,
-                                weight_dtype=s.weight_dtype, gelu=s.gelu, ln_eps=s.ln_eps,
-                                max_batch_seqs=fuse * w.max_batch,
-                                max_tokens=fuse * w.max_batch * max_len, max_len=max_len,
-                                sched_max_batch=w.max_batch, sched_c0=SCHED_C0, sched_c1=SCHED_C1)
     # fusing more batches than the stream has only enlarges the arena
-    n_sched = int(rm.schedule(make_cfg(1), st.lengths).max()) + 1
+    n_sched = int(rm.schedule(scorer_cfg(rm, s, w, 1, max_len), st.lengths).max()) + 1
     args.fuse = max(1, min(args.fuse, n_sched))
-    cfg = make_cfg(args.fuse)
-    sc = rm.Scorer(cfg, flat)
+    sc = rm.Scorer(scorer_cfg(rm, s, w, args.fuse, max_len), flat)
     del flat
-    # lanes: handles that share the weights, each on its own stream, so that
-    # consecutive batches overlap on the GPU
     lanes = [sc] + [sc.shared() for _ in range(args.lanes - 1)]
     streams = [torch.cuda.Stream() for _ in range(args.lanes)]
     stream = streams[0]
 
-    # the schedule is deterministic: pack the stream in batch order once, on the device
+    # the schedule is deterministic: pack the stream in call order once, on the device
     batch = sc.schedule(st.lengths)
     nb = int(batch.max()) + 1
-    groups = [np.nonzero(batch == b)[0] for b in range(nb)]
+    dp_groups = [np.nonzero(batch == b)[0] for b in range(nb)]
     n_dp_batches = nb
     if args.batch_index is not None:
-        # one call only (small profiling case): the step scores just this DP
-        # batch, or the `fuse` consecutive batches starting with it
-        keep = np.concatenate(groups[args.batch_index % nb:args.batch_index % nb + args.fuse])
-        sub = np.zeros(len(st.lengths), dtype=bool)
-        sub[keep] = True
+        # one call only (small profiling case): this DP batch, or the `fuse`
+        # consecutive batches starting with it
+        keep = np.concatenate(dp_groups[args.batch_index % nb:args.batch_index % nb + args.fuse])
         st = synth.Stream(lengths=st.lengths[keep], ids=st.ids, starts=st.starts[keep])
-        n_req = len(keep)
-        batch = np.zeros(n_req, dtype=np.int32)
-        nb = 1
-        groups = [np.arange(n_req)]
+        batch = None
+        groups = [np.arange(len(keep))]
         n_dp_batches = min(args.fuse, n_dp_batches)
-    elif args.fuse > 1:
+        unfused = None
+    else:
         # executor: consecutive DP batches run as one forward pass (packed, so
         # the result of every request is the same; the projections get more rows)
-        groups = [np.concatenate(groups[k:k + args.fuse]) for k in range(0, nb, args.fuse)]
-        nb = len(groups)
-    order = np.concatenate(groups)
-    packed_ids, _ = synth.pack(st, order)
-    b_tok = np.zeros(nb + 1, dtype=np.int64)
-    b_seq = np.zeros(nb + 1, dtype=np.int64)
-    b_off = []
-    for b, g in enumerate(groups):
-        lens = st.lengths[g]
-        b_off.append(synth.offsets_from_lengths(lens))
-        b_tok[b + 1] = b_tok[b] + int(lens.sum())
-        b_seq[b + 1] = b_seq[b] + len(g)
-    ids_dev = torch.from_numpy(packed_ids).cuda()
-    out_dev = torch.zeros(n_req, dtype=torch.float32, device="cuda")
-    ev_batch = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
+        groups = fused_groups(dp_groups, args.fuse)
+        unfused = dp_groups if args.fuse > 1 else None
+    ex = StreamExecutor(torch, lanes, streams, st, groups, batch)
+    n_req = ex.n_req
 
-    fork_ev = torch.cuda.Event()
-    join_ev = [torch.cuda.Event() for _ in streams]
+    # warm-up (plans every length bucket; the kernels are prebuilt)
+    ex.warm(args.warmup)
+    ex_u = None
+    if unfused is not None:
+        ex_u = StreamExecutor(torch, lanes, streams, st, unfused, batch)
+        ex_u.warm(max(3, args.warmup // 2))
 
-    def fork():
-        # every lane starts after what stream 0 has enqueued so far
-        fork_ev.record(stream)
-        for s2 in streams[1:]:
-            s2.wait_event(fork_ev)
-
-    def join():
-        for k, s2 in enumerate(streams[1:], 1):
-            join_ev[k].record(s2)
-            stream.wait_event(join_ev[k])
-
-    def step(record=False):
-        bt = sc.schedule(st.lengths)                          # S0 on the host
-        if record and args.batch_index is None and not np.array_equal(bt, batch):
-            raise RuntimeError("schedule changed between steps")
-        for b in range(nb):
-            k = b % len(lanes)
-            lanes[k].score(ids_dev[b_tok[b]:], b_off[b], out_dev[b_seq[b]:], streams[k])
-            if record:
-                ev_batch[b].record(streams[k])
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    # warm-up (plans every length bucket, compiles nothing: the kernels are prebuilt)
-    for _ in range(args.warmup):
-        fork()
-        step()
-        join()
-    torch.cuda.synchronize()
-
-    launches0 = 0
     for h in lanes:
+        # per-launch CUDA events inside the timed regions only on request
+        # (--profile-every n > 0, a diagnostic that breaks launch overlap)
         h.profile(args.profile_every)
-        launches0 += h.profile_read()["total_launches"]
-        h.profile(args.profile_every)
+    launches0 = launches_of(lanes)
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
     clocks = ClockSampler(gpu_index, clocks_log(args, f"clocks_rank{rank}.csv"))
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
     wall0 = time.perf_counter()
-    t_start.record(stream)
-    fork()
-    for k in range(args.steps):
-        step(record=(k == args.steps - 1))
-    join()
-    t_end.record(stream)
-    torch.cuda.synchronize()
+    elapsed_ms = ex.timed(args.steps, barrier, record_last=True)
     wall = time.perf_counter() - wall0
-    barrier()
+    launches = launches_of(lanes) - launches0
+    # further independent timed regions of the same K steps, for a spread
+    rep_ms = [elapsed_ms] + [ex.timed(args.steps, barrier) for _ in range(args.repeats - 1)]
+    unf_ms = ex_u.timed(args.steps, barrier) if ex_u is not None else None
     clk = clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
-    prof = None
-    for h in lanes:
-        p1 = h.profile_read()
-        h.profile(0)
-        if prof is None:
-            prof = p1
-        else:
-            for kname in KERNEL_NAMES:
-                for f in ("ms", "launches", "flops", "bytes"):
-                    prof[kname][f] += p1[kname][f]
-            prof["total_launches"] += p1["total_launches"]
-    launches = prof["total_launches"] - launches0
-    prof_timed = prof
-    if len(lanes) > 1 and args.profile_every > 0:
-        # Per-launch kernel durations from the timed region overlap across the
-        # lanes' streams; the roofline takes them from one extra step run on a
-        # single stream instead (same batches, same kernels, after the timing).
-        sc.profile(args.profile_every)
-        for b in range(nb):
-            sc.score(ids_dev[b_tok[b]:], b_off[b], out_dev[b_seq[b]:], stream)
-        torch.cuda.synchronize()
-        prof = sc.profile_read()
-        sc.profile(0)
-    # latency in the last timed step: every request is queued at the step's start
-    # and completes with its batch; the step's start is taken as the last
-    # batch's completion minus the mean step time
-    per_batch = np.array([ev_batch[0].elapsed_time(e) for e in ev_batch])
-    first_done = elapsed_ms / args.steps - per_batch[-1]
-    lat = np.empty(n_req)
-    for b in range(nb):
-        lat[b_seq[b]:b_seq[b + 1]] = per_batch[b] + first_done
-    p50 = float(np.median(lat))
-    p99 = float(np.percentile(lat, 99))
+    p50, p99 = ex.latency(elapsed_ms / args.steps)
+    # kernel table and roofline from one extra single-stream step after timing
+    prof = ex.profiled_step(sc)
 
     # ---- end to end through rm_score_host (pinned host buffers) ----
+    b_tok, b_seq, b_off = ex.b_tok, ex.b_seq, ex.b_off
     ids_pin = torch.empty(int(b_tok[-1]), dtype=torch.int32).pin_memory()
     out_pin = torch.empty(n_req, dtype=torch.float32).pin_memory()
     ids_np = ids_pin.numpy()
     host_ids = st.ids
-    # position in the arrival-ordered id array of every packed token (batch order)
-    gather = np.concatenate([np.arange(st.starts[i], st.starts[i] + st.lengths[i]) for i in order])
+    # position in the arrival-ordered id array of every packed token (call order)
+    gather = np.concatenate([np.arange(st.starts[i], st.starts[i] + st.lengths[i]) for i in ex.order])
 
     def e2e_step():
         sc.schedule(st.lengths)                               # S0
         np.take(host_ids, gather, out=ids_np)                 # S1: host gather into pinned memory
-        for b in range(nb):
+        for b in range(ex.nb):
             k = b % len(lanes)
             lanes[k].score_host(ids_pin[b_tok[b]:], b_off[b], out_pin[b_seq[b]:], streams[k])
 
@@ -500,25 +640,28 @@ def b200_arm(args):
     e1 = torch.cuda.Event(enable_timing=True)
     ew0 = time.perf_counter()
     e0.record(stream)
-    fork()
+    ex.fork()
     e_steps = max(1, args.steps)
     for _ in range(e_steps):
         e2e_step()
-    join()
+    ex.join()
     e1.record(stream)
     torch.cuda.synchronize()
     e_wall = time.perf_counter() - ew0
     barrier()
     e_ms = max(e0.elapsed_time(e1), 1000 * e_wall)
-    if not np.array_equal(out_pin.numpy(), out_dev.cpu().numpy()):
+    if not np.array_equal(out_pin.numpy(), ex.out_dev.cpu().numpy()):
         raise RuntimeError("rm_score_host and rm_score disagree")
     meta_bytes = sum(4 * (len(o)) * 2 + 8 * len(o) for o in b_off)
     h2d = 4 * int(b_tok[-1]) + meta_bytes
     d2h = 4 * n_req
 
     # ---- reduce over ranks ----
-    vals = reduce_times([elapsed_ms, e_ms], dist, "cuda")
+    vals = reduce_times([elapsed_ms, e_ms] + rep_ms + ([unf_ms] if unf_ms is not None else []),
+                        dist, "cuda")
     max_ms, max_e_ms = float(vals[0]), float(vals[1])
+    max_rep = [float(x) for x in vals[2:2 + len(rep_ms)]]
+    max_unf = float(vals[-1]) if unf_ms is not None else None
     value = whole_job_rate(world, n_req, args.steps, max_ms)
     e2e_value = whole_job_rate(world, n_req, e_steps, max_e_ms)
 
@@ -529,37 +672,32 @@ def b200_arm(args):
     traffic = (GEMM_TRAFFIC["bytes_per_launch"]
                if (GEMM_TRAFFIC["src_sha"] == sha and GEMM_TRAFFIC["workload"] == name
                    and GEMM_TRAFFIC["fuse"] == args.fuse and args.batch_index is None) else None)
-    measured_on = ("the timed region" if prof is prof_timed else
-                   "one extra single-stream step after the timed region (the timed region "
-                   f"ran {len(lanes)} overlapping streams)")
     roofline = {"kernel": "gemm_bf16_tc_kernel (QKV, output and FFN projections)",
-                "measured_on": measured_on,
+                "measured_on": "one single-stream step with per-launch CUDA events, after the timed "
+                               "regions (which ran without per-launch events)",
                 "bound": "tensor", "achieved": gemm_tflops, "peak": pk["bf16_tflops_sustained"],
                 "unit": "TFLOP/s",
                 "frac": (gemm_tflops / pk["bf16_tflops_sustained"]) if gemm_tflops else None,
                 "peak_source": f"bf16_tflops_sustained of {pk_kind} (kernel timed inside a long step)",
                 "traffic": traffic,
                 "launches_timed": g["launches"], "avg_launch_us": 1000 * g["ms"] / max(1, g["launches"])}
-    def kernel_table(pr):
-        out = {}
-        total_ms = max(1e-9, sum(pr[x]["ms"] for x in KERNEL_NAMES))
-        for kname in KERNEL_NAMES:
-            d = pr[kname]
-            if d["launches"] == 0:
-                continue
-            e = {"launches_timed": d["launches"], "avg_us": 1000 * d["ms"] / d["launches"],
-                 "share_of_timed": d["ms"] / total_ms}
-            if d["flops"] and kname in ("gemm", "attn_scores", "attn_context", "attn_fused"):
-                e["tflops"] = d["flops"] / (d["ms"] * 1e-3) / 1e12
-            if d["bytes"]:
-                e["gbs"] = d["bytes"] / (d["ms"] * 1e-3) / 1e9
-                e["hbm_frac_of_measured"] = e["gbs"] / pk["hbm_gbs"]
-            out[kname] = e
-        return out
 
-    kernels = kernel_table(prof)
-    kernels_timed = kernel_table(prof_timed) if prof is not prof_timed else None
+    total_ms = max(1e-9, sum(prof[x]["ms"] for x in KERNEL_NAMES))
+    kernels = {}
+    for kname in KERNEL_NAMES:
+        d = prof[kname]
+        if d["launches"] == 0:
+            continue
+        e = {"launches": d["launches"], "avg_us": 1000 * d["ms"] / d["launches"],
+             "share": d["ms"] / total_ms}
+        if d["flops"] and kname in ("gemm", "attn_scores", "attn_context", "attn_fused"):
+            e["tflops"] = d["flops"] / (d["ms"] * 1e-3) / 1e12
+        if d["bytes"]:
+            e["gbs"] = d["bytes"] / (d["ms"] * 1e-3) / 1e9
+            e["hbm_frac_of_measured"] = e["gbs"] / pk["hbm_gbs"]
+        kernels[kname] = e
 
+    rep_vals = [whole_job_rate(world, n_req, args.steps, m) for m in max_rep]
     result = {
         "metric": metric_for(name), "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
@@ -567,29 +705,41 @@ def b200_arm(args):
         "config": dict(workload_config(name), lanes=lanes_note(len(lanes)),
                        **({"fuse": f"{args.fuse} consecutive DP batches per rm_score call"}
                           if args.fuse > 1 else {})),
+        "repeats": dict(stat_summary(rep_vals), unit=UNIT,
+                        method=f"{len(rep_vals)} timed regions of {args.steps} steps each in this "
+                               "process (the first is `value`); 95% t-interval of the mean"),
         "p50_latency_ms": p50, "p99_latency_ms": p99, "batches_per_step": n_dp_batches,
-        "calls_per_step": nb,
+        "calls_per_step": ex.nb,
         "tokens_per_step": int(b_tok[-1]),
         "roofline": roofline,
         "kernels": kernels,
-        "kernels_timed_region": kernels_timed,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "rm_score_host, pinned host ids/scores"},
         "gpu_launches": int(launches),
         "clocks": clk,
         "wall_s_timed": wall,
+        "arena": arena_line(sc, f"{args.fuse} x {w.max_batch} sequences x {max_len} tokens"),
         "context": {"turbotransformers_req_s_len2_100": 402, "hardware": "not named on the page"},
     }
+    if max_unf is not None:
+        result["value_unfused"] = whole_job_rate(world, n_req, args.steps, max_unf)
+        result["unfused"] = {"ms_per_step": max_unf / args.steps, "calls_per_step": len(unfused),
+                             "executor": f"one DP batch (<= {w.max_batch} sequences) per rm_score call, "
+                                         f"{len(lanes)} lanes"}
+    for h in lanes:
+        h.close()
+    del ex, ex_u
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, k, el = OracleTimer(name).run(args.cpu_budget)
         result["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": oracle_threads(),
                                   "kind": "oracle",
                                   "sample": f"first {k} requests of the seeded stream scored one by "
                                             f"one by the fp64 numpy oracle ({el:.1f} s)"}
+    if world == 1 and args.batch_index is None and not args.no_extra and name == "bert-base-len2-100":
+        result["other_workloads"] = secondary_workloads(args, torch, rm)
     if rank == 0:
         print(json.dumps(result), flush=True)
-    for h in lanes:
-        h.close()
     if dist is not None:
         dist.destroy_process_group()
     return 0
@@ -1062,8 +1212,16 @@ def main():
     ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
     ap.add_argument("--workload", default="bert-base-len2-100",
                     choices=list(synth.WORKLOADS) + list(synth.PREFIX_WORKLOADS))
-    ap.add_argument("--profile-every", type=int, default=8,
-                    help="time the kernels of every n-th batch with CUDA events (0 = off)")
+    ap.add_argument("--profile-every", type=int, default=0,
+                    help="diagnostic: CUDA events around the launches of every n-th call inside the "
+                         "timed regions (0 = off; the kernel table always comes from a separate step)")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed regions of --steps steps each (median and 95%% interval reported)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads (lengths 5-500, GPT-1.3B shape, TinyBERT batch 1)")
+    ap.add_argument("--extra-steps", type=int, default=3, help="timed steps of each other workload")
+    ap.add_argument("--extra-requests", type=int, default=200,
+                    help="timed batch-1 requests per length of the TinyBERT workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clocks-dir", default=None,
@@ -1082,6 +1240,7 @@ def main():
     ap.add_argument("--batch-index", type=int, default=None,
                     help="score only this DP batch of the stream per step (small profiling case)")
     args = ap.parse_args()
+    args.repeats = max(1, args.repeats)
     if args.warmup < 3 and args.impl == "b200":
         print("note: at least 3 warm-up steps are required; using 3", file=sys.stderr)
         args.warmup = 3

@@ -20,6 +20,7 @@ __all__ = ["RmConfig", "RmError", "Scorer", "lib", "schedule", "weights_bytes", 
 
 ENC_POSTLN, DEC_PRELN = 0, 1
 F32, BF16 = 0, 1
+ROWS_RESID_F32 = 2          # res_ln rows: x fp32, y and z bf16
 GELU_ERF, GELU_TANH = 0, 1
 ATTN_FUSED, ATTN_MATERIALIZED = 0, 1
 RM_OK, RM_E_INVAL, RM_E_NOMEM, RM_E_CUDA, RM_E_RANGE, RM_E_DEVICE = 0, -1, -2, -3, -4, -5
@@ -91,6 +92,7 @@ def lib() -> ctypes.CDLL:
         "rm_get_device_error": (ctypes.c_int, [P, P]),
         "rm_arena_stats": (ctypes.c_int, [P, P]),
         "rm_selftest_bounded_wait": (ctypes.c_int, [I64, P, P]),
+        "rm_debug_fail_alloc": (ctypes.c_int, [I32]),
         "rm_destroy": (None, [P]),
         "rm_profile": (ctypes.c_int, [P, I32]),
         "rm_profile_read": (ctypes.c_int, [P, P, P, P, P, P]),
@@ -100,7 +102,7 @@ def lib() -> ctypes.CDLL:
         "rm_op_gemm_tiled": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P]),
         "rm_gemm_tile": (ctypes.c_int, [I32, I32, I32, I32, P]),
         "rm_op_vote": (ctypes.c_int, [P, I32, I32, F, P, P, P]),
-        "rm_op_embed": (ctypes.c_int, [P, P, I32, I32, P, P, P, P, F, I32, I32, I32, P, P, P]),
+        "rm_op_embed": (ctypes.c_int, [P, P, I32, I32, P, P, P, P, F, I32, I32, I32, P, I32, P, P]),
         "rm_op_attn_scores": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_softmax": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attn_context": (ctypes.c_int, [P, P, P, P, P, P, I32, I32, I32, I32, I32, P]),
@@ -295,10 +297,10 @@ class ops:
 
     @staticmethod
     def embed(ids, offsets_dev, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps, V, P, H, x,
-              err_count=None, stream=None):
+              err_count=None, stream=None, x_dtype=BF16):
         _check(lib().rm_op_embed(_ptr(ids), _ptr(offsets_dev), n_seqs, T, _ptr(emb_word),
                                  _ptr(emb_pos), _ptr(ln_g), _ptr(ln_b), eps, V, P, H, _ptr(x),
-                                 _ptr(err_count), _stream(stream)))
+                                 x_dtype, _ptr(err_count), _stream(stream)))
 
     @staticmethod
     def attn_scores(qkv, S, offsets_dev, rb_dev, so_dev, n_seqs, n_row_blocks, n_heads, head_dim,
@@ -382,6 +384,11 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def debug_fail_alloc(k: int) -> None:
+    """rm_debug_fail_alloc: the k-th library allocation from now on fails (0 disarms)."""
+    _check(lib().rm_debug_fail_alloc(int(k)))
 
 
 def selftest_bounded_wait(limit_ns: int):

@@ -1,5 +1,6 @@
 // C ABI of the scorer (include/rm.h, include/rm_ops.h): validation, weight
 // upload, the arena, per-call metadata and the forward launch sequence.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -21,6 +22,33 @@ namespace rmk {
 namespace {
 thread_local char g_msg[512] = "";
 __device__ int32_t g_err_sink[ERR_WORDS];   // error words for handle-less rm_op_* calls
+
+// Test hook (rm_debug_fail_alloc): the k-th allocation from now on fails as if
+// memory were exhausted, without reaching the allocator.
+std::atomic<int32_t> g_fail_alloc{0};
+
+bool injected_alloc_failure() {
+  int32_t k = g_fail_alloc.load();
+  while (k > 0)
+    if (g_fail_alloc.compare_exchange_weak(k, k - 1)) return k == 1;
+  return false;
+}
+
+cudaError_t dev_malloc(void** p, size_t bytes) {
+  if (injected_alloc_failure()) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaMalloc(p, bytes);
+}
+
+cudaError_t pinned_malloc(void** p, size_t bytes) {
+  if (injected_alloc_failure()) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaHostAlloc(p, bytes, cudaHostAllocDefault);
+}
 }  // namespace
 
 int set_error(int code, const char* fmt, ...) {
@@ -251,9 +279,9 @@ int upload_weights(rm_handle* h, const void* weights) {
     total += s.elems;
   }
   const size_t wbytes = static_cast<size_t>(nbf) * 2 + static_cast<size_t>(nf) * 4;
-  RM_CUDA(cudaMalloc(&h->wbuf, wbytes));
+  RM_CUDA(dev_malloc(&h->wbuf, wbytes));
   void* staging = nullptr;
-  RM_CUDA(cudaMalloc(&staging, static_cast<size_t>(total) * esz));
+  RM_CUDA(dev_malloc(&staging, static_cast<size_t>(total) * esz));
   cudaError_t e = cudaMemcpy(staging, weights, static_cast<size_t>(total) * esz, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     cudaFree(staging);
@@ -331,8 +359,11 @@ int upload_weights(rm_handle* h, const void* weights) {
 }
 
 int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
-  // length buckets: tokens rounded up to 128, score elements to 64 Ki
-  const int64_t Tb = align_up(T, 128), Sb = align_up(std::max<int64_t>(S, 1), 65536);
+  // length buckets: tokens rounded up to 128, score elements to 64 Ki; the
+  // fused attention keeps no score matrix, so its buckets are keyed on tokens alone
+  const int64_t Tb = align_up(T, 128);
+  const int64_t Sb =
+      h->cfg.attn_impl == RM_ATTN_FUSED ? 0 : align_up(std::max<int64_t>(S, 1), 65536);
   auto key = std::make_pair(Tb, Sb);
   auto it = h->buckets.find(key);
   if (it != h->buckets.end()) {
@@ -341,7 +372,7 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
   }
   const rm_config* c = &h->cfg;
   Bucket b;
-  b.plan = plan_arena(c->arch, c->hidden, c->ffn, Tb, c->attn_impl == RM_ATTN_FUSED ? 0 : Sb);
+  b.plan = plan_arena(c->arch, c->hidden, c->ffn, Tb, Sb);
   if (h->fixed_bytes + b.plan.peak > h->arena_bytes)
     return set_error(RM_E_RANGE, "arena plan (%lld bytes) exceeds the reservation",
                      (long long)b.plan.peak);
@@ -587,15 +618,21 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
   const unsigned long long w_qkv_b = 2ull * 3 * H * H, w_o_b = 2ull * H * H, w_1_b = 2ull * F * H,
                            w_2_b = 2ull * H * F;
   const L2Prefetch pf_qkv0 = pf_of(h->layers[0].w_qkv, w_qkv_b, nullptr, 0);
-  RM_KERNEL(RM_K_EMBED, 0, 6.0 * Td * Hd + 4.0 * Td,
+  // the decoder's residual stream x is fp32 (row dtype 2 of the LayerNorm:
+  // y and z bf16, x fp32); the encoder's x is the bf16 LayerNorm output
+  const int ln_dtype = dec ? 2 : 1;
+  RM_KERNEL(RM_K_EMBED, 0, (dec ? 8.0 : 6.0) * Td * Hd + 4.0 * Td,
             embed_launch(d_ids, d_off, n, T, h->emb_word, h->emb_pos, dec ? nullptr : h->ln_emb_g,
                          dec ? nullptr : h->ln_emb_b, eps, c->vocab, c->max_pos, H, x,
-                         h->d_err + ERR_CLAMPED, st, dec ? L2Prefetch{} : pf_qkv0, d_pln));
+                         h->d_err + ERR_CLAMPED, st, dec ? L2Prefetch{} : pf_qkv0, d_pln,
+                         dec ? 0 : 1));
   if (dec)
-    RM_KERNEL(RM_K_LAYERNORM, 0, 4.0 * Td * Hd,
-              res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps, 1, 2, st,
-                            pf_qkv0));
-  const double ln_bytes = (dec ? 8.0 : 6.0) * Td * Hd;
+    RM_KERNEL(RM_K_LAYERNORM, 0, 6.0 * Td * Hd,
+              res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps,
+                            ln_dtype, 2, st, pf_qkv0));
+  // algorithmic bytes per token: post-LN reads y, x and writes x (bf16); the
+  // decoder reads y (bf16) and x (fp32), writes x (fp32) and z (bf16)
+  const double ln_bytes = (dec ? 12.0 : 6.0) * Td * Hd;
   for (int l = 0; l < c->n_layers; ++l) {
     const LayerW& L = h->layers[l];
     const L2Prefetch pf_o = pf_of(L.w_o, w_o_b, nullptr, 0);
@@ -622,16 +659,16 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
             gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st));
     if (!dec) {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, 1, 0, st, pf_ffn));
+                res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, ln_dtype, 0, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
               gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
       RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
               gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st));
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, 1, 0, st, pf_next));
+                res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 0, st, pf_next));
     } else {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, 1, 1, st, pf_ffn));
+                res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 1, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
               gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
       RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
@@ -639,7 +676,8 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
       const bool last = l + 1 == c->n_layers;
       const float* g = last ? h->lnf_g : h->layers[l + 1].ln1_g;
       const float* b = last ? h->lnf_b : h->layers[l + 1].ln1_b;
-      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes, res_ln_launch(y2, x, z, g, b, T, H, eps, 1, 1, st, pf_next));
+      RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
+                res_ln_launch(y2, x, z, g, b, T, H, eps, ln_dtype, 1, st, pf_next));
     }
   }
   RM_KERNEL(RM_K_HEAD, 2.0 * n * Hd, 2.0 * n * Hd + 4.0 * n,
@@ -664,11 +702,11 @@ int alloc_runtime(rm_handle* h) {
       cfg->attn_impl == RM_ATTN_FUSED ? 0 : align_up(std::max<int64_t>(Smax, 1), 65536);
   h->arena_bytes =
       h->fixed_bytes + arena_bound(cfg->arch, cfg->hidden, cfg->ffn, align_up(T, 128), Sres);
-  cudaError_t e = cudaMalloc(&h->arena, h->arena_bytes);
-  if (e == cudaSuccess) e = cudaMalloc(&h->d_err, ERR_WORDS * sizeof(int32_t));
+  cudaError_t e = dev_malloc(reinterpret_cast<void**>(&h->arena), h->arena_bytes);
+  if (e == cudaSuccess) e = dev_malloc(reinterpret_cast<void**>(&h->d_err), ERR_WORDS * sizeof(int32_t));
   if (e == cudaSuccess) e = cudaMemset(h->d_err, 0, ERR_WORDS * sizeof(int32_t));
   if (e == cudaSuccess)
-    e = cudaHostAlloc(&h->pinned, static_cast<size_t>(kSlots) * h->meta_bytes, cudaHostAllocDefault);
+    e = pinned_malloc(reinterpret_cast<void**>(&h->pinned), static_cast<size_t>(kSlots) * h->meta_bytes);
   for (int k = 0; k < kSlots && e == cudaSuccess; ++k)
     e = cudaEventCreateWithFlags(&h->ev[k], cudaEventDisableTiming);
   if (e != cudaSuccess)
@@ -686,6 +724,12 @@ int alloc_runtime(rm_handle* h) {
 extern "C" {
 
 const char* rm_last_error(void) { return g_msg; }
+
+int rm_debug_fail_alloc(int32_t k) {
+  if (k < 0) return set_error(RM_E_INVAL, "k must be >= 0");
+  g_fail_alloc.store(k);
+  return RM_OK;
+}
 
 size_t rm_weights_bytes(const rm_config* cfg) {
   const char* why = "";
@@ -862,7 +906,7 @@ int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_
   RM_TRY(get_bucket(h, T, p_so[n], &bk));   // the arena placement and tensor maps, made now
   rm_plan* p = new rm_plan();
   p->h = h;
-  cudaError_t e = cudaMalloc(&p->d_meta, ml.base);
+  cudaError_t e = dev_malloc(reinterpret_cast<void**>(&p->d_meta), ml.base);
   if (e == cudaSuccess) e = cudaMemcpy(p->d_meta, meta.data(), ml.base, cudaMemcpyHostToDevice);
   if (e != cudaSuccess) {
     cudaFree(p->d_meta);
@@ -1087,15 +1131,17 @@ int rm_gemm_tile(int32_t M, int32_t N, int32_t K, int32_t num_sms, int32_t* out)
 
 int rm_op_embed(const int32_t* ids, const int32_t* offsets, int32_t n_seqs, int32_t T,
                 const void* emb_word, const void* emb_pos, const float* ln_g, const float* ln_b,
-                float eps, int32_t V, int32_t P, int32_t H, void* x, int32_t* err_count,
-                void* stream) {
+                float eps, int32_t V, int32_t P, int32_t H, void* x, int32_t x_dtype,
+                int32_t* err_count, void* stream) {
   if (ids == nullptr || offsets == nullptr || emb_word == nullptr || emb_pos == nullptr || x == nullptr)
     return set_error(RM_E_INVAL, "NULL argument");
   if (n_seqs < 1 || T < 0 || V < 1 || P < 1 || H < 8 || H % 8 != 0 || H > 4096)
     return set_error(RM_E_INVAL, "bad sizes");
+  if (x_dtype != RM_F32 && x_dtype != RM_BF16) return set_error(RM_E_INVAL, "bad x_dtype");
   if ((ln_g == nullptr) != (ln_b == nullptr)) return set_error(RM_E_INVAL, "ln_g and ln_b go together");
   RM_LAUNCH(embed_launch(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps, V, P, H, x,
-                         err_count, static_cast<cudaStream_t>(stream)));
+                         err_count, static_cast<cudaStream_t>(stream), L2Prefetch{}, nullptr,
+                         x_dtype));
   return RM_OK;
 }
 
@@ -1154,7 +1200,8 @@ int rm_op_res_ln(const void* y, void* x, void* z, const float* g, const float* b
   if (x == nullptr || g == nullptr || b == nullptr) return set_error(RM_E_INVAL, "NULL argument");
   if (mode < 0 || mode > 2 || (mode != 2 && y == nullptr) || (mode != 0 && z == nullptr))
     return set_error(RM_E_INVAL, "bad mode or missing y/z");
-  if (T < 0 || H < 8 || H % 8 != 0 || H > 4096 || (dtype != RM_F32 && dtype != RM_BF16))
+  if (T < 0 || H < 8 || H % 8 != 0 || H > 4096 ||
+      (dtype != RM_F32 && dtype != RM_BF16 && dtype != RM_ROWS_RESID_F32))
     return set_error(RM_E_INVAL, "bad sizes");
   RM_LAUNCH(res_ln_launch(y, x, z, g, b, T, H, eps, dtype, mode, static_cast<cudaStream_t>(stream)));
   return RM_OK;

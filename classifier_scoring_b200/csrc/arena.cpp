@@ -25,7 +25,9 @@ bool overlap_steps(const ArenaPlan& p, int a, int b) {
 
 void sizes(int arch, int H, int F, int64_t T, int64_t s_elems, ArenaPlan& p) {
   const int64_t row = 2;   // bf16 bytes
-  p.bytes[B_X] = align_up(T * H * row, kArenaAlign);
+  // the decoder's residual stream is kept in fp32 (its rounding, repeated over
+  // every layer's two additions, dominated the score error in bf16)
+  p.bytes[B_X] = align_up(T * H * (arch == RM_DEC_PRELN ? 4 : row), kArenaAlign);
   p.bytes[B_Z] = arch == RM_DEC_PRELN ? align_up(T * H * row, kArenaAlign) : 0;
   p.bytes[B_QKV] = align_up(T * 3 * H * row, kArenaAlign);
   p.bytes[B_S] = align_up(s_elems * row, kArenaAlign);

@@ -10,7 +10,10 @@
 // library holds it until the process exits.  Host code never passes the
 // array's name to a kernel (in host code that name is only a host-side
 // stand-in); it passes the device address obtained with cudaGetSymbolAddress
-// once per device.
+// once per CUDA context.
+#include <cudaTypedefs.h>
+
+#include <map>
 #include <mutex>
 
 #include "../../include/rm.h"
@@ -25,37 +28,63 @@ constexpr int64_t kNoallocMaxScoreElems = 4 * 1024 * 1024;   // bf16 score entri
 constexpr int32_t kNoallocMaxSeqs = 4096;
 constexpr int64_t kMetaBytes = 16 * (kNoallocMaxSeqs + 1);     // offsets, rb_off (int32), s_off (int64)
 constexpr int64_t kScratchBytes = kMetaBytes + 2 * kNoallocMaxScoreElems;
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-// Device address of the scratch array per device, resolved on the first call
-// made with that device current.
+// Device address of the scratch array per CUDA context.  The library's module
+// (and so the array) is loaded once per context: a caller that runs in a
+// context of its own (cuCtxCreate, or a host runtime that owns its context)
+// sees a different array than the device's primary context.  The address is
+// resolved on the first call made with that context current.
 std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {nullptr};
+std::map<CUcontext, void*> g_scratch_ptr;
 
-// Host staging of the metadata: copied into the device scratch before each
-// launch (pageable memory, so the copy has read it when cudaMemcpyAsync returns).
+// Host staging of the metadata, copied into the device scratch before each
+// launch.  These are pageable host arrays: for a pageable host-to-device
+// cudaMemcpyAsync the runtime documents (API synchronization behavior) that
+// the call returns once the source has been copied to staging memory for the
+// DMA, so the arrays may be refilled by the next call after it returns.
 std::mutex g_meta_mu;
 int32_t g_meta_off[kNoallocMaxSeqs + 1];
 int32_t g_meta_rb[kNoallocMaxSeqs + 1];
 int64_t g_meta_so[kNoallocMaxSeqs + 1];
 
-int scratch_for_current_device(unsigned char** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return set_error(RM_E_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return set_error(RM_E_DEVICE, "device index %d unsupported", dev);
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_ptr[dev] == nullptr) {
+PFN_cuCtxGetCurrent_v4000 ctx_get_current() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return set_error(RM_E_CUDA, "cudaGetSymbolAddress of the scratch array: %s",
-                       cudaGetErrorString(e));
-    g_scratch_ptr[dev] = p;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+  });
+  return fn;
+}
+
+int scratch_for_current_context(unsigned char** out) {
+  auto get = ctx_get_current();
+  if (get == nullptr) return set_error(RM_E_CUDA, "cuCtxGetCurrent is not available from the driver");
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return set_error(RM_E_CUDA, "cuCtxGetCurrent failed");
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (ctx != nullptr) {
+    auto it = g_scratch_ptr.find(ctx);
+    if (it != g_scratch_ptr.end()) {
+      *out = static_cast<unsigned char*>(it->second);
+      return RM_OK;
+    }
   }
-  *out = static_cast<unsigned char*>(g_scratch_ptr[dev]);
+  // first call in this context: with no context current, the lookup binds the
+  // device's primary context, which the launches of this call then use
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr)
+    return set_error(RM_E_CUDA, "cudaGetSymbolAddress of the scratch array: %s", cudaGetErrorString(e));
+  if (ctx == nullptr && (get(&ctx) != CUDA_SUCCESS || ctx == nullptr))
+    return set_error(RM_E_CUDA, "no current CUDA context after the scratch lookup");
+  g_scratch_ptr[ctx] = p;
+  *out = static_cast<unsigned char*>(p);
   return RM_OK;
 }
 
@@ -90,7 +119,7 @@ extern "C" int rm_op_attention_noalloc(const void* qkv, void* ctx, const int32_t
                      "(use rm_op_attn_scores/softmax/context with caller-allocated memory)",
                      (long long)elems, (long long)kNoallocMaxScoreElems);
   unsigned char* scratch = nullptr;
-  int rc = scratch_for_current_device(&scratch);
+  int rc = scratch_for_current_context(&scratch);
   if (rc != RM_OK) return rc;
   int32_t* d_off = reinterpret_cast<int32_t*>(scratch);
   int32_t* d_rb = reinterpret_cast<int32_t*>(scratch + 4 * (kNoallocMaxSeqs + 1));

@@ -60,12 +60,12 @@ __device__ __forceinline__ void normalize(float (&v)[MAXC][8], int nch, int lane
   }
 }
 
-template <int MAXC, bool LN>
+template <int MAXC, bool LN, typename TX>
 __global__ void __launch_bounds__(kWarps * 32)
     embed_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ offsets, int n_seqs,
                  int T, const bf16* __restrict__ ew, const bf16* __restrict__ ep,
                  const float* __restrict__ g, const float* __restrict__ b, float eps, int V, int H,
-                 bf16* __restrict__ x, int32_t* __restrict__ err, L2PrefetchArgs pf,
+                 TX* __restrict__ x, int32_t* __restrict__ err, L2PrefetchArgs pf,
                  const int32_t* __restrict__ pos_base) {
   pdl_launch_dependents();
   l2_prefetch_share(pf);   // static weights: no need to wait for the previous kernel
@@ -101,22 +101,24 @@ __global__ void __launch_bounds__(kWarps * 32)
     row_moments<MAXC>(v, nch, lane, H, mean, rstd, eps);
     normalize<MAXC>(v, nch, lane, mean, rstd, g, b);
   }
-  bf16* xr = x + static_cast<size_t>(t) * H;
+  TX* xr = x + static_cast<size_t>(t) * H;
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
     const int ch = lane + 32 * c;
-    if (ch < nch) Chunk8<bf16>::store(xr + ch * 8, v[c]);
+    if (ch < nch) Chunk8<TX>::store(xr + ch * 8, v[c]);
   }
 }
 
 // MODE 0: x = LN(y + x); MODE 1: x = y + x, z = LN(x); MODE 2: z = LN(x)
+// Row types: TY for y, TX for the residual stream x, TZ for z (the decoder
+// keeps x in fp32 and y, z in bf16; every other use has one type).
 // Wide rows (H > 1024) are split over WPR warps, so that a lane holds at most
 // four chunks: at H = 2048 one warp per row needs ~100 registers, which caps
 // an SM at 16 resident warps, too few to keep HBM busy.  The WPR partial sums
 // meet in shared memory (two CTA barriers per row pass).
-template <typename T, int MAXC, int MODE, int WPR>
+template <typename TY, typename TX, typename TZ, int MAXC, int MODE, int WPR>
 __global__ void __launch_bounds__(kWarps * 32)
-    res_ln_kernel(const T* __restrict__ y, T* __restrict__ x, T* __restrict__ z,
+    res_ln_kernel(const TY* __restrict__ y, TX* __restrict__ x, TZ* __restrict__ z,
                   const float* __restrict__ g, const float* __restrict__ b, int rows, int H,
                   float eps, L2PrefetchArgs pf) {
   pdl_launch_dependents();
@@ -136,10 +138,10 @@ __global__ void __launch_bounds__(kWarps * 32)
   for (int c = 0; c < MAXC; ++c) {
     const int ch = lr + LPR * c;
     if (live && ch < nch) {
-      Chunk8<T>::load(x + base + ch * 8, v[c]);
+      Chunk8<TX>::load(x + base + ch * 8, v[c]);
       if (MODE != 2) {
         float u[8];
-        Chunk8<T>::load(y + base + ch * 8, u);
+        Chunk8<TY>::load(y + base + ch * 8, u);
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[c][e] += u[e];
       }
@@ -151,9 +153,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     for (int c = 0; c < MAXC; ++c) {
       const int ch = lr + LPR * c;
       if (live && ch < nch) {
-        Chunk8<T>::store(x + base + ch * 8, v[c]);
+        Chunk8<TX>::store(x + base + ch * 8, v[c]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[c][e] = to_f32(from_f32<T>(v[c][e]));
+        for (int e = 0; e < 8; ++e) v[c][e] = to_f32(from_f32<TX>(v[c][e]));
       }
     }
   }
@@ -207,11 +209,13 @@ __global__ void __launch_bounds__(kWarps * 32)
       for (int e = 0; e < 8; ++e) v[c][e] = (v[c][e] - mean) * rstd * gg[e] + bb[e];
     }
   }
-  T* out = (MODE == 0 ? x : z) + base;
 #pragma unroll
   for (int c = 0; c < MAXC; ++c) {
     const int ch = lr + LPR * c;
-    if (ch < nch) Chunk8<T>::store(out + ch * 8, v[c]);
+    if (ch < nch) {
+      if (MODE == 0) Chunk8<TX>::store(x + base + ch * 8, v[c]);
+      else Chunk8<TZ>::store(z + base + ch * 8, v[c]);
+    }
   }
 }
 
@@ -318,55 +322,55 @@ int pick_maxc(int H) {
   return -1;
 }
 
-template <int MAXC>
+template <int MAXC, typename TX>
 cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, const void* ew,
                     const void* ep, const float* g, const float* b, float eps, int V, int H,
                     void* x, int32_t* err, cudaStream_t st, const L2Prefetch& pf,
                     const int32_t* pos_base) {
   dim3 grid((T + kWarps - 1) / kWarps);
   if (g != nullptr)
-    launch_k(embed_kernel<MAXC, true>, grid, kWarps * 32, 0, st,
+    launch_k(embed_kernel<MAXC, true, TX>, grid, kWarps * 32, 0, st,
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<bf16*>(x), err, pf_args(pf), pos_base);
+        V, H, static_cast<TX*>(x), err, pf_args(pf), pos_base);
   else
-    launch_k(embed_kernel<MAXC, false>, grid, kWarps * 32, 0, st,
+    launch_k(embed_kernel<MAXC, false, TX>, grid, kWarps * 32, 0, st,
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<bf16*>(x), err, pf_args(pf), pos_base);
+        V, H, static_cast<TX*>(x), err, pf_args(pf), pos_base);
   return cudaGetLastError();
 }
 
-template <typename T, int MAXC, int WPR>
+template <typename TY, typename TX, typename TZ, int MAXC, int WPR>
 cudaError_t res_ln_t(const void* y, void* x, void* z, const float* g, const float* b, int rows,
                      int H, float eps, int mode, cudaStream_t st, const L2Prefetch& pf) {
   dim3 grid((rows + kWarps / WPR - 1) / (kWarps / WPR));
-  const T* yy = static_cast<const T*>(y);
-  T* xx = static_cast<T*>(x);
-  T* zz = static_cast<T*>(z);
+  const TY* yy = static_cast<const TY*>(y);
+  TX* xx = static_cast<TX*>(x);
+  TZ* zz = static_cast<TZ*>(z);
   if (mode == 0)
-    launch_k(res_ln_kernel<T, MAXC, 0, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H,
-             eps, pf_args(pf));
+    launch_k(res_ln_kernel<TY, TX, TZ, MAXC, 0, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b,
+             rows, H, eps, pf_args(pf));
   else if (mode == 1)
-    launch_k(res_ln_kernel<T, MAXC, 1, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H,
-             eps, pf_args(pf));
+    launch_k(res_ln_kernel<TY, TX, TZ, MAXC, 1, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b,
+             rows, H, eps, pf_args(pf));
   else
-    launch_k(res_ln_kernel<T, MAXC, 2, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b, rows, H,
-             eps, pf_args(pf));
+    launch_k(res_ln_kernel<TY, TX, TZ, MAXC, 2, WPR>, grid, kWarps * 32, 0, st, yy, xx, zz, g, b,
+             rows, H, eps, pf_args(pf));
   return cudaGetLastError();
 }
 
 // One warp per row up to H = 1024 (at most 4 chunks a lane); 2 warps per row
 // up to 2048 and 4 up to 4096.
-template <typename T>
+template <typename TY, typename TX, typename TZ>
 cudaError_t res_ln_dispatch(const void* y, void* x, void* z, const float* g, const float* b,
                             int rows, int H, float eps, int mode, cudaStream_t st,
                             const L2Prefetch& pf) {
   const int chunks = H / 8;
-  if (chunks > 256) return res_ln_t<T, 4, 4>(y, x, z, g, b, rows, H, eps, mode, st, pf);
-  if (chunks > 128) return res_ln_t<T, 4, 2>(y, x, z, g, b, rows, H, eps, mode, st, pf);
-  if (chunks > 96) return res_ln_t<T, 4, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
-  if (chunks > 64) return res_ln_t<T, 3, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
-  if (chunks > 32) return res_ln_t<T, 2, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
-  return res_ln_t<T, 1, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 256) return res_ln_t<TY, TX, TZ, 4, 4>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 128) return res_ln_t<TY, TX, TZ, 4, 2>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 96) return res_ln_t<TY, TX, TZ, 4, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 64) return res_ln_t<TY, TX, TZ, 3, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  if (chunks > 32) return res_ln_t<TY, TX, TZ, 2, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
+  return res_ln_t<TY, TX, TZ, 1, 1>(y, x, z, g, b, rows, H, eps, mode, st, pf);
 }
 
 }  // namespace
@@ -388,12 +392,15 @@ cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs,
                          const void* emb_word, const void* emb_pos, const float* ln_g,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
                          int32_t* err_count, cudaStream_t st, const L2Prefetch& pf,
-                         const int32_t* pos_base) {
+                         const int32_t* pos_base, int x_dtype) {
   (void)P;
   if (T == 0) return cudaSuccess;
   const int maxc = pick_maxc(H);
-  RMK_MAXC_SWITCH(maxc, (embed_t<M_>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b, eps,
-                                     V, H, x, err_count, st, pf, pos_base)))
+  if (x_dtype == 0)
+    RMK_MAXC_SWITCH(maxc, (embed_t<M_, float>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g,
+                                              ln_b, eps, V, H, x, err_count, st, pf, pos_base)))
+  RMK_MAXC_SWITCH(maxc, (embed_t<M_, bf16>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b,
+                                           eps, V, H, x, err_count, st, pf, pos_base)))
 }
 
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
@@ -401,8 +408,9 @@ cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const
                           const L2Prefetch& pf) {
   if (T == 0) return cudaSuccess;
   if (H % 8 != 0 || H > 4096) return cudaErrorInvalidValue;
-  if (dtype == 0) return res_ln_dispatch<float>(y, x, z, g, b, T, H, eps, mode, st, pf);
-  return res_ln_dispatch<bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
+  if (dtype == 0) return res_ln_dispatch<float, float, float>(y, x, z, g, b, T, H, eps, mode, st, pf);
+  if (dtype == 2) return res_ln_dispatch<bf16, float, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
+  return res_ln_dispatch<bf16, bf16, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
 }
 
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,

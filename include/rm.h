@@ -227,6 +227,17 @@ int rm_get_device_error(rm_handle* h, int32_t* out);
  * NULL outputs or a limit out of range, RM_E_CUDA on a CUDA error. */
 int rm_selftest_bounded_wait(int64_t limit_ns, int32_t* out_timed_out, int64_t* out_elapsed_ns);
 
+/* Allocation fault injection for tests (the pages have no counterpart): the
+ * k-th device or pinned-host allocation that the library makes from now on
+ * (counting from 1, in this process, on any handle: rm_create makes five --
+ * weights, their upload staging, the arena, the error words, the pinned
+ * metadata ring -- rm_create_shared three and rm_plan_create one) fails as if
+ * memory were exhausted, without reaching the allocator; k = 0 disarms it.
+ * The call that meets the failure releases what it had allocated and returns
+ * RM_E_NOMEM; existing handles are untouched and stay usable.  Host only,
+ * thread-safe.  RM_E_INVAL for k < 0. */
+int rm_debug_fail_alloc(int32_t k);
+
 /* Arena figures: out[0] = bytes reserved at create, out[1] = largest plan used
  * by any call so far, out[2] = number of distinct length buckets planned.
  * out: host int64[3]. */

@@ -81,11 +81,12 @@ int rm_gemm_tile(int32_t M, int32_t N, int32_t K, int32_t num_sms, int32_t* out)
  * sequence i, then (ln_g != NULL) the embedding LayerNorm.  ids out of 0..V-1
  * are clamped and counted with atomicAdd into *err_count (may be NULL).
  * E_word: bf16 [V][H]; E_pos: bf16 [P][H]; ln_g, ln_b: fp32 [H] or NULL;
- * x: bf16 [T][H].  Requires every L_i <= P. */
+ * x: [T][H] of x_dtype (RM_BF16, or RM_F32 for the decoder's fp32 residual
+ * stream).  Requires every L_i <= P. */
 int rm_op_embed(const int32_t* ids, const int32_t* offsets, int32_t n_seqs, int32_t T,
                 const void* emb_word, const void* emb_pos, const float* ln_g, const float* ln_b,
-                float eps, int32_t V, int32_t P, int32_t H, void* x, int32_t* err_count,
-                void* stream);
+                float eps, int32_t V, int32_t P, int32_t H, void* x, int32_t x_dtype,
+                int32_t* err_count, void* stream);
 
 /* Attention scores S = (Q K^T)/sqrt(d) per sequence and head, only the valid
  * L_i x L_i block (causal: keys c <= r).  qkv: bf16 [T][3H]; S: bf16.
@@ -119,7 +120,8 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
 
 /* The materialised attention step (rm_op_attn_scores -> rm_op_softmax ->
  * rm_op_attn_context) without any device allocation: the score matrix and the
- * per-call metadata live in one file-scope device array of 8 MiB + 64 KiB that
+ * per-call metadata live in one file-scope device array of 8 MiB of scores
+ * plus 65,552 bytes of metadata (8,454,160 bytes) that
  * every device loading this library keeps until the process exits.  The pages
  * have no counterpart to this entry point; it exists for callers that cannot
  * allocate device memory where they run the step (a plugin inside another
@@ -128,9 +130,10 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
  *   qkv: bf16 [T][3H]; ctx: bf16 [T][H] (written); offsets: HOST int32[n+1].
  * Limits: n_seqs <= 4096, every L_i <= 1024 and sum_i n_heads*L_i*round_up(L_i,8)
  * <= 4 Mi score entries; larger calls return RM_E_RANGE (use the three
- * caller-allocated entry points instead).  The first call on a device looks up
- * the array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture.  The call copies its metadata into the
+ * caller-allocated entry points instead).  The first call in a CUDA context (for most
+ * callers, the device's primary context) looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it for that context; make that first call
+ * before any stream capture.  The call copies its metadata into the
  * array on stream and calls no cudaMalloc or cudaFree.  Every call shares the
  * array and it keeps the last call's contents (nothing in it needs to start at
  * zero: each call writes every entry it reads), so calls that overlap on the
@@ -140,12 +143,16 @@ int rm_op_attention_noalloc(const void* qkv, void* ctx, const int32_t* offsets, 
                             int32_t n_heads, int32_t head_dim, int32_t causal, void* stream);
 
 /* Residual + LayerNorm over rows of length H (the LayerNorm batch reduction of
- * the TurboTransformers abstract), fp32 math, rows of dtype (RM_BF16|RM_F32):
+ * the TurboTransformers abstract), fp32 math:
  *   mode 0 (post-LN): x = LN(y + x)              (z unused, may be NULL)
  *   mode 1 (pre-LN):  x = y + x;  z = LN(x)      (both written)
  *   mode 2 (plain):   z = LN(x)                  (y unused, may be NULL)
  * LN(u) = g * (u - mean)/sqrt(var + eps) + b with the biased variance.
- * y, x, z: [T][H]; g, b: fp32 [H]. */
+ * y, x, z: [T][H]; g, b: fp32 [H].  Row types by dtype: RM_F32 or RM_BF16 for
+ * all three; RM_ROWS_RESID_F32 for x in fp32 with y and z in bf16 (the pre-LN
+ * decoder's residual stream, kept in fp32 so that its sum is rounded once per
+ * addition to fp32 instead of to bf16). */
+#define RM_ROWS_RESID_F32 2
 int rm_op_res_ln(const void* y, void* x, void* z, const float* g, const float* b, int32_t T,
                  int32_t H, float eps, int32_t dtype, int32_t mode, void* stream);
 

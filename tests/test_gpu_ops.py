@@ -153,6 +153,29 @@ def test_res_ln_bf16(H):
     assert np.all(np.abs(f64(xd) - ref) <= BF16_REL * np.abs(ref) + 1e-4 * np.abs(gm))
 
 
+@pytest.mark.parametrize("H", [1024, 2048])
+@pytest.mark.parametrize("mode", [1, 2])
+def test_res_ln_fp32_residual_with_bf16_rows(H, mode):
+    """The decoder's rows: y and z bf16, the residual stream x fp32."""
+    T = 1001
+    rng = np.random.default_rng(H + 7 * mode)
+    y = rng.normal(0, 1, (T, H))
+    x = rng.normal(0.3, 3, (T, H)).astype(np.float32)
+    gm = (1 + rng.normal(0, 0.02, H)).astype(np.float32)
+    bt = rng.normal(0, 0.02, H).astype(np.float32)
+    yd, xd = dev(y, torch.bfloat16), dev(x, torch.float32)
+    zd = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    u = x.astype(np.float64) + (f64(yd) if mode == 1 else 0)
+    if mode == 1:
+        u = u.astype(np.float32).astype(np.float64)       # the stored residual: one fp32 rounding
+    rm.ops.res_ln(yd if mode == 1 else None, xd, zd, dev(gm, torch.float32), dev(bt, torch.float32),
+                  T, H, 1e-5, rm.ROWS_RESID_F32, mode)
+    torch.cuda.synchronize()
+    ref = O.layer_norm(u, gm.astype(np.float64), bt.astype(np.float64), 1e-5)
+    assert np.all(np.abs(f64(zd) - ref) <= BF16_REL * np.abs(ref) + F32_RTOL * (np.abs(ref) + np.abs(gm)))
+    assert np.array_equal(f64(xd), u if mode == 1 else x.astype(np.float64))
+
+
 # --- softmax -------------------------------------------------------------------------
 
 def varlen_rows(lens, nh, rng, dtype):
@@ -275,8 +298,9 @@ def test_attention_context(nh, d, causal):
 
 # --- embedding and head ----------------------------------------------------------------
 
-@pytest.mark.parametrize("H,ln", [(128, True), (312, True), (768, True), (2048, False)])
-def test_embed(H, ln):
+@pytest.mark.parametrize("H,ln,xdt", [(128, True, "bf16"), (312, True, "bf16"), (768, True, "bf16"),
+                                      (2048, False, "bf16"), (2048, False, "f32")])
+def test_embed(H, ln, xdt):
     V, P = 1000, 600
     lens = np.array([1, 560, 33, 8])
     off = synth.offsets_from_lengths(lens)
@@ -288,10 +312,12 @@ def test_embed(H, ln):
     ep = dev(rng.normal(0, 0.5, (P, H)), torch.bfloat16)
     g = dev(1 + rng.normal(0, 0.1, H), torch.float32)
     b = dev(rng.normal(0, 0.1, H), torch.float32)
-    x = torch.zeros(int(off[-1]), H, dtype=torch.bfloat16, device="cuda")
+    f32 = xdt == "f32"
+    x = torch.zeros(int(off[-1]), H, dtype=torch.float32 if f32 else torch.bfloat16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     rm.ops.embed(dev(ids, torch.int32), dev(off, torch.int32), len(lens), int(off[-1]), ew, ep,
-                 g if ln else None, b if ln else None, 1e-12, V, P, H, x, err)
+                 g if ln else None, b if ln else None, 1e-12, V, P, H, x, err,
+                 x_dtype=rm.F32 if f32 else rm.BF16)
     torch.cuda.synchronize()
     assert int(err.item()) == 2
     EW, EP = f64(ew), f64(ep)
@@ -300,7 +326,11 @@ def test_embed(H, ln):
         u = EW[cid[off[i]:off[i + 1]]] + EP[:L]
         ref = O.layer_norm(u, f64(g), f64(b), 1e-12) if ln else u
         got = f64(x)[off[i]:off[i + 1]]
-        assert np.all(np.abs(got - ref) <= BF16_REL * np.abs(ref) + 1e-5 * (1 + np.abs(ref)))
+        if f32:
+            # the sum of two bf16 values, rounded once to fp32
+            assert np.all(np.abs(got - ref) <= 2.0 ** -24 * np.abs(ref))
+        else:
+            assert np.all(np.abs(got - ref) <= BF16_REL * np.abs(ref) + 1e-5 * (1 + np.abs(ref)))
 
 
 @pytest.mark.parametrize("last", [0, 1])

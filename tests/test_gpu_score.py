@@ -173,18 +173,61 @@ def test_decoder_small_shape_every_sequence(attn):
     assert np.max(np.abs(got - ref)) <= SCORE_ATOL
 
 
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _report(label, err, lens):
+    """One line per whole-batch check, so the GPU log records the error profile."""
+    order = np.argsort(lens)
+    print(f"\n{label}: max |gpu - oracle| = {err.max():.3e} over {len(err)} sequences; "
+          f"8 shortest {err[order[:8]].max():.3e}, 8 longest {err[order[-8:]].max():.3e}")
+
+
 @pytest.mark.slow
-def test_gpt_1p3b_batch_sampled():
+def test_gpt_1p3b_whole_batch_every_sequence():
+    """Every sequence of a 64-sequence batch of the 1.3B-shape causal reward
+    model (lengths U[256, 560], 24 pre-LN layers) against the fp64 oracle
+    (scores written by tests/golden/make_golden.py; the shortest sequence is
+    re-scored by the oracle here to tie the stored file to it)."""
     name = "gpt-1.3b-rm"
     w = synth.WORKLOADS[name]
     st = synth.make_stream(w)
     ids, off = synth.pack(st, np.arange(w.max_batch))
+    gold = np.loadtxt(os.path.join(GOLDEN, "gpt_1p3b_rm_batch_scores.txt"))
+    assert gold.shape == (w.max_batch,)
     sc = scorer(name, max_batch_seqs=64, max_tokens=64 * 560, max_len=560)
     got = gpu_scores(sc, ids, off)
     assert np.all(np.isfinite(got))
-    i = int(np.argmin(np.diff(off)))          # the shortest sequence keeps the oracle quick
-    ref = oracle_scores(name, ids, off, [i])
-    assert abs(got[i] - ref[0]) <= SCORE_ATOL
+    lens = np.diff(off)
+    err = np.abs(got - gold)
+    _report(name, err, lens)
+    assert err.max() <= SCORE_ATOL, (err.max(), int(np.argmax(err)), int(lens[np.argmax(err)]))
+    i = int(np.argmin(lens))
+    assert abs(oracle_scores(name, ids, off, [i])[0] - gold[i]) <= 1e-9
+
+
+def test_bert_base_len5_500_longest_batch_every_sequence():
+    """Every sequence of the last (longest) DP batch of the full 10,000-request
+    lengths-5..500 stream (Bmax 32; rows up to 500 tokens) against the fp64
+    oracle's stored scores, on both attention paths."""
+    name = "bert-base-len5-500"
+    w = synth.WORKLOADS[name]
+    st = synth.make_stream(w)
+    rows = np.loadtxt(os.path.join(GOLDEN, "bert_base_len5_500_longest_batch_scores.txt"))
+    idx, gold = rows[:, 0].astype(np.int64), rows[:, 1]
+    batch, _ = OS.schedule_dp(st.lengths, w.max_batch, OS.linear_cost(20000, 1))
+    assert np.array_equal(np.nonzero(batch == batch.max())[0], idx)
+    ids, off = synth.pack(st, idx)
+    lens = np.diff(off)
+    for attn in (rm.ATTN_FUSED, rm.ATTN_MATERIALIZED):
+        sc = scorer(name, max_batch_seqs=w.max_batch, max_tokens=w.max_batch * w.len_hi, max_len=512,
+                    attn_impl=attn)
+        got = gpu_scores(sc, ids, off)
+        err = np.abs(got - gold)
+        _report(f"{name} attn_impl={attn}", err, lens)
+        assert err.max() <= SCORE_ATOL, (attn, err.max(), int(lens[np.argmax(err)]))
+    i = int(np.argmax(lens))
+    assert abs(oracle_scores(name, ids, off, [i])[0] - gold[i]) <= 1e-9
 
 
 # --- edge cases -----------------------------------------------------------------------
