@@ -13,8 +13,12 @@
 // percent of the scorer's FLOPs.
 #include <math.h>
 
+#include <algorithm>
+#include <climits>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace rmk {
 namespace {
@@ -667,6 +671,320 @@ __global__ void __launch_bounds__(128, (DP <= 64 ? 4 : 1))
   }
 }
 
+// ---------------------------------------------------------------------------
+// Packed-row attention (head dims 64 and 128).  The batch is cut into tiles of
+// 64 consecutive packed rows, whatever sequences they belong to: short
+// sequences share a tile, long ones span several, and no warp holds only
+// padding (the one-CTA-per-sequence-block layout above leaves most warps of a
+// short sequence's block idle).  A CTA takes one tile and a group of heads:
+//   warp 4, one lane : TMA producer -- per head the tile's 64 query rows,
+//                      then the K and V rows of the tile's key range
+//                      [first key of its first sequence, last key of its last
+//                      sequence) in chunks of 64 rows, into a ring of stages
+//                      that runs on across the heads (128-byte swizzle; rows
+//                      past the batch read as zeros);
+//   warps 0..3       : 16 query rows each; per chunk S = QK^T (mma.sync
+//                      m16n8k16, fragments by ldmatrix), a key admitted only
+//                      inside the row's own sequence (and c <= r when causal),
+//                      online softmax (running max and sum in fp32; P rounded
+//                      to bf16 for P.V as the materialised path stores it),
+//                      O += P V; chunks outside the warp's own key range are
+//                      skipped.  The heads pipeline: head j+1's rows are in
+//                      flight while head j is multiplied.
+// A consumer releases a buffer only after a proxy fence: its ldmatrix reads
+// are generic-proxy accesses and the TMA refill an async-proxy write (without
+// the fence a refill could overtake the reads; seen as an occasional wrong
+// (tile, head) block when the ring ran several heads ahead).
+// Every mbarrier wait is bounded; a wait that gives up counts into
+// err[ERR_TIMEOUT], the role stops, and the producer waits (bounded) for its
+// copies before the CTA exits.
+// ---------------------------------------------------------------------------
+template <int DP>
+struct TileSmem {
+  static constexpr int kBox = 64 * 64 * 2;                  // TMA box: 64 rows x 128 bytes
+  static constexpr int kNB = DP / 64;                       // boxes across a row of DP
+  static constexpr int kQ = kNB * kBox;                     // 64 query rows
+  static constexpr int kKV = 2 * kNB * kBox;                // 64 key rows of K and of V
+  static constexpr int kStages = DP == 64 ? 3 : 2;
+  static constexpr int kKVOff = 2 * kQ;                     // after two query buffers
+  static constexpr int kBarOff = kKVOff + kStages * kKV;
+  static constexpr int kBars = 4 + 2 * kStages;             // qfull[2] qempty[2] kvfull[S] kvempty[S]
+  static constexpr int kBytes = kBarOff + kBars * 8 + 1024; // + 1024-byte alignment slack
+  static constexpr int kCtasPerSm = DP == 64 ? 3 : 2;
+};
+
+// Byte offset of the 16-byte chunk `ch` (8 bf16 along the row) of row `r` in
+// a tile of 128-byte-swizzled boxes.
+__device__ __forceinline__ uint32_t sw128_off(int r, int ch) {
+  return static_cast<uint32_t>((ch >> 3) * (64 * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+
+template <int DP>
+__global__ void __launch_bounds__(160)
+    attn_tile_kernel(const __grid_constant__ CUtensorMap tm, bf16* __restrict__ ctx,
+                     const int32_t* __restrict__ offsets, int n, int T, int H, int nh, int hpc,
+                     float scale_log2, int causal, int* __restrict__ err, L2PrefetchArgs pf) {
+  using SL = TileSmem<DP>;
+  constexpr int S = SL::kStages;
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tsm_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t qfull0 = smem_u32(sm + SL::kBarOff), qempty0 = qfull0 + 16, kvfull0 = qfull0 + 32,
+                 kvempty0 = kvfull0 + 8 * S;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(qfull0 + 8 * b, 1);
+      mbar_init(qempty0 + 8 * b, 4);
+    }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(kvfull0 + 8 * s, 1);
+      mbar_init(kvempty0 + 8 * s, 4);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+  pdl_launch_dependents();
+  l2_prefetch_share(pf);
+  pdl_wait();
+
+  const int r0 = blockIdx.x * 64;
+  const int h0 = blockIdx.y * hpc;
+  const int nhl = min(hpc, nh - h0);
+  const int rlast = min(r0 + 64, T) - 1;
+  const int s_first = upper_index(offsets, n, r0);
+  const int s_last = upper_index(offsets, n, rlast);
+  const int Klo = offsets[s_first];
+  const int Khi = causal ? rlast + 1 : offsets[s_last + 1];
+  const int nch = (Khi - Klo + 63) / 64;
+
+  if (warp == 4) {
+    // ---- TMA producer ----
+    if (lane == 0) {
+      int it = 0, nq = 0;
+      bool ok = true;
+      for (int j = 0; j < nhl && ok; ++j) {
+        const int h = h0 + j, qb = j & 1;
+        if (j >= 2 && !mbar_wait(qempty0 + 8 * qb, ((j >> 1) - 1) & 1)) {
+          atomicAdd(err + ERR_TIMEOUT, 1);
+          break;
+        }
+        mbar_arrive_expect_tx(qfull0 + 8 * qb, SL::kQ);
+#pragma unroll
+        for (int b = 0; b < SL::kNB; ++b)
+          tma_load_2d(sbase + qb * SL::kQ + b * SL::kBox, &tm, h * DP + 64 * b, r0, qfull0 + 8 * qb);
+        ++nq;
+        for (int c = 0; c < nch; ++c, ++it) {
+          const int s = it % S;
+          if (it >= S && !mbar_wait(kvempty0 + 8 * s, ((it / S) - 1) & 1)) {
+            atomicAdd(err + ERR_TIMEOUT, 1);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(kvfull0 + 8 * s, SL::kKV);
+          const uint32_t dk = sbase + SL::kKVOff + s * SL::kKV, dv = dk + SL::kNB * SL::kBox;
+#pragma unroll
+          for (int b = 0; b < SL::kNB; ++b) {
+            tma_load_2d(dk + b * SL::kBox, &tm, H + h * DP + 64 * b, Klo + 64 * c, kvfull0 + 8 * s);
+            tma_load_2d(dv + b * SL::kBox, &tm, 2 * H + h * DP + 64 * b, Klo + 64 * c, kvfull0 + 8 * s);
+          }
+        }
+      }
+      // no copy into this CTA's shared memory may be in flight when it exits
+      bool drained = true;
+      for (int j = it - 1; drained && j >= 0 && j >= it - S; --j)
+        drained = mbar_wait(kvfull0 + 8 * (j % S), (j / S) & 1);
+      for (int j = nq - 1; drained && j >= 0 && j >= nq - 2; --j)
+        drained = mbar_wait(qfull0 + 8 * (j & 1), (j >> 1) & 1);
+    }
+    return;
+  }
+
+  // ---- consumers: 16 query rows per warp ----
+  const int g = lane >> 2, tq = lane & 3;
+  const int ra = r0 + warp * 16 + g, rb = ra + 8;
+  // keys a row admits: its own sequence's rows [lo, hi) (hi <= r + 1 when
+  // causal); rows past the batch admit none
+  auto key_range = [&](int r, int& lo, int& hi) {
+    if (r >= T) {
+      lo = 0;
+      hi = 0;
+      return;
+    }
+    const int s = upper_index(offsets, n, r);
+    lo = offsets[s];
+    hi = causal ? r + 1 : offsets[s + 1];
+  };
+  int lo_a, hi_a, lo_b, hi_b;
+  key_range(ra, lo_a, hi_a);
+  key_range(rb, lo_b, hi_b);
+  // the warp's key range: chunks outside it are skipped
+  const int wlo = __reduce_min_sync(0xffffffffu, min(hi_a > lo_a ? lo_a : INT_MAX, hi_b > lo_b ? lo_b : INT_MAX));
+  const int whi = __reduce_max_sync(0xffffffffu, max(hi_a, hi_b));
+
+  int it = 0;
+  for (int j = 0; j < nhl; ++j) {
+    const int h = h0 + j, qb = j & 1;
+    if (!mbar_wait(qfull0 + 8 * qb, (j >> 1) & 1)) {
+      if (lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
+      return;
+    }
+    uint32_t qa[DP / 16][4];
+    {
+      const int qr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int ks = 0; ks < DP / 16; ++ks)
+        ldmatrix_x4(qa[ks], sbase + qb * SL::kQ + sw128_off(qr, 2 * ks + (lane >> 4)));
+    }
+    // Q is in registers: the buffer may refill.  The reads are generic-proxy,
+    // the refill an async-proxy (TMA) write: fence the two before the release.
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(qempty0 + 8 * qb);
+
+    float o[DP / 8][4];
+#pragma unroll
+    for (int t = 0; t < DP / 8; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+
+    for (int c = 0; c < nch; ++c, ++it) {
+      const int s = it % S;
+      if (!mbar_wait(kvfull0 + 8 * s, (it / S) & 1)) {
+        if (lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
+        return;
+      }
+      const int c0 = Klo + 64 * c;
+      if (c0 < whi && c0 + 64 > wlo) {
+        const uint32_t kb = sbase + SL::kKVOff + s * SL::kKV, vb = kb + SL::kNB * SL::kBox;
+        float sc[8][4];
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          sc[2 * np][0] = sc[2 * np][1] = sc[2 * np][2] = sc[2 * np][3] = 0.f;
+          sc[2 * np + 1][0] = sc[2 * np + 1][1] = sc[2 * np + 1][2] = sc[2 * np + 1][3] = 0.f;
+          if (c0 + 16 * np < whi && c0 + 16 * np + 16 > wlo) {
+            const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+            for (int ks = 0; ks < DP / 16; ++ks) {
+              uint32_t kf[4];
+              ldmatrix_x4(kf, kb + sw128_off(key, 2 * ks + ((lane >> 3) & 1)));
+              mma_bf16_16816(sc[2 * np], qa[ks], kf[0], kf[1]);
+              mma_bf16_16816(sc[2 * np + 1], qa[ks], kf[2], kf[3]);
+            }
+          }
+        }
+        // mask (own sequence, causal), scale into the log2 domain, block maxima
+        float bm_a = -INFINITY, bm_b = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const int cc = c0 + nt * 8 + 2 * tq;
+          sc[nt][0] = (cc >= lo_a && cc < hi_a) ? sc[nt][0] * scale_log2 : -INFINITY;
+          sc[nt][1] = (cc + 1 >= lo_a && cc + 1 < hi_a) ? sc[nt][1] * scale_log2 : -INFINITY;
+          sc[nt][2] = (cc >= lo_b && cc < hi_b) ? sc[nt][2] * scale_log2 : -INFINITY;
+          sc[nt][3] = (cc + 1 >= lo_b && cc + 1 < hi_b) ? sc[nt][3] * scale_log2 : -INFINITY;
+          bm_a = fmaxf(bm_a, fmaxf(sc[nt][0], sc[nt][1]));
+          bm_b = fmaxf(bm_b, fmaxf(sc[nt][2], sc[nt][3]));
+        }
+        bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 1));
+        bm_a = fmaxf(bm_a, __shfl_xor_sync(0xffffffffu, bm_a, 2));
+        bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 1));
+        bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
+        const float mn_a = fmaxf(m_a, bm_a), mn_b = fmaxf(m_b, bm_b);
+        // a row with no admitted key so far keeps m = -inf; shift by 0 then
+        const float sh_a = mn_a == -INFINITY ? 0.f : mn_a, sh_b = mn_b == -INFINITY ? 0.f : mn_b;
+        const float al_a = exp2f(m_a - sh_a), al_b = exp2f(m_b - sh_b);
+        m_a = mn_a;
+        m_b = mn_b;
+        float ps_a = 0.f, ps_b = 0.f;
+        uint32_t pa[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          const float p0 = exp2f(sc[nt][0] - sh_a), p1 = exp2f(sc[nt][1] - sh_a);
+          const float p2 = exp2f(sc[nt][2] - sh_b), p3 = exp2f(sc[nt][3] - sh_b);
+          ps_a += p0 + p1;
+          ps_b += p2 + p3;
+          pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
+          pa[nt >> 1][(nt & 1) * 2 + 1] = pack_bf16x2(p2, p3);
+        }
+        l_a = l_a * al_a + ps_a;
+        l_b = l_b * al_b + ps_b;
+#pragma unroll
+        for (int t = 0; t < DP / 8; ++t) {
+          o[t][0] *= al_a;
+          o[t][1] *= al_a;
+          o[t][2] *= al_b;
+          o[t][3] *= al_b;
+        }
+        // O += P V: V fragments by ldmatrix.trans from the key-major rows
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          if (c0 + 16 * ks < whi && c0 + 16 * ks + 16 > wlo) {
+            const int key = ks * 16 + (lane & 15);
+#pragma unroll
+            for (int t = 0; t < DP / 8; t += 2) {
+              uint32_t bv[4];
+              ldmatrix_x4_trans(bv, vb + sw128_off(key, t + (lane >> 4)));
+              mma_bf16_16816(o[t], pa[ks], bv[0], bv[1]);
+              mma_bf16_16816(o[t + 1], pa[ks], bv[2], bv[3]);
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(kvempty0 + 8 * s);
+    }
+    // normalise and store this head's rows
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    const float inv_a = ra < T ? 1.0f / l_a : 0.f, inv_b = rb < T ? 1.0f / l_b : 0.f;
+    bf16* cb = ctx + h * DP;
+#pragma unroll
+    for (int t = 0; t < DP / 8; ++t) {
+      const int col = t * 8 + 2 * tq;
+      if (ra < T)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(ra) * H + col) =
+            pack_bf16x2(o[t][0] * inv_a, o[t][1] * inv_a);
+      if (rb < T)
+        *reinterpret_cast<uint32_t*>(cb + static_cast<size_t>(rb) * H + col) =
+            pack_bf16x2(o[t][2] * inv_b, o[t][3] * inv_b);
+    }
+  }
+}
+
+template <int DP>
+cudaError_t launch_tile(const void* qkv, void* ctx, const int32_t* offsets, int n, int T, int nh,
+                        int causal, int* err, int num_sms, cudaStream_t st, const L2Prefetch& pf) {
+  using SL = TileSmem<DP>;
+  const int H = nh * DP;
+  CUtensorMap tm;
+  const char* why = "";
+  // exactly T rows: key rows past the batch read as zeros
+  if (!make_tmap_bf16(&tm, qkv, static_cast<uint64_t>(T), static_cast<uint64_t>(3 * H), 64, &why))
+    return cudaErrorInvalidValue;
+  static const cudaError_t attr_err = cudaFuncSetAttribute(
+      attn_tile_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes);
+  if (attr_err != cudaSuccess) return attr_err;
+  const int tiles = (T + 63) / 64;
+  // heads per CTA: enough CTAs for two rounds of the resident ones, and as
+  // many heads per CTA as that leaves (their loads pipeline)
+  const int target = 2 * num_sms * SL::kCtasPerSm;
+  const int groups = std::min(nh, std::max(1, (target + tiles - 1) / tiles));
+  const int hpc = (nh + groups - 1) / groups;
+  dim3 grid(tiles, (nh + hpc - 1) / hpc);
+  L2PrefetchArgs pa;
+  for (int k = 0; k < 2; ++k) {
+    pa.ptr[k] = pf.ptr[k];
+    pa.bytes[k] = pf.bytes[k];
+  }
+  const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(DP));
+  launch_k(attn_tile_kernel<DP>, grid, dim3(160), SL::kBytes, st, tm, static_cast<bf16*>(ctx),
+           offsets, n, T, H, nh, hpc, scale_log2, causal, err, pa);
+  return cudaGetLastError();
+}
+
 int pad_head_dim(int d) { return d <= 32 ? 32 : (d <= 64 ? 64 : (d <= 128 ? 128 : -1)); }
 
 template <int DP, bool PFX>
@@ -772,6 +1090,17 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
     default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
+}
+
+cudaError_t attn_tile_launch(const void* qkv, void* ctx, const int32_t* offsets, int n_seqs, int T,
+                             int n_heads, int head_dim, int causal, int* err, int num_sms,
+                             cudaStream_t st, const L2Prefetch& pf) {
+  if (T == 0) return cudaSuccess;
+  if (head_dim == 64)
+    return launch_tile<64>(qkv, ctx, offsets, n_seqs, T, n_heads, causal, err, num_sms, st, pf);
+  if (head_dim == 128)
+    return launch_tile<128>(qkv, ctx, offsets, n_seqs, T, n_heads, causal, err, num_sms, st, pf);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t attn_fused_prefix_launch(const void* qkv, void* ctx, const int32_t* offsets,

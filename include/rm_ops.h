@@ -118,6 +118,19 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
                      int32_t n_seqs, int32_t n_row_blocks, int32_t n_heads, int32_t head_dim,
                      int32_t causal, void* stream);
 
+/* The same attention step on tiles of 64 consecutive packed rows: a tile
+ * holds whole short sequences and pieces of long ones, and each CTA takes one
+ * tile and a group of heads, its K/V rows (the tile's key range) arriving by
+ * TMA in 64-row chunks while the previous chunk is multiplied.  A query row
+ * admits the keys of its own sequence only (c <= r too when causal); online
+ * softmax in fp32, P rounded to bf16 for P V, as in rm_op_attn_fused.
+ * head_dim 64 or 128 (H = n_heads * head_dim); qkv: bf16 [T][3H]; ctx: bf16
+ * [T][H]; offsets: DEVICE int32[n+1] with offsets[n] = T (host value T).
+ * RM_E_INVAL for other head dims or sizes < 1; waits that give up (none in
+ * normal operation) count into an internal error word. */
+int rm_op_attn_tiles(const void* qkv, void* ctx, const int32_t* offsets, int32_t n_seqs, int32_t T,
+                     int32_t n_heads, int32_t head_dim, int32_t causal, void* stream);
+
 /* The materialised attention step (rm_op_attn_scores -> rm_op_softmax ->
  * rm_op_attn_context) without any device allocation: the score matrix and the
  * per-call metadata live in one file-scope device array of 8 MiB of scores

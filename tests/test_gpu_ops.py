@@ -382,6 +382,114 @@ def test_attention_fused(lens, nh, d, causal):
             assert np.all(np.abs(got - ref) <= tol), float((np.abs(got - ref) / tol).max())
 
 
+def _attention_ref_check(X, C, off, nh, d, causal):
+    H = nh * d
+    for i in range(len(off) - 1):
+        rows = X[off[i]:off[i + 1]]
+        for j in range(nh):
+            q = rows[:, j * d:(j + 1) * d]
+            k = rows[:, H + j * d:H + (j + 1) * d]
+            v = rows[:, 2 * H + j * d:2 * H + (j + 1) * d]
+            p = O.attention_probs(q, k, bool(causal))
+            ref = p @ v
+            # one bf16 rounding of the output and of every probability
+            tol = BF16_REL * np.abs(ref) + 2 * BF16_REL * (p @ np.abs(v)) + F32_RTOL
+            got = C[off[i]:off[i + 1], j * d:(j + 1) * d]
+            assert np.all(np.abs(got - ref) <= tol), (i, j, float((np.abs(got - ref) / tol).max()))
+
+
+@pytest.mark.parametrize("lens", [
+    [1, 65, 130, 64, 9],                              # ragged, tiles cut sequences
+    [2, 3, 1, 5, 2, 7, 1, 1, 4, 9, 2, 3, 8, 1, 6, 2],  # many sequences per 16-row warp
+    [300, 7, 560],                                    # long rows, several key chunks
+    [100] * 8,                                        # uniform, sequences straddle tiles
+    [64] * 3,                                         # tiles aligned with sequences
+    [5],                                              # one tile, shorter than 64 rows
+], ids=["ragged", "tiny", "long", "uniform", "aligned", "single"])
+@pytest.mark.parametrize("nh,d", [(2, 64), (12, 64), (16, 128)])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_attention_tiles(lens, nh, d, causal):
+    """Packed-row tiles against the oracle's attention, every row and head."""
+    H = nh * d
+    lens = np.array(lens)
+    off = synth.offsets_from_lengths(lens)
+    rng = np.random.default_rng(nh * d + causal + len(lens) + 5)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    rm.ops.attn_tiles(qkv, ctx, dev(off, torch.int32), len(lens), T, nh, d, causal)
+    torch.cuda.synchronize()
+    _attention_ref_check(f64(qkv), f64(ctx), off, nh, d, causal)
+
+
+def test_attention_tiles_bench_shape():
+    """A fused call of the BERT-base stream's shape (512 sequences of 2..100
+    tokens, 12 heads of 64): every output finite, sampled sequences against the
+    oracle, and the per-sequence fused kernel's output finite on the same input."""
+    nh, d = 12, 64
+    H = nh * d
+    rng = np.random.default_rng(2024)
+    lens = rng.integers(2, 101, 512)
+    off = synth.offsets_from_lengths(lens)
+    rb, _ = rm.ops.varlen_meta(off, nh)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    a = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    b = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    d_off = dev(off, torch.int32)
+    rm.ops.attn_tiles(qkv, a, d_off, len(lens), T, nh, d, 0)
+    rm.ops.attn_fused(qkv, b, d_off, dev(rb, torch.int32), len(lens), int(rb[-1]), nh, d, 0)
+    torch.cuda.synchronize()
+    A, B = f64(a), f64(b)
+    assert np.all(np.isfinite(A)) and np.all(np.isfinite(B))
+    pick = np.linspace(0, len(lens) - 1, 12).astype(int)
+    X = f64(qkv)
+    for i in pick:
+        sub = np.array([0, lens[i]], dtype=np.int64)
+        _attention_ref_check(X[off[i]:off[i + 1]], A[off[i]:off[i + 1]], sub, nh, d, 0)
+
+
+@pytest.mark.parametrize("kind", ["short", "mixed"])
+def test_attention_tiles_repeat_bit_identical(kind):
+    """Many heads per CTA and one key chunk per tile let the load ring run
+    several heads ahead of the warps that read it: thirty launches (other
+    launches in between change what shared memory held) must give the same
+    bits, and the first must match the oracle."""
+    nh, d = 12, 64
+    H = nh * d
+    rng = np.random.default_rng(17)
+    lens = rng.integers(1, 9, 4000) if kind == "short" else rng.integers(2, 101, 500)
+    off = synth.offsets_from_lengths(lens)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    other = dev(qkv_for(T, H, rng), torch.bfloat16)
+    d_off = dev(off, torch.int32)
+    first = None
+    junk = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    for _ in range(30):
+        rm.ops.attn_tiles(other, junk, d_off, len(lens), T, nh, d, 0)
+        ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        rm.ops.attn_tiles(qkv, ctx, d_off, len(lens), T, nh, d, 0)
+        torch.cuda.synchronize()
+        if first is None:
+            first = ctx
+            X, C = f64(qkv), f64(ctx)
+            for i in np.linspace(0, len(lens) - 1, 16).astype(int):
+                sub = np.array([0, lens[i]], dtype=np.int64)
+                _attention_ref_check(X[off[i]:off[i + 1]], C[off[i]:off[i + 1]], sub, nh, d, 0)
+        else:
+            assert torch.equal(ctx, first)
+
+
+def test_attention_tiles_rejects_other_head_dims():
+    x = torch.zeros(8, dtype=torch.bfloat16, device="cuda")
+    off = dev(np.array([0, 4], dtype=np.int32), torch.int32)
+    for d in (26, 32, 96):
+        with pytest.raises(rm.RmError) as e:
+            rm.ops.attn_tiles(x, x, off, 1, 4, 2, d, 0)
+        assert e.value.code == rm.RM_E_INVAL
+
+
 def test_gemm_gelu_epilogue_against_cuda_erf_and_oracle():
     """GELU of the epilogue (Abramowitz & Stegun 7.1.28 erf) on a dense grid of
     pre-activations: x = 0, W = 0, so y = GELU(bias)."""
