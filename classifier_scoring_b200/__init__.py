@@ -108,7 +108,7 @@ def lib() -> ctypes.CDLL:
         "rm_op_attn_context": (ctypes.c_int, [P, P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attn_fused": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attention_noalloc": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, P]),
-        "rm_op_attn_tiles": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, P]),
+        "rm_op_attn_tiles": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, I32, P]),
         "rm_op_res_ln": (ctypes.c_int, [P, P, P, P, P, I32, I32, F, I32, I32, P]),
         "rm_op_head": (ctypes.c_int, [P, P, I32, P, F, I32, I32, P, P]),
         "rm_arena_plan": (ctypes.c_int, [cfgp, I32, I32, I64, P, P, P, P, I32, P]),
@@ -329,9 +329,12 @@ class ops:
                                       n_row_blocks, n_heads, head_dim, int(causal), _stream(stream)))
 
     @staticmethod
-    def attn_tiles(qkv, ctx, offsets_dev, n_seqs, T, n_heads, head_dim, causal, stream=None):
+    def attn_tiles(qkv, ctx, offsets_dev, n_seqs, T, n_heads, head_dim, causal, stream=None,
+                   max_len=None):
+        """max_len: bound on the sequence lengths (default T)."""
         _check(lib().rm_op_attn_tiles(_ptr(qkv), _ptr(ctx), _ptr(offsets_dev), n_seqs, T, n_heads,
-                                      head_dim, causal, _stream(stream)))
+                                      head_dim, T if max_len is None else max_len, causal,
+                                      _stream(stream)))
 
     @staticmethod
     def attention_noalloc(qkv, ctx, offsets, n_heads, head_dim, causal, stream=None):

@@ -179,12 +179,6 @@ struct Bucket {
 };
 
 constexpr int kSlots = 4;
-// Longest sequence for which the fused attention runs on packed-row tiles.
-// The tiles win where most query blocks would be mostly empty (BERT-base
-// lengths 2..100: 82 vs 98 us per 28k-token call); for long rows the
-// per-sequence kernel keeps more warps busy per SM and is faster (lengths
-// 5..500: 362 vs 444 us; the causal 1.3B shape: 297 vs 324 us).
-constexpr int kTileAttnMaxLen = 128;
 
 }  // namespace
 }  // namespace rmk
@@ -650,9 +644,11 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
     if (px != nullptr) {
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
                 attn_fused_prefix_launch(qkv, ctx, d_off, d_rb, d_pst, d_pln, n, nrb, nh, d, st, pf_o));
-    } else if (c->attn_impl == RM_ATTN_FUSED && d == 64 && Lmax <= kTileAttnMaxLen) {
+    } else if (c->attn_impl == RM_ATTN_FUSED && (d == 64 || d == 128)) {
+      // packed-row tiles (head dims 64 and 128); other head dims below
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
-                attn_tile_launch(qkv, ctx, d_off, n, T, nh, d, dec, h->d_err, h->num_sms, st, pf_o));
+                attn_tile_launch(qkv, ctx, d_off, n, T, nh, d, Lmax, dec, h->d_err, h->num_sms,
+                                 st, pf_o));
     } else if (c->attn_impl == RM_ATTN_FUSED) {
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
                 attn_fused_launch(qkv, ctx, d_off, d_rb, n, nrb, nh, d, dec, st, pf_o));
@@ -1205,17 +1201,18 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
 }
 
 int rm_op_attn_tiles(const void* qkv, void* ctx, const int32_t* offsets, int32_t n_seqs, int32_t T,
-                     int32_t n_heads, int32_t head_dim, int32_t causal, void* stream) {
+                     int32_t n_heads, int32_t head_dim, int32_t max_len, int32_t causal,
+                     void* stream) {
   if (qkv == nullptr || ctx == nullptr || offsets == nullptr) return set_error(RM_E_INVAL, "NULL argument");
-  if (n_seqs < 1 || T < 1 || n_heads < 1 || (head_dim != 64 && head_dim != 128))
+  if (n_seqs < 1 || T < 1 || n_heads < 1 || max_len < 1 || (head_dim != 64 && head_dim != 128))
     return set_error(RM_E_INVAL, "bad sizes (head_dim must be 64 or 128)");
   int dev = 0, sms = 0;
   RM_CUDA(cudaGetDevice(&dev));
   RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   int32_t* err = nullptr;
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
-  RM_LAUNCH(attn_tile_launch(qkv, ctx, offsets, n_seqs, T, n_heads, head_dim, causal, err, sms,
-                             static_cast<cudaStream_t>(stream)));
+  RM_LAUNCH(attn_tile_launch(qkv, ctx, offsets, n_seqs, T, n_heads, head_dim, max_len, causal, err,
+                             sms, static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

@@ -709,7 +709,9 @@ struct TileSmem {
   static constexpr int kKVOff = 2 * kQ;                     // after two query buffers
   static constexpr int kBarOff = kKVOff + kStages * kKV;
   static constexpr int kBars = 4 + 2 * kStages;             // qfull[2] qempty[2] kvfull[S] kvempty[S]
-  static constexpr int kBytes = kBarOff + kBars * 8 + 1024; // + 1024-byte alignment slack
+  static constexpr int kSeqOff = kBarOff + kBars * 8;       // the tile's offsets window
+  static constexpr int kMaxSeqs = 66;                       // 64 rows: at most 64 sequences + 2
+  static constexpr int kBytes = kSeqOff + kMaxSeqs * 4 + 1024;   // + 1024-byte alignment slack
   static constexpr int kCtasPerSm = DP == 64 ? 3 : 2;
 };
 
@@ -753,8 +755,12 @@ __global__ void __launch_bounds__(160)
   const int h0 = blockIdx.y * hpc;
   const int nhl = min(hpc, nh - h0);
   const int rlast = min(r0 + 64, T) - 1;
-  const int s_first = upper_index(offsets, n, r0);
-  const int s_last = upper_index(offsets, n, rlast);
+  // the tile's first and last sequence: one search each, shared
+  __shared__ int s_edge[2];
+  if (threadIdx.x == 0) s_edge[0] = upper_index(offsets, n, r0);
+  if (threadIdx.x == 32) s_edge[1] = upper_index(offsets, n, rlast);
+  __syncthreads();
+  const int s_first = s_edge[0], s_last = s_edge[1];
   const int Klo = offsets[s_first];
   const int Khi = causal ? rlast + 1 : offsets[s_last + 1];
   const int nch = (Khi - Klo + 63) / 64;
@@ -802,26 +808,36 @@ __global__ void __launch_bounds__(160)
   }
 
   // ---- consumers: 16 query rows per warp ----
+  // the offsets of the tile's sequences (s_first .. s_last + 1) go to shared
+  // memory once, so that each row finds its sequence there
+  int32_t* soff = reinterpret_cast<int32_t*>(sm + SL::kSeqOff);
+  const int nseq = s_last - s_first + 2;
+  if (threadIdx.x < nseq) soff[threadIdx.x] = offsets[s_first + threadIdx.x];
+  asm volatile("bar.sync 1, 128;" ::: "memory");              // the four consumer warps
   const int g = lane >> 2, tq = lane & 3;
   const int ra = r0 + warp * 16 + g, rb = ra + 8;
-  // keys a row admits: its own sequence's rows [lo, hi) (hi <= r + 1 when
+  // keys a row admits: its own sequence's rows [lo, lo + len) (up to r when
   // causal); rows past the batch admit none
-  auto key_range = [&](int r, int& lo, int& hi) {
+  auto key_range = [&](int r, int& lo, int& len) {
     if (r >= T) {
       lo = 0;
-      hi = 0;
+      len = 0;
       return;
     }
-    const int s = upper_index(offsets, n, r);
-    lo = offsets[s];
-    hi = causal ? r + 1 : offsets[s + 1];
+    int a = 0, b2 = nseq - 2;                                   // largest i with soff[i] <= r
+    while (a < b2) {
+      const int mid = (a + b2 + 1) >> 1;
+      if (soff[mid] <= r) a = mid; else b2 = mid - 1;
+    }
+    lo = soff[a];
+    len = (causal ? r + 1 : soff[a + 1]) - lo;
   };
-  int lo_a, hi_a, lo_b, hi_b;
-  key_range(ra, lo_a, hi_a);
-  key_range(rb, lo_b, hi_b);
+  int lo_a, len_a, lo_b, len_b;
+  key_range(ra, lo_a, len_a);
+  key_range(rb, lo_b, len_b);
   // the warp's key range: chunks outside it are skipped
-  const int wlo = __reduce_min_sync(0xffffffffu, min(hi_a > lo_a ? lo_a : INT_MAX, hi_b > lo_b ? lo_b : INT_MAX));
-  const int whi = __reduce_max_sync(0xffffffffu, max(hi_a, hi_b));
+  const int wlo = __reduce_min_sync(0xffffffffu, min(len_a > 0 ? lo_a : INT_MAX, len_b > 0 ? lo_b : INT_MAX));
+  const int whi = __reduce_max_sync(0xffffffffu, max(lo_a + len_a, lo_b + len_b));
 
   int it = 0;
   for (int j = 0; j < nhl; ++j) {
@@ -873,15 +889,17 @@ __global__ void __launch_bounds__(160)
             }
           }
         }
-        // mask (own sequence, causal), scale into the log2 domain, block maxima
+        // mask to the row's own keys; block maxima of the raw scores (the
+        // log2-domain scale is positive and folds into the exponent below)
         float bm_a = -INFINITY, bm_b = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
           const int cc = c0 + nt * 8 + 2 * tq;
-          sc[nt][0] = (cc >= lo_a && cc < hi_a) ? sc[nt][0] * scale_log2 : -INFINITY;
-          sc[nt][1] = (cc + 1 >= lo_a && cc + 1 < hi_a) ? sc[nt][1] * scale_log2 : -INFINITY;
-          sc[nt][2] = (cc >= lo_b && cc < hi_b) ? sc[nt][2] * scale_log2 : -INFINITY;
-          sc[nt][3] = (cc + 1 >= lo_b && cc + 1 < hi_b) ? sc[nt][3] * scale_log2 : -INFINITY;
+          const unsigned ua = static_cast<unsigned>(cc - lo_a), ub = static_cast<unsigned>(cc - lo_b);
+          sc[nt][0] = ua < static_cast<unsigned>(len_a) ? sc[nt][0] : -INFINITY;
+          sc[nt][1] = ua + 1u < static_cast<unsigned>(len_a) ? sc[nt][1] : -INFINITY;
+          sc[nt][2] = ub < static_cast<unsigned>(len_b) ? sc[nt][2] : -INFINITY;
+          sc[nt][3] = ub + 1u < static_cast<unsigned>(len_b) ? sc[nt][3] : -INFINITY;
           bm_a = fmaxf(bm_a, fmaxf(sc[nt][0], sc[nt][1]));
           bm_b = fmaxf(bm_b, fmaxf(sc[nt][2], sc[nt][3]));
         }
@@ -890,17 +908,22 @@ __global__ void __launch_bounds__(160)
         bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 1));
         bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
         const float mn_a = fmaxf(m_a, bm_a), mn_b = fmaxf(m_b, bm_b);
-        // a row with no admitted key so far keeps m = -inf; shift by 0 then
-        const float sh_a = mn_a == -INFINITY ? 0.f : mn_a, sh_b = mn_b == -INFINITY ? 0.f : mn_b;
-        const float al_a = exp2f(m_a - sh_a), al_b = exp2f(m_b - sh_b);
+        // shift in the log2 domain; a row with no admitted key so far keeps
+        // m = -inf and shifts by 0
+        const float sh_a = mn_a == -INFINITY ? 0.f : mn_a * scale_log2;
+        const float sh_b = mn_b == -INFINITY ? 0.f : mn_b * scale_log2;
+        const float al_a = exp2f(fmaf(m_a, scale_log2, -sh_a));
+        const float al_b = exp2f(fmaf(m_b, scale_log2, -sh_b));
         m_a = mn_a;
         m_b = mn_b;
         float ps_a = 0.f, ps_b = 0.f;
         uint32_t pa[4][4];
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
-          const float p0 = exp2f(sc[nt][0] - sh_a), p1 = exp2f(sc[nt][1] - sh_a);
-          const float p2 = exp2f(sc[nt][2] - sh_b), p3 = exp2f(sc[nt][3] - sh_b);
+          const float p0 = exp2f(fmaf(sc[nt][0], scale_log2, -sh_a));
+          const float p1 = exp2f(fmaf(sc[nt][1], scale_log2, -sh_a));
+          const float p2 = exp2f(fmaf(sc[nt][2], scale_log2, -sh_b));
+          const float p3 = exp2f(fmaf(sc[nt][3], scale_log2, -sh_b));
           ps_a += p0 + p1;
           ps_b += p2 + p3;
           pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
@@ -956,7 +979,8 @@ __global__ void __launch_bounds__(160)
 
 template <int DP>
 cudaError_t launch_tile(const void* qkv, void* ctx, const int32_t* offsets, int n, int T, int nh,
-                        int causal, int* err, int num_sms, cudaStream_t st, const L2Prefetch& pf) {
+                        int max_len, int causal, int* err, int num_sms, cudaStream_t st,
+                        const L2Prefetch& pf) {
   using SL = TileSmem<DP>;
   const int H = nh * DP;
   CUtensorMap tm;
@@ -968,9 +992,14 @@ cudaError_t launch_tile(const void* qkv, void* ctx, const int32_t* offsets, int 
       attn_tile_kernel<DP>, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes);
   if (attr_err != cudaSuccess) return attr_err;
   const int tiles = (T + 63) / 64;
-  // heads per CTA: enough CTAs for two rounds of the resident ones, and as
-  // many heads per CTA as that leaves (their loads pipeline)
-  const int target = 2 * num_sms * SL::kCtasPerSm;
+  // heads per CTA: enough CTAs for a few rounds of the resident ones, and as
+  // many heads per CTA as that leaves (their loads pipeline across heads).
+  // Short rows give a tile one or two key chunks per head, so fewer, longer
+  // CTAs keep the ring busy; long rows pipeline within a head and balance
+  // better over more CTAs (measured on B200: lengths 2..100 best at 4
+  // rounds, lengths 5..500 and the causal 1.3B shape at 8).
+  const int rounds = max_len <= 128 ? 4 : 8;
+  const int target = rounds * num_sms * SL::kCtasPerSm;
   const int groups = std::min(nh, std::max(1, (target + tiles - 1) / tiles));
   const int hpc = (nh + groups - 1) / groups;
   dim3 grid(tiles, (nh + hpc - 1) / hpc);
@@ -1093,13 +1122,15 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
 }
 
 cudaError_t attn_tile_launch(const void* qkv, void* ctx, const int32_t* offsets, int n_seqs, int T,
-                             int n_heads, int head_dim, int causal, int* err, int num_sms,
-                             cudaStream_t st, const L2Prefetch& pf) {
+                             int n_heads, int head_dim, int max_len, int causal, int* err,
+                             int num_sms, cudaStream_t st, const L2Prefetch& pf) {
   if (T == 0) return cudaSuccess;
   if (head_dim == 64)
-    return launch_tile<64>(qkv, ctx, offsets, n_seqs, T, n_heads, causal, err, num_sms, st, pf);
+    return launch_tile<64>(qkv, ctx, offsets, n_seqs, T, n_heads, max_len, causal, err, num_sms, st,
+                           pf);
   if (head_dim == 128)
-    return launch_tile<128>(qkv, ctx, offsets, n_seqs, T, n_heads, causal, err, num_sms, st, pf);
+    return launch_tile<128>(qkv, ctx, offsets, n_seqs, T, n_heads, max_len, causal, err, num_sms,
+                            st, pf);
   return cudaErrorInvalidValue;
 }
 

@@ -87,10 +87,11 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
                               const L2Prefetch& pf = {});
 // Packed-row attention (head_dim 64 or 128): tiles of 64 consecutive
 // packed rows of any sequences, a group of heads per CTA, TMA-fed K/V chunks
-// of each tile's key range; err: device error words (ERR_TIMEOUT).
+// of each tile's key range; max_len (>= every L_i) sizes the head groups;
+// err: device error words (ERR_TIMEOUT).
 cudaError_t attn_tile_launch(const void* qkv, void* ctx, const int32_t* offsets, int n_seqs, int T,
-                             int n_heads, int head_dim, int causal, int* err, int num_sms,
-                             cudaStream_t st, const L2Prefetch& pf = {});
+                             int n_heads, int head_dim, int max_len, int causal, int* err,
+                             int num_sms, cudaStream_t st, const L2Prefetch& pf = {});
 // Causal fused attention over segments that may continue a shared prefix:
 // query row r of segment i attends to the pre_len[i] rows starting at packed
 // row pre_start[i] (all of them) and to rows 0..r of its own segment.

@@ -125,11 +125,13 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
  * admits the keys of its own sequence only (c <= r too when causal); online
  * softmax in fp32, P rounded to bf16 for P V, as in rm_op_attn_fused.
  * head_dim 64 or 128 (H = n_heads * head_dim); qkv: bf16 [T][3H]; ctx: bf16
- * [T][H]; offsets: DEVICE int32[n+1] with offsets[n] = T (host value T).
- * RM_E_INVAL for other head dims or sizes < 1; waits that give up (none in
+ * [T][H]; offsets: DEVICE int32[n+1] with offsets[n] = T (host value T);
+ * max_len: a host bound on every L_i (it sizes the launch: CTAs take fewer
+ * heads each when rows are long).  RM_E_INVAL for other head dims or sizes < 1; waits that give up (none in
  * normal operation) count into an internal error word. */
 int rm_op_attn_tiles(const void* qkv, void* ctx, const int32_t* offsets, int32_t n_seqs, int32_t T,
-                     int32_t n_heads, int32_t head_dim, int32_t causal, void* stream);
+                     int32_t n_heads, int32_t head_dim, int32_t max_len, int32_t causal,
+                     void* stream);
 
 /* The materialised attention step (rm_op_attn_scores -> rm_op_softmax ->
  * rm_op_attn_context) without any device allocation: the score matrix and the

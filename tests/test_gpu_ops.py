@@ -417,7 +417,10 @@ def test_attention_tiles(lens, nh, d, causal):
     T = int(off[-1])
     qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
     ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
-    rm.ops.attn_tiles(qkv, ctx, dev(off, torch.int32), len(lens), T, nh, d, causal)
+    # the launch as rm_score sizes it (max_len = the longest row), which takes
+    # more heads per CTA for short rows than the default bound (T) does
+    rm.ops.attn_tiles(qkv, ctx, dev(off, torch.int32), len(lens), T, nh, d, causal,
+                      max_len=int(lens.max()))
     torch.cuda.synchronize()
     _attention_ref_check(f64(qkv), f64(ctx), off, nh, d, causal)
 
@@ -469,7 +472,7 @@ def test_attention_tiles_repeat_bit_identical(kind):
     for _ in range(30):
         rm.ops.attn_tiles(other, junk, d_off, len(lens), T, nh, d, 0)
         ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
-        rm.ops.attn_tiles(qkv, ctx, d_off, len(lens), T, nh, d, 0)
+        rm.ops.attn_tiles(qkv, ctx, d_off, len(lens), T, nh, d, 0, max_len=int(lens.max()))
         torch.cuda.synchronize()
         if first is None:
             first = ctx
