@@ -106,6 +106,65 @@ __device__ __forceinline__ float erf_as7128(float x) {
 __device__ __forceinline__ float gelu_erf_fast(float u) {
   return 0.5f * u * (1.0f + erf_as7128(u * 0.70710678118654752f));
 }
+
+// Two fp32 lanes in one 64-bit register, for sm_100's packed arithmetic
+// (add/sub/mul/fma .rn.f32x2: one instruction, two IEEE fp32 operations, each
+// rounded as its scalar form would be).
+__device__ __forceinline__ uint64_t f32x2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f32x2_unpack(uint64_t r, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(r));
+}
+__device__ __forceinline__ uint64_t f32x2_splat(float v) { return f32x2_pack(v, v); }
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// gelu_erf_fast on two values at once: the same A&S 7.1.28 polynomial and
+// 16th power in packed fp32 (identical roundings lane by lane), the two
+// reciprocals scalar; the last step forms h + h*erf with h = u/2 (one fused
+// rounding where the scalar form rounds 1 + erf and the product).
+__device__ __forceinline__ uint64_t gelu_erf_fast_x2(uint64_t u) {
+  const uint64_t x = f32x2_mul(u, f32x2_splat(0.70710678118654752f));
+  const uint64_t ax = x & 0x7fffffff7fffffffull;
+  uint64_t p = f32x2_fma(f32x2_splat(0.0000430638f), ax, f32x2_splat(0.0002765672f));
+  p = f32x2_fma(p, ax, f32x2_splat(0.0001520143f));
+  p = f32x2_fma(p, ax, f32x2_splat(0.0092705272f));
+  p = f32x2_fma(p, ax, f32x2_splat(0.0422820123f));
+  p = f32x2_fma(p, ax, f32x2_splat(0.0705230784f));
+  p = f32x2_fma(p, ax, f32x2_splat(1.0f));
+  p = f32x2_mul(p, p);
+  p = f32x2_mul(p, p);
+  p = f32x2_mul(p, p);
+  p = f32x2_mul(p, p);                        // p^16 (inf for large |x|: erf = +-1)
+  float p0, p1;
+  f32x2_unpack(p, p0, p1);
+  // 1 - 1/p is in [0, 1): its sign bit is clear, so the sign of x is OR-ed in
+  const uint64_t y = f32x2_sub(f32x2_splat(1.0f), f32x2_pack(__fdividef(1.0f, p0), __fdividef(1.0f, p1)));
+  const uint64_t erf = y | (x & 0x8000000080000000ull);
+  const uint64_t h = f32x2_mul(u, f32x2_splat(0.5f));
+  return f32x2_fma(erf, h, h);
+}
 __device__ __forceinline__ float gelu_tanh(float u) {
   return 0.5f * u * (1.0f + tanhf(0.79788456080286536f * (u + 0.044715f * u * u * u)));
 }

@@ -16,7 +16,7 @@
 namespace rmk {
 namespace {
 
-constexpr int kWarps = 8;   // warps (rows) per CTA
+constexpr int kWarps = 4;   // warps (rows) per CTA
 
 template <int MAXC>
 __device__ __forceinline__ void row_moments(const float (&v)[MAXC][8], int nch, int lane, int H,
