@@ -793,13 +793,21 @@ def kernel_bench(args):
         d_off = torch.from_numpy(off).cuda()
         d_so = torch.from_numpy(so).cuda()
         n, T = len(lens), int(off[-1])
-        # the kernel's rows are independent, so a launch covers at most 2^31 rows: fine here
-        ms = timed(lambda: rm.ops.softmax(S, rm.BF16, d_off, d_so, n, T, nh, int(lens.max()), causal, st))
         entries = nh * float(np.sum(lens * (lens + 1) / 2 if causal else lens * lens))
         gb = 4.0 * entries / 1e9
-        out["kernels"][label] = {"ms": ms, "algorithmic_GB": gb, "gbs": gb / (ms * 1e-3),
-                                 "frac_of_measured": gb / (ms * 1e-3) / pk["hbm_gbs"],
-                                 "sequences": n, "heads": nh}
+        scratch = torch.empty(rm.ops.softmax_scratch_bytes(n, T, nh), dtype=torch.uint8, device="cuda")
+        # by length class (the path rm_score takes; the row-index kernels are
+        # inside the timing) and with batch-wide lane groups
+        for name, fn in (
+                (label, lambda: rm.ops.softmax_classes(S, rm.BF16, d_off, d_so, n, T, nh,
+                                                       int(lens.max()), causal, scratch, st)),
+                (label + "_batchwide", lambda: rm.ops.softmax(S, rm.BF16, d_off, d_so, n, T, nh,
+                                                              int(lens.max()), causal, st))):
+            ms = timed(fn)
+            out["kernels"][name] = {"ms": ms, "algorithmic_GB": gb, "gbs": gb / (ms * 1e-3),
+                                    "frac_of_measured": gb / (ms * 1e-3) / pk["hbm_gbs"],
+                                    "sequences": n, "heads": nh}
+        del scratch
         del S
     for label, H, T, mode in (("res_ln_post_H768", 768, 1 << 20, 0), ("res_ln_pre_H2048", 2048, 1 << 18, 1)):
         y = torch.randn(T, H, dtype=torch.bfloat16, device="cuda")

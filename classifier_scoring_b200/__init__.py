@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         "rm_op_embed": (ctypes.c_int, [P, P, I32, I32, P, P, P, P, F, I32, I32, I32, P, I32, P, P]),
         "rm_op_attn_scores": (ctypes.c_int, [P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_softmax": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P]),
+        "rm_op_softmax_classes": (ctypes.c_int, [P, I32, P, P, I32, I32, I32, I32, I32, P, P]),
+        "rm_softmax_scratch_bytes": (SZ, [I32, I32, I32]),
         "rm_op_attn_context": (ctypes.c_int, [P, P, P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attn_fused": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attention_noalloc": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, P]),
@@ -314,6 +316,17 @@ class ops:
     def softmax(S, s_dtype, offsets_dev, so_dev, n_seqs, T, n_heads, max_len, causal, stream=None):
         _check(lib().rm_op_softmax(_ptr(S), s_dtype, _ptr(offsets_dev), _ptr(so_dev), n_seqs, T,
                                    n_heads, max_len, int(causal), _stream(stream)))
+
+    @staticmethod
+    def softmax_scratch_bytes(n_seqs, T, n_heads):
+        return int(lib().rm_softmax_scratch_bytes(int(n_seqs), int(T), int(n_heads)))
+
+    @staticmethod
+    def softmax_classes(S, s_dtype, offsets_dev, so_dev, n_seqs, T, n_heads, max_len, causal, scratch,
+                        stream=None):
+        """scratch: device buffer of softmax_scratch_bytes(n_seqs, T, n_heads) bytes."""
+        _check(lib().rm_op_softmax_classes(_ptr(S), s_dtype, _ptr(offsets_dev), _ptr(so_dev), n_seqs,
+                                           T, n_heads, max_len, causal, _ptr(scratch), _stream(stream)))
 
     @staticmethod
     def attn_context(S, qkv, ctx, offsets_dev, rb_dev, so_dev, n_seqs, n_row_blocks, n_heads,

@@ -200,6 +200,7 @@ struct rm_handle {
   int64_t arena_bytes = 0, fixed_bytes = 0, meta_bytes = 0;
   int32_t* d_ids = nullptr;
   float* d_scores = nullptr;
+  void* d_sm_scratch = nullptr;   // row index of the materialised softmax
   uint8_t* d_meta = nullptr;
   uint8_t* planned = nullptr;
   int32_t* d_err = nullptr;
@@ -656,7 +657,8 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
       RM_KERNEL(RM_K_SCORES, att_flops, 2.0 * Td * Hd * 2 + 2.0 * att,
                 attn_scores_launch(qkv, s, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
       RM_KERNEL(RM_K_SOFTMAX, 0, sm_bytes,
-                softmax_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, h->d_err, st));
+                softmax_classes_launch(s, 1, d_off, d_so, n, T, nh, Lmax, dec, h->d_sm_scratch,
+                                       h->num_sms, st));
       RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
                 attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
     }
@@ -702,7 +704,16 @@ int alloc_runtime(rm_handle* h) {
   const int64_t Smax = static_cast<int64_t>(cfg->n_heads) * T * Lp;
   const MetaLayout ml(cfg->max_batch_seqs);
   h->meta_bytes = align_up(ml.bytes, 256);
-  h->fixed_bytes = h->meta_bytes + align_up(4 * T, 256) + align_up(4 * cfg->max_batch_seqs, 256);
+  // fixed part: metadata | ids (rm_score_host) | scores (rm_score_host) |
+  // the materialised softmax's row index (none with the fused attention)
+  const int64_t sm_scratch =
+      cfg->attn_impl == RM_ATTN_FUSED
+          ? 0
+          : align_up(static_cast<int64_t>(softmax_classes_scratch_bytes(cfg->max_batch_seqs,
+                                                                        static_cast<int>(T),
+                                                                        cfg->n_heads)), 256);
+  h->fixed_bytes = h->meta_bytes + align_up(4 * T, 256) + align_up(4 * cfg->max_batch_seqs, 256) +
+                   sm_scratch;
   const int64_t Sres =
       cfg->attn_impl == RM_ATTN_FUSED ? 0 : align_up(std::max<int64_t>(Smax, 1), 65536);
   h->arena_bytes =
@@ -720,6 +731,8 @@ int alloc_runtime(rm_handle* h) {
   h->d_meta = h->arena;
   h->d_ids = reinterpret_cast<int32_t*>(h->arena + h->meta_bytes);
   h->d_scores = reinterpret_cast<float*>(h->arena + h->meta_bytes + align_up(4 * T, 256));
+  h->d_sm_scratch = h->arena + h->meta_bytes + align_up(4 * T, 256) +
+                    align_up(4 * cfg->max_batch_seqs, 256);
   h->planned = h->arena + h->fixed_bytes;
   return RM_OK;
 }
@@ -1197,6 +1210,29 @@ int rm_op_attn_fused(const void* qkv, void* ctx, const int32_t* offsets, const i
     return set_error(RM_E_INVAL, "bad sizes");
   RM_LAUNCH(attn_fused_launch(qkv, ctx, offsets, rb_off, n_seqs, n_row_blocks, n_heads, head_dim,
                               causal != 0, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+size_t rm_softmax_scratch_bytes(int32_t n_seqs, int32_t T, int32_t n_heads) {
+  if (n_seqs < 0 || T < 0 || n_heads < 1) return 0;
+  return softmax_classes_scratch_bytes(n_seqs, T, n_heads);
+}
+
+int rm_op_softmax_classes(void* S, int32_t s_dtype, const int32_t* offsets, const int64_t* s_off,
+                          int32_t n_seqs, int32_t T, int32_t n_heads, int32_t max_len,
+                          int32_t causal, void* scratch, void* stream) {
+  if (S == nullptr || offsets == nullptr || s_off == nullptr || scratch == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || T < 1 || n_heads < 1 || max_len < 1 || max_len > 1024 ||
+      (s_dtype != RM_F32 && s_dtype != RM_BF16))
+    return set_error(RM_E_INVAL, "bad sizes");
+  if ((reinterpret_cast<uintptr_t>(scratch) & 15) != 0)
+    return set_error(RM_E_INVAL, "scratch must be 16-byte aligned");
+  int dev = 0, sms = 0;
+  RM_CUDA(cudaGetDevice(&dev));
+  RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  RM_LAUNCH(softmax_classes_launch(S, s_dtype, offsets, s_off, n_seqs, T, n_heads, max_len,
+                                   causal != 0, scratch, sms, static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

@@ -15,6 +15,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -117,6 +118,63 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// One lane group's softmax over its U rows (row[u] of valid length len[u];
+// len 0 = no row): each lane holds MAXC 8-element chunks of each row in
+// registers, all loads issued before the first reduction so that short rows
+// still keep enough bytes in flight.  Every lane of the warp calls it (the
+// group reductions are warp shuffles).
+template <typename T, int G, int MAXC, int U>
+__device__ __forceinline__ void softmax_group(T* const (&row)[U], const int (&len)[U], int sub) {
+  float v[U][MAXC][8];
+#pragma unroll
+  for (int u = 0; u < U; ++u)
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) Chunk8<T>::load(row[u] + col, v[u][c]);
+    }
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    float m = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (col + e >= len[u]) v[u][c][e] = -INFINITY;
+          m = fmaxf(m, v[u][c][e]);
+        }
+      }
+    }
+    m = group_max<G>(m);
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float p = (col + e < len[u]) ? __expf(v[u][c][e] - m) : 0.f;
+          v[u][c][e] = p;
+          sum += p;
+        }
+      }
+    }
+    sum = group_sum<G>(sum);
+    const float inv = 1.0f / sum;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int col = (c * G + sub) * 8;
+      if (col < len[u]) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[u][c][e] *= inv;
+        Chunk8<T>::store(row[u] + col, v[u][c]);
+      }
+    }
+  }
+}
+
 // Masked softmax.  A group of G lanes owns U consecutive rows; each lane
 // holds MAXC 8-element chunks of each of them in registers.  All U*MAXC loads
 // of a lane are issued before the first reduction, so short rows still keep
@@ -167,54 +225,293 @@ __global__ void __launch_bounds__(256)
       row[u] = S;
     }
   }
-  float v[U][MAXC][8];
+  softmax_group<T, G, MAXC, U>(row, len, sub);
+}
+
+// softmax_group for bf16 rows, written for instruction count and registers
+// (the class kernel below is bound by the latency of its loads, so it keeps
+// the next rows' loads in flight while it computes): the row maximum over
+// packed bf16 pairs (exact in any precision), the masking of a row's last
+// partial chunk at 16-bit granularity (-inf), and the exponent's argument
+// and the sum in packed fp32 pairs; exp2 of -inf gives the masked entries
+// exactly 0.  The exponentials are formed twice (for the sum, then for the
+// output) rather than held.
+template <int G, int MAXC, int U>
+__device__ __forceinline__ void softmax_load_bf16(bf16* const (&row)[U], const int (&len)[U], int sub,
+                                                  uint32_t (&w)[U][MAXC][4]) {
 #pragma unroll
   for (int u = 0; u < U; ++u)
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int col = (c * G + sub) * 8;
-      if (col < len[u]) Chunk8<T>::load(row[u] + col, v[u][c]);
+      if (col < len[u]) {
+        const uint4 q = *reinterpret_cast<const uint4*>(row[u] + col);
+        w[u][c][0] = q.x;
+        w[u][c][1] = q.y;
+        w[u][c][2] = q.z;
+        w[u][c][3] = q.w;
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) w[u][c][j] = 0xff80ff80u;   // -inf pairs
+      }
     }
+}
+
+template <int G, int MAXC, int U>
+__device__ __forceinline__ void softmax_compute_bf16(bf16* const (&row)[U], const int (&len)[U],
+                                                     int sub, uint32_t (&w)[U][MAXC][4]) {
+  constexpr float kLog2e = 1.4426950408889634f;
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    float m = -INFINITY;
+    // entries past the row inside its last chunk read as -inf
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
-      const int col = (c * G + sub) * 8;
-      if (col < len[u]) {
+      const int nv = len[u] - (c * G + sub) * 8;
+      if (nv > 0 && nv < 8) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          if (col + e >= len[u]) v[u][c][e] = -INFINITY;
-          m = fmaxf(m, v[u][c][e]);
+        for (int j = 0; j < 4; ++j) {
+          if (2 * j >= nv) w[u][c][j] = 0xff80ff80u;
+          else if (2 * j + 1 >= nv) w[u][c][j] = (w[u][c][j] & 0x0000ffffu) | 0xff800000u;
         }
       }
     }
+    __nv_bfloat162 mx = *reinterpret_cast<const __nv_bfloat162*>(&w[u][0][0]);
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        mx = __hmax2(mx, *reinterpret_cast<const __nv_bfloat162*>(&w[u][c][j]));
+    float m = fmaxf(__low2float(mx), __high2float(mx));
     m = group_max<G>(m);
-    float sum = 0.f;
+    // a row with no entry (len 0) keeps m = -inf: shift by 0 then
+    const uint64_t shift = f32x2_splat(m == -INFINITY ? 0.f : -m * kLog2e);
+    const uint64_t l2e = f32x2_splat(kLog2e);
+    uint64_t acc = 0;                                         // +0.0 in both lanes
 #pragma unroll
-    for (int c = 0; c < MAXC; ++c) {
-      const int col = (c * G + sub) * 8;
-      if (col < len[u]) {
+    for (int c = 0; c < MAXC; ++c)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float p = (col + e < len[u]) ? __expf(v[u][c][e] - m) : 0.f;
-          v[u][c][e] = p;
-          sum += p;
-        }
+      for (int j = 0; j < 4; ++j) {
+        float x0, x1;
+        f32x2_unpack(f32x2_fma(f32x2_pack(bf16_lo(w[u][c][j]), bf16_hi(w[u][c][j])), l2e, shift), x0, x1);
+        acc = f32x2_add(acc, f32x2_pack(exp2f(x0), exp2f(x1)));
       }
-    }
-    sum = group_sum<G>(sum);
-    const float inv = 1.0f / sum;
+    float a0, a1;
+    f32x2_unpack(acc, a0, a1);
+    const float inv = 1.0f / group_sum<G>(a0 + a1);
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int col = (c * G + sub) * 8;
       if (col < len[u]) {
+        uint32_t o[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[u][c][e] *= inv;
-        Chunk8<T>::store(row[u] + col, v[u][c]);
+        for (int j = 0; j < 4; ++j) {
+          float x0, x1;
+          f32x2_unpack(f32x2_fma(f32x2_pack(bf16_lo(w[u][c][j]), bf16_hi(w[u][c][j])), l2e, shift), x0, x1);
+          o[j] = pack_bf16x2(exp2f(x0) * inv, exp2f(x1) * inv);
+        }
+        *reinterpret_cast<uint4*>(row[u] + col) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
   }
+}
+
+// ---------------------------------------------------------------------------
+// Masked softmax by row-length class.  The batch-wide kernel above sizes its
+// lane groups for the longest row and finds each group's sequence by a binary
+// search over the offsets: with many short rows most lanes idle and the
+// search's dependent loads cost more than the rows.  Here the rows are first
+// regrouped, on the device, by the class of their length (8-element chunks
+// <= 1, 2, 4, 8, 16, 32, 64, 96, 128):
+//   softmax_count_kernel: rows per class (n_heads * L_i per sequence);
+//   softmax_index_kernel: each sequence reserves a stretch of its class's
+//     segment of a class-ordered row space and writes, for every row of the
+//     stretch, its sequence (row_seq) and the stretch's start (seq_base);
+//   softmax_class_kernel: one persistent pass per class, lane groups sized
+//     to the class, each group finding its sequence with one load.
+// The order of sequences inside a class (reservation order) does not matter:
+// every row is computed on its own, with the same arithmetic whatever its
+// position.
+// ---------------------------------------------------------------------------
+constexpr int kSmClasses = 9;
+
+__host__ __device__ constexpr int softmax_class_of(int L) {
+  return (L + 7) / 8 <= 1 ? 0 : (L + 7) / 8 <= 2 ? 1 : (L + 7) / 8 <= 4 ? 2 : (L + 7) / 8 <= 8 ? 3
+       : (L + 7) / 8 <= 16 ? 4 : (L + 7) / 8 <= 32 ? 5 : (L + 7) / 8 <= 64 ? 6
+       : (L + 7) / 8 <= 96 ? 7 : 8;
+}
+
+// scratch: counters int64[2 * kSmClasses] (rows per class, reservation
+// cursors) | seq_base int64[n] | row_seq int32[n_heads * T]
+struct SoftmaxIndexLayout {
+  size_t base, rows, bytes;
+  SoftmaxIndexLayout(long long n, long long rows_total) {
+    base = 16 * kSmClasses;
+    rows = base + 8 * static_cast<size_t>(n);
+    bytes = rows + 4 * static_cast<size_t>(rows_total);
+  }
+};
+
+__global__ void __launch_bounds__(256)
+    softmax_count_kernel(const int32_t* __restrict__ offsets, int n, int nh,
+                         unsigned long long* __restrict__ ctr) {
+  __shared__ unsigned long long part[kSmClasses];
+  if (threadIdx.x < kSmClasses) part[threadIdx.x] = 0;
+  pdl_launch_dependents();
+  pdl_wait();
+  __syncthreads();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int L = offsets[i + 1] - offsets[i];
+    atomicAdd(&part[softmax_class_of(L)], static_cast<unsigned long long>(nh) * L);
+  }
+  __syncthreads();
+  if (threadIdx.x < kSmClasses && part[threadIdx.x] != 0) atomicAdd(&ctr[threadIdx.x], part[threadIdx.x]);
+}
+
+__global__ void __launch_bounds__(256)
+    softmax_index_kernel(const int32_t* __restrict__ offsets, int n, int nh,
+                         unsigned long long* __restrict__ ctr, long long* __restrict__ seq_base,
+                         int32_t* __restrict__ row_seq) {
+  __shared__ long long seg[kSmClasses];
+  pdl_launch_dependents();
+  pdl_wait();
+  if (threadIdx.x == 0) {
+    long long a = 0;
+    for (int k = 0; k < kSmClasses; ++k) {
+      seg[k] = a;
+      a += static_cast<long long>(ctr[k]);
+    }
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  for (int i = blockIdx.x * 8 + (threadIdx.x >> 5); i < n; i += gridDim.x * 8) {
+    const int L = offsets[i + 1] - offsets[i];
+    const int k = softmax_class_of(L);
+    const long long cnt = static_cast<long long>(nh) * L;
+    long long base = 0;
+    if (lane == 0)
+      base = seg[k] + static_cast<long long>(atomicAdd(&ctr[kSmClasses + k], static_cast<unsigned long long>(cnt)));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (lane == 0) seq_base[i] = base;
+    for (long long r = lane; r < cnt; r += 32) row_seq[base + r] = i;
+  }
+}
+
+// Rows [R0, R0 + U) of the class-ordered row space (those below Re): their
+// addresses and lengths (length 0 for none).
+template <typename T, int U>
+__device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ offsets,
+                                              const int64_t* __restrict__ s_off,
+                                              const long long* __restrict__ seq_base,
+                                              const int32_t* __restrict__ row_seq, long long R0,
+                                              long long Re, int nh, int causal, T* (&row)[U],
+                                              int (&len)[U]) {
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    len[u] = 0;
+    row[u] = S;
+  }
+  if (R0 >= Re) return;
+  int i = row_seq[R0];
+  long long b = seq_base[i];
+  int L = offsets[i + 1] - offsets[i];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const long long R = R0 + u;
+    if (R < Re) {
+      if (R - b >= static_cast<long long>(nh) * L) {         // the next sequence's stretch
+        i = row_seq[R];
+        b = seq_base[i];
+        L = offsets[i + 1] - offsets[i];
+      }
+      const long long rr = R - b;                            // row inside the sequence's block
+      len[u] = causal ? static_cast<int>(rr % L) + 1 : L;
+      row[u] = S + s_off[i] + rr * ((L + 7) & ~7);
+    }
+  }
+}
+
+// One class: lane groups of G lanes, U consecutive rows (of the class-ordered
+// row space) each, grid-striding.  The loop bound is uniform across a warp
+// (groups past the end get empty rows): the group reductions are warp
+// shuffles.  For bf16 rows the next iteration's rows are loaded before the
+// current ones are computed, so that loads stay in flight.
+template <typename T, int G, int MAXC, int U>
+__device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restrict__ offsets,
+                                                   const int64_t* __restrict__ s_off,
+                                                   const long long* __restrict__ seq_base,
+                                                   const int32_t* __restrict__ row_seq,
+                                                   long long Rb, long long Re, int nh, int causal) {
+  if (Rb >= Re) return;
+  const int lane = threadIdx.x & 31, sub = lane % G;
+  constexpr int kGpw = 32 / G;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  long long wg = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (Rb + wg * kGpw * U >= Re) return;                      // uniform across the warp
+  int len[U];
+  T* row[U];
+  class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re, nh,
+                      causal, row, len);
+  if constexpr (std::is_same<T, bf16>::value) {
+    uint32_t w[U][MAXC][4];
+    softmax_load_bf16<G, MAXC, U>(row, len, sub, w);
+    for (;;) {
+      const long long nwg = wg + warps;
+      const bool more = Rb + nwg * kGpw * U < Re;            // uniform across the warp
+      int nlen[U];
+      T* nrow[U];
+      uint32_t nw[U][MAXC][4];
+      if (more) {
+        class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (nwg * kGpw + lane / G) * U,
+                            Re, nh, causal, nrow, nlen);
+        softmax_load_bf16<G, MAXC, U>(nrow, nlen, sub, nw);
+      }
+      softmax_compute_bf16<G, MAXC, U>(row, len, sub, w);
+      if (!more) break;
+      wg = nwg;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        row[u] = nrow[u];
+        len[u] = nlen[u];
+#pragma unroll
+        for (int c = 0; c < MAXC; ++c)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) w[u][c][j] = nw[u][c][j];
+      }
+    }
+  } else {
+    for (;;) {
+      softmax_group<T, G, MAXC, U>(row, len, sub);
+      wg += warps;
+      if (Rb + wg * kGpw * U >= Re) break;
+      class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re,
+                          nh, causal, row, len);
+    }
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256, 3)
+    softmax_class_kernel(T* __restrict__ S, const int32_t* __restrict__ offsets,
+                         const int64_t* __restrict__ s_off, const unsigned long long* __restrict__ ctr,
+                         const long long* __restrict__ seq_base, const int32_t* __restrict__ row_seq,
+                         int k_max, int nh, int causal) {
+  pdl_launch_dependents();
+  pdl_wait();
+  long long seg[kSmClasses + 1];
+  seg[0] = 0;
+#pragma unroll
+  for (int k = 0; k < kSmClasses; ++k) seg[k + 1] = seg[k] + static_cast<long long>(ctr[k]);
+  // lanes per row: the smallest power of two covering the class's chunks (at
+  // most 32), rows per lane group so that a lane has about four chunks in flight
+  softmax_class_pass<T, 1, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[0], seg[1], nh, causal);
+  if (k_max >= 1) softmax_class_pass<T, 2, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[1], seg[2], nh, causal);
+  if (k_max >= 2) softmax_class_pass<T, 4, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[2], seg[3], nh, causal);
+  if (k_max >= 3) softmax_class_pass<T, 8, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[3], seg[4], nh, causal);
+  if (k_max >= 4) softmax_class_pass<T, 16, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[4], seg[5], nh, causal);
+  if (k_max >= 5) softmax_class_pass<T, 32, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[5], seg[6], nh, causal);
+  if (k_max >= 6) softmax_class_pass<T, 32, 2, 2>(S, offsets, s_off, seq_base, row_seq, seg[6], seg[7], nh, causal);
+  if (k_max >= 7) softmax_class_pass<T, 32, 3, 1>(S, offsets, s_off, seq_base, row_seq, seg[7], seg[8], nh, causal);
+  if (k_max >= 8) softmax_class_pass<T, 32, 4, 1>(S, offsets, s_off, seq_base, row_seq, seg[8], seg[9], nh, causal);
 }
 
 template <int DP>
@@ -1081,6 +1378,42 @@ cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
     case 128: launch_k(attn_scores_kernel<128>, grid, 128, 0, st, q, s, offsets, rb_off, s_off, n_seqs, H, head_dim, scale, causal); break;
     default: return cudaErrorInvalidValue;
   }
+  return cudaGetLastError();
+}
+
+size_t softmax_classes_scratch_bytes(int n_seqs, int T, int n_heads) {
+  return SoftmaxIndexLayout(n_seqs, static_cast<long long>(n_heads) * T).bytes;
+}
+
+cudaError_t softmax_classes_launch(void* S, int s_dtype, const int32_t* offsets,
+                                   const int64_t* s_off, int n_seqs, int T, int n_heads,
+                                   int max_len, int causal, void* scratch, int num_sms,
+                                   cudaStream_t st) {
+  if (n_seqs == 0 || T == 0) return cudaSuccess;
+  if (max_len < 1 || max_len > 1024) return cudaErrorInvalidValue;
+  const SoftmaxIndexLayout lay(n_seqs, static_cast<long long>(n_heads) * T);
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  unsigned long long* ctr = reinterpret_cast<unsigned long long*>(base);
+  long long* seq_base = reinterpret_cast<long long*>(base + lay.base);
+  int32_t* row_seq = reinterpret_cast<int32_t*>(base + lay.rows);
+  cudaError_t e = cudaMemsetAsync(ctr, 0, 16 * kSmClasses, st);
+  if (e != cudaSuccess) return e;
+  const int seq_blocks = std::max(1, std::min((n_seqs + 255) / 256, num_sms * 4));
+  launch_k(softmax_count_kernel, dim3(seq_blocks), dim3(256), 0, st, offsets, n_seqs, n_heads, ctr);
+  const int idx_blocks = std::max(1, std::min((n_seqs + 7) / 8, num_sms * 8));
+  launch_k(softmax_index_kernel, dim3(idx_blocks), dim3(256), 0, st, offsets, n_seqs, n_heads, ctr,
+           seq_base, row_seq);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int k_max = softmax_class_of(max_len);
+  // three CTAs of 256 threads per SM (the kernel's register bound: it holds
+  // two iterations' rows), grid-striding over each class
+  if (s_dtype == 0)
+    launch_k(softmax_class_kernel<float>, dim3(num_sms * 3), dim3(256), 0, st, static_cast<float*>(S),
+             offsets, s_off, ctr, seq_base, row_seq, k_max, n_heads, causal);
+  else
+    launch_k(softmax_class_kernel<bf16>, dim3(num_sms * 3), dim3(256), 0, st, static_cast<bf16*>(S),
+             offsets, s_off, ctr, seq_base, row_seq, k_max, n_heads, causal);
   return cudaGetLastError();
 }
 

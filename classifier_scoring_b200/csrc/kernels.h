@@ -80,6 +80,16 @@ cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
 cudaError_t softmax_launch(void* S, int s_dtype, const int32_t* offsets, const int64_t* s_off,
                            int n_seqs, int T, int n_heads, int max_len, int causal, int* err,
                            cudaStream_t st);
+// The masked softmax by row-length class: the rows are regrouped on the device
+// by the class of their length into scratch (device,
+// softmax_classes_scratch_bytes(n_seqs, T, n_heads) bytes, 16-byte aligned),
+// then one persistent kernel takes each class up to that of max_len with lane
+// groups sized to it.
+size_t softmax_classes_scratch_bytes(int n_seqs, int T, int n_heads);
+cudaError_t softmax_classes_launch(void* S, int s_dtype, const int32_t* offsets,
+                                   const int64_t* s_off, int n_seqs, int T, int n_heads,
+                                   int max_len, int causal, void* scratch, int num_sms,
+                                   cudaStream_t st);
 // scores + masked softmax + context in one kernel (probabilities stay in registers)
 cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets,
                               const int32_t* rb_off, int n_seqs, int n_row_blocks, int n_heads,

@@ -103,6 +103,24 @@ int rm_op_softmax(void* S, int32_t s_dtype, const int32_t* offsets, const int64_
                   int32_t n_seqs, int32_t T, int32_t n_heads, int32_t max_len, int32_t causal,
                   void* stream);
 
+/* The same softmax by row-length class: the rows are first regrouped on the
+ * device by the 8-element chunks of their length (<= 1, 2, 4, 8, 16, 32, 64,
+ * 96, 128) into scratch, each row recording its sequence, and one persistent
+ * kernel then takes each class with lanes per row fitted to it (one lane for
+ * rows of up to 8 keys ... 32 lanes holding 4 chunks each for 1024), so that
+ * short rows leave no lanes idle when the batch also holds long ones and no
+ * lane group searches the offsets.  Same arguments as rm_op_softmax, plus
+ * scratch: device memory of rm_softmax_scratch_bytes(n_seqs, T, n_heads) bytes
+ * (about 4 bytes per row), 16-byte aligned, overwritten by the call.  The
+ * per-row arithmetic is rm_op_softmax's; only the order in which a row's
+ * exponentials are summed follows its lanes per row.  RM_E_INVAL for NULL
+ * pointers or bad sizes. */
+int rm_op_softmax_classes(void* S, int32_t s_dtype, const int32_t* offsets, const int64_t* s_off,
+                          int32_t n_seqs, int32_t T, int32_t n_heads, int32_t max_len,
+                          int32_t causal, void* scratch, void* stream);
+/* Host only: the scratch bytes rm_op_softmax_classes needs (0 for bad sizes). */
+size_t rm_softmax_scratch_bytes(int32_t n_seqs, int32_t T, int32_t n_heads);
+
 /* Context C = P V per sequence and head into ctx[T][H] (head j in columns
  * j*d..j*d+d-1).  S holds P (bf16), qkv: bf16 [T][3H], ctx: bf16 [T][H]. */
 int rm_op_attn_context(const void* S, const void* qkv, void* ctx, const int32_t* offsets,

@@ -222,6 +222,76 @@ def test_softmax(lens, causal, dtype):
             assert np.all(got[:, r, lim:end] == 0)
 
 
+@pytest.mark.parametrize("lens", [[1, 2, 3, 100, 57], [64, 128, 256], [513, 560, 7], [1024, 1000],
+                                  [5, 33, 65, 129, 257, 513, 769, 31, 8, 1]],
+                         ids=["short", "tinybert", "long", "max", "mixed"])
+@pytest.mark.parametrize("causal", [0, 1])
+@pytest.mark.parametrize("dtype", [rm.F32, rm.BF16], ids=["f32", "bf16"])
+def test_softmax_classes(lens, causal, dtype):
+    """Length-class softmax against the oracle, every row of every sequence,
+    the masked tail of each written chunk exactly 0, entries outside the rows
+    untouched; twice in a row on the same scratch (the index is rebuilt)."""
+    nh = 3
+    rng = np.random.default_rng(len(lens) + causal + 101)
+    lens = np.array(lens)
+    off, rb, so, S = varlen_rows(lens, nh, rng, dtype)
+    tdt = torch.float32 if dtype == rm.F32 else torch.bfloat16
+    T = int(off[-1])
+    d_off, d_so = dev(off, torch.int32), dev(so, torch.int64)
+    nbytes = rm.ops.softmax_scratch_bytes(len(lens), T, nh)
+    scratch = torch.full((nbytes,), 255, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        Sd = dev(S, tdt)
+        S_in = f64(Sd)
+        rm.ops.softmax_classes(Sd, dtype, d_off, d_so, len(lens), T, nh, int(lens.max()), causal,
+                               scratch)
+        torch.cuda.synchronize()
+        P = f64(Sd)
+        for i, L in enumerate(lens):
+            Lp = (L + 7) // 8 * 8
+            got = P[so[i]:so[i + 1]].reshape(nh, L, Lp)
+            s_in = S_in[so[i]:so[i + 1]].reshape(nh, L, Lp)[:, :, :L]
+            allowed = np.tril(np.ones((L, L), bool)) if causal else np.ones((L, L), bool)
+            ref = O.softmax_masked(s_in, np.broadcast_to(allowed, (nh, L, L)))
+            g = got[:, :, :L]
+            ok = np.broadcast_to(allowed, g.shape)
+            tol = F32_RTOL if dtype == rm.F32 else BF16_REL
+            assert np.all(np.abs(g[ok] - ref[ok]) <= tol * ref[ok] + 1e-37)
+            before = S_in[so[i]:so[i + 1]].reshape(nh, L, Lp)
+            for r in (0, L - 1):
+                lim = r + 1 if causal else L
+                end = min(Lp, (lim + 7) // 8 * 8)
+                assert np.all(got[:, r, lim:end] == 0)
+                # past the last written chunk the buffer is untouched
+                assert np.array_equal(got[:, r, end:], before[:, r, end:], equal_nan=True)
+
+
+def test_softmax_classes_many_sequences_against_the_oracle():
+    """Thousands of sequences of every class (the planning kernels loop), sampled
+    against the oracle, the longest included."""
+    nh = 2
+    rng = np.random.default_rng(5)
+    lens = rng.integers(1, 40, 3000)
+    lens[rng.integers(0, 3000, 40)] = rng.integers(40, 1025, 40)
+    off, rb, so, S = varlen_rows(lens, nh, rng, rm.F32)
+    T = int(off[-1])
+    Sd = dev(S, torch.float32)
+    S_in = f64(Sd)
+    scratch = torch.empty(rm.ops.softmax_scratch_bytes(len(lens), T, nh), dtype=torch.uint8,
+                          device="cuda")
+    rm.ops.softmax_classes(Sd, rm.F32, dev(off, torch.int32), dev(so, torch.int64), len(lens), T, nh,
+                           int(lens.max()), 0, scratch)
+    torch.cuda.synchronize()
+    P = f64(Sd)
+    for i in list(np.linspace(0, len(lens) - 1, 40).astype(int)) + list(np.argsort(lens)[-5:]):
+        L = int(lens[i])
+        Lp = (L + 7) // 8 * 8
+        got = P[so[i]:so[i + 1]].reshape(nh, L, Lp)[:, :, :L]
+        s_in = S_in[so[i]:so[i + 1]].reshape(nh, L, Lp)[:, :, :L]
+        ref = O.softmax_masked(s_in, np.ones((nh, L, L), bool))
+        assert np.all(np.abs(got - ref) <= F32_RTOL * ref + 1e-37)
+
+
 # --- attention scores and context -----------------------------------------------------
 
 def qkv_for(T, H, rng):
