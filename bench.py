@@ -900,8 +900,12 @@ def prefix_bench(args):
         shared()
         unshared()
     torch.cuda.synchronize()
-    if np.max(np.abs(out.cpu().numpy() - out_cat.cpu().numpy())) > 2e-3:
-        raise RuntimeError("shared-prefix and unshared scores disagree")
+    # the two paths run different attention kernels (bf16 P rounded against
+    # other running maxima), each meant to be within 2e-2 of the fp64 oracle:
+    # their difference is reported, and only one beyond twice that is an error
+    path_diff = float(np.max(np.abs(out.cpu().numpy() - out_cat.cpu().numpy())))
+    if path_diff > 4e-2:
+        raise RuntimeError(f"shared-prefix and unshared scores disagree by {path_diff}")
     l0 = sc.profile_read()["total_launches"]
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
@@ -952,7 +956,8 @@ def prefix_bench(args):
                    "parallelism": "replicas"},
         "unshared": {"value": whole_job_rate(world, n_c, args.steps, float(vals[1])),
                      "ms_per_step": float(vals[1]) / args.steps,
-                     "api": "rm_score on the prefix + candidate concatenations"},
+                     "api": "rm_score on the prefix + candidate concatenations",
+                     "max_abs_score_diff_vs_shared": path_diff},
         "roofline": {"kernel": "gemm_bf16_tc_kernel (QKV, output and FFN projections)",
                      "measured_on": "one profiled step after the timed region",
                      "bound": "tensor", "achieved": gemm_tflops, "peak": pk["bf16_tflops_sustained"],

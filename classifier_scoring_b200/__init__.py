@@ -21,6 +21,7 @@ __all__ = ["RmConfig", "RmError", "Scorer", "lib", "schedule", "weights_bytes", 
 ENC_POSTLN, DEC_PRELN = 0, 1
 F32, BF16 = 0, 1
 ROWS_RESID_F32 = 2          # res_ln rows: x fp32, y and z bf16
+ROWS_F32_IN = 3             # res_ln rows: y and x fp32, z bf16
 GELU_ERF, GELU_TANH = 0, 1
 ATTN_FUSED, ATTN_MATERIALIZED = 0, 1
 RM_OK, RM_E_INVAL, RM_E_NOMEM, RM_E_CUDA, RM_E_RANGE, RM_E_DEVICE = 0, -1, -2, -3, -4, -5

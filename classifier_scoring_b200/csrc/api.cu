@@ -391,9 +391,9 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
 }
 
 int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCount], int M, int N,
-         int K, const float* bias, void* y, int act, cudaStream_t st) {
+         int K, const float* bias, void* y, int act, cudaStream_t st, bool out_f32 = false) {
   const GemmTile tile = gemm_pick(M, N, K, h->num_sms, act);
-  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], tile, M, N, K, bias, y, false,
+  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], tile, M, N, K, bias, y, out_f32,
                               act, h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return RM_OK;
@@ -599,7 +599,10 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
   const double att = ci.att;
   const double Td = T, Hd = H, Fd = F;
   auto gemm_flops = [&](double N, double K) { return 2.0 * Td * N * K; };
-  auto gemm_bytes = [&](double N, double K) { return 2.0 * (Td * K + N * K + Td * N); };
+  auto gemm_bytes = [&](double N, double K, double out_bytes = 2.0) {
+    return 2.0 * (Td * K + N * K) + out_bytes * Td * N;
+  };
+  const double y_bytes = dec ? 4.0 : 2.0;   // the decoder's sublayer outputs are fp32
   const double att_flops = 2.0 * att * d;            // one of the two contractions
   const double sm_bytes = 4.0 * att;                 // bf16 read + write per admitted entry
   const double ctx_bytes = 2.0 * att + 2.0 * Td * Hd * 2;   // P, V, ctx
@@ -619,9 +622,10 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
   const unsigned long long w_qkv_b = 2ull * 3 * H * H, w_o_b = 2ull * H * H, w_1_b = 2ull * F * H,
                            w_2_b = 2ull * H * F;
   const L2Prefetch pf_qkv0 = pf_of(h->layers[0].w_qkv, w_qkv_b, nullptr, 0);
-  // the decoder's residual stream x is fp32 (row dtype 2 of the LayerNorm:
-  // y and z bf16, x fp32); the encoder's x is the bf16 LayerNorm output
-  const int ln_dtype = dec ? 2 : 1;
+  // the decoder keeps its residual stream x and the sublayer outputs y in
+  // fp32 (LayerNorm row dtype 3: y and x fp32, z bf16); the encoder's x is
+  // the bf16 LayerNorm output
+  const int ln_dtype = dec ? 3 : 1;
   RM_KERNEL(RM_K_EMBED, 0, (dec ? 8.0 : 6.0) * Td * Hd + 4.0 * Td,
             embed_launch(d_ids, d_off, n, T, h->emb_word, h->emb_pos, dec ? nullptr : h->ln_emb_g,
                          dec ? nullptr : h->ln_emb_b, eps, c->vocab, c->max_pos, H, x,
@@ -632,8 +636,8 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
               res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps,
                             ln_dtype, 2, st, pf_qkv0));
   // algorithmic bytes per token: post-LN reads y, x and writes x (bf16); the
-  // decoder reads y (bf16) and x (fp32), writes x (fp32) and z (bf16)
-  const double ln_bytes = (dec ? 12.0 : 6.0) * Td * Hd;
+  // decoder reads y and x (fp32), writes x (fp32) and z (bf16)
+  const double ln_bytes = (dec ? 14.0 : 6.0) * Td * Hd;
   for (int l = 0; l < c->n_layers; ++l) {
     const LayerW& L = h->layers[l];
     const L2Prefetch pf_o = pf_of(L.w_o, w_o_b, nullptr, 0);
@@ -662,8 +666,9 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
       RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
                 attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
     }
-    RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd),
-            gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st));
+    // the decoder's sublayer outputs stay fp32 up to the fp32 residual add
+    RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd, y_bytes),
+            gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st, dec));
     if (!dec) {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
                 res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, ln_dtype, 0, st, pf_ffn));
@@ -678,8 +683,8 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
                 res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 1, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
               gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
-      RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
-              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st));
+      RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd, y_bytes),
+              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st, true));
       const bool last = l + 1 == c->n_layers;
       const float* g = last ? h->lnf_g : h->layers[l + 1].ln1_g;
       const float* b = last ? h->lnf_b : h->layers[l + 1].ln1_b;
@@ -1258,7 +1263,8 @@ int rm_op_res_ln(const void* y, void* x, void* z, const float* g, const float* b
   if (mode < 0 || mode > 2 || (mode != 2 && y == nullptr) || (mode != 0 && z == nullptr))
     return set_error(RM_E_INVAL, "bad mode or missing y/z");
   if (T < 0 || H < 8 || H % 8 != 0 || H > 4096 ||
-      (dtype != RM_F32 && dtype != RM_BF16 && dtype != RM_ROWS_RESID_F32))
+      (dtype != RM_F32 && dtype != RM_BF16 && dtype != RM_ROWS_RESID_F32 &&
+       dtype != RM_ROWS_F32_IN))
     return set_error(RM_E_INVAL, "bad sizes");
   RM_LAUNCH(res_ln_launch(y, x, z, g, b, T, H, eps, dtype, mode, static_cast<cudaStream_t>(stream)));
   return RM_OK;

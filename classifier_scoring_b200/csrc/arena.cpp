@@ -25,16 +25,18 @@ bool overlap_steps(const ArenaPlan& p, int a, int b) {
 
 void sizes(int arch, int H, int F, int64_t T, int64_t s_elems, ArenaPlan& p) {
   const int64_t row = 2;   // bf16 bytes
-  // the decoder's residual stream is kept in fp32 (its rounding, repeated over
-  // every layer's two additions, dominated the score error in bf16)
+  // the decoder's residual stream is kept in fp32 (its rounding to bf16,
+  // repeated over every layer's two additions, dominated the score error)
   p.bytes[B_X] = align_up(T * H * (arch == RM_DEC_PRELN ? 4 : row), kArenaAlign);
   p.bytes[B_Z] = arch == RM_DEC_PRELN ? align_up(T * H * row, kArenaAlign) : 0;
   p.bytes[B_QKV] = align_up(T * 3 * H * row, kArenaAlign);
   p.bytes[B_S] = align_up(s_elems * row, kArenaAlign);
   p.bytes[B_CTX] = align_up(T * H * row, kArenaAlign);
-  p.bytes[B_Y1] = align_up(T * H * row, kArenaAlign);
+  // the decoder's sublayer outputs y stay fp32 up to the residual add
+  const int64_t yrow = arch == RM_DEC_PRELN ? 4 : row;
+  p.bytes[B_Y1] = align_up(T * H * yrow, kArenaAlign);
   p.bytes[B_F] = align_up(T * F * row, kArenaAlign);
-  p.bytes[B_Y2] = align_up(T * H * row, kArenaAlign);
+  p.bytes[B_Y2] = align_up(T * H * yrow, kArenaAlign);
   static const int32_t first[B_COUNT] = {0, 0, 1, 2, 4, 5, 7, 8};
   static const int32_t last[B_COUNT] = {9, 9, 4, 4, 5, 6, 8, 9};
   for (int k = 0; k < B_COUNT; ++k) {

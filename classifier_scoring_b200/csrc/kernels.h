@@ -50,8 +50,8 @@ cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
                          int32_t* err_count, cudaStream_t st, const L2Prefetch& pf = {},
                          const int32_t* pos_base = nullptr, int x_dtype = 1);
-// dtype: 0 fp32, 1 bf16, 2 residual x fp32 with y, z bf16; mode 0 post, 1 pre,
-// 2 plain (see rm_ops.h)
+// dtype: 0 fp32, 1 bf16, 2 residual x fp32 with y, z bf16, 3 y and x fp32 with
+// z bf16; mode 0 post, 1 pre, 2 plain (see rm_ops.h)
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
                           int H, float eps, int dtype, int mode, cudaStream_t st,
                           const L2Prefetch& pf = {});

@@ -410,6 +410,7 @@ cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const
   if (H % 8 != 0 || H > 4096) return cudaErrorInvalidValue;
   if (dtype == 0) return res_ln_dispatch<float, float, float>(y, x, z, g, b, T, H, eps, mode, st, pf);
   if (dtype == 2) return res_ln_dispatch<bf16, float, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
+  if (dtype == 3) return res_ln_dispatch<float, float, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
   return res_ln_dispatch<bf16, bf16, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
 }
 

@@ -182,10 +182,12 @@ int rm_op_attention_noalloc(const void* qkv, void* ctx, const int32_t* offsets, 
  *   mode 2 (plain):   z = LN(x)                  (y unused, may be NULL)
  * LN(u) = g * (u - mean)/sqrt(var + eps) + b with the biased variance.
  * y, x, z: [T][H]; g, b: fp32 [H].  Row types by dtype: RM_F32 or RM_BF16 for
- * all three; RM_ROWS_RESID_F32 for x in fp32 with y and z in bf16 (the pre-LN
- * decoder's residual stream, kept in fp32 so that its sum is rounded once per
- * addition to fp32 instead of to bf16). */
+ * all three; RM_ROWS_RESID_F32 for x in fp32 with y and z in bf16;
+ * RM_ROWS_F32_IN for y and x in fp32 with z in bf16 (the pre-LN decoder's
+ * layout: its residual stream and the sublayer outputs added to it stay fp32,
+ * so that each addition is rounded once to fp32 instead of to bf16). */
 #define RM_ROWS_RESID_F32 2
+#define RM_ROWS_F32_IN 3
 int rm_op_res_ln(const void* y, void* x, void* z, const float* g, const float* b, int32_t T,
                  int32_t H, float eps, int32_t dtype, int32_t mode, void* stream);
 

@@ -10,6 +10,11 @@ Only the seeded generators (synth) and the oracle are used.  Files:
                          64-sequence batch of the 1.3B-shape causal reward
                          model stream (24 layers, d 2048, 16 heads, FFN 8192,
                          bf16 weights, lengths U[256, 560], seed 4).
+  gpt_1p3b_best_of_8_scores.txt -- scores of all 64 candidates of the
+                         best-of-8 workload (8 posts of U[208, 512] tokens, 8
+                         summaries of U[24, 48] each, the 1.3B-shape weights
+                         of seed 4, requests of seed 5), each candidate scored
+                         as its own post + summary sequence.
   bert_base_len5_500_longest_batch_scores.txt -- request index and score of
                          every sequence of the last (longest) DP batch of the
                          10,000-request BERT-base stream with lengths
@@ -26,6 +31,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 
 import synth  # noqa: E402
+from oracle import best_of_n as OB  # noqa: E402
 from oracle import schedule as OS  # noqa: E402
 from oracle import scorer  # noqa: E402
 
@@ -72,6 +78,18 @@ def bert_base_len5_500_longest_batch():
     return idx, ids, off
 
 
+def gpt_best_of_8_scores():
+    w = synth.PREFIX_WORKLOADS["gpt-1.3b-best-of-8"]
+    ids, prefix_len, n_cand, cand_len = synth.make_prefix_groups(w)
+    m = _model("gpt-1.3b-rm")
+    out = []
+    for p, cands in OB.split_groups(ids, prefix_len, n_cand, cand_len):
+        for c in cands:
+            out.append(scorer.score_one(m, np.concatenate([p, c])))
+            print(f"best-of-8: {len(out)}/{int(n_cand.sum())}", flush=True)
+    return np.array(out)
+
+
 def write(name):
     path = os.path.join(HERE, name)
     if name == "tiny_enc_scores.txt":
@@ -83,6 +101,10 @@ def write(name):
         np.savetxt(path, s, fmt="%.17g",
                    header="fp64 oracle scores, gpt-1.3b-rm workload (seed 4), first 64 requests, "
                           "one per sequence")
+    elif name == "gpt_1p3b_best_of_8_scores.txt":
+        np.savetxt(path, gpt_best_of_8_scores(), fmt="%.17g",
+                   header="fp64 oracle scores, gpt-1.3b-best-of-8 (weights seed 4, requests seed 5), "
+                          "every candidate as its own prefix + candidate sequence, group-major")
     elif name == "bert_base_len5_500_longest_batch_scores.txt":
         idx, ids, off = bert_base_len5_500_longest_batch()
         s = _score_all(_model("bert-base-len5-500"), ids, off, name)
@@ -95,7 +117,7 @@ def write(name):
 
 
 ALL = ["tiny_enc_scores.txt", "gpt_1p3b_rm_batch_scores.txt",
-       "bert_base_len5_500_longest_batch_scores.txt"]
+       "bert_base_len5_500_longest_batch_scores.txt", "gpt_1p3b_best_of_8_scores.txt"]
 
 if __name__ == "__main__":
     for n in (sys.argv[1:] or ALL):

@@ -155,21 +155,24 @@ def test_res_ln_bf16(H):
 
 @pytest.mark.parametrize("H", [1024, 2048])
 @pytest.mark.parametrize("mode", [1, 2])
-def test_res_ln_fp32_residual_with_bf16_rows(H, mode):
-    """The decoder's rows: y and z bf16, the residual stream x fp32."""
+@pytest.mark.parametrize("ydt", ["bf16", "f32"])
+def test_res_ln_fp32_residual_with_bf16_rows(H, mode, ydt):
+    """The decoder's rows: z bf16, the residual stream x fp32, y bf16
+    (RM_ROWS_RESID_F32) or fp32 (RM_ROWS_F32_IN)."""
     T = 1001
     rng = np.random.default_rng(H + 7 * mode)
     y = rng.normal(0, 1, (T, H))
     x = rng.normal(0.3, 3, (T, H)).astype(np.float32)
     gm = (1 + rng.normal(0, 0.02, H)).astype(np.float32)
     bt = rng.normal(0, 0.02, H).astype(np.float32)
-    yd, xd = dev(y, torch.bfloat16), dev(x, torch.float32)
+    yd = dev(y, torch.bfloat16 if ydt == "bf16" else torch.float32)
+    xd = dev(x, torch.float32)
     zd = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
     u = x.astype(np.float64) + (f64(yd) if mode == 1 else 0)
     if mode == 1:
         u = u.astype(np.float32).astype(np.float64)       # the stored residual: one fp32 rounding
     rm.ops.res_ln(yd if mode == 1 else None, xd, zd, dev(gm, torch.float32), dev(bt, torch.float32),
-                  T, H, 1e-5, rm.ROWS_RESID_F32, mode)
+                  T, H, 1e-5, rm.ROWS_RESID_F32 if ydt == "bf16" else rm.ROWS_F32_IN, mode)
     torch.cuda.synchronize()
     ref = O.layer_norm(u, gm.astype(np.float64), bt.astype(np.float64), 1e-5)
     assert np.all(np.abs(f64(zd) - ref) <= BF16_REL * np.abs(ref) + F32_RTOL * (np.abs(ref) + np.abs(gm)))

@@ -79,12 +79,16 @@ def test_prefix_scores_match_oracle_and_unshared_path(scorer, flat, case):
     got, best, lo = run_prefix(scorer, ids, prefix_len, n_cand, cand_len)
     ref = B.score_candidates(oracle_model(DEC, flat), ids, prefix_len, n_cand, cand_len)
     assert np.max(np.abs(got - ref)) <= SCORE_ATOL
-    # the same concatenations through rm_score: same arithmetic, prefix recomputed per candidate
+    # the same concatenations through rm_score, the prefix recomputed per
+    # candidate: the same projections, but another attention kernel (packed-row
+    # tiles rather than the per-segment prefix kernel), whose online softmax
+    # rounds P to bf16 against running maxima over other key blocks; half the
+    # score tolerance bounds the difference
     cat_ids, cat_off = concatenations(ids, prefix_len, n_cand, cand_len)
     plain = torch.full((len(cat_off) - 1,), float("nan"), device="cuda")
     scorer.score(torch.from_numpy(cat_ids).cuda(), cat_off, plain)
     torch.cuda.synchronize()
-    assert np.max(np.abs(got - plain.cpu().numpy())) <= 2e-3
+    assert np.max(np.abs(got - plain.cpu().numpy())) <= SCORE_ATOL / 2
     # selection on the kernel's own fp32 scores: the oracle's rule, same decision
     b_ref, lo_ref = B.select(got, n_cand)
     assert best.tolist() == b_ref.tolist()
