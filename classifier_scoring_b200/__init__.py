@@ -27,7 +27,11 @@ ATTN_FUSED, ATTN_MATERIALIZED = 0, 1
 RM_OK, RM_E_INVAL, RM_E_NOMEM, RM_E_CUDA, RM_E_RANGE, RM_E_DEVICE = 0, -1, -2, -3, -4, -5
 SCHED_THROUGHPUT, SCHED_LATENCY = 0, 1
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmscore.so")
+# RMSCORE_LIB names another build of the library (the checked build,
+# librmscore_checked.so, for tests of its bounds checks)
+LIB_PATH = os.environ.get("RMSCORE_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                                                         "librmscore.so")
+CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmscore_checked.so")
 
 
 class RmError(RuntimeError):
@@ -94,6 +98,8 @@ def lib() -> ctypes.CDLL:
         "rm_arena_stats": (ctypes.c_int, [P, P]),
         "rm_selftest_bounded_wait": (ctypes.c_int, [I64, P, P]),
         "rm_debug_fail_alloc": (ctypes.c_int, [I32]),
+        "rm_build_checked": (ctypes.c_int, []),
+        "rm_bounds_errors": (ctypes.c_int, [P]),
         "rm_destroy": (None, [P]),
         "rm_profile": (ctypes.c_int, [P, I32]),
         "rm_profile_read": (ctypes.c_int, [P, P, P, P, P, P]),
@@ -407,6 +413,18 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+
+def build_checked() -> bool:
+    """True in the checked build (librmscore_checked.so)."""
+    return bool(lib().rm_build_checked())
+
+
+def bounds_errors() -> int:
+    """rm_bounds_errors: failed bounds tests since the last call (checked build)."""
+    out = np.zeros(1, dtype=np.int64)
+    _check(lib().rm_bounds_errors(out.ctypes.data))
+    return int(out[0])
 
 
 def debug_fail_alloc(k: int) -> None:

@@ -1003,6 +1003,18 @@ int rm_get_device_error(rm_handle* h, int32_t* out) {
   return RM_OK;
 }
 
+int rm_build_checked(void) { return RMK_CHECKED; }
+
+int rm_bounds_errors(int64_t* out) {
+  if (out == nullptr) return set_error(RM_E_INVAL, "NULL argument");
+  int32_t a = 0, b = 0;
+  RM_CUDA(cudaDeviceSynchronize());
+  RM_CUDA(bounds_errors_rowops(&a, true));
+  RM_CUDA(bounds_errors_attention(&b, true));
+  *out = static_cast<int64_t>(a) + b;
+  return RM_OK;
+}
+
 int rm_profile(rm_handle* h, int32_t every) {
   if (h == nullptr || every < 0) return set_error(RM_E_INVAL, "bad argument");
   for (auto& r : h->prof) {

@@ -24,6 +24,8 @@
 namespace rmk {
 namespace {
 
+RMK_BOUNDS_UNIT(attention)
+
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
   asm volatile(
@@ -62,6 +64,7 @@ __global__ void __launch_bounds__(128)
   pdl_launch_dependents();
   pdl_wait();
   const BlockSeq q = locate_block(offsets, rb_off, s_off, n, blockIdx.x);
+  if (!in_bounds(q.L >= 1 && q.row0 < q.L)) return;   // checked build: inconsistent row blocks
   const int hd = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const size_t H3 = 3 * static_cast<size_t>(H);
@@ -207,12 +210,13 @@ __global__ void __launch_bounds__(256)
       len[u] = 0;
       row[u] = S;
       if (R < rows) {
-        while (R >= seq_row1) {
+        while (R >= seq_row1 && in_bounds(i + 1 < n)) {
           ++i;
           seq_row0 = seq_row1;
           seq_row1 = static_cast<long long>(nh) * offsets[i + 1];
         }
         const int L = offsets[i + 1] - offsets[i];
+        if (!in_bounds(R < seq_row1 && L >= 1)) continue;   // rows past offsets[n]
         const long long rr = R - seq_row0;
         len[u] = causal ? static_cast<int>(rr % L) + 1 : L;
         row[u] = S + s_off[i] + rr * ((L + 7) & ~7);
@@ -403,8 +407,8 @@ __device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ 
                                               const int64_t* __restrict__ s_off,
                                               const long long* __restrict__ seq_base,
                                               const int32_t* __restrict__ row_seq, long long R0,
-                                              long long Re, int nh, int causal, T* (&row)[U],
-                                              int (&len)[U]) {
+                                              long long Re, int n, int nh, int causal,
+                                              T* (&row)[U], int (&len)[U]) {
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     len[u] = 0;
@@ -412,6 +416,7 @@ __device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ 
   }
   if (R0 >= Re) return;
   int i = row_seq[R0];
+  if (!in_bounds(i >= 0 && i < n)) return;
   long long b = seq_base[i];
   int L = offsets[i + 1] - offsets[i];
 #pragma unroll
@@ -420,10 +425,12 @@ __device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ 
     if (R < Re) {
       if (R - b >= static_cast<long long>(nh) * L) {         // the next sequence's stretch
         i = row_seq[R];
+        if (!in_bounds(i >= 0 && i < n)) return;
         b = seq_base[i];
         L = offsets[i + 1] - offsets[i];
       }
       const long long rr = R - b;                            // row inside the sequence's block
+      if (!in_bounds(L >= 1 && rr >= 0 && rr < static_cast<long long>(nh) * L)) return;
       len[u] = causal ? static_cast<int>(rr % L) + 1 : L;
       row[u] = S + s_off[i] + rr * ((L + 7) & ~7);
     }
@@ -440,7 +447,8 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
                                                    const int64_t* __restrict__ s_off,
                                                    const long long* __restrict__ seq_base,
                                                    const int32_t* __restrict__ row_seq,
-                                                   long long Rb, long long Re, int nh, int causal) {
+                                                   long long Rb, long long Re, int n, int nh,
+                                                   int causal) {
   if (Rb >= Re) return;
   const int lane = threadIdx.x & 31, sub = lane % G;
   constexpr int kGpw = 32 / G;
@@ -449,8 +457,8 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
   if (Rb + wg * kGpw * U >= Re) return;                      // uniform across the warp
   int len[U];
   T* row[U];
-  class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re, nh,
-                      causal, row, len);
+  class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re, n,
+                      nh, causal, row, len);
   if constexpr (std::is_same<T, bf16>::value) {
     uint32_t w[U][MAXC][4];
     softmax_load_bf16<G, MAXC, U>(row, len, sub, w);
@@ -462,7 +470,7 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
       uint32_t nw[U][MAXC][4];
       if (more) {
         class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (nwg * kGpw + lane / G) * U,
-                            Re, nh, causal, nrow, nlen);
+                            Re, n, nh, causal, nrow, nlen);
         softmax_load_bf16<G, MAXC, U>(nrow, nlen, sub, nw);
       }
       softmax_compute_bf16<G, MAXC, U>(row, len, sub, w);
@@ -484,7 +492,7 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
       wg += warps;
       if (Rb + wg * kGpw * U >= Re) break;
       class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re,
-                          nh, causal, row, len);
+                          n, nh, causal, row, len);
     }
   }
 }
@@ -494,7 +502,7 @@ __global__ void __launch_bounds__(256, 3)
     softmax_class_kernel(T* __restrict__ S, const int32_t* __restrict__ offsets,
                          const int64_t* __restrict__ s_off, const unsigned long long* __restrict__ ctr,
                          const long long* __restrict__ seq_base, const int32_t* __restrict__ row_seq,
-                         int k_max, int nh, int causal) {
+                         int k_max, int n, int nh, int causal) {
   pdl_launch_dependents();
   pdl_wait();
   long long seg[kSmClasses + 1];
@@ -503,15 +511,15 @@ __global__ void __launch_bounds__(256, 3)
   for (int k = 0; k < kSmClasses; ++k) seg[k + 1] = seg[k] + static_cast<long long>(ctr[k]);
   // lanes per row: the smallest power of two covering the class's chunks (at
   // most 32), rows per lane group so that a lane has about four chunks in flight
-  softmax_class_pass<T, 1, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[0], seg[1], nh, causal);
-  if (k_max >= 1) softmax_class_pass<T, 2, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[1], seg[2], nh, causal);
-  if (k_max >= 2) softmax_class_pass<T, 4, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[2], seg[3], nh, causal);
-  if (k_max >= 3) softmax_class_pass<T, 8, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[3], seg[4], nh, causal);
-  if (k_max >= 4) softmax_class_pass<T, 16, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[4], seg[5], nh, causal);
-  if (k_max >= 5) softmax_class_pass<T, 32, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[5], seg[6], nh, causal);
-  if (k_max >= 6) softmax_class_pass<T, 32, 2, 2>(S, offsets, s_off, seq_base, row_seq, seg[6], seg[7], nh, causal);
-  if (k_max >= 7) softmax_class_pass<T, 32, 3, 1>(S, offsets, s_off, seq_base, row_seq, seg[7], seg[8], nh, causal);
-  if (k_max >= 8) softmax_class_pass<T, 32, 4, 1>(S, offsets, s_off, seq_base, row_seq, seg[8], seg[9], nh, causal);
+  softmax_class_pass<T, 1, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[0], seg[1], n, nh, causal);
+  if (k_max >= 1) softmax_class_pass<T, 2, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[1], seg[2], n, nh, causal);
+  if (k_max >= 2) softmax_class_pass<T, 4, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[2], seg[3], n, nh, causal);
+  if (k_max >= 3) softmax_class_pass<T, 8, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[3], seg[4], n, nh, causal);
+  if (k_max >= 4) softmax_class_pass<T, 16, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[4], seg[5], n, nh, causal);
+  if (k_max >= 5) softmax_class_pass<T, 32, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[5], seg[6], n, nh, causal);
+  if (k_max >= 6) softmax_class_pass<T, 32, 2, 2>(S, offsets, s_off, seq_base, row_seq, seg[6], seg[7], n, nh, causal);
+  if (k_max >= 7) softmax_class_pass<T, 32, 3, 1>(S, offsets, s_off, seq_base, row_seq, seg[7], seg[8], n, nh, causal);
+  if (k_max >= 8) softmax_class_pass<T, 32, 4, 1>(S, offsets, s_off, seq_base, row_seq, seg[8], seg[9], n, nh, causal);
 }
 
 template <int DP>
@@ -524,6 +532,7 @@ __global__ void __launch_bounds__(128)
   pdl_launch_dependents();
   pdl_wait();
   const BlockSeq q = locate_block(offsets, rb_off, s_off, n, blockIdx.x);
+  if (!in_bounds(q.L >= 1 && q.row0 < q.L)) return;   // checked build: inconsistent row blocks
   const int hd = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const size_t H3 = 3 * static_cast<size_t>(H);
@@ -618,6 +627,7 @@ __global__ void __launch_bounds__(128)
   const int t0 = offsets[i];
   const int L = offsets[i + 1] - t0;
   const int row0 = (b - rb_off[i]) * 64;
+  if (!in_bounds(L >= 1 && row0 < L)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const size_t H3 = 3 * static_cast<size_t>(H);
   const bf16* qb = qkv + static_cast<size_t>(t0) * H3 + hd * d;
@@ -804,6 +814,7 @@ __global__ void __launch_bounds__(128, (DP <= 64 ? 4 : 1))
   const int ps = PFX ? pre_start[i] : 0;
   const int Lk = P0 + L;                               // keys of the segment
   const int row0 = (b - rb_off[i]) * 64;
+  if (!in_bounds(L >= 1 && row0 < L && P0 >= 0)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
   const size_t H3 = 3 * static_cast<size_t>(H);
   const bf16* qb = qkv + static_cast<size_t>(t0) * H3 + hd * d;
@@ -1061,6 +1072,11 @@ __global__ void __launch_bounds__(160)
   const int Klo = offsets[s_first];
   const int Khi = causal ? rlast + 1 : offsets[s_last + 1];
   const int nch = (Khi - Klo + 63) / 64;
+  // checked build: the tile's sequences must fit the offsets window, and its
+  // key range must hold its rows (the same test in every thread of the CTA)
+  if (!in_bounds(s_last - s_first + 2 <= SL::kMaxSeqs && Klo >= 0 && Klo <= r0 && Khi > rlast &&
+                 Khi <= T))
+    return;
 
   if (warp == 4) {
     // ---- TMA producer ----
@@ -1362,6 +1378,15 @@ cudaError_t softmax_dispatch(void* S, const int32_t* offsets, const int64_t* s_o
 
 }  // namespace
 
+cudaError_t bounds_errors_attention(int32_t* out, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_bounds_attention, sizeof(int32_t));
+  if (e == cudaSuccess && reset) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_bounds_attention, &zero, sizeof(int32_t));
+  }
+  return e;
+}
+
 cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
                                const int32_t* rb_off, const int64_t* s_off, int n_seqs,
                                int n_row_blocks, int n_heads, int head_dim, int causal,
@@ -1410,10 +1435,10 @@ cudaError_t softmax_classes_launch(void* S, int s_dtype, const int32_t* offsets,
   // two iterations' rows), grid-striding over each class
   if (s_dtype == 0)
     launch_k(softmax_class_kernel<float>, dim3(num_sms * 3), dim3(256), 0, st, static_cast<float*>(S),
-             offsets, s_off, ctr, seq_base, row_seq, k_max, n_heads, causal);
+             offsets, s_off, ctr, seq_base, row_seq, k_max, n_seqs, n_heads, causal);
   else
     launch_k(softmax_class_kernel<bf16>, dim3(num_sms * 3), dim3(256), 0, st, static_cast<bf16*>(S),
-             offsets, s_off, ctr, seq_base, row_seq, k_max, n_heads, causal);
+             offsets, s_off, ctr, seq_base, row_seq, k_max, n_seqs, n_heads, causal);
   return cudaGetLastError();
 }
 

@@ -208,6 +208,24 @@ __device__ __forceinline__ void l2_prefetch_share(const L2PrefetchArgs& pf) {
 // that gave up.
 enum { ERR_CLAMPED = 0, ERR_TIMEOUT = 1, ERR_WORDS = 2 };
 
+// The checked build (-DRM_CHECKED, librmscore_checked.so): kernels test the
+// indices they derive from offsets and other metadata before the accesses
+// those indices address; a failed test adds one to the translation unit's
+// bounds counter (rm_bounds_errors sums and clears them) and the access is
+// skipped.  No trap, no assert.  In the product build in_bounds() is
+// constant true and the tests compile away.
+#ifdef RM_CHECKED
+#define RMK_CHECKED 1
+#else
+#define RMK_CHECKED 0
+#endif
+#define RMK_BOUNDS_UNIT(unit)                                                      \
+  __device__ int32_t g_bounds_##unit = 0;                                          \
+  __device__ __forceinline__ bool in_bounds(bool ok) {                             \
+    if (RMK_CHECKED && !ok) atomicAdd(&g_bounds_##unit, 1);                        \
+    return !RMK_CHECKED || ok;                                                     \
+  }
+
 }  // namespace rmk
 
 namespace rmk {

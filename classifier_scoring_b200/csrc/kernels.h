@@ -71,6 +71,11 @@ cudaError_t cvt_to_bf16_launch(const void* src, int src_dtype, void* dst, size_t
 cudaError_t cvt_to_f32_launch(const void* src, int src_dtype, float* dst, size_t n,
                               cudaStream_t st);
 
+// Bounds counters of the checked build (RM_CHECKED), per translation unit:
+// read into *out, cleared when reset.  Always 0 in the product build.
+cudaError_t bounds_errors_rowops(int32_t* out, bool reset);
+cudaError_t bounds_errors_attention(int32_t* out, bool reset);
+
 // ---- attention (attention.cu) ----
 cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
                                const int32_t* rb_off, const int64_t* s_off, int n_seqs,

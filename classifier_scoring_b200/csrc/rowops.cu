@@ -16,6 +16,8 @@
 namespace rmk {
 namespace {
 
+RMK_BOUNDS_UNIT(rowops)
+
 constexpr int kWarps = 4;   // warps (rows) per CTA
 
 template <int MAXC>
@@ -66,7 +68,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                  int T, const bf16* __restrict__ ew, const bf16* __restrict__ ep,
                  const float* __restrict__ g, const float* __restrict__ b, float eps, int V, int H,
                  TX* __restrict__ x, int32_t* __restrict__ err, L2PrefetchArgs pf,
-                 const int32_t* __restrict__ pos_base) {
+                 const int32_t* __restrict__ pos_base, int P) {
   pdl_launch_dependents();
   l2_prefetch_share(pf);   // static weights: no need to wait for the previous kernel
   pdl_wait();
@@ -76,6 +78,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int i = upper_index(offsets, n_seqs, t);
   // a segment that continues a shared prefix starts at position pos_base[i]
   const int pos = t - offsets[i] + (pos_base != nullptr ? pos_base[i] : 0);
+  if (!in_bounds(pos >= 0 && pos < P)) return;   // checked build: offsets past the position table
   int id = ids[t];
   if (id < 0 || id >= V) {
     if (lane == 0 && err != nullptr) atomicAdd(err, 1);
@@ -231,6 +234,7 @@ __global__ void __launch_bounds__(kWarps * 32)
   // out_index maps segments to output slots; a negative slot is not scored
   const int slot = out_index != nullptr ? out_index[i] : i;
   if (slot < 0) return;
+  if (!in_bounds(offsets[i] >= 0 && offsets[i + 1] > offsets[i])) return;
   const int t = last ? offsets[i + 1] - 1 : offsets[i];
   const bf16* xr = x + static_cast<size_t>(t) * H;
   float acc = 0.f;
@@ -279,6 +283,7 @@ __global__ void __launch_bounds__(128)
   const int g = blockIdx.x * blockDim.x + threadIdx.x;
   if (g >= n_groups) return;
   const int a = group_off[g], e = group_off[g + 1];
+  if (!in_bounds(a >= 0 && e > a)) return;
   int arg = 0;
   float top = scores[a];
   for (int k = a + 1; k < e; ++k) {
@@ -324,18 +329,18 @@ int pick_maxc(int H) {
 
 template <int MAXC, typename TX>
 cudaError_t embed_t(const int32_t* ids, const int32_t* offsets, int n, int T, const void* ew,
-                    const void* ep, const float* g, const float* b, float eps, int V, int H,
+                    const void* ep, const float* g, const float* b, float eps, int V, int P, int H,
                     void* x, int32_t* err, cudaStream_t st, const L2Prefetch& pf,
                     const int32_t* pos_base) {
   dim3 grid((T + kWarps - 1) / kWarps);
   if (g != nullptr)
     launch_k(embed_kernel<MAXC, true, TX>, grid, kWarps * 32, 0, st,
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<TX*>(x), err, pf_args(pf), pos_base);
+        V, H, static_cast<TX*>(x), err, pf_args(pf), pos_base, P);
   else
     launch_k(embed_kernel<MAXC, false, TX>, grid, kWarps * 32, 0, st,
         ids, offsets, n, T, static_cast<const bf16*>(ew), static_cast<const bf16*>(ep), g, b, eps,
-        V, H, static_cast<TX*>(x), err, pf_args(pf), pos_base);
+        V, H, static_cast<TX*>(x), err, pf_args(pf), pos_base, P);
   return cudaGetLastError();
 }
 
@@ -393,14 +398,13 @@ cudaError_t embed_launch(const int32_t* ids, const int32_t* offsets, int n_seqs,
                          const float* ln_b, float eps, int V, int P, int H, void* x,
                          int32_t* err_count, cudaStream_t st, const L2Prefetch& pf,
                          const int32_t* pos_base, int x_dtype) {
-  (void)P;
   if (T == 0) return cudaSuccess;
   const int maxc = pick_maxc(H);
   if (x_dtype == 0)
     RMK_MAXC_SWITCH(maxc, (embed_t<M_, float>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g,
-                                              ln_b, eps, V, H, x, err_count, st, pf, pos_base)))
+                                              ln_b, eps, V, P, H, x, err_count, st, pf, pos_base)))
   RMK_MAXC_SWITCH(maxc, (embed_t<M_, bf16>(ids, offsets, n_seqs, T, emb_word, emb_pos, ln_g, ln_b,
-                                           eps, V, H, x, err_count, st, pf, pos_base)))
+                                           eps, V, P, H, x, err_count, st, pf, pos_base)))
 }
 
 cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const float* b, int T,
@@ -412,6 +416,15 @@ cudaError_t res_ln_launch(const void* y, void* x, void* z, const float* g, const
   if (dtype == 2) return res_ln_dispatch<bf16, float, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
   if (dtype == 3) return res_ln_dispatch<float, float, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
   return res_ln_dispatch<bf16, bf16, bf16>(y, x, z, g, b, T, H, eps, mode, st, pf);
+}
+
+cudaError_t bounds_errors_rowops(int32_t* out, bool reset) {
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_bounds_rowops, sizeof(int32_t));
+  if (e == cudaSuccess && reset) {
+    const int32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_bounds_rowops, &zero, sizeof(int32_t));
+  }
+  return e;
 }
 
 cudaError_t head_launch(const void* x, const int32_t* offsets, int n_seqs, const float* w_r,

@@ -238,6 +238,20 @@ int rm_selftest_bounded_wait(int64_t limit_ns, int32_t* out_timed_out, int64_t* 
  * thread-safe.  RM_E_INVAL for k < 0. */
 int rm_debug_fail_alloc(int32_t k);
 
+/* The checked build (the pages have no counterpart): librmscore_checked.so is
+ * the same library compiled with RM_CHECKED, in which the kernels test the
+ * indices they derive from offsets and other per-call metadata (positions in
+ * the position table, sequence and row-block indices, a tile's offsets
+ * window, the softmax's row index) before the accesses those indices address,
+ * and skip the access and count it when a test fails (no trap, no assert).
+ * rm_build_checked() returns 1 in that library and 0 in the product one.
+ * rm_bounds_errors: waits for the device, writes the number of failed tests
+ * since the last call (all handles and rm_op_* calls of this process on the
+ * current device) and clears it; always 0 in the product library.  RM_E_INVAL
+ * for NULL out, RM_E_CUDA on a CUDA error. */
+int rm_build_checked(void);
+int rm_bounds_errors(int64_t* out);
+
 /* Arena figures: out[0] = bytes reserved at create, out[1] = largest plan used
  * by any call so far, out[2] = number of distinct length buckets planned.
  * out: host int64[3]. */
