@@ -119,3 +119,43 @@ def test_invalid_prefix_calls(scorer, flat):
     with rm.Scorer(config_for(enc), synth.make_weights(enc, 0)) as e:
         with pytest.raises(rm.RmError):                   # the encoder's prefix sees the candidate
             e.score_prefix(ids_d, [3], [1], [2], out)
+
+
+@pytest.mark.slow
+def test_gpt_1p3b_best_of_8_every_candidate_against_the_stored_oracle():
+    """The best-of-8 workload at the 1.3B shape (8 posts of 208..512 tokens, 8
+    summaries of 24..48 each): every candidate's score, shared prefix and
+    unshared concatenation alike, within the score tolerance of the fp64
+    oracle's stored scores (tests/golden/make_golden.py; one candidate is
+    re-scored here to tie the file to the oracle); each group's choice is the
+    first maximum of the kernel's own scores."""
+    import os
+    from oracle import scorer as O
+    w = synth.PREFIX_WORKLOADS["gpt-1.3b-best-of-8"]
+    s = w.shape
+    ids, prefix_len, n_cand, cand_len = synth.make_prefix_groups(w)
+    gold = np.loadtxt(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                                   "gpt_1p3b_best_of_8_scores.txt"))
+    nc, ng = int(n_cand.sum()), len(n_cand)
+    assert gold.shape == (nc,)
+    cat_ids, cat_off = concatenations(ids, prefix_len, n_cand, cand_len)
+    big = synth.make_weights(s, w.weight_seed)
+    cfg = config_for(s, max_batch_seqs=ng + nc, max_tokens=int(cat_off[-1]),
+                     max_len=int(np.diff(cat_off).max()))
+    with rm.Scorer(cfg, big) as sc:
+        got, best, lo = run_prefix(sc, ids, prefix_len, n_cand, cand_len)
+        plain = torch.full((nc,), float("nan"), device="cuda")
+        sc.score(torch.from_numpy(cat_ids).cuda(), cat_off, plain)
+        torch.cuda.synchronize()
+        plain = plain.cpu().numpy().astype(np.float64)
+    e_shared, e_plain = np.abs(got - gold), np.abs(plain - gold)
+    print(f"\ngpt-1.3b-best-of-8: max |gpu - oracle| shared {e_shared.max():.3e}, "
+          f"unshared {e_plain.max():.3e} over {nc} candidates")
+    assert e_shared.max() <= SCORE_ATOL and e_plain.max() <= SCORE_ATOL
+    b_ref, lo_ref = B.select(got, n_cand)
+    assert best.tolist() == b_ref.tolist()
+    assert np.allclose(lo, lo_ref, rtol=1e-6, atol=1e-6)
+    m = oracle_model(s, big)
+    del big
+    k = int(np.argmin(np.diff(cat_off)))
+    assert abs(O.score_one(m, cat_ids[cat_off[k]:cat_off[k + 1]]) - gold[k]) <= 1e-9
