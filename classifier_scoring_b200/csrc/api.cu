@@ -175,7 +175,8 @@ struct LayerW {
 
 struct Bucket {
   ArenaPlan plan;
-  CUtensorMap a_in, a_ctx, a_f;   // A operands: x (encoder) or z (decoder), ctx, f
+  CUtensorMap a_in, a_ctx, a_f;      // A operands: x (encoder) or z (decoder), ctx, f
+  CUtensorMap y_qkv, y_o, y_f, y_2;  // outputs: qkv, y1, f, y2 (the bucket's rows)
 };
 
 constexpr int kSlots = 4;
@@ -384,6 +385,15 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
       !make_tmap_bf16(&b.a_ctx, base + b.plan.off[B_CTX], Tb, c->hidden, 128, &why) ||
       !make_tmap_bf16(&b.a_f, base + b.plan.off[B_F], Tb, c->ffn, 128, &why))
     return set_error(RM_E_CUDA, "activation tensor map: %s", why);
+  // output maps cover the bucket's Tb rows (the buffers' extent): the rows of
+  // a call's last 128-row tile past its T tokens land in their own buffer's
+  // padding rows, which no later step reads
+  const bool dec = c->arch == RM_DEC_PRELN;
+  if (!make_tmap_store(&b.y_qkv, base + b.plan.off[B_QKV], Tb, 3 * c->hidden, false, &why) ||
+      !make_tmap_store(&b.y_o, base + b.plan.off[B_Y1], Tb, c->hidden, dec, &why) ||
+      !make_tmap_store(&b.y_f, base + b.plan.off[B_F], Tb, c->ffn, false, &why) ||
+      !make_tmap_store(&b.y_2, base + b.plan.off[B_Y2], Tb, c->hidden, dec, &why))
+    return set_error(RM_E_CUDA, "output tensor map: %s", why);
   h->max_peak = std::max(h->max_peak, b.plan.peak);
   auto res = h->buckets.emplace(key, b);
   *out = &res.first->second;
@@ -391,9 +401,10 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
 }
 
 int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCount], int M, int N,
-         int K, const float* bias, void* y, int act, cudaStream_t st, bool out_f32 = false) {
+         int K, const float* bias, const CUtensorMap& y, int act, cudaStream_t st,
+         bool out_f32 = false) {
   const GemmTile tile = gemm_pick(M, N, K, h->num_sms, act);
-  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], tile, M, N, K, bias, y, out_f32,
+  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], y, tile, M, N, K, bias, out_f32,
                               act, h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return RM_OK;
@@ -645,7 +656,7 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
     const L2Prefetch pf_next =
         l + 1 < c->n_layers ? pf_of(h->layers[l + 1].w_qkv, w_qkv_b, nullptr, 0) : L2Prefetch{};
     RM_GEMM(gemm_flops(3 * Hd, Hd), gemm_bytes(3 * Hd, Hd),
-            gemm(h, bk->a_in, L.tm[0], T, 3 * H, H, L.b_qkv, qkv, 0, st));
+            gemm(h, bk->a_in, L.tm[0], T, 3 * H, H, L.b_qkv, bk->y_qkv, 0, st));
     if (px != nullptr) {
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
                 attn_fused_prefix_launch(qkv, ctx, d_off, d_rb, d_pst, d_pln, n, nrb, nh, d, st, pf_o));
@@ -668,23 +679,23 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
     }
     // the decoder's sublayer outputs stay fp32 up to the fp32 residual add
     RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd, y_bytes),
-            gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, y1, 0, st, dec));
+            gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, bk->y_o, 0, st, dec));
     if (!dec) {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
                 res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, ln_dtype, 0, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
-              gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
+              gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, bk->y_f, act, st));
       RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd),
-              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st));
+              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, bk->y_2, 0, st));
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
                 res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 0, st, pf_next));
     } else {
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
                 res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 1, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
-              gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, f, act, st));
+              gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, bk->y_f, act, st));
       RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd, y_bytes),
-              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, y2, 0, st, true));
+              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, bk->y_2, 0, st, true));
       const bool last = l + 1 == c->n_layers;
       const float* g = last ? h->lnf_g : h->layers[l + 1].ln1_g;
       const float* b = last ? h->lnf_b : h->layers[l + 1].ln1_b;
@@ -1137,13 +1148,14 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
   RM_CUDA(cudaGetDevice(&dev));
   RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const GemmTile tile = cg != 0 ? GemmTile{cg, bn} : gemm_pick(M, N, K, sms, act);
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   const char* why = "";
-  if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, tile.b_box(), &why))
+  if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, tile.b_box(), &why) ||
+      !make_tmap_store(&ty, y, M, N, y_dtype == RM_F32, &why))
     return set_error(RM_E_INVAL, "tensor map: %s", why);
   int32_t* err = nullptr;
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
-  RM_LAUNCH(gemm_launch(ta, tb, tile, M, N, K, bias, y, y_dtype == RM_F32, act, err, sms,
+  RM_LAUNCH(gemm_launch(ta, tb, ty, tile, M, N, K, bias, y_dtype == RM_F32, act, err, sms,
                         static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }

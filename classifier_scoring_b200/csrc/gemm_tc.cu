@@ -21,10 +21,11 @@
 //                      and marks the accumulator full;
 //   warps 2..        : epilogue (four warps, or sixteen when the epilogue applies
 //                      GELU) -- tcgen05.ld (warp w reads TMEM lanes
-//                      32*(w%4)..+31 = tile rows), + bias, optional GELU,
-//                      staged through shared memory into whole row segments of
-//                      bf16 or fp32, then release the accumulator.  The
-//                      epilogue of tile i overlaps the mainloop of tile i+1.
+//                      32*(w%4)..+31 = tile rows), + bias, optional GELU, into
+//                      swizzled 32 x 32 boxes in shared memory that one lane
+//                      writes out with bulk tensor stores (TMA), then release
+//                      the accumulator.  The epilogue of tile i overlaps the
+//                      mainloop of tile i+1.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that
 // gives up counts into err[ERR_TIMEOUT] and the role leaves its loop; the CTA
 // then waits (bounded) for its own copies, frees its TMEM and returns.
@@ -40,11 +41,13 @@ namespace {
 constexpr int BM = 128;
 constexpr int BK = 64;                      // 64 bf16 = one 128-byte swizzle row
 
-// Epilogue warps: four (one per TMEM lane quarter) for a plain epilogue;
-// sixteen (four per quarter, taking the column rounds in turn) when the
-// epilogue applies GELU, whose arithmetic otherwise outlasts a short mainloop
-// (B200, FFN1 of 27.8k tokens: 128.9 us with eight, 122.9 us with sixteen).
-constexpr int epi_warps(int act) { return act != 0 ? 16 : 4; }
+// Epilogue warps: eight (two per TMEM lane quarter, taking the column rounds
+// in turn) for a plain epilogue, sixteen when it applies GELU, whose
+// arithmetic otherwise outlasts a short mainloop (B200, 27.8k tokens: the
+// QKV projection in a power-capped loop 97.9 us with eight against 104.3 us
+// with four; FFN1 with L2 flushed 122.9 us with sixteen against 128.9 us with
+// eight).
+constexpr int epi_warps(int act) { return act != 0 ? 16 : 8; }
 constexpr int gemm_threads(int act) { return 64 + 32 * epi_warps(act); }
 // Time per column of a CTA-pair tile relative to a single-CTA tile, and the
 // smallest products for which pairs are considered (measured on B200 with
@@ -129,15 +132,6 @@ __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32]
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
-__device__ __forceinline__ void tmem_ld_16cols(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
-      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -147,50 +141,44 @@ constexpr uint32_t tmem_cols_for(int bn) {
   return 2 * bn <= 32 ? 32 : (2 * bn <= 64 ? 64 : (2 * bn <= 128 ? 128 : (2 * bn <= 256 ? 256 : 512)));
 }
 
-template <int BN, int CG, int EW>
+template <int BN, int CG, int EW, int ESZ>
 struct GemmSmem {
   static constexpr int kA = BM * BK * 2;
   static constexpr int kB = (BN / CG) * BK * 2;   // this CTA's share of the B tile
   static constexpr int kStage = kA + kB;          // multiple of 1024 for BN/CG % 8 == 0
-  // epilogue staging: per epilogue warp 32 rows x one round of output (128 B
-  // with four epilogue warps, 64 B with more), row pitch padded by 16 B so
-  // that both the row-wise writes and the segment-wise reads spread over the
-  // bank groups
-  static constexpr int kRoundBytes = EW == 4 ? 128 : 64;
-  static constexpr int kStagePitch = kRoundBytes + 16;
-  static constexpr int kStageWarpBytes = 32 * kStagePitch;
-  // bias of the tile per epilogue warp (no cross-warp barrier): two buffers
-  // (one per accumulator) with four warps, one with more
-  static constexpr int kBiasFloatsPerWarp = EW == 4 ? 2 * BN : BN;
-  static constexpr int kBiasBytes = EW * kBiasFloatsPerWarp * 4;
-  // as many 64-deep K stages as fit beside the rest (227 KB per CTA), at most 8
-  static constexpr int kFixed = EW * kStageWarpBytes + kBiasBytes + 20 * 8 + 16 + 1024;
-  static constexpr int kStagesFit = (232448 - kFixed) / kStage;
-  static constexpr int kStages = kStagesFit < 8 ? kStagesFit : 8;
-  static constexpr int kEpiOff = kStages * kStage;
-  static constexpr int kBiasOff = kEpiOff + EW * kStageWarpBytes;
-  static constexpr int kBarOff = kBiasOff + kBiasBytes;   // full[S], empty[S], accf[2], acce[2]
+  // epilogue: per warp, kEpiBufs staging boxes of 32 rows x 32 output columns
+  // (64-byte rows of bf16 or 128-byte rows of fp32) in the swizzled layout of
+  // the output tensor map, written out by bulk tensor stores
+  static constexpr int kRowBytes = 32 * ESZ;
+  static constexpr int kBoxBytes = 32 * kRowBytes;
+  // barriers (full[S], empty[S], accf[2], acce[2], S <= 8), TMEM slot, and
+  // the slack that aligns the dynamic shared memory to 1024 bytes
+  static constexpr int kTail = (2 * 8 + 4) * 8 + 16 + 1024;
+  // as many 64-deep K stages as fit beside the rest (227 KB per CTA), at most
+  // 8; two staging boxes per warp unless that costs a stage
+  static constexpr int stages_with(int bufs) {
+    return (232448 - EW * bufs * kBoxBytes - kTail) / kStage < 8
+               ? (232448 - EW * bufs * kBoxBytes - kTail) / kStage
+               : 8;
+  }
+  static constexpr int kEpiBufs = stages_with(2) >= stages_with(1) ? 2 : 1;
+  static constexpr int kStages = stages_with(kEpiBufs);
+  static constexpr int kEpiOff = kStages * kStage;   // 1024-byte aligned: the boxes are too
+  static constexpr int kBarOff = kEpiOff + EW * kEpiBufs * kBoxBytes;
   static constexpr int kSlotOff = kBarOff + (2 * kStages + 4) * 8;
   static constexpr int kBytes = kSlotOff + 16 + 1024;   // + alignment slack
   static_assert(kStages >= 3, "at least three stages");
   static_assert(kBytes <= 232448, "fits one CTA's shared memory");
 };
 
-template <int ACT>
-__device__ __forceinline__ float epilogue_act(float t) {
-  if (ACT == 1) return gelu_erf_fast(t);
-  if (ACT == 2) return gelu_tanh(t);
-  return t;
-}
-
 template <int BN, int CG, int ACT, bool OUT_F32>
 __global__ void __launch_bounds__(gemm_threads(ACT), 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, int M, int N, int K,
-                        const float* __restrict__ bias, void* __restrict__ y,
-                        int* __restrict__ err, int n_fastest) {
+                        const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmY, int M, int N, int K,
+                        const float* __restrict__ bias, int* __restrict__ err, int n_fastest) {
   constexpr int EW = epi_warps(ACT);
-  using L = GemmSmem<BN, CG, EW>;
+  using L = GemmSmem<BN, CG, EW, OUT_F32 ? 4 : 2>;
   constexpr int S = L::kStages;
   constexpr uint32_t kTmemCols = tmem_cols_for(BN);
   static_assert(L::kStage % 1024 == 0, "stage size keeps the 1024-byte swizzle alignment");
@@ -347,35 +335,24 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
       }
     }
   } else {
-    // ---- epilogue: TMEM -> registers -> bias/GELU -> smem staging -> global ----
-    // Each thread owns one tile row (its TMEM lane).  A round takes
-    // kRoundBytes of that row, writes it to the warp's staging rows, then the
-    // warp stores whole row segments.  With more than four warps the warps of
-    // a lane quarter take the rounds in turn.
-    constexpr int ESZ = OUT_F32 ? 4 : 2;
-    constexpr int RB = L::kRoundBytes;
-    constexpr int CPR = RB / ESZ;                // columns per round
+    // ---- epilogue: TMEM -> registers -> bias/GELU -> swizzled smem box -> TMA store ----
+    // Each thread owns one tile row (its TMEM lane).  A round takes 32
+    // columns of that row, adds the bias (and GELU), writes the warp's 32 x 32
+    // box into one of its staging buffers and lane 0 stores the box with one
+    // bulk tensor copy; rows and columns outside Y are clipped by the copy.
+    // With more than four warps the warps of a lane quarter take the rounds
+    // in turn.
+    constexpr int NB = L::kEpiBufs;
     constexpr int NH = EW / 4;                   // warps per TMEM lane quarter
     const int ew = warp - 2;
     const int q = warp & 3;                      // TMEM lane quarter of this warp
     const int h0 = ew >> 2;                      // this warp's first round
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    uint8_t* stg = smem + L::kEpiOff + ew * L::kStageWarpBytes;
-    float* sbias_warp = reinterpret_cast<float*>(smem + L::kBiasOff) + ew * L::kBiasFloatsPerWarp;
+    uint8_t* stg0 = smem + L::kEpiOff + ew * NB * L::kBoxBytes;
+    int nst = 0;                                 // boxes this warp has stored
     int local = 0;
     for (int t = unit; t < tiles; t += units, ++local) {
       const int acc = local & 1, use = local >> 1;
-      // stage this tile's bias while the mainloop still runs (with two
-      // buffers, the one for this accumulator was last read two tiles ago;
-      // with one, this warp's reads of the previous tile ended before its
-      // arrival below)
-      float* sbias = sbias_warp + (EW == 4 ? acc * BN : 0);
-      {
-        const int nb0 = n_blk(t) * BN;
-        for (int j = lane; j < BN; j += 32)
-          sbias[j] = (bias != nullptr && nb0 + j < N) ? __ldg(bias + nb0 + j) : 0.0f;
-        __syncwarp();
-      }
       const bool ready = mbar_wait(accf0 + 8 * acc, use & 1);
       if (!__all_sync(0xffffffffu, ready)) {
         if (lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
@@ -386,82 +363,77 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
       const int n0 = n_blk(t) * BN;
       const int row0 = m0 + q * 32;
       const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
-#pragma unroll 1
-      for (int c = h0 * CPR; c < BN; c += NH * CPR) {
-        if (n0 + c >= N) break;                  // uniform across the warp
-        float v[CPR];
-        if (CPR >= 32) {
-          uint32_t r[32];
+      if (row0 < M) {                            // uniform across the warp
+        // TMEM loads run one round ahead: round c+1's columns are in flight
+        // while round c's values go through the bias, GELU and the store
+        int c = h0 * 32;
+        bool have = c < BN && n0 + c < N;        // uniform across the warp
+        uint32_t r[32];
+        if (have) tmem_ld_32cols(base + c, r);
+        while (have) {
+          // the bias of these columns: the same address in every lane (L1)
+          float4 b4[8];
 #pragma unroll
-          for (int h = 0; h < CPR / 32; ++h) {
-            tmem_ld_32cols(base + c + 32 * h, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[32 * h + j] = __uint_as_float(r[j]);
-          }
-        } else {
-          uint32_t r[16];
-          tmem_ld_16cols(base + c, r);
+          for (int g = 0; g < 8; ++g)
+            b4[g] = (bias != nullptr && n0 + c + 4 * g < N)
+                        ? __ldg(reinterpret_cast<const float4*>(bias + n0 + c + 4 * g))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
           tmem_wait_ld();
+          uint64_t p2[16];                       // bias added, two columns per register
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
-        }
-#pragma unroll
-        for (int g = 0; g < CPR / 4; ++g) {
-          // c + 4g < BN except in a partial last round, whose columns are not stored
-          const float4 b4 = (c + 4 * g < BN) ? *reinterpret_cast<const float4*>(sbias + c + 4 * g)
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-          if (ACT == 1) {
-            // bias and GELU two columns per packed instruction
-            uint64_t lo = f32x2_add(f32x2_pack(v[4 * g + 0], v[4 * g + 1]), f32x2_pack(b4.x, b4.y));
-            uint64_t hi = f32x2_add(f32x2_pack(v[4 * g + 2], v[4 * g + 3]), f32x2_pack(b4.z, b4.w));
-            lo = gelu_erf_fast_x2(lo);
-            hi = gelu_erf_fast_x2(hi);
-            f32x2_unpack(lo, v[4 * g + 0], v[4 * g + 1]);
-            f32x2_unpack(hi, v[4 * g + 2], v[4 * g + 3]);
-          } else {
-            v[4 * g + 0] = epilogue_act<ACT>(v[4 * g + 0] + b4.x);
-            v[4 * g + 1] = epilogue_act<ACT>(v[4 * g + 1] + b4.y);
-            v[4 * g + 2] = epilogue_act<ACT>(v[4 * g + 2] + b4.z);
-            v[4 * g + 3] = epilogue_act<ACT>(v[4 * g + 3] + b4.w);
+          for (int g = 0; g < 8; ++g) {
+            p2[2 * g] = f32x2_add(f32x2_pack(__uint_as_float(r[4 * g]), __uint_as_float(r[4 * g + 1])),
+                                  f32x2_pack(b4[g].x, b4[g].y));
+            p2[2 * g + 1] = f32x2_add(
+                f32x2_pack(__uint_as_float(r[4 * g + 2]), __uint_as_float(r[4 * g + 3])),
+                f32x2_pack(b4[g].z, b4[g].w));
           }
-        }
-        __syncwarp();                            // the previous round's reads are done
-        uint8_t* my_row = stg + lane * L::kStagePitch;
+          const int cn = c + NH * 32;
+          const bool next = cn < BN && n0 + cn < N;
+          if (next) tmem_ld_32cols(base + cn, r);
+          float v[32];
 #pragma unroll
-        for (int j = 0; j < RB / 16; ++j) {
-          uint4 u;
+          for (int k = 0; k < 16; ++k) {
+            if (ACT == 1) p2[k] = gelu_erf_fast_x2(p2[k]);
+            f32x2_unpack(p2[k], v[2 * k], v[2 * k + 1]);
+            if (ACT == 2) {
+              v[2 * k] = gelu_tanh(v[2 * k]);
+              v[2 * k + 1] = gelu_tanh(v[2 * k + 1]);
+            }
+          }
+          // this buffer's previous box has been read out by its store
+          const int buf = NB == 1 ? 0 : (nst & 1);
+          if (nst >= NB) {
+            if (lane == 0) bulk_wait_group_read<NB - 1>();
+            __syncwarp();
+          }
+          uint8_t* box = stg0 + buf * L::kBoxBytes;
           if (OUT_F32) {
-            u = make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
-                           __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-          } else {
-            u = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                           pack_bf16x2(v[8 * j + 4], v[8 * j + 5]), pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-          }
-          *reinterpret_cast<uint4*>(my_row + 16 * j) = u;
-        }
-        __syncwarp();
-        // RB/16 16-byte chunks per row; a store instruction covers 32/(RB/16)
-        // rows (128-byte rows: 4, lanes along the row; 64-byte rows: 8, lanes
-        // down the rows, which keeps the 80-byte pitch free of bank conflicts)
-        constexpr int CH = RB / 16;
-        constexpr int RPI = 32 / CH;
-        const int ch = RB == 128 ? (lane & 7) : (lane >> 3);
-        const int rsub = RB == 128 ? (lane >> 3) : (lane & 7);
-        const int tcol = c + ch * (16 / ESZ);    // column inside the tile
-        const int gcol = n0 + tcol;
-        // a round can run past the tile (BN not a multiple of the round width):
-        // those columns belong to the next tile and are not stored
-        const bool col_ok = tcol < BN && gcol < N;
+            // 128-byte rows, 128-byte swizzle: 16-byte chunk j of row r at j ^ (r % 8)
 #pragma unroll
-        for (int it = 0; it < 32 / RPI; ++it) {
-          const int rr = it * RPI + rsub;
-          const int grow = row0 + rr;
-          if (grow < M && col_ok) {
-            const uint4 u = *reinterpret_cast<const uint4*>(stg + rr * L::kStagePitch + ch * 16);
-            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(y) +
-                                      (static_cast<size_t>(grow) * N + gcol) * ESZ) = u;
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                  make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                             __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+          } else {
+            // 64-byte rows, 64-byte swizzle: 16-byte chunk j of row r at j ^ ((r / 2) % 4)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                  make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                             pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                             pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
           }
+          // the box's generic-proxy writes before the async-proxy store reads them
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, smem_u32(box), n0 + c, row0);
+            bulk_commit_group();
+          }
+          ++nst;
+          c = cn;
+          have = next;
         }
       }
       tc_fence_before();
@@ -472,6 +444,8 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
         else mbar_arrive_cluster(map_to_rank(acce0 + 8 * acc, 0));
       }
     }
+    // every store of this warp has finished before the CTA's shared memory goes
+    if (lane == 0) bulk_wait_group<0>();
   }
   __syncwarp();
   tc_fence_before();
@@ -494,9 +468,9 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
 // Host side
 // ---------------------------------------------------------------------------
 template <int BN, int CG, int ACT, bool OUT_F32>
-cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
-                       const float* bias, void* y, int* err, int num_sms, cudaStream_t st) {
-  using L = GemmSmem<BN, CG, epi_warps(ACT)>;
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, int M,
+                       int N, int K, const float* bias, int* err, int num_sms, cudaStream_t st) {
+  using L = GemmSmem<BN, CG, epi_warps(ACT), OUT_F32 ? 4 : 2>;
   auto kern = gemm_bf16_tc_kernel<BN, CG, ACT, OUT_F32>;
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(gemm_threads(ACT));
@@ -545,21 +519,21 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, int M, int N,
   cfg.numAttrs = na;
   // the activations (A, M rows) are at least as large as the weights (B, N rows)
   const int n_fastest = M >= N ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, a, b, M, N, K, bias, y, err, n_fastest);
+  return cudaLaunchKernelEx(&cfg, kern, a, b, y, M, N, K, bias, err, n_fastest);
 }
 
 template <int BN, int CG>
-cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, int M, int N, int K,
-                       const float* bias, void* y, bool out_f32, int act, int* err, int num_sms,
-                       cudaStream_t st) {
+cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, int M,
+                       int N, int K, const float* bias, bool out_f32, int act, int* err,
+                       int num_sms, cudaStream_t st) {
   if (out_f32) {
-    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, M, N, K, bias, y, err, num_sms, st);
-    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, M, N, K, bias, y, err, num_sms, st);
-    return launch_one<BN, CG, 0, true>(a, b, M, N, K, bias, y, err, num_sms, st);
+    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, y, M, N, K, bias, err, num_sms, st);
+    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, y, M, N, K, bias, err, num_sms, st);
+    return launch_one<BN, CG, 0, true>(a, b, y, M, N, K, bias, err, num_sms, st);
   }
-  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, M, N, K, bias, y, err, num_sms, st);
-  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, M, N, K, bias, y, err, num_sms, st);
-  return launch_one<BN, CG, 0, false>(a, b, M, N, K, bias, y, err, num_sms, st);
+  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, y, M, N, K, bias, err, num_sms, st);
+  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, y, M, N, K, bias, err, num_sms, st);
+  return launch_one<BN, CG, 0, false>(a, b, y, M, N, K, bias, err, num_sms, st);
 }
 
 }  // namespace
@@ -597,27 +571,30 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms, int act) {
   return best;
 }
 
-cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, GemmTile tile, int M, int N,
-                        int K, const float* bias, void* y, bool out_f32, int act, int* err,
-                        int num_sms, cudaStream_t st) {
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y,
+                        GemmTile tile, int M, int N, int K, const float* bias, bool out_f32,
+                        int act, int* err, int num_sms, cudaStream_t st) {
+#define RM_GEMM_TILE(cg, bn) \
+  case bn: return launch_act<bn, cg>(a, b, y, M, N, K, bias, out_f32, act, err, num_sms, st)
   if (tile.cg == 2) {
     switch (tile.bn) {
-      case 128: return launch_act<128, 2>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-      case 192: return launch_act<192, 2>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-      case 256: return launch_act<256, 2>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+      RM_GEMM_TILE(2, 128);
+      RM_GEMM_TILE(2, 192);
+      RM_GEMM_TILE(2, 256);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (tile.bn) {
-    case 64: return launch_act<64, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 96: return launch_act<96, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 128: return launch_act<128, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 160: return launch_act<160, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 192: return launch_act<192, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 224: return launch_act<224, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
-    case 256: return launch_act<256, 1>(a, b, M, N, K, bias, y, out_f32, act, err, num_sms, st);
+    RM_GEMM_TILE(1, 64);
+    RM_GEMM_TILE(1, 96);
+    RM_GEMM_TILE(1, 128);
+    RM_GEMM_TILE(1, 160);
+    RM_GEMM_TILE(1, 192);
+    RM_GEMM_TILE(1, 224);
+    RM_GEMM_TILE(1, 256);
     default: return cudaErrorInvalidValue;
   }
+#undef RM_GEMM_TILE
 }
 
 // Failure detection without a fault: one thread waits on an mbarrier that

@@ -24,17 +24,23 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms, int act = 0);
 cudaError_t bounded_wait_selftest(unsigned long long limit_ns, int* d_timed_out,
                                   unsigned long long* d_elapsed_ns, cudaStream_t st);
 inline int gemm_tile_index(int box_rows) { return (box_rows - 64) / 32; }
-// a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, tile.b_box()}.
+// a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, tile.b_box()};
+// y: [>= M][N] output map of make_tmap_store (fp32 when out_f32, else bf16).
 // Persistent grid of min(tiles, num_sms / cg) units of cg CTAs.
-cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, GemmTile tile, int M, int N,
-                        int K, const float* bias, void* y, bool out_f32, int act, int* err,
-                        int num_sms, cudaStream_t st);
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y,
+                        GemmTile tile, int M, int N, int K, const float* bias, bool out_f32,
+                        int act, int* err, int num_sms, cudaStream_t st);
 
 // ---- TMA descriptors (tma.cpp) ----
 // 2-D bf16 row-major [rows][cols] tensor, box {64 cols, box_rows}, 128-byte swizzle,
 // zero fill outside.  Returns false (message in *why) if the driver refuses it.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                     uint32_t box_rows, const char** why);
+// 2-D row-major [rows][cols] output of the GEMM (bf16, or fp32 when f32), box
+// {32 cols, 32 rows}, 64-byte (bf16) or 128-byte (fp32) swizzle: the layout of
+// the GEMM epilogue's staging boxes.  Stores outside the tensor are clipped.
+bool make_tmap_store(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, bool f32,
+                     const char** why);
 
 // Weights of the next GEMMs to pull into L2 while a latency-bound kernel runs
 // (the whole model does not stay in L2, so a GEMM would otherwise start on

@@ -51,4 +51,32 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t 
   return true;
 }
 
+bool make_tmap_store(CUtensorMap* map, void* base, uint64_t rows, uint64_t cols, bool f32,
+                     const char** why) {
+  auto fn = encode_fn();
+  if (fn == nullptr) {
+    *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return false;
+  }
+  const uint64_t esz = f32 ? 4 : 2;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (cols * esz) % 16 != 0) {
+    *why = "TMA needs a 16-byte aligned base and a row pitch that is a multiple of 16 bytes";
+    return false;
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * esz};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims,
+         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    *why = "cuTensorMapEncodeTiled rejected the tensor";
+    return false;
+  }
+  return true;
+}
+
 }  // namespace rmk

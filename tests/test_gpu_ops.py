@@ -56,8 +56,8 @@ def test_gemm_fp32_out(M, N, K, act):
     assert np.all(err <= bound), float((err / bound).max())
 
 
-# bf16 output: the epilogue stores 64 columns per round, so widths that are not
-# a multiple of 64 (96, 160, 224) end in a partial round
+# bf16 output: the epilogue stores boxes of 32 columns, so widths that are not
+# a multiple of 32 (936, 1200) end in a box the store clips
 @pytest.mark.parametrize("M,N,K", [(3264, 2304, 768), (77, 936, 312), (3328, 768, 768),
                                    (1000, 1200, 312), (4000, 2304, 768)])
 def test_gemm_bf16_out_and_no_bias(M, N, K):
@@ -75,6 +75,8 @@ def test_gemm_bf16_out_and_no_bias(M, N, K):
 # Every output tile forced, on a ragged problem (partial last row and column
 # tiles -- with a CTA pair the second CTA's rows or weight half can lie wholly
 # outside -- and a partial last K block) and on a multi-round projection shape.
+# Y is the head of a larger buffer whose rows past M must stay untouched (the
+# epilogue's box stores are clipped to M rows).
 GEMM_TILES = [(1, bn) for bn in (64, 96, 128, 160, 192, 224, 256)] + [(2, bn) for bn in (128, 192, 256)]
 
 
@@ -89,20 +91,23 @@ def test_gemm_every_tile(cg, bn, shape, out):
     b = torch.randn(N, generator=g, dtype=torch.float32) * 0.1
     X, W, B = f64(x), f64(w), f64(b)
     scale = np.abs(X) @ np.abs(W).T + np.abs(B)
-    if out == "f32-gelu":
-        y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    f32 = out == "f32-gelu"
+    buf = torch.full((M + 300, N), float("nan"), dtype=torch.float32 if f32 else torch.bfloat16,
+                     device="cuda")
+    y = buf[:M]
+    if f32:
         rm.ops.gemm_tiled(x.cuda(), w.cuda(), b.cuda(), y, rm.F32, M, N, K, 1, cg, bn)
         torch.cuda.synchronize()
         ref = O.gelu(O.linear(X, W, B), O.GELU_ERF)
         bound = F32_RTOL * scale * 1.2 + 4e-7 * np.abs(ref)
     else:
-        y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         rm.ops.gemm_tiled(x.cuda(), w.cuda(), b.cuda(), y, rm.BF16, M, N, K, 0, cg, bn)
         torch.cuda.synchronize()
         ref = O.linear(X, W, B)
         bound = BF16_REL * np.abs(ref) + F32_RTOL * scale
     err = np.abs(f64(y) - ref)
     assert np.all(err <= bound), float(np.nanmax(err / bound))
+    assert bool(torch.isnan(buf[M:]).all())
 
 
 def test_gemm_rejects_bad_shapes():
