@@ -118,6 +118,8 @@ def lib() -> ctypes.CDLL:
         "rm_op_attn_fused": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_attention_noalloc": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, P]),
         "rm_op_attn_tiles": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, I32, P]),
+        "rm_attn_tc_tiles": (ctypes.c_int, [P, I32, P]),
+        "rm_op_attn_tc": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_res_ln": (ctypes.c_int, [P, P, P, P, P, I32, I32, F, I32, I32, P]),
         "rm_op_head": (ctypes.c_int, [P, P, I32, P, F, I32, I32, P, P]),
         "rm_arena_plan": (ctypes.c_int, [cfgp, I32, I32, I64, P, P, P, P, I32, P]),
@@ -355,6 +357,20 @@ class ops:
         _check(lib().rm_op_attn_tiles(_ptr(qkv), _ptr(ctx), _ptr(offsets_dev), n_seqs, T, n_heads,
                                       head_dim, T if max_len is None else max_len, causal,
                                       _stream(stream)))
+
+    @staticmethod
+    def attn_tc_tiles(offsets):
+        """rm_attn_tc_tiles: host offsets -> int32 tile boundaries (sequence indices)."""
+        off = _i32(offsets)
+        n = len(off) - 1
+        out = np.zeros(n + 1, dtype=np.int32)
+        k = _check(lib().rm_attn_tc_tiles(off.ctypes.data, n, out.ctypes.data))
+        return out[:k + 1].copy()
+
+    @staticmethod
+    def attn_tc(qkv, ctx, offsets_dev, tiles_dev, n_tiles, n_seqs, T, n_heads, causal, stream=None):
+        _check(lib().rm_op_attn_tc(_ptr(qkv), _ptr(ctx), _ptr(offsets_dev), _ptr(tiles_dev), n_tiles,
+                                   n_seqs, T, n_heads, causal, _stream(stream)))
 
     @staticmethod
     def attention_noalloc(qkv, ctx, offsets, n_heads, head_dim, causal, stream=None):

@@ -224,16 +224,18 @@ struct rm_handle {
 namespace {
 
 // Metadata of one call in a staging slot / the device meta region:
-// offsets int32[n+1] | rb_off int32[n+1] | s_off int64[n+1]  (16-byte aligned
-// parts), then for shared-prefix calls pre_start int32[n] | pre_len int32[n] |
+// offsets int32[n+1] | rb_off int32[n+1] | s_off int64[n+1] | tiles int32[n+1]
+// (16-byte aligned parts; tiles: the tensor-core attention's sequence tiles),
+// then for shared-prefix calls pre_start int32[n] | pre_len int32[n] |
 // out_index int32[n] | group_off int32[n+1].  `base` bytes are copied for a
 // plain call, `bytes` for a shared-prefix call.
 struct MetaLayout {
-  int64_t rb, so, base, pst, pln, oix, gof, bytes;
+  int64_t rb, so, tl, base, pst, pln, oix, gof, bytes;
   explicit MetaLayout(int64_t n) {
     rb = align_up(4 * (n + 1), 16);
     so = rb + align_up(4 * (n + 1), 16);
-    base = so + align_up(8 * (n + 1), 16);
+    tl = so + align_up(8 * (n + 1), 16);
+    base = tl + align_up(4 * (n + 1), 16);
     pst = base;
     pln = pst + align_up(4 * n, 16);
     oix = pln + align_up(4 * n, 16);
@@ -472,6 +474,8 @@ struct ProfScope {
 // What the launch sequence of one call needs to know on the host.
 struct CallInfo {
   int32_t n = 0, T = 0, nrb = 0, Lmax = 0;
+  int32_t ntc = 0;                   // tensor-core attention tiles (0: that kernel does not apply)
+  const int32_t* d_tl = nullptr;
   int64_t S = 0;
   double att = 0;   // attention entries the mask admits, summed over heads
   const int32_t* d_off = nullptr;
@@ -497,6 +501,12 @@ double attention_entries(const rm_config* c, const int32_t* offsets, int32_t n,
 
 int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, float* d_out,
                     cudaStream_t st);
+
+// The tensor-core attention takes a plain call of the fused attention when
+// the head dim is 64 and no sequence is longer than its 128-row tiles.
+bool tc_attention_applies(const rm_config* c, int32_t max_len, bool prefix) {
+  return !prefix && c->attn_impl == RM_ATTN_FUSED && c->hidden / c->n_heads == 64 && max_len <= 128;
+}
 
 // host_ids != NULL: copy the ids host->device (into the arena) once the call
 // has been validated, and the scores back into host_out at the end.
@@ -532,6 +542,8 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   RM_TRY(host_varlen_meta(offsets, n, c->n_heads, p_rb, p_so, &Lmax));
   const int32_t nrb = p_rb[n];
   const int64_t S = p_so[n];
+  const int32_t ntc =
+      tc_attention_applies(c, Lmax, px != nullptr) ? attn_tc_tiles(offsets, n, reinterpret_cast<int32_t*>(ps + ml.tl)) : 0;
   if (host_ids != nullptr) {
     RM_CUDA(cudaMemcpyAsync(h->d_ids, host_ids, 4 * static_cast<size_t>(T), cudaMemcpyHostToDevice, st));
     d_ids = h->d_ids;
@@ -557,6 +569,8 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   ci.T = T;
   ci.nrb = nrb;
   ci.Lmax = Lmax;
+  ci.ntc = ntc;
+  ci.d_tl = reinterpret_cast<const int32_t*>(h->d_meta + ml.tl);
   ci.S = S;
   ci.att = attention_entries(c, offsets, n, px);
   ci.d_off = d_off;
@@ -660,6 +674,11 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
     if (px != nullptr) {
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
                 attn_fused_prefix_launch(qkv, ctx, d_off, d_rb, d_pst, d_pln, n, nrb, nh, d, st, pf_o));
+    } else if (ci.ntc > 0) {
+      // tensor-core attention on tiles of whole sequences (head dim 64, L <= 128)
+      RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
+                attn_tc_launch(qkv, ctx, d_off, ci.d_tl, ci.ntc, n, T, nh, dec, h->d_err,
+                               h->num_sms, st, pf_o));
     } else if (c->attn_impl == RM_ATTN_FUSED && (d == 64 || d == 128)) {
       // packed-row tiles (head dims 64 and 128); other head dims below
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
@@ -936,6 +955,9 @@ int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_
   std::memcpy(p_off, seq_offsets, 4 * static_cast<size_t>(n + 1));
   int32_t Lmax = 0;
   RM_TRY(host_varlen_meta(seq_offsets, n, c->n_heads, p_rb, p_so, &Lmax));
+  const int32_t ntc = tc_attention_applies(c, Lmax, false)
+                          ? attn_tc_tiles(seq_offsets, n, reinterpret_cast<int32_t*>(meta.data() + ml.tl))
+                          : 0;
   Bucket* bk = nullptr;
   RM_TRY(get_bucket(h, T, p_so[n], &bk));   // the arena placement and tensor maps, made now
   rm_plan* p = new rm_plan();
@@ -953,6 +975,8 @@ int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_
   ci.T = T;
   ci.nrb = p_rb[n];
   ci.Lmax = Lmax;
+  ci.ntc = ntc;
+  ci.d_tl = reinterpret_cast<const int32_t*>(p->d_meta + ml.tl);
   ci.S = p_so[n];
   ci.att = attention_entries(c, seq_offsets, n, nullptr);
   ci.d_off = reinterpret_cast<const int32_t*>(p->d_meta);
@@ -1018,11 +1042,12 @@ int rm_build_checked(void) { return RMK_CHECKED; }
 
 int rm_bounds_errors(int64_t* out) {
   if (out == nullptr) return set_error(RM_E_INVAL, "NULL argument");
-  int32_t a = 0, b = 0;
+  int32_t a = 0, b = 0, c = 0;
   RM_CUDA(cudaDeviceSynchronize());
   RM_CUDA(bounds_errors_rowops(&a, true));
   RM_CUDA(bounds_errors_attention(&b, true));
-  *out = static_cast<int64_t>(a) + b;
+  RM_CUDA(bounds_errors_attention_tc(&c, true));
+  *out = static_cast<int64_t>(a) + b + c;
   return RM_OK;
 }
 
@@ -1278,6 +1303,34 @@ int rm_op_attn_tiles(const void* qkv, void* ctx, const int32_t* offsets, int32_t
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
   RM_LAUNCH(attn_tile_launch(qkv, ctx, offsets, n_seqs, T, n_heads, head_dim, max_len, causal, err,
                              sms, static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_attn_tc_tiles(const int32_t* offsets, int32_t n_seqs, int32_t* tiles) {
+  if (offsets == nullptr || tiles == nullptr || n_seqs < 1) return set_error(RM_E_INVAL, "bad arguments");
+  if (offsets[0] != 0) return set_error(RM_E_INVAL, "seq_offsets[0] must be 0");
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const int64_t L = static_cast<int64_t>(offsets[i + 1]) - offsets[i];
+    if (L < 1 || L > 128)
+      return set_error(RM_E_RANGE, "sequence %d has length %lld (tiles need 1..128)", i, (long long)L);
+  }
+  return attn_tc_tiles(offsets, n_seqs, tiles);
+}
+
+int rm_op_attn_tc(const void* qkv, void* ctx, const int32_t* offsets, const int32_t* tiles,
+                  int32_t n_tiles, int32_t n_seqs, int32_t T, int32_t n_heads, int32_t causal,
+                  void* stream) {
+  if (qkv == nullptr || ctx == nullptr || offsets == nullptr || tiles == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || T < 1 || n_heads < 1 || n_tiles < 1 || n_tiles > n_seqs)
+    return set_error(RM_E_INVAL, "bad sizes");
+  int dev = 0, sms = 0;
+  RM_CUDA(cudaGetDevice(&dev));
+  RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  int32_t* err = nullptr;
+  RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
+  RM_LAUNCH(attn_tc_launch(qkv, ctx, offsets, tiles, n_tiles, n_seqs, T, n_heads, causal, err, sms,
+                           static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

@@ -81,6 +81,7 @@ cudaError_t cvt_to_f32_launch(const void* src, int src_dtype, float* dst, size_t
 // read into *out, cleared when reset.  Always 0 in the product build.
 cudaError_t bounds_errors_rowops(int32_t* out, bool reset);
 cudaError_t bounds_errors_attention(int32_t* out, bool reset);
+cudaError_t bounds_errors_attention_tc(int32_t* out, bool reset);
 
 // ---- attention (attention.cu) ----
 cudaError_t attn_scores_launch(const void* qkv, void* S, const int32_t* offsets,
@@ -113,6 +114,16 @@ cudaError_t attn_fused_launch(const void* qkv, void* ctx, const int32_t* offsets
 cudaError_t attn_tile_launch(const void* qkv, void* ctx, const int32_t* offsets, int n_seqs, int T,
                              int n_heads, int head_dim, int max_len, int causal, int* err,
                              int num_sms, cudaStream_t st, const L2Prefetch& pf = {});
+// Tensor-core attention (attention_tc.cu): head dim 64, every sequence at
+// most 128 tokens.  tiles: DEVICE int32[n_tiles + 1], tile k holds sequences
+// [tiles[k], tiles[k+1]) (at most 128 rows), as attn_tc_tiles builds them.
+cudaError_t attn_tc_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                           const int32_t* tiles, int n_tiles, int n, int T, int nh, int causal,
+                           int* err, int num_sms, cudaStream_t st, const L2Prefetch& pf = {});
+// Greedy cut of the packed batch into tiles of whole sequences of at most 128
+// rows (host; every sequence at most 128 tokens): writes tiles[0..n_tiles],
+// returns n_tiles.
+int32_t attn_tc_tiles(const int32_t* offsets, int32_t n, int32_t* tiles);
 // Causal fused attention over segments that may continue a shared prefix:
 // query row r of segment i attends to the pre_len[i] rows starting at packed
 // row pre_start[i] (all of them) and to rows 0..r of its own segment.

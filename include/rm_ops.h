@@ -151,6 +151,31 @@ int rm_op_attn_tiles(const void* qkv, void* ctx, const int32_t* offsets, int32_t
                      int32_t n_heads, int32_t head_dim, int32_t max_len, int32_t causal,
                      void* stream);
 
+/* Tiles of the tensor-core attention (rm_op_attn_tc): a greedy cut of the
+ * packed batch into runs of whole sequences of at most 128 rows each.
+ * offsets: HOST int32[n_seqs+1] with offsets[0] = 0 and every length in
+ * 1..128; tiles: HOST int32[n_seqs+1] (caller-owned), receives tiles[0..k]
+ * with tiles[0] = 0 and tiles[k] = n_seqs, tile j holding sequences
+ * [tiles[j], tiles[j+1]).  Returns k (>= 1), or RM_E_INVAL / RM_E_RANGE.
+ * This cut of the batch has no counterpart in the pages; it is the layout
+ * of the kernel below. */
+int rm_attn_tc_tiles(const int32_t* offsets, int32_t n_seqs, int32_t* tiles);
+
+/* The attention step of rm_op_attn_tiles on the 5th-generation tensor cores,
+ * for head_dim 64 and sequences of at most 128 tokens (the TurboTransformers
+ * proposed-method section's batched QK^T, batch softmax and PV, fused): per
+ * tile of rm_attn_tc_tiles and head, S = QK^T (tcgen05.mma into tensor
+ * memory), the row softmax over the row's own sequence (c <= r too when
+ * causal) in fp32 with P rounded to bf16, and C = P V (tcgen05.mma), written
+ * to ctx.  qkv: bf16 [T][3H], H = 64 * n_heads; ctx: bf16 [T][H]; offsets:
+ * DEVICE int32[n_seqs+1] with offsets[n_seqs] = T (host value T); tiles:
+ * DEVICE int32[n_tiles+1] as rm_attn_tc_tiles wrote them for the same
+ * offsets.  RM_E_INVAL for NULL pointers or sizes < 1; waits that give up
+ * (none in normal operation) count into an internal error word. */
+int rm_op_attn_tc(const void* qkv, void* ctx, const int32_t* offsets, const int32_t* tiles,
+                  int32_t n_tiles, int32_t n_seqs, int32_t T, int32_t n_heads, int32_t causal,
+                  void* stream);
+
 /* The materialised attention step (rm_op_attn_scores -> rm_op_softmax ->
  * rm_op_attn_context) without any device allocation: the score matrix and the
  * per-call metadata live in one file-scope device array of 8 MiB of scores

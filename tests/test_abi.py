@@ -116,6 +116,33 @@ def test_varlen_meta_layout():
         rm.ops.varlen_meta(bad, 3)
 
 
+@pytest.mark.parametrize("seed", range(6))
+def test_attn_tc_tiles_cut_whole_sequences_greedily(seed):
+    """Tiles of the tensor-core attention: consecutive runs of whole sequences
+    that cover the batch, each at most 128 rows, and maximal (the next
+    sequence would not have fit) -- checked against the definition, not a
+    second implementation of the cut."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(1, 129, int(rng.integers(1, 400)))
+    if seed == 0:
+        lens = np.array([128, 1, 127, 128, 64, 64, 65])
+    off = synth.offsets_from_lengths(lens)
+    tiles = rm.ops.attn_tc_tiles(off)
+    assert tiles[0] == 0 and tiles[-1] == len(lens)
+    assert np.all(np.diff(tiles) >= 1)
+    rows = off[tiles[1:]] - off[tiles[:-1]]
+    assert np.all(rows <= 128)
+    # greedy: each tile but the last could not take the next tile's first sequence
+    assert np.all(rows[:-1] + lens[tiles[1:-1]] > 128)
+
+
+def test_attn_tc_tiles_reject_long_or_empty_sequences():
+    for lens in ([5, 129, 3], [4, 0, 2]):
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        with pytest.raises(rm.RmError):
+            rm.ops.attn_tc_tiles(off)
+
+
 def test_gemm_tile_pick_is_a_known_tile():
     tiles = {(1, bn) for bn in (64, 96, 128, 160, 192, 224, 256)} | {(2, bn) for bn in (128, 192, 256)}
     for M in (1, 77, 128, 300, 3328, 26112):

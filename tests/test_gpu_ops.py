@@ -571,6 +571,99 @@ def test_attention_tiles_rejects_other_head_dims():
         assert e.value.code == rm.RM_E_INVAL
 
 
+# --- tensor-core attention (head dim 64, sequences of at most 128 tokens) ------
+
+def _attn_tc(qkv, ctx, off, nh, causal):
+    tiles = rm.ops.attn_tc_tiles(off)
+    rm.ops.attn_tc(qkv, ctx, dev(off, torch.int32), dev(tiles, torch.int32), len(tiles) - 1,
+                   len(off) - 1, int(off[-1]), nh, causal)
+    return tiles
+
+
+@pytest.mark.parametrize("lens", [
+    [1, 65, 128, 64, 9],                                # ragged; a full 128-row tile
+    [2, 3, 1, 5, 2, 7, 1, 1, 4, 9, 2, 3, 8, 1, 6, 2],    # many sequences per tile and warp
+    [100] * 8,                                          # one sequence per tile
+    [127, 1, 128, 128, 2],                              # tiles of exactly 128 rows
+    [5],                                                # one short tile
+    [33, 31, 32, 32, 64, 17, 47],                       # sequences across 32-row warps
+], ids=["ragged", "tiny", "uniform", "full", "single", "warps"])
+@pytest.mark.parametrize("nh", [2, 12])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_attention_tc(lens, nh, causal):
+    """tcgen05 attention on sequence tiles against the oracle's attention,
+    every row and head."""
+    d = 64
+    H = nh * d
+    lens = np.array(lens)
+    off = synth.offsets_from_lengths(lens)
+    rng = np.random.default_rng(nh * 7 + causal + len(lens))
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    _attn_tc(qkv, ctx, off, nh, causal)
+    torch.cuda.synchronize()
+    _attention_ref_check(f64(qkv), f64(ctx), off, nh, d, causal)
+
+
+def test_attention_tc_bench_shape_against_tiles_and_oracle():
+    """A fused call of the BERT-base stream's shape (512 sequences of 2..100
+    tokens, 12 heads of 64): every output finite, within bf16 rounding of the
+    packed-row tile kernel everywhere, sampled sequences against the oracle."""
+    nh, d = 12, 64
+    H = nh * d
+    rng = np.random.default_rng(2024)
+    lens = rng.integers(2, 101, 512)
+    off = synth.offsets_from_lengths(lens)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    a = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    b = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    _attn_tc(qkv, a, off, nh, 0)
+    rm.ops.attn_tiles(qkv, b, dev(off, torch.int32), len(lens), T, nh, d, 0, max_len=100)
+    torch.cuda.synchronize()
+    A, B = f64(a), f64(b)
+    assert np.all(np.isfinite(A))
+    X = f64(qkv)
+    # Each kernel rounds every P entry to bf16 (half an ulp, 2^-9 relative:
+    # at most 2^-9 * max_k |v_kc| on output column c after the division by
+    # the row sum) and the output once (2^-9 |out|); the two differ by at
+    # most twice that.  max_k runs over the row's own sequence.
+    vmax = np.repeat(np.maximum.reduceat(np.abs(X[:, 2 * H:]), off[:-1], axis=0), lens, axis=0)
+    assert np.all(np.abs(A - B) <= 1.5 * BF16_REL * (vmax + np.abs(B)) + 1e-6)
+    for i in np.linspace(0, len(lens) - 1, 16).astype(int):
+        sub = np.array([0, lens[i]], dtype=np.int64)
+        _attention_ref_check(X[off[i]:off[i + 1]], A[off[i]:off[i + 1]], sub, nh, d, 0)
+
+
+def test_attention_tc_repeat_bit_identical():
+    """Twelve heads through three load slots, four TMEM regions and two softmax
+    groups: thirty launches with other launches in between give the same bits."""
+    nh, d = 12, 64
+    H = nh * d
+    rng = np.random.default_rng(23)
+    lens = rng.integers(1, 129, 300)
+    off = synth.offsets_from_lengths(lens)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    other = dev(qkv_for(T, H, rng), torch.bfloat16)
+    junk = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    first = None
+    for _ in range(30):
+        _attn_tc(other, junk, off, nh, 0)
+        ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        _attn_tc(qkv, ctx, off, nh, 0)
+        torch.cuda.synchronize()
+        if first is None:
+            first = ctx
+            X, C = f64(qkv), f64(ctx)
+            for i in np.linspace(0, len(lens) - 1, 12).astype(int):
+                sub = np.array([0, lens[i]], dtype=np.int64)
+                _attention_ref_check(X[off[i]:off[i + 1]], C[off[i]:off[i + 1]], sub, nh, d, 0)
+        else:
+            assert torch.equal(ctx, first)
+
+
 def test_gemm_gelu_epilogue_against_cuda_erf_and_oracle():
     """GELU of the epilogue (Abramowitz & Stegun 7.1.28 erf) on a dense grid of
     pre-activations: x = 0, W = 0, so y = GELU(bias)."""
