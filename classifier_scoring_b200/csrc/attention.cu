@@ -238,8 +238,8 @@ __global__ void __launch_bounds__(256)
 // packed bf16 pairs (exact in any precision), the masking of a row's last
 // partial chunk at 16-bit granularity (-inf), and the exponent's argument
 // and the sum in packed fp32 pairs; exp2 of -inf gives the masked entries
-// exactly 0.  The exponentials are formed twice (for the sum, then for the
-// output) rather than held.
+// exactly 0.  A row's exponentials are held (two per 64-bit register) from
+// the sum to the output, which is one packed multiply per pair.
 template <int G, int MAXC, int U>
 __device__ __forceinline__ void softmax_load_bf16(bf16* const (&row)[U], const int (&len)[U], int sub,
                                                   uint32_t (&w)[U][MAXC][4]) {
@@ -291,17 +291,19 @@ __device__ __forceinline__ void softmax_compute_bf16(bf16* const (&row)[U], cons
     const uint64_t shift = f32x2_splat(m == -INFINITY ? 0.f : -m * kLog2e);
     const uint64_t l2e = f32x2_splat(kLog2e);
     uint64_t acc = 0;                                         // +0.0 in both lanes
+    uint64_t e2[MAXC][4];                                     // the exponentials, two per register
 #pragma unroll
     for (int c = 0; c < MAXC; ++c)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float x0, x1;
         f32x2_unpack(f32x2_fma(f32x2_pack(bf16_lo(w[u][c][j]), bf16_hi(w[u][c][j])), l2e, shift), x0, x1);
-        acc = f32x2_add(acc, f32x2_pack(exp2f(x0), exp2f(x1)));
+        e2[c][j] = f32x2_pack(ex2_approx_ftz(x0), ex2_approx_ftz(x1));
+        acc = f32x2_add(acc, e2[c][j]);
       }
     float a0, a1;
     f32x2_unpack(acc, a0, a1);
-    const float inv = 1.0f / group_sum<G>(a0 + a1);
+    const uint64_t inv2 = f32x2_splat(1.0f / group_sum<G>(a0 + a1));
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int col = (c * G + sub) * 8;
@@ -309,9 +311,9 @@ __device__ __forceinline__ void softmax_compute_bf16(bf16* const (&row)[U], cons
         uint32_t o[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float x0, x1;
-          f32x2_unpack(f32x2_fma(f32x2_pack(bf16_lo(w[u][c][j]), bf16_hi(w[u][c][j])), l2e, shift), x0, x1);
-          o[j] = pack_bf16x2(exp2f(x0) * inv, exp2f(x1) * inv);
+          float y0, y1;
+          f32x2_unpack(f32x2_mul(e2[c][j], inv2), y0, y1);
+          o[j] = pack_bf16x2(y0, y1);
         }
         *reinterpret_cast<uint4*>(row[u] + col) = make_uint4(o[0], o[1], o[2], o[3]);
       }
@@ -336,12 +338,14 @@ __device__ __forceinline__ void softmax_compute_bf16(bf16* const (&row)[U], cons
 // every row is computed on its own, with the same arithmetic whatever its
 // position.
 // ---------------------------------------------------------------------------
-constexpr int kSmClasses = 9;
+constexpr int kSmClasses = 13;
 
+// 8-element chunks of a row: <= 1, 2, 4, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128
 __host__ __device__ constexpr int softmax_class_of(int L) {
-  return (L + 7) / 8 <= 1 ? 0 : (L + 7) / 8 <= 2 ? 1 : (L + 7) / 8 <= 4 ? 2 : (L + 7) / 8 <= 8 ? 3
-       : (L + 7) / 8 <= 16 ? 4 : (L + 7) / 8 <= 32 ? 5 : (L + 7) / 8 <= 64 ? 6
-       : (L + 7) / 8 <= 96 ? 7 : 8;
+  return (L + 7) / 8 <= 1 ? 0 : (L + 7) / 8 <= 2 ? 1 : (L + 7) / 8 <= 4 ? 2 : (L + 7) / 8 <= 6 ? 3
+       : (L + 7) / 8 <= 8 ? 4 : (L + 7) / 8 <= 12 ? 5 : (L + 7) / 8 <= 16 ? 6
+       : (L + 7) / 8 <= 24 ? 7 : (L + 7) / 8 <= 32 ? 8 : (L + 7) / 8 <= 48 ? 9
+       : (L + 7) / 8 <= 64 ? 10 : (L + 7) / 8 <= 96 ? 11 : 12;
 }
 
 // scratch: counters int64[2 * kSmClasses] (rows per class, reservation
@@ -400,6 +404,16 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// The sequence a lane's rows belong to: its index, the start of its stretch
+// in the class-ordered row space, its length and score offset.  Kept across
+// iterations so that a lane walking consecutive rows looks a sequence up
+// only when it crosses into the next one.
+struct SeqCache {
+  long long b = 0;             // stretch [b, b + rows)
+  int rows = 0, L = 0;
+  long long soff = 0;
+};
+
 // Rows [R0, R0 + U) of the class-ordered row space (those below Re): their
 // addresses and lengths (length 0 for none).
 template <typename T, int U>
@@ -408,118 +422,185 @@ __device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ 
                                               const long long* __restrict__ seq_base,
                                               const int32_t* __restrict__ row_seq, long long R0,
                                               long long Re, int n, int nh, int causal,
-                                              T* (&row)[U], int (&len)[U]) {
+                                              SeqCache& sc, T* (&row)[U], int (&len)[U]) {
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     len[u] = 0;
     row[u] = S;
   }
-  if (R0 >= Re) return;
-  int i = row_seq[R0];
-  if (!in_bounds(i >= 0 && i < n)) return;
-  long long b = seq_base[i];
-  int L = offsets[i + 1] - offsets[i];
 #pragma unroll
   for (int u = 0; u < U; ++u) {
     const long long R = R0 + u;
     if (R < Re) {
-      if (R - b >= static_cast<long long>(nh) * L) {         // the next sequence's stretch
-        i = row_seq[R];
+      if (R < sc.b || R - sc.b >= sc.rows) {                 // another sequence's stretch
+        const int i = row_seq[R];
         if (!in_bounds(i >= 0 && i < n)) return;
-        b = seq_base[i];
-        L = offsets[i + 1] - offsets[i];
+        sc.b = seq_base[i];
+        sc.L = offsets[i + 1] - offsets[i];
+        sc.rows = nh * sc.L;
+        sc.soff = s_off[i];
       }
-      const long long rr = R - b;                            // row inside the sequence's block
-      if (!in_bounds(L >= 1 && rr >= 0 && rr < static_cast<long long>(nh) * L)) return;
-      len[u] = causal ? static_cast<int>(rr % L) + 1 : L;
-      row[u] = S + s_off[i] + rr * ((L + 7) & ~7);
+      const long long rr = R - sc.b;                         // row inside the sequence's block
+      if (!in_bounds(sc.L >= 1 && rr >= 0 && rr < sc.rows)) return;
+      len[u] = causal ? static_cast<int>(rr % sc.L) + 1 : sc.L;
+      row[u] = S + sc.soff + rr * ((sc.L + 7) & ~7);
     }
   }
 }
 
+// The bf16 class kernel stages its rows through shared memory with cp.async:
+// per warp a ring of kSmStages iterations, each up to kSmChunks 16-byte chunks
+// per lane (chunk-major, so a warp's accesses to one chunk are contiguous).
+// The loads in flight are then not bounded by registers: about 8 KB per warp.
+constexpr int kSmStages = 4;
+constexpr int kSmChunks = 4;
+constexpr int kSmRingWarpBytes = kSmStages * kSmChunks * 32 * 16;
+constexpr int kSmClassThreads = 256;
+
+__device__ __forceinline__ void sm_cp16(uint32_t saddr, const void* g) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(saddr), "l"(g) : "memory");
+}
+__device__ __forceinline__ void sm_cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void sm_cp_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // One class: lane groups of G lanes, U consecutive rows (of the class-ordered
-// row space) each, grid-striding.  The loop bound is uniform across a warp
-// (groups past the end get empty rows): the group reductions are warp
-// shuffles.  For bf16 rows the next iteration's rows are loaded before the
-// current ones are computed, so that loads stay in flight.
+// row space) each.  Each warp walks one contiguous stretch of the class's
+// rows (an equal share of its warp-iterations), so consecutive iterations of
+// a lane group stay inside one sequence's rows and its address arithmetic
+// needs no lookup (the class-ordered row space keeps a sequence's rows
+// together).  The loop bound is uniform across a warp (groups past the end
+// get empty rows): the group reductions are warp shuffles.  bf16 rows are
+// loaded kSmStages - 1 iterations ahead into the warp's shared-memory ring.
 template <typename T, int G, int MAXC, int U>
 __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restrict__ offsets,
                                                    const int64_t* __restrict__ s_off,
                                                    const long long* __restrict__ seq_base,
                                                    const int32_t* __restrict__ row_seq,
                                                    long long Rb, long long Re, int n, int nh,
-                                                   int causal) {
+                                                   int causal, uint32_t ring) {
   if (Rb >= Re) return;
   const int lane = threadIdx.x & 31, sub = lane % G;
   constexpr int kGpw = 32 / G;
+  constexpr long long GU = static_cast<long long>(kGpw) * U;   // rows per warp-iteration
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  long long wg = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (Rb + wg * kGpw * U >= Re) return;                      // uniform across the warp
+  const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const long long iters = (Re - Rb + GU - 1) / GU;
+  const long long per = (iters + warps - 1) / warps;
+  long long it = w * per;
+  const long long it_end = min(iters, it + per);
+  if (it >= it_end) return;                                  // uniform across the warp
+  const long long lane_off = static_cast<long long>(lane / G) * U;
+  SeqCache sc;
   int len[U];
   T* row[U];
-  class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re, n,
-                      nh, causal, row, len);
   if constexpr (std::is_same<T, bf16>::value) {
-    uint32_t w[U][MAXC][4];
-    softmax_load_bf16<G, MAXC, U>(row, len, sub, w);
-    for (;;) {
-      const long long nwg = wg + warps;
-      const bool more = Rb + nwg * kGpw * U < Re;            // uniform across the warp
-      int nlen[U];
-      T* nrow[U];
-      uint32_t nw[U][MAXC][4];
-      if (more) {
-        class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (nwg * kGpw + lane / G) * U,
-                            Re, n, nh, causal, nrow, nlen);
-        softmax_load_bf16<G, MAXC, U>(nrow, nlen, sub, nw);
-      }
-      softmax_compute_bf16<G, MAXC, U>(row, len, sub, w);
-      if (!more) break;
-      wg = nwg;
+    constexpr int D = kSmStages;
+    static_assert(U * MAXC <= kSmChunks, "a lane's chunks fit its ring slot");
+    // this lane's chunk k of stage st
+    auto slot = [&](int st, int k) { return ring + static_cast<uint32_t>((st * kSmChunks + k) * 512); };
+    SeqCache sci;                                            // the issuing side's sequence
+    auto issue = [&](long long t) {
+      int il[U];
+      T* ir[U];
+      class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + t * GU + lane_off, Re, n, nh,
+                          causal, sci, ir, il);
+      const int st = static_cast<int>(t & (D - 1));
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        row[u] = nrow[u];
-        len[u] = nlen[u];
+      for (int u = 0; u < U; ++u)
 #pragma unroll
-        for (int c = 0; c < MAXC; ++c)
+        for (int c = 0; c < MAXC; ++c) {
+          const int col = (c * G + sub) * 8;
+          if (col < il[u]) sm_cp16(slot(st, u * MAXC + c), ir[u] + col);
+        }
+    };
 #pragma unroll
-          for (int j = 0; j < 4; ++j) w[u][c][j] = nw[u][c][j];
-      }
+    for (int k = 0; k < D - 1; ++k) {
+      if (it + k < it_end) issue(it + k);
+      sm_cp_commit();
     }
+    for (; it < it_end; ++it) {
+      if (it + D - 1 < it_end) issue(it + D - 1);
+      sm_cp_commit();
+      sm_cp_wait<D - 1>();                                   // iteration it has landed
+      class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
+                          causal, sc, row, len);
+      const int st = static_cast<int>(it & (D - 1));
+      uint32_t w4[U][MAXC][4];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int c = 0; c < MAXC; ++c) {
+          const int col = (c * G + sub) * 8;
+          if (col < len[u]) {
+            uint32_t q0, q1, q2, q3;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(q0), "=r"(q1), "=r"(q2), "=r"(q3)
+                         : "r"(slot(st, u * MAXC + c)));
+            w4[u][c][0] = q0;
+            w4[u][c][1] = q1;
+            w4[u][c][2] = q2;
+            w4[u][c][3] = q3;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w4[u][c][j] = 0xff80ff80u;   // -inf pairs
+          }
+        }
+      softmax_compute_bf16<G, MAXC, U>(row, len, sub, w4);
+    }
+    sm_cp_wait<0>();
   } else {
+    class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
+                        causal, sc, row, len);
     for (;;) {
       softmax_group<T, G, MAXC, U>(row, len, sub);
-      wg += warps;
-      if (Rb + wg * kGpw * U >= Re) break;
-      class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + (wg * kGpw + lane / G) * U, Re,
-                          n, nh, causal, row, len);
+      if (++it >= it_end) break;
+      class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
+                          causal, sc, row, len);
     }
   }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(256, 3)
+__global__ void __launch_bounds__(kSmClassThreads, 3)
     softmax_class_kernel(T* __restrict__ S, const int32_t* __restrict__ offsets,
                          const int64_t* __restrict__ s_off, const unsigned long long* __restrict__ ctr,
                          const long long* __restrict__ seq_base, const int32_t* __restrict__ row_seq,
                          int k_max, int n, int nh, int causal) {
+  extern __shared__ __align__(16) uint8_t sm_ring_raw[];
+  // this warp's ring (bf16 rows), offset by the lane's 16 bytes
+  const uint32_t ring = smem_u32(sm_ring_raw) + (threadIdx.x >> 5) * kSmRingWarpBytes + (threadIdx.x & 31) * 16;
   pdl_launch_dependents();
   pdl_wait();
   long long seg[kSmClasses + 1];
   seg[0] = 0;
 #pragma unroll
   for (int k = 0; k < kSmClasses; ++k) seg[k + 1] = seg[k] + static_cast<long long>(ctr[k]);
-  // lanes per row: the smallest power of two covering the class's chunks (at
-  // most 32), rows per lane group so that a lane has about four chunks in flight
-  softmax_class_pass<T, 1, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[0], seg[1], n, nh, causal);
-  if (k_max >= 1) softmax_class_pass<T, 2, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[1], seg[2], n, nh, causal);
-  if (k_max >= 2) softmax_class_pass<T, 4, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[2], seg[3], n, nh, causal);
-  if (k_max >= 3) softmax_class_pass<T, 8, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[3], seg[4], n, nh, causal);
-  if (k_max >= 4) softmax_class_pass<T, 16, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[4], seg[5], n, nh, causal);
-  if (k_max >= 5) softmax_class_pass<T, 32, 1, 4>(S, offsets, s_off, seq_base, row_seq, seg[5], seg[6], n, nh, causal);
-  if (k_max >= 6) softmax_class_pass<T, 32, 2, 2>(S, offsets, s_off, seq_base, row_seq, seg[6], seg[7], n, nh, causal);
-  if (k_max >= 7) softmax_class_pass<T, 32, 3, 1>(S, offsets, s_off, seq_base, row_seq, seg[7], seg[8], n, nh, causal);
-  if (k_max >= 8) softmax_class_pass<T, 32, 4, 1>(S, offsets, s_off, seq_base, row_seq, seg[8], seg[9], n, nh, causal);
+  // lanes per row G and chunks per lane MAXC with G * MAXC covering the
+  // class's chunks and MAXC three or four: a lane holds up to four chunks of
+  // one row, so the per-row work (addresses, masks, reductions) is spread
+  // over up to 32 entries; rows of one or two chunks take four or two rows
+  // per lane
+#define RM_SM_PASS(k, G, MAXC, U)                                                               \
+  if (k_max >= k)                                                                              \
+    softmax_class_pass<T, G, MAXC, U>(S, offsets, s_off, seq_base, row_seq, seg[k], seg[k + 1], n, \
+                                      nh, causal, ring)
+  RM_SM_PASS(0, 1, 1, 4);
+  RM_SM_PASS(1, 1, 2, 2);
+  RM_SM_PASS(2, 1, 4, 1);
+  RM_SM_PASS(3, 2, 3, 1);
+  RM_SM_PASS(4, 2, 4, 1);
+  RM_SM_PASS(5, 4, 3, 1);
+  RM_SM_PASS(6, 4, 4, 1);
+  RM_SM_PASS(7, 8, 3, 1);
+  RM_SM_PASS(8, 8, 4, 1);
+  RM_SM_PASS(9, 16, 3, 1);
+  RM_SM_PASS(10, 16, 4, 1);
+  RM_SM_PASS(11, 32, 3, 1);
+  RM_SM_PASS(12, 32, 4, 1);
+#undef RM_SM_PASS
 }
 
 template <int DP>
@@ -698,15 +779,15 @@ __global__ void __launch_bounds__(128)
     const float mn_a = fmaxf(m_a, bm_a), mn_b = fmaxf(m_b, bm_b);
     // rows whose keys are all masked so far keep m = -inf; use 0 as the shift then
     const float sh_a = mn_a == -INFINITY ? 0.f : mn_a, sh_b = mn_b == -INFINITY ? 0.f : mn_b;
-    const float al_a = exp2f(m_a - sh_a), al_b = exp2f(m_b - sh_b);
+    const float al_a = ex2_approx_ftz(m_a - sh_a), al_b = ex2_approx_ftz(m_b - sh_b);
     m_a = mn_a;
     m_b = mn_b;
     float ps_a = 0.f, ps_b = 0.f;
     uint32_t pa[4][4];   // P as the A operand of four k=16 steps
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
-      const float p0 = exp2f(sc[nt][0] - sh_a), p1 = exp2f(sc[nt][1] - sh_a);
-      const float p2 = exp2f(sc[nt][2] - sh_b), p3 = exp2f(sc[nt][3] - sh_b);
+      const float p0 = ex2_approx_ftz(sc[nt][0] - sh_a), p1 = ex2_approx_ftz(sc[nt][1] - sh_a);
+      const float p2 = ex2_approx_ftz(sc[nt][2] - sh_b), p3 = ex2_approx_ftz(sc[nt][3] - sh_b);
       ps_a += p0 + p1;
       ps_b += p2 + p3;
       pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
@@ -915,15 +996,15 @@ __global__ void __launch_bounds__(128, (DP <= 64 ? 4 : 1))
       bm_b = fmaxf(bm_b, __shfl_xor_sync(0xffffffffu, bm_b, 2));
       const float mn_a = fmaxf(m_a, bm_a), mn_b = fmaxf(m_b, bm_b);
       const float sh_a = mn_a == -INFINITY ? 0.f : mn_a, sh_b = mn_b == -INFINITY ? 0.f : mn_b;
-      const float al_a = exp2f(m_a - sh_a), al_b = exp2f(m_b - sh_b);
+      const float al_a = ex2_approx_ftz(m_a - sh_a), al_b = ex2_approx_ftz(m_b - sh_b);
       m_a = mn_a;
       m_b = mn_b;
       float ps_a = 0.f, ps_b = 0.f;
       uint32_t pa[4][4];
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
-        const float p0 = exp2f(sc[nt][0] - sh_a), p1 = exp2f(sc[nt][1] - sh_a);
-        const float p2 = exp2f(sc[nt][2] - sh_b), p3 = exp2f(sc[nt][3] - sh_b);
+        const float p0 = ex2_approx_ftz(sc[nt][0] - sh_a), p1 = ex2_approx_ftz(sc[nt][1] - sh_a);
+        const float p2 = ex2_approx_ftz(sc[nt][2] - sh_b), p3 = ex2_approx_ftz(sc[nt][3] - sh_b);
         ps_a += p0 + p1;
         ps_b += p2 + p3;
         pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
@@ -1225,18 +1306,18 @@ __global__ void __launch_bounds__(160)
         // m = -inf and shifts by 0
         const float sh_a = mn_a == -INFINITY ? 0.f : mn_a * scale_log2;
         const float sh_b = mn_b == -INFINITY ? 0.f : mn_b * scale_log2;
-        const float al_a = exp2f(fmaf(m_a, scale_log2, -sh_a));
-        const float al_b = exp2f(fmaf(m_b, scale_log2, -sh_b));
+        const float al_a = ex2_approx_ftz(fmaf(m_a, scale_log2, -sh_a));
+        const float al_b = ex2_approx_ftz(fmaf(m_b, scale_log2, -sh_b));
         m_a = mn_a;
         m_b = mn_b;
         float ps_a = 0.f, ps_b = 0.f;
         uint32_t pa[4][4];
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
-          const float p0 = exp2f(fmaf(sc[nt][0], scale_log2, -sh_a));
-          const float p1 = exp2f(fmaf(sc[nt][1], scale_log2, -sh_a));
-          const float p2 = exp2f(fmaf(sc[nt][2], scale_log2, -sh_b));
-          const float p3 = exp2f(fmaf(sc[nt][3], scale_log2, -sh_b));
+          const float p0 = ex2_approx_ftz(fmaf(sc[nt][0], scale_log2, -sh_a));
+          const float p1 = ex2_approx_ftz(fmaf(sc[nt][1], scale_log2, -sh_a));
+          const float p2 = ex2_approx_ftz(fmaf(sc[nt][2], scale_log2, -sh_b));
+          const float p3 = ex2_approx_ftz(fmaf(sc[nt][3], scale_log2, -sh_b));
           ps_a += p0 + p1;
           ps_b += p2 + p3;
           pa[nt >> 1][(nt & 1) * 2 + 0] = pack_bf16x2(p0, p1);
@@ -1431,14 +1512,21 @@ cudaError_t softmax_classes_launch(void* S, int s_dtype, const int32_t* offsets,
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int k_max = softmax_class_of(max_len);
-  // three CTAs of 256 threads per SM (the kernel's register bound: it holds
-  // two iterations' rows), grid-striding over each class
-  if (s_dtype == 0)
-    launch_k(softmax_class_kernel<float>, dim3(num_sms * 3), dim3(256), 0, st, static_cast<float*>(S),
-             offsets, s_off, ctr, seq_base, row_seq, k_max, n_seqs, n_heads, causal);
-  else
-    launch_k(softmax_class_kernel<bf16>, dim3(num_sms * 3), dim3(256), 0, st, static_cast<bf16*>(S),
-             offsets, s_off, ctr, seq_base, row_seq, k_max, n_seqs, n_heads, causal);
+  // three CTAs of 256 threads per SM, each warp walking one stretch of each
+  // class; bf16 rows through the warps' shared-memory rings (64 KB per CTA)
+  if (s_dtype == 0) {
+    launch_k(softmax_class_kernel<float>, dim3(num_sms * 3), dim3(kSmClassThreads), 0, st,
+             static_cast<float*>(S), offsets, s_off, ctr, seq_base, row_seq, k_max, n_seqs, n_heads,
+             causal);
+  } else {
+    constexpr int kRing = (kSmClassThreads / 32) * kSmRingWarpBytes;
+    static const cudaError_t attr_err = cudaFuncSetAttribute(
+        softmax_class_kernel<bf16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kRing);
+    if (attr_err != cudaSuccess) return attr_err;
+    launch_k(softmax_class_kernel<bf16>, dim3(num_sms * 3), dim3(kSmClassThreads), kRing, st,
+             static_cast<bf16*>(S), offsets, s_off, ctr, seq_base, row_seq, k_max, n_seqs, n_heads,
+             causal);
+  }
   return cudaGetLastError();
 }
 

@@ -85,14 +85,6 @@ __device__ __forceinline__ uint32_t low_bits(int x) {
   return x <= 0 ? 0u : (x >= 32 ? 0xffffffffu : ((1u << x) - 1u));
 }
 
-// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32): subnormal
-// inputs and results flush to zero.
-__device__ __forceinline__ float ex2_approx_ftz(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 // The same with A read from tensor memory (M = 128 lanes, two 16-bit
 // elements of a row per 32-bit column).
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,

@@ -107,6 +107,16 @@ __device__ __forceinline__ float gelu_erf_fast(float u) {
   return 0.5f * u * (1.0f + erf_as7128(u * 0.70710678118654752f));
 }
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32): one
+// special-function-unit instruction; subnormal inputs and results flush to
+// zero (for the softmax kernels: terms below 2^-126 of the row maximum's
+// term, far under one bf16 ulp of the largest probability).
+__device__ __forceinline__ float ex2_approx_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Two fp32 lanes in one 64-bit register, for sm_100's packed arithmetic
 // (add/sub/mul/fma .rn.f32x2: one instruction, two IEEE fp32 operations, each
 // rounded as its scalar form would be).
