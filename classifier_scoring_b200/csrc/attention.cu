@@ -348,19 +348,38 @@ __host__ __device__ constexpr int softmax_class_of(int L) {
        : (L + 7) / 8 <= 64 ? 10 : (L + 7) / 8 <= 96 ? 11 : 12;
 }
 
+// Largest chunk count of class k.
+__host__ __device__ constexpr int softmax_class_hi(int k) {
+  return k == 0 ? 1 : k == 1 ? 2 : k == 2 ? 4 : k == 3 ? 6 : k == 4 ? 8 : k == 5 ? 12 : k == 6 ? 16
+       : k == 7 ? 24 : k == 8 ? 32 : k == 9 ? 48 : k == 10 ? 64 : k == 11 ? 96 : 128;
+}
+// The rows of a sequence of length L that class k takes, per head: every
+// row when not causal (when k is L's class); when causal, the rows r whose
+// own length r + 1 falls in the class: [r_lo, r_lo + run).
+struct ClassRun {
+  int r_lo, run;
+};
+__host__ __device__ inline ClassRun softmax_class_run(int L, int k, int causal) {
+  if (!causal) return ClassRun{0, softmax_class_of(L) == k ? L : 0};
+  const int lo = k == 0 ? 0 : 8 * softmax_class_hi(k - 1);       // first row of the class
+  const int hi = 8 * softmax_class_hi(k) < L ? 8 * softmax_class_hi(k) : L;   // one past its last
+  return ClassRun{lo, hi > lo ? hi - lo : 0};
+}
+
 // scratch: counters int64[2 * kSmClasses] (rows per class, reservation
-// cursors) | seq_base int64[n] | row_seq int32[n_heads * T]
+// cursors) | seq_base int64[n][kSmClasses] (the start of each sequence's
+// stretch in each class) | row_seq int32[n_heads * T]
 struct SoftmaxIndexLayout {
   size_t base, rows, bytes;
   SoftmaxIndexLayout(long long n, long long rows_total) {
     base = 16 * kSmClasses;
-    rows = base + 8 * static_cast<size_t>(n);
+    rows = base + 8 * static_cast<size_t>(n) * kSmClasses;
     bytes = rows + 4 * static_cast<size_t>(rows_total);
   }
 };
 
 __global__ void __launch_bounds__(256)
-    softmax_count_kernel(const int32_t* __restrict__ offsets, int n, int nh,
+    softmax_count_kernel(const int32_t* __restrict__ offsets, int n, int nh, int causal,
                          unsigned long long* __restrict__ ctr) {
   __shared__ unsigned long long part[kSmClasses];
   if (threadIdx.x < kSmClasses) part[threadIdx.x] = 0;
@@ -369,14 +388,21 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     const int L = offsets[i + 1] - offsets[i];
-    atomicAdd(&part[softmax_class_of(L)], static_cast<unsigned long long>(nh) * L);
+    if (!causal) {
+      atomicAdd(&part[softmax_class_of(L)], static_cast<unsigned long long>(nh) * L);
+    } else {
+      for (int k = 0; k <= softmax_class_of(L); ++k) {
+        const ClassRun cr = softmax_class_run(L, k, 1);
+        if (cr.run > 0) atomicAdd(&part[k], static_cast<unsigned long long>(nh) * cr.run);
+      }
+    }
   }
   __syncthreads();
   if (threadIdx.x < kSmClasses && part[threadIdx.x] != 0) atomicAdd(&ctr[threadIdx.x], part[threadIdx.x]);
 }
 
 __global__ void __launch_bounds__(256)
-    softmax_index_kernel(const int32_t* __restrict__ offsets, int n, int nh,
+    softmax_index_kernel(const int32_t* __restrict__ offsets, int n, int nh, int causal,
                          unsigned long long* __restrict__ ctr, long long* __restrict__ seq_base,
                          int32_t* __restrict__ row_seq) {
   __shared__ long long seg[kSmClasses];
@@ -393,35 +419,44 @@ __global__ void __launch_bounds__(256)
   const int lane = threadIdx.x & 31;
   for (int i = blockIdx.x * 8 + (threadIdx.x >> 5); i < n; i += gridDim.x * 8) {
     const int L = offsets[i + 1] - offsets[i];
-    const int k = softmax_class_of(L);
-    const long long cnt = static_cast<long long>(nh) * L;
-    long long base = 0;
-    if (lane == 0)
-      base = seg[k] + static_cast<long long>(atomicAdd(&ctr[kSmClasses + k], static_cast<unsigned long long>(cnt)));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    if (lane == 0) seq_base[i] = base;
-    for (long long r = lane; r < cnt; r += 32) row_seq[base + r] = i;
+    // one stretch per class the sequence's rows fall in: its own class, or
+    // when causal every class of a row length 1..L
+    for (int k = causal ? 0 : softmax_class_of(L); k <= softmax_class_of(L); ++k) {
+      const ClassRun cr = softmax_class_run(L, k, causal);
+      if (cr.run == 0) continue;
+      const long long cnt = static_cast<long long>(nh) * cr.run;
+      long long base = 0;
+      if (lane == 0)
+        base = seg[k] + static_cast<long long>(atomicAdd(&ctr[kSmClasses + k], static_cast<unsigned long long>(cnt)));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (lane == 0) seq_base[static_cast<long long>(i) * kSmClasses + k] = base;
+      for (long long r = lane; r < cnt; r += 32) row_seq[base + r] = i;
+    }
   }
 }
 
-// The sequence a lane's rows belong to: its index, the start of its stretch
-// in the class-ordered row space, its length and score offset.  Kept across
+// The sequence a lane's rows belong to: the start of its stretch in the
+// class-ordered row space, the stretch's rows per head (run, from row r_lo
+// of each head block), its length and score offset.  Kept across
 // iterations so that a lane walking consecutive rows looks a sequence up
 // only when it crosses into the next one.
 struct SeqCache {
   long long b = 0;             // stretch [b, b + rows)
-  int rows = 0, L = 0;
+  int rows = 0, L = 0, r_lo = 0, run = 1;
+  float inv_run = 1.f;
   long long soff = 0;
 };
 
-// Rows [R0, R0 + U) of the class-ordered row space (those below Re): their
-// addresses and lengths (length 0 for none).
+// Rows [R0, R0 + U) of class k's row space (those below Re): their addresses
+// and lengths (length 0 for none).  A stretch row rr is row r_lo + rr % run
+// of head rr / run (the quotient from a float reciprocal, corrected: exact
+// for rr < 2^24).
 template <typename T, int U>
 __device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ offsets,
                                               const int64_t* __restrict__ s_off,
                                               const long long* __restrict__ seq_base,
                                               const int32_t* __restrict__ row_seq, long long R0,
-                                              long long Re, int n, int nh, int causal,
+                                              long long Re, int n, int nh, int causal, int k,
                                               SeqCache& sc, T* (&row)[U], int (&len)[U]) {
 #pragma unroll
   for (int u = 0; u < U; ++u) {
@@ -433,17 +468,37 @@ __device__ __forceinline__ void class_rows_at(T* S, const int32_t* __restrict__ 
     const long long R = R0 + u;
     if (R < Re) {
       if (R < sc.b || R - sc.b >= sc.rows) {                 // another sequence's stretch
-        const int i = row_seq[R];
+        // the index is rewritten by every call's index kernel: read it from L2
+        const int i = __ldcg(row_seq + R);
         if (!in_bounds(i >= 0 && i < n)) return;
-        sc.b = seq_base[i];
+        sc.b = __ldcg(seq_base + static_cast<long long>(i) * kSmClasses + k);
         sc.L = offsets[i + 1] - offsets[i];
-        sc.rows = nh * sc.L;
+        const ClassRun cr = softmax_class_run(sc.L, k, causal);
+        sc.r_lo = cr.r_lo;
+        sc.run = cr.run > 0 ? cr.run : 1;
+        sc.inv_run = 1.0f / static_cast<float>(sc.run);
+        sc.rows = nh * cr.run;
         sc.soff = s_off[i];
       }
-      const long long rr = R - sc.b;                         // row inside the sequence's block
+      const int rr = static_cast<int>(R - sc.b);             // row inside the stretch
       if (!in_bounds(sc.L >= 1 && rr >= 0 && rr < sc.rows)) return;
-      len[u] = causal ? static_cast<int>(rr % sc.L) + 1 : sc.L;
-      row[u] = S + sc.soff + rr * ((sc.L + 7) & ~7);
+      if (!causal) {
+        len[u] = sc.L;
+        row[u] = S + sc.soff + static_cast<long long>(rr) * ((sc.L + 7) & ~7);
+      } else {
+        int h = __float2int_rz(static_cast<float>(rr) * sc.inv_run);
+        int r = rr - h * sc.run;
+        if (r < 0) {
+          --h;
+          r += sc.run;
+        } else if (r >= sc.run) {
+          ++h;
+          r -= sc.run;
+        }
+        r += sc.r_lo;
+        len[u] = r + 1;
+        row[u] = S + sc.soff + static_cast<long long>(h * sc.L + r) * ((sc.L + 7) & ~7);
+      }
     }
   }
 }
@@ -467,31 +522,28 @@ __device__ __forceinline__ void sm_cp_wait() {
 }
 
 // One class: lane groups of G lanes, U consecutive rows (of the class-ordered
-// row space) each.  Each warp walks one contiguous stretch of the class's
-// rows (an equal share of its warp-iterations), so consecutive iterations of
-// a lane group stay inside one sequence's rows and its address arithmetic
+// row space) each; a warp-iteration takes 32 / G * U consecutive rows.  The
+// warp runs iterations [it, it_end) of the class: consecutive iterations of
+// a lane group stay inside one sequence's rows, so its address arithmetic
 // needs no lookup (the class-ordered row space keeps a sequence's rows
 // together).  The loop bound is uniform across a warp (groups past the end
 // get empty rows): the group reductions are warp shuffles.  bf16 rows are
 // loaded kSmStages - 1 iterations ahead into the warp's shared-memory ring.
+template <int G, int U>
+__host__ __device__ constexpr long long class_rows_per_iter() {
+  return static_cast<long long>(32 / G) * U;
+}
 template <typename T, int G, int MAXC, int U>
 __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restrict__ offsets,
                                                    const int64_t* __restrict__ s_off,
                                                    const long long* __restrict__ seq_base,
                                                    const int32_t* __restrict__ row_seq,
-                                                   long long Rb, long long Re, int n, int nh,
-                                                   int causal, uint32_t ring) {
-  if (Rb >= Re) return;
-  const int lane = threadIdx.x & 31, sub = lane % G;
-  constexpr int kGpw = 32 / G;
-  constexpr long long GU = static_cast<long long>(kGpw) * U;   // rows per warp-iteration
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const long long iters = (Re - Rb + GU - 1) / GU;
-  const long long per = (iters + warps - 1) / warps;
-  long long it = w * per;
-  const long long it_end = min(iters, it + per);
+                                                   long long Rb, long long Re, long long it,
+                                                   long long it_end, int n, int nh, int causal,
+                                                   int k, uint32_t ring) {
   if (it >= it_end) return;                                  // uniform across the warp
+  const int lane = threadIdx.x & 31, sub = lane % G;
+  constexpr long long GU = class_rows_per_iter<G, U>();      // rows per warp-iteration
   const long long lane_off = static_cast<long long>(lane / G) * U;
   SeqCache sc;
   int len[U];
@@ -506,7 +558,7 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
       int il[U];
       T* ir[U];
       class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + t * GU + lane_off, Re, n, nh,
-                          causal, sci, ir, il);
+                          causal, k, sci, ir, il);
       const int st = static_cast<int>(t & (D - 1));
 #pragma unroll
       for (int u = 0; u < U; ++u)
@@ -526,7 +578,7 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
       sm_cp_commit();
       sm_cp_wait<D - 1>();                                   // iteration it has landed
       class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
-                          causal, sc, row, len);
+                          causal, k, sc, row, len);
       const int st = static_cast<int>(it & (D - 1));
       uint32_t w4[U][MAXC][4];
 #pragma unroll
@@ -553,12 +605,12 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
     sm_cp_wait<0>();
   } else {
     class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
-                        causal, sc, row, len);
+                        causal, k, sc, row, len);
     for (;;) {
       softmax_group<T, G, MAXC, U>(row, len, sub);
       if (++it >= it_end) break;
       class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
-                          causal, sc, row, len);
+                          causal, k, sc, row, len);
     }
   }
 }
@@ -582,11 +634,31 @@ __global__ void __launch_bounds__(kSmClassThreads, 3)
   // class's chunks and MAXC three or four: a lane holds up to four chunks of
   // one row, so the per-row work (addresses, masks, reductions) is spread
   // over up to 32 entries; rows of one or two chunks take four or two rows
-  // per lane
-#define RM_SM_PASS(k, G, MAXC, U)                                                               \
-  if (k_max >= k)                                                                              \
-    softmax_class_pass<T, G, MAXC, U>(S, offsets, s_off, seq_base, row_seq, seg[k], seg[k + 1], n, \
-                                      nh, causal, ring)
+  // per lane.  Each class's warp-iterations are split evenly over all warps,
+  // one contiguous share each (laying the classes end to end and cutting
+  // that sequence into equal shares measured slower on B200: 2..100 scores
+  // 67% -> 28% of HBM, causal 50% -> 24%).
+  constexpr long long kRpi[kSmClasses] = {
+      class_rows_per_iter<1, 4>(),  class_rows_per_iter<1, 2>(),  class_rows_per_iter<1, 1>(),
+      class_rows_per_iter<2, 1>(),  class_rows_per_iter<2, 1>(),  class_rows_per_iter<4, 1>(),
+      class_rows_per_iter<4, 1>(),  class_rows_per_iter<8, 1>(),  class_rows_per_iter<8, 1>(),
+      class_rows_per_iter<16, 1>(), class_rows_per_iter<16, 1>(), class_rows_per_iter<32, 1>(),
+      class_rows_per_iter<32, 1>()};
+  long long ibase[kSmClasses + 1];
+  ibase[0] = 0;
+#pragma unroll
+  for (int k = 0; k < kSmClasses; ++k)
+    ibase[k + 1] = ibase[k] + (k <= k_max ? (seg[k + 1] - seg[k] + kRpi[k] - 1) / kRpi[k] : 0);
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+#define RM_SM_PASS(k, G, MAXC, U)                                                                \
+  if (k_max >= k) {                                                                             \
+    const long long nit = ibase[k + 1] - ibase[k];                                              \
+    const long long pk = (nit + warps - 1) / warps;                                             \
+    softmax_class_pass<T, G, MAXC, U>(S, offsets, s_off, seq_base, row_seq, seg[k], seg[k + 1],  \
+                                      w * pk < nit ? w * pk : nit, (w + 1) * pk < nit ? (w + 1) * pk : nit, \
+                                      n, nh, causal, k, ring);                                  \
+  }
   RM_SM_PASS(0, 1, 1, 4);
   RM_SM_PASS(1, 1, 2, 2);
   RM_SM_PASS(2, 1, 4, 1);
@@ -1498,6 +1570,16 @@ cudaError_t softmax_classes_launch(void* S, int s_dtype, const int32_t* offsets,
   if (n_seqs == 0 || T == 0) return cudaSuccess;
   if (max_len < 1 || max_len > 1024) return cudaErrorInvalidValue;
   const SoftmaxIndexLayout lay(n_seqs, static_cast<long long>(n_heads) * T);
+  // The count, index and class kernels run in plain stream order (no
+  // programmatic dependent launch), each after the previous kernel has
+  // completed.  With all three launched programmatically after the scores
+  // kernel, rm_score on B200 gave rows of P that had not been normalised
+  // (decoder, materialised attention, wrong in some calls and not in others);
+  // with either the class kernel or the two index kernels in plain order the
+  // scores matched the oracle in every call.  Every kernel of the chain waits
+  // (griddepcontrol.wait) before it touches global memory; the cause was not
+  // isolated.
+  PdlScope plain(false);
   uint8_t* base = static_cast<uint8_t*>(scratch);
   unsigned long long* ctr = reinterpret_cast<unsigned long long*>(base);
   long long* seq_base = reinterpret_cast<long long*>(base + lay.base);
@@ -1505,10 +1587,11 @@ cudaError_t softmax_classes_launch(void* S, int s_dtype, const int32_t* offsets,
   cudaError_t e = cudaMemsetAsync(ctr, 0, 16 * kSmClasses, st);
   if (e != cudaSuccess) return e;
   const int seq_blocks = std::max(1, std::min((n_seqs + 255) / 256, num_sms * 4));
-  launch_k(softmax_count_kernel, dim3(seq_blocks), dim3(256), 0, st, offsets, n_seqs, n_heads, ctr);
+  launch_k(softmax_count_kernel, dim3(seq_blocks), dim3(256), 0, st, offsets, n_seqs, n_heads, causal,
+           ctr);
   const int idx_blocks = std::max(1, std::min((n_seqs + 7) / 8, num_sms * 8));
-  launch_k(softmax_index_kernel, dim3(idx_blocks), dim3(256), 0, st, offsets, n_seqs, n_heads, ctr,
-           seq_base, row_seq);
+  launch_k(softmax_index_kernel, dim3(idx_blocks), dim3(256), 0, st, offsets, n_seqs, n_heads, causal,
+           ctr, seq_base, row_seq);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int k_max = softmax_class_of(max_len);
