@@ -758,6 +758,7 @@ def kernel_bench(args):
     pk, pk_kind = peaks()
     st = torch.cuda.Stream()
     reps = max(3, args.steps)
+    only = set(args.only.split(",")) if args.only else set()
     out = {"metric": "HBM GB/s of the softmax and residual+LayerNorm kernels alone",
            "unit": "GB/s", "peak_hbm_gbs": pk["hbm_gbs"], "peak_source": f"hbm_gbs of {pk_kind}",
            "kernels": {}}
@@ -787,6 +788,8 @@ def kernel_bench(args):
             lens.append(L)
             tot += nh * L * ((L + 7) // 8 * 8)
         lens = np.array(lens)
+        if only and label not in only and label + "_batchwide" not in only:
+            continue                             # the lengths are drawn all the same
         off = synth.offsets_from_lengths(lens)
         rb, so = rm.ops.varlen_meta(off, nh)
         S = torch.randn(int(so[-1]), dtype=torch.bfloat16, device="cuda")
@@ -803,6 +806,8 @@ def kernel_bench(args):
                                                        int(lens.max()), causal, scratch, st)),
                 (label + "_batchwide", lambda: rm.ops.softmax(S, rm.BF16, d_off, d_so, n, T, nh,
                                                               int(lens.max()), causal, st))):
+            if only and name not in only:
+                continue
             ms = timed(fn)
             out["kernels"][name] = {"ms": ms, "algorithmic_GB": gb, "gbs": gb / (ms * 1e-3),
                                     "frac_of_measured": gb / (ms * 1e-3) / pk["hbm_gbs"],
@@ -810,6 +815,8 @@ def kernel_bench(args):
         del scratch
         del S
     for label, H, T, mode in (("res_ln_post_H768", 768, 1 << 20, 0), ("res_ln_pre_H2048", 2048, 1 << 18, 1)):
+        if only and label not in only:
+            continue
         y = torch.randn(T, H, dtype=torch.bfloat16, device="cuda")
         x = torch.randn(T, H, dtype=torch.bfloat16, device="cuda")
         z = torch.empty_like(x) if mode == 1 else None
@@ -1239,6 +1246,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--clocks-dir", default=None,
                     help="also write the raw clock samples of the timed region as CSV here")
+    ap.add_argument("--only", default="",
+                    help="with --kernel-bench: comma-separated entries to run (e.g. softmax_len2_100)")
     ap.add_argument("--kernel-bench", action="store_true",
                     help="time the softmax and residual+LayerNorm kernels alone on GB-scale inputs")
     ap.add_argument("--fuse", type=int, default=8,
