@@ -18,6 +18,10 @@ inside the timed region.  Multi-GPU (torchrun): independent replicas, one
 stream per rank, no collective on the data path (weak scaling); the time is
 the max over ranks.
 
+`repeats` holds five timed regions of this process; `processes` repeats the
+measurement in independent processes (default five in total, one after
+another on the same GPU), each reporting its first timed region.
+
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same stream (rank 0 only).
 """
@@ -738,11 +742,36 @@ def b200_arm(args):
                                             f"one by the fp64 numpy oracle ({el:.1f} s)"}
     if world == 1 and args.batch_index is None and not args.no_extra and name == "bert-base-len2-100":
         result["other_workloads"] = secondary_workloads(args, torch, rm)
+    if world == 1 and args.batch_index is None and args.processes > 1:
+        result["processes"] = process_repeats(args, name, value)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if dist is not None:
         dist.destroy_process_group()
     return 0
+
+
+def process_repeats(args, name, first):
+    """The same measurement repeated in independent processes (fresh CUDA
+    context, weights and arena each), run one after another on this GPU once
+    this process is idle: the value of each process's first timed region,
+    with this process's as the first."""
+    vals, errors = [first], []
+    cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(args.steps),
+           "--warmup", str(args.warmup), "--fuse", str(args.fuse), "--lanes", str(args.lanes),
+           "--repeats", "1", "--processes", "1", "--no-extra", "--no-cpu-baseline"]
+    for _ in range(args.processes - 1):
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        try:
+            vals.append(float(json.loads(r.stdout.strip().splitlines()[-1])["value"]))
+        except (ValueError, IndexError, KeyError):
+            errors.append(f"exit {r.returncode}: {r.stderr.strip().splitlines()[-1:] or ''}")
+    out = dict(stat_summary(vals), unit=UNIT,
+               method=f"{len(vals)} independent processes, each: {args.warmup} warm-up and "
+                      f"{args.steps} timed steps, one timed region; 95% t-interval of the mean")
+    if errors:
+        out["errors"] = errors
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -1237,6 +1266,9 @@ def main():
                          "timed regions (0 = off; the kernel table always comes from a separate step)")
     ap.add_argument("--repeats", type=int, default=5,
                     help="timed regions of --steps steps each (median and 95%% interval reported)")
+    ap.add_argument("--processes", type=int, default=5,
+                    help="also repeat the measurement in this many independent processes in total "
+                         "(this one included; 1 = none)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads (lengths 5-500, GPT-1.3B shape, TinyBERT batch 1)")
     ap.add_argument("--extra-steps", type=int, default=3, help="timed steps of each other workload")
