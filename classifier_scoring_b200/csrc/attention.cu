@@ -554,7 +554,13 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
     // this lane's chunk k of stage st
     auto slot = [&](int st, int k) { return ring + static_cast<uint32_t>((st * kSmChunks + k) * 512); };
     SeqCache sci;                                            // the issuing side's sequence
-    auto issue = [&](long long t) {
+    // With one row per lane group the issuing side's row address and length
+    // are kept for the computing side, D iterations deep (a register queue
+    // shifted once per iteration); with more rows per group they are
+    // recomputed (the queue would cost 3 * D * U registers).
+    T* qrow[D];
+    int qlen[D];
+    auto issue = [&](long long t, int q) {
       int il[U];
       T* ir[U];
       class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + t * GU + lane_off, Re, n, nh,
@@ -567,18 +573,36 @@ __device__ __forceinline__ void softmax_class_pass(T* S, const int32_t* __restri
           const int col = (c * G + sub) * 8;
           if (col < il[u]) sm_cp16(slot(st, u * MAXC + c), ir[u] + col);
         }
+      if (U == 1) {
+        qrow[q] = ir[0];
+        qlen[q] = il[0];
+      }
     };
 #pragma unroll
-    for (int k = 0; k < D - 1; ++k) {
-      if (it + k < it_end) issue(it + k);
+    for (int q = 0; q < D - 1; ++q) {
+      qrow[q] = S;
+      qlen[q] = 0;
+      if (it + q < it_end) issue(it + q, q);
       sm_cp_commit();
     }
     for (; it < it_end; ++it) {
-      if (it + D - 1 < it_end) issue(it + D - 1);
+      qrow[D - 1] = S;
+      qlen[D - 1] = 0;
+      if (it + D - 1 < it_end) issue(it + D - 1, D - 1);
       sm_cp_commit();
       sm_cp_wait<D - 1>();                                   // iteration it has landed
-      class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n, nh,
-                          causal, k, sc, row, len);
+      if (U == 1) {
+        row[0] = qrow[0];
+        len[0] = qlen[0];
+#pragma unroll
+        for (int q = 0; q < D - 1; ++q) {
+          qrow[q] = qrow[q + 1];
+          qlen[q] = qlen[q + 1];
+        }
+      } else {
+        class_rows_at<T, U>(S, offsets, s_off, seq_base, row_seq, Rb + it * GU + lane_off, Re, n,
+                            nh, causal, k, sc, row, len);
+      }
       const int st = static_cast<int>(it & (D - 1));
       uint32_t w4[U][MAXC][4];
 #pragma unroll
