@@ -107,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "rm_varlen_meta": (ctypes.c_int, [P, I32, I32, P, P]),
         "rm_op_gemm": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_gemm_tiled": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P]),
+        "rm_op_gemm_accumulate": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, I32, I32, P]),
         "rm_gemm_tile": (ctypes.c_int, [I32, I32, I32, I32, P]),
         "rm_op_vote": (ctypes.c_int, [P, I32, I32, F, P, P, P]),
         "rm_op_embed": (ctypes.c_int, [P, P, I32, I32, P, P, P, P, F, I32, I32, I32, P, I32, P, P]),
@@ -295,6 +296,11 @@ class ops:
     def gemm_tiled(x, w, bias, y, y_dtype, M, N, K, act=0, cg=0, bn=0, stream=None):
         _check(lib().rm_op_gemm_tiled(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), y_dtype, M, N, K,
                                       act, cg, bn, _stream(stream)))
+
+    @staticmethod
+    def gemm_accumulate(x, w, bias, y, y_dtype, M, N, K, act=0, cg=0, bn=0, stream=None):
+        _check(lib().rm_op_gemm_accumulate(_ptr(x), _ptr(w), _ptr(bias), _ptr(y), y_dtype, M, N,
+                                           K, act, cg, bn, _stream(stream)))
 
     @staticmethod
     def vote(scores, K, n, threshold=0.0, decision=None, votes=None, stream=None):

@@ -390,11 +390,16 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
   // output maps cover the bucket's Tb rows (the buffers' extent): the rows of
   // a call's last 128-row tile past its T tokens land in their own buffer's
   // padding rows, which no later step reads
+  // (y1, y2: the encoder's sublayer outputs; the decoder adds its sublayer
+  // outputs straight into its fp32 residual stream and has neither, so its
+  // maps stand in for them unused)
   const bool dec = c->arch == RM_DEC_PRELN;
+  const int64_t y1 = dec ? b.plan.off[B_F] : b.plan.off[B_Y1];
+  const int64_t y2 = dec ? b.plan.off[B_F] : b.plan.off[B_Y2];
   if (!make_tmap_store(&b.y_qkv, base + b.plan.off[B_QKV], Tb, 3 * c->hidden, false, &why) ||
-      !make_tmap_store(&b.y_o, base + b.plan.off[B_Y1], Tb, c->hidden, dec, &why) ||
+      !make_tmap_store(&b.y_o, base + y1, Tb, c->hidden, false, &why) ||
       !make_tmap_store(&b.y_f, base + b.plan.off[B_F], Tb, c->ffn, false, &why) ||
-      !make_tmap_store(&b.y_2, base + b.plan.off[B_Y2], Tb, c->hidden, dec, &why))
+      !make_tmap_store(&b.y_2, base + y2, Tb, c->hidden, false, &why))
     return set_error(RM_E_CUDA, "output tensor map: %s", why);
   h->max_peak = std::max(h->max_peak, b.plan.peak);
   auto res = h->buckets.emplace(key, b);
@@ -402,12 +407,14 @@ int get_bucket(rm_handle* h, int64_t T, int64_t S, Bucket** out) {
   return RM_OK;
 }
 
+// y: the output map; yacc (when not null, act 0 and out_f32 only): the fp32
+// [M][N] tensor the product is added to instead (y then unused)
 int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCount], int M, int N,
          int K, const float* bias, const CUtensorMap& y, int act, cudaStream_t st,
-         bool out_f32 = false) {
+         bool out_f32 = false, void* yacc = nullptr) {
   const GemmTile tile = gemm_pick(M, N, K, h->num_sms, act);
-  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], y, tile, M, N, K, bias, out_f32,
-                              act, h->d_err, h->num_sms, st);
+  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], y, yacc, tile, M, N, K, bias,
+                              out_f32, act, h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return RM_OK;
 }
@@ -607,9 +614,9 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
   bf16* qkv = reinterpret_cast<bf16*>(base + bk->plan.off[B_QKV]);
   bf16* s = reinterpret_cast<bf16*>(base + bk->plan.off[B_S]);
   bf16* ctx = reinterpret_cast<bf16*>(base + bk->plan.off[B_CTX]);
-  bf16* y1 = reinterpret_cast<bf16*>(base + bk->plan.off[B_Y1]);
+  bf16* y1 = reinterpret_cast<bf16*>(base + bk->plan.off[B_Y1]);   // encoder only
   bf16* f = reinterpret_cast<bf16*>(base + bk->plan.off[B_F]);
-  bf16* y2 = reinterpret_cast<bf16*>(base + bk->plan.off[B_Y2]);
+  bf16* y2 = reinterpret_cast<bf16*>(base + bk->plan.off[B_Y2]);   // encoder only
   const int H = c->hidden, F = c->ffn, nh = c->n_heads, d = H / nh;
   const int act = c->gelu == RM_GELU_TANH ? 2 : 1;
   const bool dec = c->arch == RM_DEC_PRELN;
@@ -627,7 +634,6 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
   auto gemm_bytes = [&](double N, double K, double out_bytes = 2.0) {
     return 2.0 * (Td * K + N * K) + out_bytes * Td * N;
   };
-  const double y_bytes = dec ? 4.0 : 2.0;   // the decoder's sublayer outputs are fp32
   const double att_flops = 2.0 * att * d;            // one of the two contractions
   const double sm_bytes = 4.0 * att;                 // bf16 read + write per admitted entry
   const double ctx_bytes = 2.0 * att + 2.0 * Td * Hd * 2;   // P, V, ctx
@@ -661,8 +667,8 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
               res_ln_launch(nullptr, x, z, h->layers[0].ln1_g, h->layers[0].ln1_b, T, H, eps,
                             ln_dtype, 2, st, pf_qkv0));
   // algorithmic bytes per token: post-LN reads y, x and writes x (bf16); the
-  // decoder reads y and x (fp32), writes x (fp32) and z (bf16)
-  const double ln_bytes = (dec ? 14.0 : 6.0) * Td * Hd;
+  // decoder reads x (fp32, the sublayer output already added) and writes z (bf16)
+  const double ln_bytes = 6.0 * Td * Hd;
   for (int l = 0; l < c->n_layers; ++l) {
     const LayerW& L = h->layers[l];
     const L2Prefetch pf_o = pf_of(L.w_o, w_o_b, nullptr, 0);
@@ -696,10 +702,9 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
       RM_KERNEL(RM_K_CONTEXT, att_flops, ctx_bytes,
                 attn_context_launch(s, qkv, ctx, d_off, d_rb, d_so, n, nrb, nh, d, dec, st));
     }
-    // the decoder's sublayer outputs stay fp32 up to the fp32 residual add
-    RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd, y_bytes),
-            gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, bk->y_o, 0, st, dec));
     if (!dec) {
+      RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd),
+              gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, bk->y_o, 0, st));
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
                 res_ln_launch(y1, x, nullptr, L.ln1_g, L.ln1_b, T, H, eps, ln_dtype, 0, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
@@ -709,17 +714,22 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
                 res_ln_launch(y2, x, nullptr, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 0, st, pf_next));
     } else {
+      // The output projection and FFN2 add their outputs straight into the
+      // fp32 residual stream x (in L2, each sum rounded once to fp32, as the
+      // separate addition would round it); the LayerNorm after each reads x.
+      RM_GEMM(gemm_flops(Hd, Hd), gemm_bytes(Hd, Hd, 8.0),
+              gemm(h, bk->a_ctx, L.tm[1], T, H, H, L.b_o, bk->y_o, 0, st, true, x));
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y1, x, z, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 1, st, pf_ffn));
+                res_ln_launch(nullptr, x, z, L.ln2_g, L.ln2_b, T, H, eps, ln_dtype, 2, st, pf_ffn));
       RM_GEMM(gemm_flops(Fd, Hd), gemm_bytes(Fd, Hd),
               gemm(h, bk->a_in, L.tm[2], T, F, H, L.b_1, bk->y_f, act, st));
-      RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd, y_bytes),
-              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, bk->y_2, 0, st, true));
+      RM_GEMM(gemm_flops(Hd, Fd), gemm_bytes(Hd, Fd, 8.0),
+              gemm(h, bk->a_f, L.tm[3], T, H, F, L.b_2, bk->y_2, 0, st, true, x));
       const bool last = l + 1 == c->n_layers;
       const float* g = last ? h->lnf_g : h->layers[l + 1].ln1_g;
       const float* b = last ? h->lnf_b : h->layers[l + 1].ln1_b;
       RM_KERNEL(RM_K_LAYERNORM, 0, ln_bytes,
-                res_ln_launch(y2, x, z, g, b, T, H, eps, ln_dtype, 1, st, pf_next));
+                res_ln_launch(nullptr, x, z, g, b, T, H, eps, ln_dtype, 2, st, pf_next));
     }
   }
   RM_KERNEL(RM_K_HEAD, 2.0 * n * Hd, 2.0 * n * Hd + 4.0 * n,
@@ -1152,13 +1162,17 @@ int rm_op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t
   return rm_op_gemm_tiled(x, w, bias, y, y_dtype, M, N, K, act, 0, 0, stream);
 }
 
-int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
-                     int32_t M, int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn,
-                     void* stream) {
+namespace {
+// rm_op_gemm_tiled and rm_op_gemm_accumulate: store the product into y, or
+// add it to y
+int op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype, int32_t M,
+            int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn, bool accumulate,
+            void* stream) {
   if (x == nullptr || w == nullptr || y == nullptr) return set_error(RM_E_INVAL, "NULL argument");
   if (M < 1 || N < 8 || K < 8 || N % 8 != 0 || K % 8 != 0)
     return set_error(RM_E_INVAL, "need M >= 1 and N, K positive multiples of 8");
-  if (act < 0 || act > 2 || (y_dtype != RM_F32 && y_dtype != RM_BF16))
+  if (act < 0 || act > 2 || (y_dtype != RM_F32 && y_dtype != RM_BF16) ||
+      (accumulate && (act != 0 || y_dtype != RM_F32)))
     return set_error(RM_E_INVAL, "bad act or y_dtype");
   if ((reinterpret_cast<uintptr_t>(y) & 15) != 0 || (reinterpret_cast<uintptr_t>(bias) & 15) != 0)
     return set_error(RM_E_INVAL, "y and bias must be 16-byte aligned");
@@ -1180,9 +1194,22 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
     return set_error(RM_E_INVAL, "tensor map: %s", why);
   int32_t* err = nullptr;
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
-  RM_LAUNCH(gemm_launch(ta, tb, ty, tile, M, N, K, bias, y_dtype == RM_F32, act, err, sms,
-                        static_cast<cudaStream_t>(stream)));
+  RM_LAUNCH(gemm_launch(ta, tb, ty, accumulate ? y : nullptr, tile, M, N, K, bias,
+                        y_dtype == RM_F32, act, err, sms, static_cast<cudaStream_t>(stream)));
   return RM_OK;
+}
+}  // namespace
+
+int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, int32_t y_dtype,
+                     int32_t M, int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn,
+                     void* stream) {
+  return op_gemm(x, w, bias, y, y_dtype, M, N, K, act, cg, bn, false, stream);
+}
+
+int rm_op_gemm_accumulate(const void* x, const void* w, const float* bias, void* y,
+                          int32_t y_dtype, int32_t M, int32_t N, int32_t K, int32_t act,
+                          int32_t cg, int32_t bn, void* stream) {
+  return op_gemm(x, w, bias, y, y_dtype, M, N, K, act, cg, bn, true, stream);
 }
 
 int rm_op_vote(const float* scores, int32_t K, int32_t n, float threshold, int32_t* decision,

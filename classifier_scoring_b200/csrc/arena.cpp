@@ -32,8 +32,9 @@ void sizes(int arch, int H, int F, int64_t T, int64_t s_elems, ArenaPlan& p) {
   p.bytes[B_QKV] = align_up(T * 3 * H * row, kArenaAlign);
   p.bytes[B_S] = align_up(s_elems * row, kArenaAlign);
   p.bytes[B_CTX] = align_up(T * H * row, kArenaAlign);
-  // the decoder's sublayer outputs y stay fp32 up to the residual add
-  const int64_t yrow = arch == RM_DEC_PRELN ? 4 : row;
+  // the decoder's output projection and FFN2 add into its fp32 x: no buffer
+  // for their outputs
+  const int64_t yrow = arch == RM_DEC_PRELN ? 0 : row;
   p.bytes[B_Y1] = align_up(T * H * yrow, kArenaAlign);
   p.bytes[B_F] = align_up(T * F * row, kArenaAlign);
   p.bytes[B_Y2] = align_up(T * H * yrow, kArenaAlign);

@@ -1,7 +1,9 @@
 // Y[M][N] = act(X[M][K] . W[N][K]^T + bias) on the 5th-generation tensor
 // cores: the QKV, attention-output and FFN projections of the scorer (the
 // "BLAS routines" of the TurboTransformers abstract, on tensor cores as its
-// proposed-method section does; here bf16 in, fp32 accumulation).
+// proposed-method section does; here bf16 in, fp32 accumulation).  With an
+// fp32 accumulation target the tile is added to Y instead (Y += X.W^T + bias),
+// which folds a residual add into the projection that produces its addend.
 //
 // Persistent, warp-specialised kernel: one CTA per SM (CG = 1) or one CTA pair
 // per two SMs (CG = 2) walks the (128*CG) x BN output tiles t = unit,
@@ -23,7 +25,9 @@
 //                      GELU) -- tcgen05.ld (warp w reads TMEM lanes
 //                      32*(w%4)..+31 = tile rows), + bias, optional GELU, into
 //                      swizzled 32 x 32 boxes in shared memory that one lane
-//                      writes out with bulk tensor stores (TMA), then release
+//                      writes out with bulk tensor stores (TMA), or, when
+//                      accumulating into fp32, row-contiguous boxes that every
+//                      lane adds to its row of Y with a bulk reduction; then release
 //                      the accumulator.  The epilogue of tile i overlaps the
 //                      mainloop of tile i+1.
 // Every mbarrier wait is bounded (about 2 s of %globaltimer); a wait that
@@ -126,7 +130,8 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmY, int M, int N, int K,
-                        const float* __restrict__ bias, int* __restrict__ err, int n_fastest) {
+                        const float* __restrict__ bias, int* __restrict__ err, int n_fastest,
+                        void* __restrict__ yacc) {
   constexpr int EW = epi_warps(ACT);
   using L = GemmSmem<BN, CG, EW, OUT_F32 ? 4 : 2>;
   constexpr int S = L::kStages;
@@ -354,32 +359,71 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
           // this buffer's previous box has been read out by its store
           const int buf = NB == 1 ? 0 : (nst & 1);
           if (nst >= NB) {
-            if (lane == 0) bulk_wait_group_read<NB - 1>();
+            bulk_wait_group_read<NB - 1>();      // no-op in lanes without copies in flight
             __syncwarp();
           }
           uint8_t* box = stg0 + buf * L::kBoxBytes;
-          if (OUT_F32) {
-            // 128-byte rows, 128-byte swizzle: 16-byte chunk j of row r at j ^ (r % 8)
+          if (ACT == 0 && OUT_F32 && yacc != nullptr) {
+            // Y += the tile: each lane adds its own row's 32 columns with one
+            // bulk reduction in L2 (fp32 adds: the sum is rounded once, as a
+            // separate addition would round it), so the row stays contiguous
+            // (no swizzle).  The
+            // lane writes its 16-byte chunks in an order rotated by its
+            // position, which spreads each quarter warp over all banks.
+            constexpr int NCH = 8;
+            uint4 ch[NCH];
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) =
-                  make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
-                             __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-          } else {
-            // 64-byte rows, 64-byte swizzle: 16-byte chunk j of row r at j ^ ((r / 2) % 4)
+            for (int j = 0; j < NCH; ++j)
+              ch[j] = make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                                 __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+            const int key = lane & 7;
+            // rotate left by key (register indices stay compile-time)
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
-                  make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]), pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                             pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                             pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-          }
-          // the box's generic-proxy writes before the async-proxy store reads them
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, smem_u32(box), n0 + c, row0);
+            for (int bit = 1; bit < NCH; bit <<= 1) {
+              const bool rot = (key & bit) != 0;
+              uint4 t[NCH];
+#pragma unroll
+              for (int j = 0; j < NCH; ++j) t[j] = rot ? ch[(j + bit) % NCH] : ch[j];
+#pragma unroll
+              for (int j = 0; j < NCH; ++j) ch[j] = t[j];
+            }
+            uint8_t* row = box + lane * (NCH * 16);
+#pragma unroll
+            for (int j = 0; j < NCH; ++j)
+              *reinterpret_cast<uint4*>(row + (((j + key) % NCH) << 4)) = ch[j];
+            fence_proxy_async_smem();
+            const int grow = row0 + lane, gcol = n0 + c;
+            if (grow < M) {
+              const int cols = N - gcol < 32 ? N - gcol : 32;   // a multiple of 8
+              float* dst = static_cast<float*>(yacc) + static_cast<size_t>(grow) * N + gcol;
+              bulk_reduce_add_f32(dst, smem_u32(row), cols * 4);
+            }
             bulk_commit_group();
+          } else {
+            if (OUT_F32) {
+              // 128-byte rows, 128-byte swizzle: 16-byte chunk j of row r at j ^ (r % 8)
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4*>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                    make_uint4(__float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                               __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+            } else {
+              // 64-byte rows, 64-byte swizzle: 16-byte chunk j of row r at j ^ ((r / 2) % 4)
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                    make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
+                               pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                               pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                               pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+            }
+            // the box's generic-proxy writes before the async-proxy store reads them
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, smem_u32(box), n0 + c, row0);
+              bulk_commit_group();
+            }
           }
           ++nst;
           c = cn;
@@ -395,7 +439,7 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
       }
     }
     // every store of this warp has finished before the CTA's shared memory goes
-    if (lane == 0) bulk_wait_group<0>();
+    bulk_wait_group<0>();
   }
   __syncwarp();
   tc_fence_before();
@@ -418,8 +462,9 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
 // Host side
 // ---------------------------------------------------------------------------
 template <int BN, int CG, int ACT, bool OUT_F32>
-cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, int M,
-                       int N, int K, const float* bias, int* err, int num_sms, cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, void* yacc,
+                       int M, int N, int K, const float* bias, int* err, int num_sms,
+                       cudaStream_t st) {
   using L = GemmSmem<BN, CG, epi_warps(ACT), OUT_F32 ? 4 : 2>;
   auto kern = gemm_bf16_tc_kernel<BN, CG, ACT, OUT_F32>;
   cudaLaunchConfig_t cfg = {};
@@ -469,21 +514,21 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   cfg.numAttrs = na;
   // the activations (A, M rows) are at least as large as the weights (B, N rows)
   const int n_fastest = M >= N ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, a, b, y, M, N, K, bias, err, n_fastest);
+  return cudaLaunchKernelEx(&cfg, kern, a, b, y, M, N, K, bias, err, n_fastest, yacc);
 }
 
 template <int BN, int CG>
-cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, int M,
-                       int N, int K, const float* bias, bool out_f32, int act, int* err,
+cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, void* yacc,
+                       int M, int N, int K, const float* bias, bool out_f32, int act, int* err,
                        int num_sms, cudaStream_t st) {
   if (out_f32) {
-    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, y, M, N, K, bias, err, num_sms, st);
-    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, y, M, N, K, bias, err, num_sms, st);
-    return launch_one<BN, CG, 0, true>(a, b, y, M, N, K, bias, err, num_sms, st);
+    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
+    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
+    return launch_one<BN, CG, 0, true>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
   }
-  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, y, M, N, K, bias, err, num_sms, st);
-  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, y, M, N, K, bias, err, num_sms, st);
-  return launch_one<BN, CG, 0, false>(a, b, y, M, N, K, bias, err, num_sms, st);
+  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
+  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
+  return launch_one<BN, CG, 0, false>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
 }
 
 }  // namespace
@@ -522,10 +567,10 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms, int act) {
 }
 
 cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y,
-                        GemmTile tile, int M, int N, int K, const float* bias, bool out_f32,
-                        int act, int* err, int num_sms, cudaStream_t st) {
+                        void* yacc, GemmTile tile, int M, int N, int K, const float* bias,
+                        bool out_f32, int act, int* err, int num_sms, cudaStream_t st) {
 #define RM_GEMM_TILE(cg, bn) \
-  case bn: return launch_act<bn, cg>(a, b, y, M, N, K, bias, out_f32, act, err, num_sms, st)
+  case bn: return launch_act<bn, cg>(a, b, y, yacc, M, N, K, bias, out_f32, act, err, num_sms, st)
   if (tile.cg == 2) {
     switch (tile.bn) {
       RM_GEMM_TILE(2, 128);

@@ -30,6 +30,7 @@ int schedule_dp(const SchedCost& cost, const int32_t* lengths, int32_t n, int32_
 //   0 LN1 (decoder)  1 QKV GEMM  2 scores  3 softmax  4 context  5 out-proj GEMM
 //   6 residual+LN   7 FFN1 GEMM  8 FFN2 GEMM  9 residual+LN
 // x (and z for the decoder) live through every step; the rest are planned.
+// The decoder's out-proj and FFN2 add into x, so its y1 and y2 take no bytes.
 enum Buf { B_X = 0, B_Z, B_QKV, B_S, B_CTX, B_Y1, B_F, B_Y2, B_COUNT };
 struct ArenaPlan {
   int64_t off[B_COUNT] = {0};

@@ -26,10 +26,13 @@ cudaError_t bounded_wait_selftest(unsigned long long limit_ns, int* d_timed_out,
 inline int gemm_tile_index(int box_rows) { return (box_rows - 64) / 32; }
 // a: bf16 [M][K] map with box {64, 128}; b: bf16 [N][K] map with box {64, tile.b_box()};
 // y: [>= M][N] output map of make_tmap_store (fp32 when out_f32, else bf16).
+// yacc: nullptr to store the tile through y; else (act 0 and out_f32 only)
+// the 16-byte aligned row-major fp32 [M][N] tensor that the tile is added to
+// in L2 (each sum rounded once to fp32); y is then not used.
 // Persistent grid of min(tiles, num_sms / cg) units of cg CTAs.
 cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y,
-                        GemmTile tile, int M, int N, int K, const float* bias, bool out_f32,
-                        int act, int* err, int num_sms, cudaStream_t st);
+                        void* yacc, GemmTile tile, int M, int N, int K, const float* bias,
+                        bool out_f32, int act, int* err, int num_sms, cudaStream_t st);
 
 // ---- TMA descriptors (tma.cpp) ----
 // 2-D bf16 row-major [rows][cols] tensor, box {64 cols, box_rows}, 128-byte swizzle,

@@ -59,6 +59,20 @@ int rm_op_gemm_tiled(const void* x, const void* w, const float* bias, void* y, i
                      int32_t M, int32_t N, int32_t K, int32_t act, int32_t cg, int32_t bn,
                      void* stream);
 
+/* Y[M][N] += X[M][K] . W[N][K]^T + bias[N] with Y in fp32: the pre-LN
+ * decoder's output projection and FFN2 added straight into its fp32 residual
+ * stream (the residual additions of the layer equations, which the
+ * TurboTransformers abstract pairs with the LayerNorm batch reduction; here
+ * folded into the GEMM that produces the addend).  The tile is accumulated in
+ * fp32 and added to y in L2; each element of y is added to exactly once, with
+ * one fp32 rounding, so the result equals a separate fp32 addition of the
+ * rm_op_gemm output and does not depend on the order of the tiles.  Same
+ * arguments as rm_op_gemm_tiled with y_dtype = RM_F32 and act = 0 (RM_E_INVAL
+ * for any other); y must be 16-byte aligned and is read and written. */
+int rm_op_gemm_accumulate(const void* x, const void* w, const float* bias, void* y,
+                          int32_t y_dtype, int32_t M, int32_t N, int32_t K, int32_t act,
+                          int32_t cg, int32_t bn, void* stream);
+
 /* Majority vote of an ensemble of K scorer replicas ("experts"), the SambaNova
  * blog's accuracy section (Figs. 4-5: several TinyBERT instances vote on each
  * input).  scores: device float[K][n], expert k's score of input i at

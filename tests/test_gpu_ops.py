@@ -110,6 +110,54 @@ def test_gemm_every_tile(cg, bn, shape, out):
     assert bool(torch.isnan(buf[M:]).all())
 
 
+# Y += X.W^T + b with Y in fp32 (the decoder's residual add folded into its
+# output projection and FFN2): every tile, ragged and projection shapes.  Y
+# starts from seeded values; rows past M (the rest of the buffer) must keep
+# theirs bit for bit.  Each element is added to once, so the result equals the
+# stored product added in fp32 (the unfolded path) and repeats bit for bit.
+@pytest.mark.parametrize("cg,bn", GEMM_TILES, ids=[f"cg{c}-bn{b}" for c, b in GEMM_TILES])
+@pytest.mark.parametrize("shape", ["ragged", "proj"])
+def test_gemm_accumulate_every_tile(cg, bn, shape):
+    M, N, K = (555, 2 * bn + 40, 200) if shape == "ragged" else (3328, 768, 768)
+    g = torch.Generator().manual_seed(cg * 1000 + bn + M + 1)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    b = torch.randn(N, generator=g, dtype=torch.float32) * 0.1
+    y0 = torch.randn(M + 300, N, generator=g) * 2.0
+    X, W, B = f64(x), f64(w), f64(b)
+    ref = O.linear(X, W, B)
+    scale = np.abs(X) @ np.abs(W).T + np.abs(B)
+    Y0 = f64(y0[:M])
+    xd, wd, bd = x.cuda(), w.cuda(), b.cuda()
+    runs = []
+    for _ in range(2):
+        buf = y0.cuda()
+        rm.ops.gemm_accumulate(xd, wd, bd, buf[:M], rm.F32, M, N, K, 0, cg, bn)
+        torch.cuda.synchronize()
+        runs.append(buf)
+    buf = runs[0]
+    # the tile's fp32 accumulation, then one fp32 rounding of the sum
+    err = np.abs(f64(buf[:M]) - (Y0 + ref))
+    bound = 2.0 ** -24 * np.abs(Y0 + ref) + F32_RTOL * scale * (1.0 + 2.0 ** -23)
+    assert np.all(err <= bound), float(np.nanmax(err / bound))
+    assert torch.equal(buf[M:].cpu(), y0[M:])
+    assert torch.equal(runs[0], runs[1])
+    # the same as storing the product and adding it in fp32
+    prod = torch.empty(M, N, dtype=torch.float32, device="cuda")
+    rm.ops.gemm_tiled(xd, wd, bd, prod, rm.F32, M, N, K, 0, cg, bn)
+    torch.cuda.synchronize()
+    assert torch.equal(buf[:M], y0[:M].cuda() + prod)
+
+
+def test_gemm_accumulate_takes_fp32_without_activation_only():
+    x = torch.zeros(16, 16, dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros(16, 16, dtype=torch.float32, device="cuda")
+    with pytest.raises(rm.RmError):
+        rm.ops.gemm_accumulate(x, x, None, y, rm.F32, 16, 16, 16, 1)
+    with pytest.raises(rm.RmError):
+        rm.ops.gemm_accumulate(x, x, None, x, rm.BF16, 16, 16, 16, 0)
+
+
 def test_gemm_rejects_bad_shapes():
     x = torch.zeros(16, 12, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(rm.RmError):
