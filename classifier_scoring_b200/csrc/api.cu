@@ -413,8 +413,10 @@ int gemm(rm_handle* h, const CUtensorMap& a, const CUtensorMap (&b)[kGemmTileCou
          int K, const float* bias, const CUtensorMap& y, int act, cudaStream_t st,
          bool out_f32 = false, void* yacc = nullptr) {
   const GemmTile tile = gemm_pick(M, N, K, h->num_sms, act);
-  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())], y, yacc, tile, M, N, K, bias,
-                              out_f32, act, h->d_err, h->num_sms, st);
+  const int split = gemm_tail_split(tile, M, N, h->num_sms);
+  cudaError_t e = gemm_launch(a, b[gemm_tile_index(tile.b_box())],
+                              b[gemm_tile_index(tile.b_box() / split)], y, yacc, tile, M, N, K,
+                              bias, out_f32, act, h->d_err, h->num_sms, st);
   if (e != cudaSuccess) return set_error(RM_E_CUDA, "gemm launch: %s", cudaGetErrorString(e));
   return RM_OK;
 }
@@ -1187,14 +1189,16 @@ int op_gemm(const void* x, const void* w, const float* bias, void* y, int32_t y_
   RM_CUDA(cudaGetDevice(&dev));
   RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
   const GemmTile tile = cg != 0 ? GemmTile{cg, bn} : gemm_pick(M, N, K, sms, act);
-  CUtensorMap ta, tb, ty;
+  const int split = gemm_tail_split(tile, M, N, sms);
+  CUtensorMap ta, tb, tbs, ty;
   const char* why = "";
   if (!make_tmap_bf16(&ta, x, M, K, 128, &why) || !make_tmap_bf16(&tb, w, N, K, tile.b_box(), &why) ||
+      !make_tmap_bf16(&tbs, w, N, K, tile.b_box() / split, &why) ||
       !make_tmap_store(&ty, y, M, N, y_dtype == RM_F32, &why))
     return set_error(RM_E_INVAL, "tensor map: %s", why);
   int32_t* err = nullptr;
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
-  RM_LAUNCH(gemm_launch(ta, tb, ty, accumulate ? y : nullptr, tile, M, N, K, bias,
+  RM_LAUNCH(gemm_launch(ta, tb, tbs, ty, accumulate ? y : nullptr, tile, M, N, K, bias,
                         y_dtype == RM_F32, act, err, sms, static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }

@@ -129,9 +129,10 @@ template <int BN, int CG, int ACT, bool OUT_F32>
 __global__ void __launch_bounds__(gemm_threads(ACT), 1)
     gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB2,
                         const __grid_constant__ CUtensorMap tmY, int M, int N, int K,
                         const float* __restrict__ bias, int* __restrict__ err, int n_fastest,
-                        void* __restrict__ yacc) {
+                        void* __restrict__ yacc, int full, int split) {
   constexpr int EW = epi_warps(ACT);
   using L = GemmSmem<BN, CG, EW, OUT_F32 ? 4 : 2>;
   constexpr int S = L::kStages;
@@ -155,6 +156,27 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
   // M fastest: they share a few B column panels.
   auto m_blk = [&](int t) { return n_fastest ? t / tiles_n : t % tiles_m; };
   auto n_blk = [&](int t) { return n_fastest ? t % tiles_n : t / tiles_m; };
+  // Work items: tiles 0..full-1 whole, then each remaining tile (the last,
+  // partial round of the persistent grid) as `split` slices of BN/split
+  // columns, so that SMs that would idle in that round take a slice each
+  // (1-CTA tiles only; a slice loads its own narrower box of B, tmB2).  Not
+  // with the tanh GELU, whose epilogue has no registers to spare.
+  if (ACT == 2) {
+    split = 1;
+    full = tiles;
+  }
+  const int cols_split = BN / split;
+  const int works = full + (tiles - full) * split;
+  auto work_tile = [&](int w, int& t, int& c0) {
+    if (w < full) {
+      t = w;
+      c0 = 0;
+      return BN;
+    }
+    t = full + (w - full) / split;
+    c0 = ((w - full) % split) * cols_split;
+    return cols_split;
+  };
   const int nk = (K + BK - 1) / BK;
   const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S),
                  accf0 = smem_u32(bars + 2 * S), acce0 = smem_u32(bars + 2 * S + 2);
@@ -199,9 +221,12 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
       // ---- TMA producer ----
       int it = 0;
       bool ok = true;
-      for (int t = unit; t < tiles && ok; t += units) {
+      for (int w = unit; w < works && ok; w += units) {
+        int t, c0;
+        const int cols = work_tile(w, t, c0);
         const int m0 = m_blk(t) * BM * CG + static_cast<int>(rank) * BM;
-        const int nb0 = n_blk(t) * BN + static_cast<int>(rank) * (BN / CG);
+        const int nb0 = n_blk(t) * BN + c0 + static_cast<int>(rank) * (BN / CG);
+        const bool whole = cols == BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = (it / S) & 1;
@@ -212,9 +237,9 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
           }
           const uint32_t dA = smem_u32(smem + s * L::kStage), dB = dA + L::kA;
           if (CG == 1) {
-            mbar_arrive_expect_tx(full0 + 8 * s, L::kStage);
+            mbar_arrive_expect_tx(full0 + 8 * s, whole ? L::kStage : L::kA + cols * BK * 2);
             tma_load_2d(dA, &tmA, kb * BK, m0, full0 + 8 * s);
-            tma_load_2d(dB, &tmB, kb * BK, nb0, full0 + 8 * s);
+            tma_load_2d(dB, whole ? &tmB : &tmB2, kb * BK, nb0, full0 + 8 * s);
           } else {
             // the leader expects the bytes of both CTAs on its own barrier
             if (rank == 0) mbar_arrive_expect_tx(full0 + 8 * s, 2 * L::kStage);
@@ -240,10 +265,13 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
   } else if (warp == 1) {
     if (lane == 0 && rank == 0) {
       // ---- MMA issuer (the leader issues for the pair) ----
-      constexpr uint32_t idesc = idesc_bf16_f32(BM * CG, BN);
+      constexpr uint32_t idesc_whole = idesc_bf16_f32(BM * CG, BN);
+      const uint32_t idesc_slice = idesc_bf16_f32(BM * CG, cols_split);
       int it = 0, local = 0;
       bool ok = true;
-      for (int t = unit; t < tiles && ok; t += units, ++local) {
+      for (int w = unit; w < works && ok; w += units, ++local) {
+        int t, c0;
+        const uint32_t idesc = work_tile(w, t, c0) == BN ? idesc_whole : idesc_slice;
         const int acc = local & 1, use = local >> 1;
         if (use > 0 && !mbar_wait(acce0 + 8 * acc, (use - 1) & 1)) {
           atomicAdd(err + ERR_TIMEOUT, 1);
@@ -306,7 +334,9 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
     uint8_t* stg0 = smem + L::kEpiOff + ew * NB * L::kBoxBytes;
     int nst = 0;                                 // boxes this warp has stored
     int local = 0;
-    for (int t = unit; t < tiles; t += units, ++local) {
+    for (int w = unit; w < works; w += units, ++local) {
+      int t, c0;
+      const int cols = work_tile(w, t, c0);
       const int acc = local & 1, use = local >> 1;
       const bool ready = mbar_wait(accf0 + 8 * acc, use & 1);
       if (!__all_sync(0xffffffffu, ready)) {
@@ -315,14 +345,14 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
       }
       tc_fence_after();
       const int m0 = m_blk(t) * BM * CG + static_cast<int>(rank) * BM;
-      const int n0 = n_blk(t) * BN;
+      const int n0 = n_blk(t) * BN + c0;
       const int row0 = m0 + q * 32;
       const uint32_t base = tmem + lane_base + static_cast<uint32_t>(acc) * (kTmemCols / 2);
       if (row0 < M) {                            // uniform across the warp
         // TMEM loads run one round ahead: round c+1's columns are in flight
         // while round c's values go through the bias, GELU and the store
         int c = h0 * 32;
-        bool have = c < BN && n0 + c < N;        // uniform across the warp
+        bool have = c < cols && n0 + c < N;      // uniform across the warp
         uint32_t r[32];
         if (have) tmem_ld_32cols(base + c, r);
         while (have) {
@@ -344,7 +374,7 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
                 f32x2_pack(b4[g].z, b4[g].w));
           }
           const int cn = c + NH * 32;
-          const bool next = cn < BN && n0 + cn < N;
+          const bool next = cn < cols && n0 + cn < N;
           if (next) tmem_ld_32cols(base + cn, r);
           float v[32];
 #pragma unroll
@@ -462,9 +492,9 @@ __global__ void __launch_bounds__(gemm_threads(ACT), 1)
 // Host side
 // ---------------------------------------------------------------------------
 template <int BN, int CG, int ACT, bool OUT_F32>
-cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, void* yacc,
-                       int M, int N, int K, const float* bias, int* err, int num_sms,
-                       cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b_split,
+                       const CUtensorMap& y, void* yacc, int M, int N, int K, const float* bias,
+                       int* err, int num_sms, cudaStream_t st) {
   using L = GemmSmem<BN, CG, epi_warps(ACT), OUT_F32 ? 4 : 2>;
   auto kern = gemm_bf16_tc_kernel<BN, CG, ACT, OUT_F32>;
   cudaLaunchConfig_t cfg = {};
@@ -504,7 +534,13 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   int max_units = num_sms / CG;
   if (CG == 2 && setup.resident_units > 0 && setup.resident_units < max_units)
     max_units = setup.resident_units;
-  cfg.gridDim = dim3(CG * (tiles < max_units ? tiles : max_units));
+  // the last partial round's tiles as column slices (1-CTA tiles, not with
+  // the tanh GELU)
+  const int split = CG == 1 && ACT != 2 ? gemm_tail_split(GemmTile{CG, BN}, M, N, num_sms) : 1;
+  const int rem = tiles >= max_units ? tiles % max_units : tiles;
+  const int full = split > 1 ? tiles - rem : tiles;
+  const int works = full + (tiles - full) * split;
+  cfg.gridDim = dim3(CG * (works < max_units ? works : max_units));
   if (g_pdl) {
     attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[na].val.programmaticStreamSerializationAllowed = 1;
@@ -514,21 +550,22 @@ cudaError_t launch_one(const CUtensorMap& a, const CUtensorMap& b, const CUtenso
   cfg.numAttrs = na;
   // the activations (A, M rows) are at least as large as the weights (B, N rows)
   const int n_fastest = M >= N ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, a, b, y, M, N, K, bias, err, n_fastest, yacc);
+  return cudaLaunchKernelEx(&cfg, kern, a, b, b_split, y, M, N, K, bias, err, n_fastest, yacc,
+                            full, split);
 }
 
 template <int BN, int CG>
-cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y, void* yacc,
-                       int M, int N, int K, const float* bias, bool out_f32, int act, int* err,
-                       int num_sms, cudaStream_t st) {
+cudaError_t launch_act(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& bs,
+                       const CUtensorMap& y, void* yacc, int M, int N, int K, const float* bias,
+                       bool out_f32, int act, int* err, int num_sms, cudaStream_t st) {
   if (out_f32) {
-    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
-    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
-    return launch_one<BN, CG, 0, true>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
+    if (act == 1) return launch_one<BN, CG, 1, true>(a, b, bs, y, yacc, M, N, K, bias, err, num_sms, st);
+    if (act == 2) return launch_one<BN, CG, 2, true>(a, b, bs, y, yacc, M, N, K, bias, err, num_sms, st);
+    return launch_one<BN, CG, 0, true>(a, b, bs, y, yacc, M, N, K, bias, err, num_sms, st);
   }
-  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
-  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
-  return launch_one<BN, CG, 0, false>(a, b, y, yacc, M, N, K, bias, err, num_sms, st);
+  if (act == 1) return launch_one<BN, CG, 1, false>(a, b, bs, y, yacc, M, N, K, bias, err, num_sms, st);
+  if (act == 2) return launch_one<BN, CG, 2, false>(a, b, bs, y, yacc, M, N, K, bias, err, num_sms, st);
+  return launch_one<BN, CG, 0, false>(a, b, bs, y, yacc, M, N, K, bias, err, num_sms, st);
 }
 
 }  // namespace
@@ -566,11 +603,27 @@ GemmTile gemm_pick(int M, int N, int K, int num_sms, int act) {
   return best;
 }
 
-cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y,
-                        void* yacc, GemmTile tile, int M, int N, int K, const float* bias,
-                        bool out_f32, int act, int* err, int num_sms, cudaStream_t st) {
-#define RM_GEMM_TILE(cg, bn) \
-  case bn: return launch_act<bn, cg>(a, b, y, yacc, M, N, K, bias, out_f32, act, err, num_sms, st)
+int gemm_tail_split(GemmTile tile, int M, int N, int num_sms) {
+  if (tile.cg != 1 || num_sms < 1) return 1;
+  const long long tiles = ((M + 127LL) / 128) * ((N + tile.bn - 1LL) / tile.bn);
+  const long long rem = tiles >= num_sms ? tiles % num_sms : tiles;
+  if (rem == 0) return 1;
+  for (int f : {4, 2}) {
+    if (tile.bn % f != 0 || rem * f > num_sms) continue;
+    for (int i = 0; i < kGemmTileCount; ++i)
+      if (kGemmTileWidths[i] == tile.bn / f) return f;
+  }
+  return 1;
+}
+
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b_split,
+                        const CUtensorMap& y, void* yacc, GemmTile tile, int M, int N, int K,
+                        const float* bias, bool out_f32, int act, int* err, int num_sms,
+                        cudaStream_t st) {
+#define RM_GEMM_TILE(cg, bn)                                                                  \
+  case bn:                                                                                    \
+    return launch_act<bn, cg>(a, b, b_split, y, yacc, M, N, K, bias, out_f32, act, err, num_sms, \
+                              st)
   if (tile.cg == 2) {
     switch (tile.bn) {
       RM_GEMM_TILE(2, 128);

@@ -29,10 +29,16 @@ inline int gemm_tile_index(int box_rows) { return (box_rows - 64) / 32; }
 // yacc: nullptr to store the tile through y; else (act 0 and out_f32 only)
 // the 16-byte aligned row-major fp32 [M][N] tensor that the tile is added to
 // in L2 (each sum rounded once to fp32); y is then not used.
-// Persistent grid of min(tiles, num_sms / cg) units of cg CTAs.
-cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& y,
-                        void* yacc, GemmTile tile, int M, int N, int K, const float* bias,
-                        bool out_f32, int act, int* err, int num_sms, cudaStream_t st);
+// Persistent grid of units of cg CTAs, each walking its share of the tiles.
+// With 1-CTA tiles, the tiles of a last partial round (or of a single round
+// that fills at most half of the SMs) are cut into gemm_tail_split column
+// slices of bn / split columns each; b_split is the weights' map with boxes
+// of bn / split rows (b itself when the split is 1).
+int gemm_tail_split(GemmTile tile, int M, int N, int num_sms);
+cudaError_t gemm_launch(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b_split,
+                        const CUtensorMap& y, void* yacc, GemmTile tile, int M, int N, int K,
+                        const float* bias, bool out_f32, int act, int* err, int num_sms,
+                        cudaStream_t st);
 
 // ---- TMA descriptors (tma.cpp) ----
 // 2-D bf16 row-major [rows][cols] tensor, box {64 cols, box_rows}, 128-byte swizzle,

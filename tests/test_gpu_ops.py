@@ -158,6 +158,33 @@ def test_gemm_accumulate_takes_fp32_without_activation_only():
         rm.ops.gemm_accumulate(x, x, None, x, rm.BF16, 16, 16, 16, 0)
 
 
+# The tiles of the persistent grid's last, partial round run as 2 or 4 column
+# slices each when the slices fit the idle SMs.  Shapes where that happens on
+# a 148-SM B200 (widths 256 -> 4 slices of 64, 192 -> 2 of 96, 128 -> 2 of 64;
+# and a single round of few tiles), against the oracle and bit for bit against
+# 64-column tiles, which are never sliced: an element's value does not depend
+# on the tile or slice it was computed in.
+@pytest.mark.parametrize("bn,M,N,K", [(256, 20000, 768, 320), (192, 19000, 768, 256),
+                                      (128, 9700, 768, 192), (256, 1000, 1000, 200)])
+def test_gemm_tail_slices(bn, M, N, K):
+    g = torch.Generator().manual_seed(bn + M)
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16)
+    w = (torch.randn(N, K, generator=g) * 0.05).to(torch.bfloat16)
+    b = torch.randn(N, generator=g, dtype=torch.float32) * 0.1
+    xd, wd, bd = x.cuda(), w.cuda(), b.cuda()
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    y64 = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    rm.ops.gemm_tiled(xd, wd, bd, y, rm.F32, M, N, K, 0, 1, bn)
+    rm.ops.gemm_tiled(xd, wd, bd, y64, rm.F32, M, N, K, 0, 1, 64)
+    torch.cuda.synchronize()
+    X, W, B = f64(x), f64(w), f64(b)
+    ref = O.linear(X, W, B)
+    scale = np.abs(X) @ np.abs(W).T + np.abs(B)
+    err = np.abs(f64(y) - ref)
+    assert np.all(err <= F32_RTOL * scale), float(np.nanmax(err / (F32_RTOL * scale)))
+    assert torch.equal(y, y64)
+
+
 def test_gemm_rejects_bad_shapes():
     x = torch.zeros(16, 12, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(rm.RmError):
