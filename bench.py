@@ -406,6 +406,17 @@ class StreamExecutor:
             lat[self.b_seq[b]:self.b_seq[b + 1]] = per_batch[b] + first_done
         return float(np.median(lat)), float(np.percentile(lat, 99))
 
+    def cupti_step(self, sc):
+        """The same single-stream step without events, its kernels timed by CUPTI."""
+        def run():
+            for b in range(self.nb):
+                sc.score(self.ids_dev[self.b_tok[b]:], self.b_off[b], self.out_dev[self.b_seq[b]:],
+                         self.stream)
+        try:
+            return cupti_kernel_times(self.torch, run)
+        except Exception as e:                      # a profiler that cannot start
+            return {"error": f"{type(e).__name__}: {e}"}
+
     def profiled_step(self, sc):
         """One step on a single stream with per-launch CUDA events (after timing)."""
         sc.profile(1)
@@ -416,6 +427,45 @@ class StreamExecutor:
         prof = sc.profile_read()
         sc.profile(0)
         return prof
+
+
+# kernel name fragment -> the library's kernel kind (KERNEL_NAMES)
+CUPTI_KINDS = (("gemm_bf16_tc_kernel", "gemm"), ("res_ln_kernel", "layernorm"),
+               ("attn_tc_kernel", "attn_fused"), ("attn_tile_kernel", "attn_fused"),
+               ("attn_fused", "attn_fused"), ("attn_scores_kernel", "attn_scores"),
+               ("attn_context_kernel", "attn_context"), ("softmax", "softmax"),
+               ("embed_kernel", "embed"), ("head_kernel", "head"), ("best_of_n_kernel", "head"))
+
+
+def cupti_kernel_times(torch, run):
+    """Each kernel's share of the device timeline of run() (one stream), by
+    kind, from CUPTI activity records (torch.profiler): a launch's end minus
+    the later of its start and the previous kernel's end.  With programmatic
+    dependent launch a kernel starts while its predecessor runs and waits for
+    it, so its own start-to-end time would count that wait; its share does
+    not, and no event sits between two launches.  None where the profiler has
+    no CUDA activity."""
+    from torch.autograd import DeviceType
+    from torch.profiler import ProfilerActivity, profile
+    if ProfilerActivity.CUDA not in torch.profiler.supported_activities():
+        return None
+    with profile(activities=[ProfilerActivity.CUDA]) as p:
+        run()
+        torch.cuda.synchronize()
+    ks = sorted(((e.time_range.start, e.time_range.end, e.name) for e in p.events()
+                 if e.device_type == DeviceType.CUDA), key=lambda k: k[0])
+    out = {}
+    prev_end = None
+    for start, end, name in ks:
+        share = end - (start if prev_end is None else max(start, prev_end))
+        prev_end = end if prev_end is None else max(prev_end, end)
+        kind = next((k for frag, k in CUPTI_KINDS if frag in name), None)
+        if kind is None:
+            continue
+        d = out.setdefault(kind, {"launches": 0, "us": 0.0})
+        d["launches"] += 1
+        d["us"] += max(0.0, float(share))
+    return out
 
 
 def launches_of(lanes):
@@ -620,6 +670,8 @@ def b200_arm(args):
     p50, p99 = ex.latency(elapsed_ms / args.steps)
     # kernel table and roofline from one extra single-stream step after timing
     prof = ex.profiled_step(sc)
+    # and the same step's kernels timed by CUPTI, without per-launch events
+    cup = ex.cupti_step(sc)
 
     # ---- end to end through rm_score_host (pinned host buffers) ----
     b_tok, b_seq, b_off = ex.b_tok, ex.b_seq, ex.b_off
@@ -699,6 +751,16 @@ def b200_arm(args):
         if d["bytes"]:
             e["gbs"] = d["bytes"] / (d["ms"] * 1e-3) / 1e9
             e["hbm_frac_of_measured"] = e["gbs"] / pk["hbm_gbs"]
+        c = (cup or {}).get(kname)
+        if isinstance(c, dict) and c["launches"] == d["launches"] and c["us"] > 0:
+            # the same launches' shares of the device timeline (CUPTI), no events between them
+            cu = {"avg_us": c["us"] / c["launches"]}
+            if "tflops" in e:
+                cu["tflops"] = d["flops"] / (c["us"] * 1e-6) / 1e12
+            if d["bytes"]:
+                cu["gbs"] = d["bytes"] / (c["us"] * 1e-6) / 1e9
+                cu["hbm_frac_of_measured"] = cu["gbs"] / pk["hbm_gbs"]
+            e["cupti"] = cu
         kernels[kname] = e
 
     rep_vals = [whole_job_rate(world, n_req, args.steps, m) for m in max_rep]
@@ -717,6 +779,13 @@ def b200_arm(args):
         "tokens_per_step": int(b_tok[-1]),
         "roofline": roofline,
         "kernels": kernels,
+        "kernels_method": "avg_us, gbs, tflops: per-launch CUDA events in one single-stream step after "
+                          "the timed regions (an event between two launches ends their programmatic "
+                          "overlap, so short kernels read slow); cupti: in a second such step without "
+                          "events, each launch's share of the device timeline from CUPTI activity "
+                          "records (its end minus the later of its start and the previous kernel's end)"
+                          + ("" if not (isinstance(cup, dict) and "error" in cup)
+                             else f" (unavailable: {cup['error']})"),
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": "rm_score_host, pinned host ids/scores"},
         "gpu_launches": int(launches),
