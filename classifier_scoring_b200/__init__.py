@@ -121,6 +121,8 @@ def lib() -> ctypes.CDLL:
         "rm_op_attn_tiles": (ctypes.c_int, [P, P, P, I32, I32, I32, I32, I32, I32, P]),
         "rm_attn_tc_tiles": (ctypes.c_int, [P, I32, P]),
         "rm_op_attn_tc": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
+        "rm_attn_tcl_items": (ctypes.c_int, [P, I32, I32, P]),
+        "rm_op_attn_tcl": (ctypes.c_int, [P, P, P, P, I32, I32, I32, I32, I32, P]),
         "rm_op_res_ln": (ctypes.c_int, [P, P, P, P, P, I32, I32, F, I32, I32, P]),
         "rm_op_head": (ctypes.c_int, [P, P, I32, P, F, I32, I32, P, P]),
         "rm_arena_plan": (ctypes.c_int, [cfgp, I32, I32, I64, P, P, P, P, I32, P]),
@@ -372,6 +374,20 @@ class ops:
         out = np.zeros(n + 1, dtype=np.int32)
         k = _check(lib().rm_attn_tc_tiles(off.ctypes.data, n, out.ctypes.data))
         return out[:k + 1].copy()
+
+    @staticmethod
+    def attn_tcl_items(offsets, causal=0):
+        """rm_attn_tcl_items: host offsets -> int32 work items of the long-row kernel."""
+        off = _i32(offsets)
+        n = len(off) - 1
+        out = np.zeros(4 * n, dtype=np.int32)
+        k = _check(lib().rm_attn_tcl_items(off.ctypes.data, n, causal, out.ctypes.data))
+        return out[:k].copy()
+
+    @staticmethod
+    def attn_tcl(qkv, ctx, offsets_dev, items_dev, n_items, n_seqs, T, n_heads, causal, stream=None):
+        _check(lib().rm_op_attn_tcl(_ptr(qkv), _ptr(ctx), _ptr(offsets_dev), _ptr(items_dev), n_items,
+                                    n_seqs, T, n_heads, causal, _stream(stream)))
 
     @staticmethod
     def attn_tc(qkv, ctx, offsets_dev, tiles_dev, n_tiles, n_seqs, T, n_heads, causal, stream=None):

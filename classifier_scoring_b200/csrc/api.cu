@@ -235,7 +235,7 @@ struct MetaLayout {
     rb = align_up(4 * (n + 1), 16);
     so = rb + align_up(4 * (n + 1), 16);
     tl = so + align_up(8 * (n + 1), 16);
-    base = tl + align_up(4 * (n + 1), 16);
+    base = tl + align_up(4 * (4 * n + 1), 16);   // tiles (n + 1) or long-row items (<= 4n)
     pst = base;
     pln = pst + align_up(4 * n, 16);
     oix = pln + align_up(4 * n, 16);
@@ -484,7 +484,8 @@ struct ProfScope {
 struct CallInfo {
   int32_t n = 0, T = 0, nrb = 0, Lmax = 0;
   int32_t ntc = 0;                   // tensor-core attention tiles (0: that kernel does not apply)
-  const int32_t* d_tl = nullptr;
+  int32_t ntcl = 0;                  // or its long-row work items (0: does not apply)
+  const int32_t* d_tl = nullptr;     // the tiles or the items
   int64_t S = 0;
   double att = 0;   // attention entries the mask admits, summed over heads
   const int32_t* d_off = nullptr;
@@ -515,6 +516,13 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
 // the head dim is 64 and no sequence is longer than its 128-row tiles.
 bool tc_attention_applies(const rm_config* c, int32_t max_len, bool prefix) {
   return !prefix && c->attn_impl == RM_ATTN_FUSED && c->hidden / c->n_heads == 64 && max_len <= 128;
+}
+// Its long-row form takes the other plain encoder calls with head dim 64 and
+// sequences of up to 512 tokens (causal calls measured faster on the
+// packed-row tiles, which skip the keys past each row in 16-key steps).
+bool tcl_attention_applies(const rm_config* c, int32_t max_len, bool prefix) {
+  return !prefix && c->attn_impl == RM_ATTN_FUSED && c->hidden / c->n_heads == 64 &&
+         c->arch != RM_DEC_PRELN && max_len > 128 && max_len <= 512;
 }
 
 // host_ids != NULL: copy the ids host->device (into the arena) once the call
@@ -551,8 +559,12 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   RM_TRY(host_varlen_meta(offsets, n, c->n_heads, p_rb, p_so, &Lmax));
   const int32_t nrb = p_rb[n];
   const int64_t S = p_so[n];
+  const bool dec_c = c->arch == RM_DEC_PRELN;
   const int32_t ntc =
       tc_attention_applies(c, Lmax, px != nullptr) ? attn_tc_tiles(offsets, n, reinterpret_cast<int32_t*>(ps + ml.tl)) : 0;
+  const int32_t ntcl = tcl_attention_applies(c, Lmax, px != nullptr)
+                           ? attn_tcl_items(offsets, n, dec_c ? 1 : 0, reinterpret_cast<int32_t*>(ps + ml.tl))
+                           : 0;
   if (host_ids != nullptr) {
     RM_CUDA(cudaMemcpyAsync(h->d_ids, host_ids, 4 * static_cast<size_t>(T), cudaMemcpyHostToDevice, st));
     d_ids = h->d_ids;
@@ -579,6 +591,7 @@ int score_impl(rm_handle* h, const int32_t* d_ids, const int32_t* host_ids, cons
   ci.nrb = nrb;
   ci.Lmax = Lmax;
   ci.ntc = ntc;
+  ci.ntcl = ntcl;
   ci.d_tl = reinterpret_cast<const int32_t*>(h->d_meta + ml.tl);
   ci.S = S;
   ci.att = attention_entries(c, offsets, n, px);
@@ -687,6 +700,11 @@ int enqueue_forward(rm_handle* h, const CallInfo& ci, const int32_t* d_ids, floa
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
                 attn_tc_launch(qkv, ctx, d_off, ci.d_tl, ci.ntc, n, T, nh, dec, h->d_err,
                                h->num_sms, st, pf_o));
+    } else if (ci.ntcl > 0) {
+      // its long-row form: 128-row query tiles of one sequence (head dim 64, L <= 512)
+      RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
+                attn_tcl_launch(qkv, ctx, d_off, ci.d_tl, ci.ntcl, n, T, nh, dec, h->d_err,
+                                h->num_sms, st, pf_o));
     } else if (c->attn_impl == RM_ATTN_FUSED && (d == 64 || d == 128)) {
       // packed-row tiles (head dims 64 and 128); other head dims below
       RM_KERNEL(RM_K_ATTN_FUSED, 2.0 * att_flops, 2.0 * Td * 3 * Hd + 2.0 * Td * Hd,
@@ -970,6 +988,10 @@ int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_
   const int32_t ntc = tc_attention_applies(c, Lmax, false)
                           ? attn_tc_tiles(seq_offsets, n, reinterpret_cast<int32_t*>(meta.data() + ml.tl))
                           : 0;
+  const int32_t ntcl = tcl_attention_applies(c, Lmax, false)
+                           ? attn_tcl_items(seq_offsets, n, c->arch == RM_DEC_PRELN ? 1 : 0,
+                                            reinterpret_cast<int32_t*>(meta.data() + ml.tl))
+                           : 0;
   Bucket* bk = nullptr;
   RM_TRY(get_bucket(h, T, p_so[n], &bk));   // the arena placement and tensor maps, made now
   rm_plan* p = new rm_plan();
@@ -988,6 +1010,7 @@ int rm_plan_create(rm_handle* h, const int32_t* seq_offsets, int32_t n_seqs, rm_
   ci.nrb = p_rb[n];
   ci.Lmax = Lmax;
   ci.ntc = ntc;
+  ci.ntcl = ntcl;
   ci.d_tl = reinterpret_cast<const int32_t*>(p->d_meta + ml.tl);
   ci.S = p_so[n];
   ci.att = attention_entries(c, seq_offsets, n, nullptr);
@@ -1362,6 +1385,34 @@ int rm_op_attn_tc(const void* qkv, void* ctx, const int32_t* offsets, const int3
   RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
   RM_LAUNCH(attn_tc_launch(qkv, ctx, offsets, tiles, n_tiles, n_seqs, T, n_heads, causal, err, sms,
                            static_cast<cudaStream_t>(stream)));
+  return RM_OK;
+}
+
+int rm_attn_tcl_items(const int32_t* offsets, int32_t n_seqs, int32_t causal, int32_t* items) {
+  if (offsets == nullptr || items == nullptr || n_seqs < 1) return set_error(RM_E_INVAL, "bad arguments");
+  if (offsets[0] != 0) return set_error(RM_E_INVAL, "seq_offsets[0] must be 0");
+  for (int32_t i = 0; i < n_seqs; ++i) {
+    const int64_t L = static_cast<int64_t>(offsets[i + 1]) - offsets[i];
+    if (L < 1 || L > 512)
+      return set_error(RM_E_RANGE, "sequence %d has length %lld (items need 1..512)", i, (long long)L);
+  }
+  return attn_tcl_items(offsets, n_seqs, causal != 0 ? 1 : 0, items);
+}
+
+int rm_op_attn_tcl(const void* qkv, void* ctx, const int32_t* offsets, const int32_t* items,
+                   int32_t n_items, int32_t n_seqs, int32_t T, int32_t n_heads, int32_t causal,
+                   void* stream) {
+  if (qkv == nullptr || ctx == nullptr || offsets == nullptr || items == nullptr)
+    return set_error(RM_E_INVAL, "NULL argument");
+  if (n_seqs < 1 || T < 1 || n_heads < 1 || n_items < 1 || n_items > 4 * n_seqs)
+    return set_error(RM_E_INVAL, "bad sizes");
+  int dev = 0, sms = 0;
+  RM_CUDA(cudaGetDevice(&dev));
+  RM_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+  int32_t* err = nullptr;
+  RM_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_err_sink));
+  RM_LAUNCH(attn_tcl_launch(qkv, ctx, offsets, items, n_items, n_seqs, T, n_heads, causal, err, sms,
+                            static_cast<cudaStream_t>(stream)));
   return RM_OK;
 }
 

@@ -85,6 +85,23 @@ __device__ __forceinline__ uint32_t low_bits(int x) {
   return x <= 0 ? 0u : (x >= 32 ? 0xffffffffu : ((1u << x) - 1u));
 }
 
+// Named barrier 1 over the 512 softmax threads that also ANDs a flag across
+// them: every thread leaves with the same answer, so a bounded wait that gave
+// up in one thread ends the loop in all of them together (none is left at a
+// barrier that the others will not reach).
+__device__ __forceinline__ bool softmax_bar_and(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 512, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u)
+      : "memory");
+  return r != 0;
+}
+
 // The same with A read from tensor memory (M = 128 lanes, two 16-bit
 // elements of a row per 32-bit column).
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
@@ -408,6 +425,311 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Longer rows: head dim 64, sequences of up to 512 tokens.  A CTA takes a
+// work item -- 128 consecutive query rows of one sequence -- and a group of
+// heads, one head at a time:
+//   warp 0, one lane : TMA producer -- Q (the item's 128 rows) and the K
+//                      chunks of the sequence (128 key rows each, at most 4)
+//                      once the previous head's S is computed; the V chunks
+//                      once the previous head's P V is done;
+//   warp 1, one lane : tcgen05.mma -- S_c = Q K_c^T for every chunk c into
+//                      TMEM columns 128c.., then, chunk by chunk as the
+//                      softmax releases P_c, O += P_c V_c (A = P_c from TMEM,
+//                      B = V_c through the MN-major descriptor) into columns
+//                      64..127, which chunk 0's scores no longer need by then;
+//   warps 2..17      : four softmax groups, group g owning key chunk g of
+//                      every row (one thread per row and group).  Each group
+//                      takes its chunk's maximum; the four maxima meet in
+//                      shared memory, so the row's exponentials use the
+//                      row's own maximum (the exact softmax, no rescaling);
+//                      P_c goes over the scores as bf16, the four partial sums
+//                      meet the same way, and group g writes context dims
+//                      16g..16g+15 of the row.
+// The whole of TMEM (512 columns) holds one head's scores, so heads do not
+// overlap in TMEM; the next head's loads overlap this head's softmax.
+constexpr int kTclChunks = 4;                          // key chunks: up to 512 keys
+constexpr int kTclThreads = 64 + 4 * 128;
+
+struct TclSmem {
+  static constexpr int kBox = kTcRows * kTcDim * 2;    // 16 KB
+  static constexpr int kQ = 0;
+  static constexpr int kK = kBox;                      // K chunk c at kK + c * kBox
+  static constexpr int kV = kK + kTclChunks * kBox;    // V chunk c at kV + c * kBox
+  static constexpr int kRed = kV + kTclChunks * kBox;  // float [2][4][128]: partial max, sum
+  // qk_full v_full s_full o_full p_full[4] tmem_free
+  static constexpr int kBarOff = kRed + 2 * 4 * 128 * 4;
+  static constexpr int kBars = 9;
+  static constexpr int kTmemSlotOff = kBarOff + kBars * 8;
+  static constexpr int kBytes = kTmemSlotOff + 16 + 1024;   // + 1024-byte alignment slack
+  static_assert(kBytes <= 232448, "fits one CTA's shared memory");
+};
+
+__global__ void __launch_bounds__(kTclThreads, 1)
+    attn_tcl_kernel(const __grid_constant__ CUtensorMap tm, bf16* __restrict__ ctx,
+                    const int32_t* __restrict__ offsets, const int32_t* __restrict__ items,
+                    int n, int T, int H, int nh, int hpc, float scale_log2, int causal,
+                    int* __restrict__ err, L2PrefetchArgs pf) {
+  using SL = TclSmem;
+  extern __shared__ uint8_t tc_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tc_raw) + 1023) &
+                                           ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t bar0 = sbase + SL::kBarOff;
+  const uint32_t qk_full = bar0, v_full = bar0 + 8, s_full = bar0 + 16, o_full = bar0 + 24;
+  auto p_full = [&](int c) { return bar0 + 32u + 8u * c; };
+  const uint32_t tmem_free = bar0 + 64;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + SL::kTmemSlotOff);
+  float* red_max = reinterpret_cast<float*>(sm + SL::kRed);   // [4][128]
+  float* red_sum = red_max + 4 * 128;                          // [4][128]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qk_full, 1);
+    mbar_init(v_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(o_full, 1);
+    for (int c = 0; c < kTclChunks; ++c) mbar_init(p_full(c), 4);   // the group's four warps
+    mbar_init(tmem_free, 16);                                      // every softmax warp
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(tmem_slot))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_launch_dependents();
+  l2_prefetch_share(pf);
+  pdl_wait();
+
+  // work item: sequence s, query rows [q0, q0 + 128) of it
+  const int it = items[blockIdx.x];
+  const int s = it >> 2, qt = it & 3;
+  const int h0 = blockIdx.y * hpc;
+  const bool seq_ok = in_bounds(s >= 0 && s < n);
+  const int r0 = seq_ok ? offsets[s] : 0;
+  const int L = seq_ok ? offsets[s + 1] - r0 : 0;
+  const int q0 = qt * kTcRows;
+  // checked build: whole sequences of 1..512 tokens inside the batch, a query
+  // tile inside its sequence; a failed item does no work
+  const bool item_ok = in_bounds(seq_ok && L >= 1 && L <= kTclChunks * kTcRows && r0 >= 0 &&
+                                 r0 + L <= T && q0 < L);
+  const int nhl = item_ok ? min(hpc, nh - h0) : 0;
+  const int nc = (L + kTcRows - 1) / kTcRows;                // key chunks of this sequence
+  // causal: a query tile sees keys up to its last row only
+  const int kend_tile = causal ? min(L, q0 + kTcRows) : L;
+  const int nc_used = (kend_tile + kTcRows - 1) / kTcRows;
+
+  if (warp == 0) {
+    // ---- TMA producer ----
+    if (lane == 0) {
+      int nqk = 0, nv = 0;
+      for (int j = 0; j < nhl; ++j) {
+        const int col = (h0 + j) * kTcDim;
+        if (j > 0 && !mbar_wait(s_full, (j - 1) & 1)) {        // Q and K of head j-1 consumed
+          atomicAdd(err + ERR_TIMEOUT, 1);
+          break;
+        }
+        mbar_arrive_expect_tx(qk_full, (1 + nc_used) * SL::kBox);
+        tma_load_2d(sbase + SL::kQ, &tm, col, r0 + q0, qk_full);
+        for (int c = 0; c < nc_used; ++c)
+          tma_load_2d(sbase + SL::kK + c * SL::kBox, &tm, H + col, r0 + c * kTcRows, qk_full);
+        ++nqk;
+        if (j > 0 && !mbar_wait(o_full, (j - 1) & 1)) {        // V of head j-1 consumed
+          atomicAdd(err + ERR_TIMEOUT, 1);
+          break;
+        }
+        mbar_arrive_expect_tx(v_full, nc_used * SL::kBox);
+        for (int c = 0; c < nc_used; ++c)
+          tma_load_2d(sbase + SL::kV + c * SL::kBox, &tm, 2 * H + col, r0 + c * kTcRows, v_full);
+        ++nv;
+      }
+      // no copy into this CTA's shared memory may be in flight when it exits
+      bool drained = true;
+      if (nqk > 0) drained = mbar_wait(qk_full, (nqk - 1) & 1);
+      if (drained && nv > 0) mbar_wait(v_full, (nv - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(kTcRows, kTcRows);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(kTcRows, kTcDim) | (1u << 16);   // B MN-major
+      int js = 0, jo = 0;
+      for (int j = 0; j < nhl; ++j) {
+        if (!mbar_wait(qk_full, j & 1) || (j > 0 && !mbar_wait(tmem_free, (j - 1) & 1))) {
+          atomicAdd(err + ERR_TIMEOUT, 1);
+          break;
+        }
+        tc_fence_after();
+        const uint64_t qd = smem_desc_k_sw128(sbase + SL::kQ);
+        for (int c = 0; c < nc_used; ++c) {
+          const uint64_t kd = smem_desc_k_sw128(sbase + SL::kK + c * SL::kBox);
+          const uint32_t d = tmem + static_cast<uint32_t>(c * kTcRows);
+#pragma unroll
+          for (int ks = 0; ks < kTcDim / 16; ++ks)
+            mma_bf16_ss(d, qd + 2ull * ks, kd + 2ull * ks, idesc_s, ks > 0);
+        }
+        tc_commit<1>(s_full);
+        ++js;
+        bool ok = mbar_wait(v_full, j & 1);
+        for (int c = 0; c < nc_used && ok; ++c) {
+          if (!mbar_wait(p_full(c), j & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          // 16-key steps holding a key some row of the tile admits
+          const int nk16 = min((kend_tile - c * kTcRows + 15) / 16, kTcRows / 16);
+          const uint32_t v = sbase + SL::kV + c * SL::kBox;
+          const uint32_t pc = tmem + static_cast<uint32_t>(c * kTcRows);
+          for (int kb = 0; kb < nk16; ++kb)
+            mma_bf16_ts(tmem + kTcDim, pc + kb * 8, smem_desc_mn_sw128(v + kb * 16 * 128), idesc_o,
+                        c > 0 || kb > 0);
+        }
+        if (!ok) {
+          atomicAdd(err + ERR_TIMEOUT, 1);
+          break;
+        }
+        tc_commit<1>(o_full);
+        ++jo;
+      }
+      // TMEM is freed after the last MMAs have completed (bounded waits)
+      bool drained = true;
+      if (js > 0) drained = mbar_wait(s_full, (js - 1) & 1);
+      if (drained && jo > 0) mbar_wait(o_full, (jo - 1) & 1);
+    }
+  } else {
+    // ---- softmax groups: group g = key chunk g, one tile row per thread ----
+    const int g = (warp - 2) >> 2;
+    const int qtr = warp & 3;                   // TMEM lane quarter of this warp
+    const int i = qtr * 32 + lane;              // tile row = TMEM lane
+    const bool row_ok = q0 + i < L;
+    // keys [0, kend) of the sequence; those of chunk g as chunk columns [0, klen)
+    const int kend = !row_ok ? 0 : (causal ? q0 + i + 1 : L);
+    const int klen = max(0, min(kend - g * kTcRows, kTcRows));
+    // 32-column groups of chunk g that some row of this warp admits
+    const int wlen = __reduce_max_sync(0xffffffffu, klen);
+    bool need[4];
+#pragma unroll
+    for (int gi = 0; gi < 4; ++gi) need[gi] = gi * 32 < wlen;
+    const bool active = g < nc_used;
+    const uint32_t treg = tmem + (static_cast<uint32_t>(qtr * 32) << 16) + g * kTcRows;
+    const int r = r0 + q0 + i;
+
+    for (int j = 0; j < nhl; ++j) {
+      int klen_h;
+      asm volatile("mov.b32 %0, %1;" : "=r"(klen_h) : "r"(klen));
+      const bool s_ok = mbar_wait(s_full, j & 1);
+      if (!s_ok && lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
+      tc_fence_after();
+      uint32_t vm[4];
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) vm[gi] = low_bits(klen_h - 32 * gi);
+      float m = -INFINITY;
+      if (active && s_ok) {
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          if (!need[gi]) continue;
+          uint32_t sv[32];
+          tmem_ld_32cols(treg + gi * 32, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (vm[gi] & (1u << c)) m = fmaxf(m, __uint_as_float(sv[c]));
+        }
+      }
+      red_max[g * 128 + i] = m;
+      if (!softmax_bar_and(s_ok)) break;          // the softmax warps, all or none
+      float mrow = red_max[i];
+#pragma unroll
+      for (int gg = 1; gg < kTclChunks; ++gg) mrow = fmaxf(mrow, red_max[gg * 128 + i]);
+      const float msc = kend > 0 ? mrow * scale_log2 : 0.f;
+      // P = exp2(s * scale_log2 - max * scale_log2) on the row's keys of
+      // this chunk, 0 elsewhere, written over the scores as bf16 pairs (keys
+      // 32gi.. to columns 16gi.., already read); the sum in fp32 before P is
+      // rounded to bf16
+      const uint64_t sc2 = f32x2_splat(scale_log2), nm2 = f32x2_splat(-msc);
+      uint64_t l2 = 0ull;
+      if (active) {
+#pragma unroll
+        for (int gi = 0; gi < 4; ++gi) {
+          uint32_t pk[16];
+          if (need[gi]) {
+            uint32_t sv[32];
+            tmem_ld_32cols(treg + gi * 32, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c2 = 0; c2 < 16; ++c2) {
+              const bool in0 = (vm[gi] >> (2 * c2)) & 1u, in1 = (vm[gi] >> (2 * c2 + 1)) & 1u;
+              float x0, x1;
+              f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[2 * c2]),
+                                                __uint_as_float(sv[2 * c2 + 1])),
+                                     sc2, nm2),
+                           x0, x1);
+              const float p0 = in0 ? ex2_approx_ftz(x0) : 0.f;
+              const float p1 = in1 ? ex2_approx_ftz(x1) : 0.f;
+              l2 = f32x2_add(l2, f32x2_pack(p0, p1));
+              pk[c2] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int c2 = 0; c2 < 16; ++c2) pk[c2] = 0u;
+          }
+          tmem_st_16cols(treg + gi * 16, pk);
+        }
+        // P's stores complete before the MMA reads them
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full(g));
+      }
+      float l0, l1;
+      f32x2_unpack(l2, l0, l1);
+      red_sum[g * 128 + i] = l0 + l1;
+      const bool o_ok = mbar_wait(o_full, j & 1);
+      if (!o_ok && lane == 0) atomicAdd(err + ERR_TIMEOUT, 1);
+      if (!softmax_bar_and(o_ok)) break;
+      tc_fence_after();
+      float l = red_sum[i];
+#pragma unroll
+      for (int gg = 1; gg < kTclChunks; ++gg) l += red_sum[gg * 128 + i];
+      // context dims 16g..16g+15 of the row: O columns 64 + 16g..
+      uint32_t ov[16];
+      tmem_ld_16cols(tmem + (static_cast<uint32_t>(qtr * 32) << 16) + kTcDim + 16 * g, ov);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tmem_free);   // TMEM may take the next head's S
+      if (kend > 0) {
+        const float inv = 1.0f / l;
+        uint4* dst = reinterpret_cast<uint4*>(ctx + static_cast<size_t>(r) * H + (h0 + j) * kTcDim +
+                                              16 * g);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            wv[e] = pack_bf16x2(__uint_as_float(ov[8 * u + 2 * e]) * inv,
+                                __uint_as_float(ov[8 * u + 2 * e + 1]) * inv);
+          dst[u] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
 }  // namespace
 
 int32_t attn_tc_tiles(const int32_t* offsets, int32_t n, int32_t* tiles) {
@@ -452,6 +774,59 @@ cudaError_t attn_tc_launch(const void* qkv, void* ctx, const int32_t* offsets,
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kTcDim));
   launch_k(attn_tc_kernel, grid, dim3(kTcThreads), SL::kBytes, st, tm, static_cast<bf16*>(ctx), offsets,
            tiles, n, T, H, nh, hpc, scale_log2, causal, err, pa);
+  return cudaGetLastError();
+}
+
+int32_t attn_tcl_items(const int32_t* offsets, int32_t n, int32_t causal, int32_t* items) {
+  // (sequence, query tile) pairs, those with the most key chunks first so that
+  // the grid's last CTAs are short ones
+  int32_t count[kTclChunks + 1] = {0};
+  auto chunks = [&](int32_t i, int32_t q) {
+    const int32_t L = offsets[i + 1] - offsets[i];
+    const int32_t kend = causal ? std::min(L, (q + 1) * kTcRows) : L;
+    return (kend + kTcRows - 1) / kTcRows;
+  };
+  for (int32_t i = 0; i < n; ++i)
+    for (int32_t q = 0; q * kTcRows < offsets[i + 1] - offsets[i]; ++q) ++count[chunks(i, q)];
+  int32_t start[kTclChunks + 1];
+  int32_t k = 0;
+  for (int32_t c = kTclChunks; c >= 1; --c) {
+    start[c] = k;
+    k += count[c];
+  }
+  for (int32_t i = 0; i < n; ++i)
+    for (int32_t q = 0; q * kTcRows < offsets[i + 1] - offsets[i]; ++q)
+      items[start[chunks(i, q)]++] = (i << 2) | q;
+  return k;
+}
+
+cudaError_t attn_tcl_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                            const int32_t* items, int n_items, int n, int T, int nh, int causal,
+                            int* err, int num_sms, cudaStream_t st, const L2Prefetch& pf) {
+  using SL = TclSmem;
+  if (n_items < 1 || T < 1) return cudaSuccess;
+  const int H = nh * kTcDim;
+  CUtensorMap tm;
+  const char* why = "";
+  // exactly T rows: rows past the batch read as zeros
+  if (!make_tmap_bf16(&tm, qkv, static_cast<uint64_t>(T), static_cast<uint64_t>(3 * H), kTcRows,
+                      &why))
+    return cudaErrorInvalidValue;
+  static const cudaError_t attr_err =
+      cudaFuncSetAttribute(attn_tcl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kBytes);
+  if (attr_err != cudaSuccess) return attr_err;
+  // one CTA per SM: all heads of an item in one CTA unless that leaves SMs idle
+  const int groups = std::min(nh, std::max(1, (num_sms + n_items - 1) / n_items));
+  const int hpc = (nh + groups - 1) / groups;
+  dim3 grid(n_items, (nh + hpc - 1) / hpc);
+  L2PrefetchArgs pa;
+  for (int k = 0; k < 2; ++k) {
+    pa.ptr[k] = pf.ptr[k];
+    pa.bytes[k] = pf.bytes[k];
+  }
+  const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(kTcDim));
+  launch_k(attn_tcl_kernel, grid, dim3(kTclThreads), SL::kBytes, st, tm, static_cast<bf16*>(ctx),
+           offsets, items, n, T, H, nh, hpc, scale_log2, causal, err, pa);
   return cudaGetLastError();
 }
 

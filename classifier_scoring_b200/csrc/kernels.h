@@ -129,6 +129,15 @@ cudaError_t attn_tile_launch(const void* qkv, void* ctx, const int32_t* offsets,
 cudaError_t attn_tc_launch(const void* qkv, void* ctx, const int32_t* offsets,
                            const int32_t* tiles, int n_tiles, int n, int T, int nh, int causal,
                            int* err, int num_sms, cudaStream_t st, const L2Prefetch& pf = {});
+// Tensor-core attention for sequences of up to 512 tokens, head dim 64: work
+// items of 128 query rows of one sequence, item = (sequence << 2) | tile.
+// attn_tcl_items writes the items of every sequence (offsets: host, n + 1
+// entries, every length 1..512; items: capacity sum of ceil(L / 128) <= 4n),
+// those with the most key chunks first, and returns their count.
+int32_t attn_tcl_items(const int32_t* offsets, int32_t n, int32_t causal, int32_t* items);
+cudaError_t attn_tcl_launch(const void* qkv, void* ctx, const int32_t* offsets,
+                            const int32_t* items, int n_items, int n, int T, int nh, int causal,
+                            int* err, int num_sms, cudaStream_t st, const L2Prefetch& pf = {});
 // Greedy cut of the packed batch into tiles of whole sequences of at most 128
 // rows (host; every sequence at most 128 tokens): writes tiles[0..n_tiles],
 // returns n_tiles.

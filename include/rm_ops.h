@@ -190,6 +190,32 @@ int rm_op_attn_tc(const void* qkv, void* ctx, const int32_t* offsets, const int3
                   int32_t n_tiles, int32_t n_seqs, int32_t T, int32_t n_heads, int32_t causal,
                   void* stream);
 
+/* Work items of the long-row tensor-core attention (rm_op_attn_tcl): every
+ * run of 128 query rows of a sequence, item = (sequence << 2) | tile (tile
+ * 0..3 covers rows 128*tile ..), those that read the most 128-key chunks
+ * first (causal != 0: a tile reads keys up to its own last row only).
+ * offsets: HOST int32[n_seqs+1] with offsets[0] = 0 and every length in
+ * 1..512; items: HOST int32[4 * n_seqs] (caller-owned).  Returns the item
+ * count (sum over sequences of ceil(L / 128)), or RM_E_INVAL / RM_E_RANGE.
+ * This cut has no counterpart in the pages; it is the layout of the kernel
+ * below. */
+int rm_attn_tcl_items(const int32_t* offsets, int32_t n_seqs, int32_t causal, int32_t* items);
+
+/* rm_op_attn_tc for sequences of up to 512 tokens (head_dim 64): per item of
+ * rm_attn_tcl_items and head, S = Q K^T for the item's 128 query rows against
+ * every 128-key chunk of its sequence (tcgen05.mma into tensor memory), the
+ * row softmax over the row's own sequence (c <= r too when causal) in fp32
+ * with P rounded to bf16, and C = P V (tcgen05.mma), written to ctx.  qkv:
+ * bf16 [T][3H], H = 64 * n_heads; ctx: bf16 [T][H]; offsets: DEVICE
+ * int32[n_seqs+1] with offsets[n_seqs] = T (host value T); items: DEVICE
+ * int32[n_items] as rm_attn_tcl_items wrote them for the same offsets and
+ * causal flag.  RM_E_INVAL for NULL pointers, sizes < 1 or n_items >
+ * 4 * n_seqs; waits that give up (none in normal operation) count into an
+ * internal error word. */
+int rm_op_attn_tcl(const void* qkv, void* ctx, const int32_t* offsets, const int32_t* items,
+                   int32_t n_items, int32_t n_seqs, int32_t T, int32_t n_heads, int32_t causal,
+                   void* stream);
+
 /* The materialised attention step (rm_op_attn_scores -> rm_op_softmax ->
  * rm_op_attn_context) without any device allocation: the score matrix and the
  * per-call metadata live in one file-scope device array of 8 MiB of scores

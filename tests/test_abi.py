@@ -136,6 +136,27 @@ def test_attn_tc_tiles_cut_whole_sequences_greedily(seed):
     assert np.all(rows[:-1] + lens[tiles[1:-1]] > 128)
 
 
+def test_attn_tcl_items_cover_every_query_tile_heaviest_first():
+    rng = np.random.default_rng(5)
+    for causal in (0, 1):
+        lens = rng.integers(1, 513, 40)
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        items = rm.ops.attn_tcl_items(off, causal)
+        want = sorted((i, q) for i, L in enumerate(lens) for q in range((L + 127) // 128))
+        assert sorted((int(it) >> 2, int(it) & 3) for it in items) == want
+        chunks = [(min(lens[it >> 2], 128 * ((it & 3) + 1)) if causal else lens[it >> 2]) for it in items]
+        chunks = [(c + 127) // 128 for c in chunks]
+        assert chunks == sorted(chunks, reverse=True)
+
+
+def test_attn_tcl_items_reject_long_or_empty_sequences():
+    out = np.zeros(8, dtype=np.int32)
+    for lens in ([513], [3, 0, 2]):
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        rc = rm.lib().rm_attn_tcl_items(off.ctypes.data, len(lens), 0, out.ctypes.data)
+        assert rc < 0
+
+
 def test_attn_tc_tiles_reject_long_or_empty_sequences():
     for lens in ([5, 129, 3], [4, 0, 2]):
         off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)

@@ -681,6 +681,64 @@ def test_attention_tc(lens, nh, causal):
     _attention_ref_check(f64(qkv), f64(ctx), off, nh, d, causal)
 
 
+def _attn_tcl(qkv, ctx, off, nh, causal):
+    items = rm.ops.attn_tcl_items(off, causal)
+    rm.ops.attn_tcl(qkv, ctx, dev(off, torch.int32), dev(items, torch.int32), len(items),
+                    len(off) - 1, int(off[-1]), nh, causal)
+    return items
+
+
+@pytest.mark.parametrize("lens", [
+    [129],                                              # two key chunks, one row past a tile
+    [512],                                              # four full chunks and query tiles
+    [1, 512, 130, 7, 300, 256, 128],                    # ragged, chunk and tile edges
+    [200] * 6,                                          # uniform
+    [383, 385, 5],                                      # around the third chunk edge
+], ids=["129", "512", "ragged", "uniform", "edges"])
+@pytest.mark.parametrize("nh", [2, 12])
+@pytest.mark.parametrize("causal", [0, 1])
+def test_attention_tcl(lens, nh, causal):
+    """tcgen05 attention on 128-row query tiles of sequences up to 512 tokens
+    against the oracle's attention, every row and head."""
+    d = 64
+    H = nh * d
+    lens = np.array(lens)
+    off = synth.offsets_from_lengths(lens)
+    rng = np.random.default_rng(nh * 11 + causal + len(lens))
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    ctx = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    _attn_tcl(qkv, ctx, off, nh, causal)
+    torch.cuda.synchronize()
+    _attention_ref_check(f64(qkv), f64(ctx), off, nh, d, causal)
+
+
+def test_attention_tcl_long_stream_against_tiles_and_oracle():
+    """A fused call of the lengths-5..500 stream's shape (256 sequences, 12
+    heads of 64): every output finite, within bf16 rounding of the packed-row
+    tile kernel everywhere, and bit-identical on a repeat."""
+    nh, d = 12, 64
+    H = nh * d
+    rng = np.random.default_rng(77)
+    lens = rng.integers(5, 501, 256)
+    off = synth.offsets_from_lengths(lens)
+    T = int(off[-1])
+    qkv = dev(qkv_for(T, H, rng) * 1.5, torch.bfloat16)
+    a = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    a2 = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    b = torch.full((T, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+    _attn_tcl(qkv, a, off, nh, 0)
+    _attn_tcl(qkv, a2, off, nh, 0)
+    rm.ops.attn_tiles(qkv, b, dev(off, torch.int32), len(lens), T, nh, d, 0, max_len=500)
+    torch.cuda.synchronize()
+    A, B = f64(a), f64(b)
+    assert np.all(np.isfinite(A))
+    assert torch.equal(a, a2)
+    X = f64(qkv)
+    vmax = np.repeat(np.maximum.reduceat(np.abs(X[:, 2 * H:]), off[:-1], axis=0), lens, axis=0)
+    assert np.all(np.abs(A - B) <= 1.5 * BF16_REL * (vmax + np.abs(B)) + 1e-6)
+
+
 def test_attention_tc_bench_shape_against_tiles_and_oracle():
     """A fused call of the BERT-base stream's shape (512 sequences of 2..100
     tokens, 12 heads of 64): every output finite, within bf16 rounding of the
