@@ -58,8 +58,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic per launch of the dominant kernel (tcgen05 GEMM) from one ncu
 # capture; valid only for the code it was taken on (code_sha of gemm_tc.cu).  Mean of the 48 projections of one fused call of eight DP
 # batches, T = 27829 (the default step's calls average T = 25457).
-GEMM_TRAFFIC = {"src_sha": "0cc3c5de254ba009", "workload": "bert-base-len2-100", "fuse": 8,
-                "bytes_per_launch": 131918603}
+GEMM_TRAFFIC = {"src_sha": "3db551ef7a0e0283", "workload": "bert-base-len2-100", "fuse": 8,
+                "bytes_per_launch": 131929445}
 
 
 def code_sha(path):
@@ -671,7 +671,8 @@ def b200_arm(args):
     # kernel table and roofline from one extra single-stream step after timing
     prof = ex.profiled_step(sc)
     # and the same step's kernels timed by CUPTI, without per-launch events
-    cup = ex.cupti_step(sc)
+    # (not under another profiler such as ncu)
+    cup = ex.cupti_step(sc) if not args.no_cupti else None
 
     # ---- end to end through rm_score_host (pinned host buffers) ----
     b_tok, b_seq, b_off = ex.b_tok, ex.b_seq, ex.b_off
@@ -828,7 +829,7 @@ def process_repeats(args, name, first):
     vals, errors = [first], []
     cmd = [sys.executable, os.path.abspath(__file__), "--workload", name, "--steps", str(args.steps),
            "--warmup", str(args.warmup), "--fuse", str(args.fuse), "--lanes", str(args.lanes),
-           "--repeats", "1", "--processes", "1", "--no-extra", "--no-cpu-baseline"]
+           "--repeats", "1", "--processes", "1", "--no-extra", "--no-cpu-baseline", "--no-cupti"]
     for _ in range(args.processes - 1):
         r = subprocess.run(cmd, capture_output=True, text=True)
         try:
@@ -1345,6 +1346,8 @@ def main():
                     help="timed batch-1 requests per length of the TinyBERT workload")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cupti", action="store_true",
+                    help="skip the CUPTI-timed step of the kernel table (for runs under ncu)")
     ap.add_argument("--clocks-dir", default=None,
                     help="also write the raw clock samples of the timed region as CSV here")
     ap.add_argument("--only", default="",
