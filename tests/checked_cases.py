@@ -34,6 +34,19 @@ def valid_inputs():
         cfg = config_for(w.shape, max_batch_seqs=8, max_tokens=256, max_len=64, attn_impl=attn)
         with rm.Scorer(cfg, synth.make_weights(w.shape, w.seed)) as sc:
             res[f"tiny_err_{attn}"] = float(np.max(np.abs(gpu_scores(sc, ids, off) - gold)))
+    # an encoder with rows past 128 tokens: the long-row tensor-core attention
+    enc = synth.ModelShape(synth.ENC_POSTLN, 2, 256, 4, 1024, 5000, 600, synth.W_BF16,
+                           synth.GELU_ERF, 1e-12)
+    eflat = synth.make_weights(enc, 11)
+    em = oracle_model(enc, eflat)
+    cfg = config_for(enc, max_batch_seqs=16, max_tokens=2048, max_len=600, attn_impl=rm.ATTN_FUSED)
+    with rm.Scorer(cfg, eflat) as sc:
+        lens = np.array([1, 200, 130, 7, 300])
+        o = synth.offsets_from_lengths(lens)
+        tids = synth.make_token_ids(int(o[-1]), enc.vocab, 6)
+        got = gpu_scores(sc, tids, o)
+        want = np.array([O.score_one(em, tids[o[i]:o[i + 1]]) for i in range(len(lens))])
+        res["enc_long_err_0"] = float(np.max(np.abs(got - want)))
     # the decoder paths: tiles, materialised, and shared prefixes with the vote of best-of-N
     dec = synth.ModelShape(synth.DEC_PRELN, 2, 256, 4, 1024, 5000, 600, synth.W_BF16,
                            synth.GELU_ERF, 1e-5)
