@@ -631,6 +631,11 @@ __global__ void __launch_bounds__(kTclThreads, 1)
 #pragma unroll
       for (int gi = 0; gi < 4; ++gi) vm[gi] = low_bits(klen_h - 32 * gi);
       float m = -INFINITY;
+      // groups that every row of the warp admits in full (most of a long
+      // sequence) take no per-column mask
+      bool full[4];
+#pragma unroll
+      for (int gi = 0; gi < 4; ++gi) full[gi] = __all_sync(0xffffffffu, vm[gi] == 0xffffffffu);
       if (active && s_ok) {
 #pragma unroll
         for (int gi = 0; gi < 4; ++gi) {
@@ -638,9 +643,14 @@ __global__ void __launch_bounds__(kTclThreads, 1)
           uint32_t sv[32];
           tmem_ld_32cols(treg + gi * 32, sv);
           tmem_wait_ld();
+          if (full[gi]) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (vm[gi] & (1u << c)) m = fmaxf(m, __uint_as_float(sv[c]));
+            for (int c = 0; c < 32; ++c) m = fmaxf(m, __uint_as_float(sv[c]));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (vm[gi] & (1u << c)) m = fmaxf(m, __uint_as_float(sv[c]));
+          }
         }
       }
       red_max[g * 128 + i] = m;
@@ -663,18 +673,32 @@ __global__ void __launch_bounds__(kTclThreads, 1)
             uint32_t sv[32];
             tmem_ld_32cols(treg + gi * 32, sv);
             tmem_wait_ld();
+            if (full[gi]) {
 #pragma unroll
-            for (int c2 = 0; c2 < 16; ++c2) {
-              const bool in0 = (vm[gi] >> (2 * c2)) & 1u, in1 = (vm[gi] >> (2 * c2 + 1)) & 1u;
-              float x0, x1;
-              f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[2 * c2]),
-                                                __uint_as_float(sv[2 * c2 + 1])),
-                                     sc2, nm2),
-                           x0, x1);
-              const float p0 = in0 ? ex2_approx_ftz(x0) : 0.f;
-              const float p1 = in1 ? ex2_approx_ftz(x1) : 0.f;
-              l2 = f32x2_add(l2, f32x2_pack(p0, p1));
-              pk[c2] = pack_bf16x2(p0, p1);
+              for (int c2 = 0; c2 < 16; ++c2) {
+                float x0, x1;
+                f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[2 * c2]),
+                                                  __uint_as_float(sv[2 * c2 + 1])),
+                                       sc2, nm2),
+                             x0, x1);
+                const float p0 = ex2_approx_ftz(x0), p1 = ex2_approx_ftz(x1);
+                l2 = f32x2_add(l2, f32x2_pack(p0, p1));
+                pk[c2] = pack_bf16x2(p0, p1);
+              }
+            } else {
+#pragma unroll
+              for (int c2 = 0; c2 < 16; ++c2) {
+                const bool in0 = (vm[gi] >> (2 * c2)) & 1u, in1 = (vm[gi] >> (2 * c2 + 1)) & 1u;
+                float x0, x1;
+                f32x2_unpack(f32x2_fma(f32x2_pack(__uint_as_float(sv[2 * c2]),
+                                                  __uint_as_float(sv[2 * c2 + 1])),
+                                       sc2, nm2),
+                             x0, x1);
+                const float p0 = in0 ? ex2_approx_ftz(x0) : 0.f;
+                const float p1 = in1 ? ex2_approx_ftz(x1) : 0.f;
+                l2 = f32x2_add(l2, f32x2_pack(p0, p1));
+                pk[c2] = pack_bf16x2(p0, p1);
+              }
             }
           } else {
 #pragma unroll
