@@ -46,3 +46,17 @@ def test_sharing_saves_memory_on_bert():
     S = 12 * 64 * 51 * 56
     off, nb, first, last, peak = rm.ops.arena_plan(cfg, T, 64, S)
     assert peak < 0.75 * int(nb.sum())
+
+
+def test_decoder_plans_no_sublayer_output_buffers():
+    """The decoder adds its out-projection and FFN2 outputs straight into its
+    fp32 residual stream, so its plans give y1 and y2 (buffers 5 and 7) no
+    bytes; the encoder's keep one bf16 row per token each."""
+    T, S = 3000, 0
+    dec = config_for(synth.GPT_1P3B, max_len=560)
+    off, nb, first, last, peak = rm.ops.arena_plan(dec, T, 8, S)
+    assert nb[5] == 0 and nb[7] == 0
+    assert nb[0] == T * synth.GPT_1P3B.hidden * 4          # x in fp32
+    enc = config_for(synth.BERT_BASE, max_len=100)
+    off, nb, first, last, peak = rm.ops.arena_plan(enc, T, 64, S)
+    assert nb[5] == nb[7] == T * synth.BERT_BASE.hidden * 2
